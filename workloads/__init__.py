@@ -1,0 +1,3 @@
+"""Seeded synthetic inputs (random draws only; none of the layer's arithmetic)."""
+from .synth import (HIDDEN, INTER, NUM_EXPERTS, TOP_K, GROUP, LayerWeights, layer_weights,
+                    tokens, token_stream, zipf_router_bias, stack_token_seed, WORKLOADS)
