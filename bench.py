@@ -1,0 +1,373 @@
+"""Benchmark of the W4 g32 MoE layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode_e512_t1|verify_e512_t4|stack40_e512_t1|prefill_e512_t2048_zipf|reduced_e32_t1]
+
+A step is one pass of the whole layer (router, top-k, routed gate/up, down,
+shared expert, combine) over one batch of synthetic input: one token for the
+default batch-1 decode workload, each step a new seeded token.  Inputs and
+weights are resident in HBM when the timed region starts; L2 is flushed
+(256 MiB write) before every step, outside the per-step CUDA events.
+Rank 0 prints one JSON line.  With N > 1 (torchrun) every rank runs its own
+independent token stream on its own GPU: replicas, no collective on the data
+path; time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer decode tokens/s and achieved HBM GB/s (W4 g32, 512e top-8, T=1)"
+H, I = 2560, 768
+ROUTED_BYTES = 3_317_760        # per expert: int4 codes + bf16 scales
+SHARED_BYTES = 11_796_480       # bf16 shared expert
+L2_FLUSH_BYTES = 256 << 20
+
+
+def router_bytes(E):
+    return E * H * 2
+
+
+def decode_bytes(E, union):
+    """Algorithmic bytes of one call: distinct routed experts + shared + router."""
+    return union * ROUTED_BYTES + SHARED_BYTES + router_bytes(E)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.rows = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                r = subprocess.run(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                    "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                   timeout=5)
+                if r.returncode == 0 and r.stdout.strip():
+                    self.rows.append([c.strip() for c in r.stdout.strip().split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._t.join(timeout=10)
+
+    def summary(self):
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4)
+                          if len(r) > 5 + i and r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ------------------------------------------------------------------ reference arm (the oracle)
+
+def cpu_oracle_rate(workload: str, seconds: float = 15.0, max_tokens: int = 64):
+    """Time the fp64 oracle on a bounded sample of the workload (rank 0 only)."""
+    import numpy as np
+    import torch
+    import oracle
+    import workloads
+    wl = workloads.WORKLOADS[workload]
+    E = wl["num_experts"]
+    lw = workloads.layer_weights(E, seed=wl.get("weight_seed", 100), device="cpu" if E <= 32 else
+                                 ("cuda" if torch.cuda.is_available() else "cpu"))
+    host = lw.host_arrays()
+    if workload.startswith("prefill"):
+        host["router_bias"] = workloads.zipf_router_bias(E, wl["zipf_s"]).numpy()
+    T = min(wl["T"], 4)
+    seeds = wl.get("token_seeds") or wl.get("call_seeds") or [1 + t for t in range(1000)]
+    n, t0 = 0, time.perf_counter()
+    calls = 0
+    while calls < max_tokens and (time.perf_counter() - t0) < seconds:
+        x = workloads.tokens(T, seed=seeds[calls % len(seeds)], device="cpu")
+        xb = x.view(torch.int16).numpy().view(np.uint16)
+        oracle.moe_layer(xb, host, 8)
+        n += T
+        calls += 1
+    dt = time.perf_counter() - t0
+    cores = len(os.sched_getaffinity(0))
+    threads = torch.get_num_threads()
+    return {"value": n / dt, "unit": "tokens/s", "cores": cores, "threads": threads,
+            "kind": "oracle",
+            "sample": f"{calls} calls of T={T} of {workload} through the fp64 numpy oracle "
+                      f"({dt:.1f} s of host time, numpy/BLAS threads as configured: {threads})"}
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    steps, warm = args.steps, args.warmup
+    import numpy as np
+    import torch
+    import oracle
+    import workloads
+    wl = workloads.WORKLOADS[args.workload]
+    E = wl["num_experts"]
+    lw = workloads.layer_weights(E, seed=wl.get("weight_seed", 100),
+                                 device="cuda" if torch.cuda.is_available() else "cpu")
+    host = lw.host_arrays()
+    del lw
+    T = wl["T"] if wl["T"] <= 4 else 4
+    seeds = wl.get("token_seeds") or wl.get("call_seeds") or [1 + t for t in range(1000)]
+    def step(i):
+        x = workloads.tokens(T, seed=seeds[i % len(seeds)], device="cpu")
+        oracle.moe_layer(x.view(torch.int16).numpy().view(np.uint16), host, 8)
+    for i in range(warm):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(steps):
+        step(warm + i)
+    dt = time.perf_counter() - t0
+    v = steps * T / dt
+    line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": ws, "steps": steps,
+            "warmup": warm, "ms_per_step": dt * 1e3 / steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": args.workload, "T": T, "experts": E, "top_k": 8, "hidden": H,
+                       "inter": I},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": len(os.sched_getaffinity(0)),
+                             "kind": "oracle",
+                             "sample": f"{steps} calls of T={T} through the fp64 numpy oracle"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+
+def build_layers(workload, device):
+    import torch
+    import workloads
+    import weight_only_int4_fp32_b200 as lm
+    wl = workloads.WORKLOADS[workload]
+    E = wl["num_experts"]
+    T = wl["T"]
+    nlayers = wl.get("layers", 1)
+    seeds = wl.get("layer_seeds") or [wl["weight_seed"]]
+    layers = []
+    for l in range(nlayers):
+        lw = workloads.layer_weights(E, seed=seeds[l], device=device)
+        w = lw.tensors()
+        if workload.startswith("prefill"):
+            w = dict(w)
+            w["router_bias"] = workloads.zipf_router_bias(E, wl["zipf_s"]).to(device)
+        layers.append(lm.MoELayer(w, top_k=8, max_tokens=max(T, 1)))
+        del lw, w
+        torch.cuda.empty_cache()
+    return layers, E, T
+
+
+def make_inputs(workload, n, T, device):
+    import torch
+    import workloads
+    wl = workloads.WORKLOADS[workload]
+    if workload.startswith("decode") or workload.startswith("reduced"):
+        seeds = [1 + t for t in range(n)] if workload.startswith("decode") else list(range(n))
+        return [workloads.tokens(1, seed=s, device=device) for s in seeds]
+    if workload.startswith("verify"):
+        return [workloads.tokens(4, seed=10000 + i, device=device) for i in range(n)]
+    if workload.startswith("stack"):
+        return [torch.stack([workloads.tokens(1, seed=workloads.stack_token_seed(t, l), device=device)[0]
+                             for l in range(wl["layers"])]) for t in range(n)]
+    return [workloads.tokens(T, seed=wl["token_seed"] + i, device=device) for i in range(n)]
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    ws, rank, local = dist_env()
+    if ws > 1:
+        dist.init_process_group("nccl", init_method="env://", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import weight_only_int4_fp32_b200 as lm
+    layers, E, T = build_layers(args.workload, dev)
+    nsteps, nwarm = args.steps, args.warmup
+    inputs = make_inputs(args.workload, nsteps + nwarm, T, dev)
+    stack = args.workload.startswith("stack")
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def one_step(x):
+        if stack:
+            for l, layer in enumerate(layers):
+                layer.forward(x[l:l + 1], out)
+        else:
+            layers[0].forward(x, out)
+
+    # union of routed experts per step (bytes the method must read), from the routing
+    def union_of(x):
+        if stack:
+            return [8] * len(layers)
+        _, idx, _ = layers[0].forward(x, return_routing=True)
+        return [int(torch.unique(idx).numel())]
+
+    for i in range(nwarm):
+        flush.fill_(float(i))
+        one_step(inputs[i])
+    torch.cuda.synchronize()
+    unions = [union_of(inputs[nwarm + i]) for i in range(nsteps)]
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(nsteps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(nsteps)]
+    n0 = sum(l.launch_count() for l in layers)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter()
+    with ClockSampler(local) as clk:
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for i in range(nsteps):
+            flush.fill_(float(i))
+            starts[i].record(stream)
+            one_step(inputs[nwarm + i])
+            ends[i].record(stream)
+        g1.record(stream)
+        torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall
+    if ws > 1:
+        dist.barrier()
+    launches = sum(l.launch_count() for l in layers) - n0
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    kern_ms = sum(step_ms)
+    if ws > 1:
+        tt = torch.tensor([kern_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        kern_ms = float(tt.item())
+    status = [l.status() for l in layers]
+    if any(s != lm.LING_MOE_OK for s in status):
+        raise RuntimeError(f"device status {status}")
+
+    # end to end through the host-buffer entry point (pinned buffers, copies timed)
+    e2e = None
+    if not stack:
+        xh = [inputs[nwarm + i].cpu().pin_memory() for i in range(nsteps)]
+        oh = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+        for i in range(min(nwarm, 5)):
+            layers[0].forward_host(xh[i], oh)
+        torch.cuda.synchronize()
+        if ws > 1:
+            dist.barrier()
+        te = time.perf_counter()
+        for i in range(nsteps):
+            flush.fill_(float(i))
+            layers[0].forward_host(xh[i], oh)
+        te = time.perf_counter() - te
+        tt = torch.tensor([te], device=dev)
+        if ws > 1:
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e = {"value": ws * nsteps * T / float(tt.item()), "unit": "tokens/s",
+               "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2,
+               "note": "ling_moe_forward_host per step: pinned H2D copy + layer + D2H copy + "
+                       "stream sync; the L2 flush fill runs between steps inside this wall clock"}
+
+    per_call_bytes = [sum(decode_bytes(E, u) for u in us) for us in unions]
+    if args.workload.startswith("prefill"):
+        per_call_bytes = [b + 2 * T * H * 2 for b in per_call_bytes]
+    avg_bytes = sum(per_call_bytes) / len(per_call_bytes)
+    calls_per_step = len(layers)
+    avg_launch_ms = kern_ms / nsteps / calls_per_step
+    achieved = (avg_bytes / calls_per_step) / (avg_launch_ms * 1e-3) / 1e9
+    peak, peak_kind = peaks()
+    tokens = ws * nsteps * T
+    value = tokens / (kern_ms * 1e-3)
+    if rank == 0:
+        cpu = cpu_oracle_rate(args.workload if not stack else "decode_e512_t1",
+                              seconds=args.cpu_seconds) if ws == 1 and args.cpu_seconds > 0 else None
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": nsteps,
+            "warmup": nwarm, "ms_per_step": kern_ms / nsteps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "w4a16, fp32 accumulate",
+            "data": "synthetic (seeded weights and tokens, recipe in DESIGN.md)",
+            "config": {"workload": args.workload, "T": T, "experts": E, "top_k": 8, "hidden": H,
+                       "inter": I, "layers": len(layers),
+                       "l2": "flushed before every step (256 MiB write), outside the per-step events",
+                       "parallelism": f"replicas x{ws}"},
+            "us_per_layer": avg_launch_ms * 1e3,
+            "achieved_gbs": achieved,
+            "frac_of_8tbs": achieved / 8000.0,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_kind": peak_kind,
+                         "bytes_per_launch": avg_bytes / calls_per_step},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+            "wall_s_timed_region": t_wall,
+            "step_us_p10_p50_p90": [sorted(step_ms)[int(q * (nsteps - 1))] * 1e3 for q in (0.1, 0.5, 0.9)],
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    for l in layers:
+        l.close()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode_e512_t1")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

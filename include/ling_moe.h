@@ -1,0 +1,151 @@
+/*
+ * ling_moe.h -- C ABI of a B200 (sm_100a) library for the routed-expert
+ * mixture-of-experts layer of a Ling-3.0-flash-shaped model with W4 g32
+ * routed-expert weights.
+ *
+ * What one call computes (for each of T tokens x[t], hidden H):
+ *
+ *   logits[e] = sum_h x[h] * Wr[e,h] (+ b[e])                    fp32
+ *   S         = the k experts with the largest logits, ties to the lower index
+ *   w_e       = exp(logits[e]) / sum_{j in S} exp(logits[j]),  e in S
+ *               (softmax over all experts renormalised over S; sums to 1)
+ *   out       = sum_{e in S} w_e * Wd_e (SiLU(Wg_e x) * (Wu_e x))
+ *             + Wd_s (SiLU(Wg_s x) * (Wu_s x))                   -> bf16
+ *
+ * Sources for the structure: the vLLM recipe page "inclusionAI/Ling-3.0-flash"
+ * (section Overview: 512 routed experts, 8 active per token, one shared
+ * expert; section "Single-GPU int4": symmetric W4, group_size 32, routed
+ * experts only, shared expert in bf16) and the bpdata article "Harom
+ * optimalizacio a Ling-3.0-flash MoE inferenciajanak" (section "Modell es
+ * kiindulo konfiguracio": 8 of 512 routed experts plus one shared expert,
+ * hidden 2,560; section "Optimalizacio 1": moe_intermediate_size 768).  The
+ * pages do not state the gate function or the FFN form; this library fixes
+ * softmax -> top-k (ties to the lower index) -> renormalise, and the SwiGLU
+ * FFN above.  Routed weights are w = q * s with q a signed 4-bit code in
+ * [-8, 7] and s one bf16 scale per 32 consecutive elements along K.
+ *
+ * Canonical int4 packing at this boundary: two's-complement nibbles, two per
+ * byte, the LOW nibble holds the EVEN index along K, bytes run along K,
+ * rows are row-major [rows, K/2].  The library copies and repacks weights
+ * into its own layout inside ling_moe_create.
+ *
+ * Threading / streams: a handle owns a workspace, so one handle must not be
+ * used by two streams (or two host threads) at the same time.  Different
+ * handles are independent.
+ */
+#ifndef LING_MOE_H
+#define LING_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes of every entry point. */
+typedef enum {
+  LING_MOE_OK = 0,
+  LING_MOE_ERR_INVALID_ARG = -1,   /* bad pointer, size, alignment or aliasing; nothing enqueued */
+  LING_MOE_ERR_CUDA = -2,          /* a CUDA runtime call failed; see ling_moe_last_error() */
+  LING_MOE_ERR_OOM = -3,           /* device allocation failed in ling_moe_create */
+  LING_MOE_ERR_UNSUPPORTED = -4,   /* shape outside what the kernels are built for */
+  LING_MOE_ERR_DEVICE_TIMEOUT = -5 /* a bounded device-side wait gave up (sticky) */
+} ling_moe_status_t;
+
+/* Layer shape.  Supported: hidden == 2560, inter == 768 (the Ling-3.0-flash
+ * MoE shape; the kernels are specialised for it), group_size == 32,
+ * 1 <= top_k <= 8, top_k <= num_experts <= 512, max_tokens >= 1. */
+typedef struct {
+  int hidden;       /* H */
+  int inter;        /* I, per expert (moe_intermediate_size) */
+  int num_experts;  /* E, routed experts */
+  int top_k;        /* k */
+  int group_size;   /* g, int4 scale group along K */
+  int max_tokens;   /* largest T any forward call on this handle will pass */
+} ling_moe_config_t;
+
+/* Weights in the canonical layout, all DEVICE pointers on the current device.
+ * Read only during ling_moe_create (copied and repacked); the caller may free
+ * them as soon as it returns.  bf16 tensors are raw 16-bit patterns. */
+typedef struct {
+  const void *router_w;     /* bf16 [E, H] row-major */
+  const float *router_bias; /* fp32 [E], added to the logits before selection, or NULL */
+  const uint8_t *gate_q;    /* int4 [E, I, H/2] packed as described above */
+  const void *gate_s;       /* bf16 [E, I, H/g] */
+  const uint8_t *up_q;      /* int4 [E, I, H/2] */
+  const void *up_s;         /* bf16 [E, I, H/g] */
+  const uint8_t *down_q;    /* int4 [E, H, I/2] */
+  const void *down_s;       /* bf16 [E, H, I/g] */
+  const void *sh_gate;      /* bf16 [I, H] shared expert */
+  const void *sh_up;        /* bf16 [I, H] */
+  const void *sh_down;      /* bf16 [H, I] */
+} ling_moe_weights_t;
+
+typedef struct ling_moe ling_moe_t; /* opaque handle */
+
+/* Validate cfg and weights, allocate library-owned device memory (repacked
+ * weights + workspace sized for cfg->max_tokens), repack, synchronise.
+ * The only entry point that allocates or synchronises the device.
+ * On success *out is a new handle; on failure *out is NULL and nothing leaks.
+ * Errors: INVALID_ARG (NULL pointers, nonsensical sizes), UNSUPPORTED (a shape
+ * the kernels are not built for), OOM, CUDA. */
+int ling_moe_create(const ling_moe_config_t *cfg, const ling_moe_weights_t *w,
+                    ling_moe_t **out);
+
+/* out[T, H] (bf16) = layer(x[T, H] bf16) on `stream` (a cudaStream_t, NULL =
+ * legacy default stream).  x and out are DEVICE pointers owned by the caller,
+ * contiguous row-major, 16-byte aligned; out must not overlap x.
+ * 0 <= T <= max_tokens; T == 0 returns OK and enqueues nothing.
+ * Asynchronous: no host synchronisation and no allocation, so the call can be
+ * captured into a CUDA graph.  Device-detected failures (a bounded wait that
+ * gave up) are reported later by ling_moe_status.
+ * Errors: INVALID_ARG (checked on the host before anything is enqueued), CUDA. */
+int ling_moe_forward(ling_moe_t *h, const void *x, int T, void *out, void *stream);
+
+/* As ling_moe_forward, and also writes the routing: topk_idx int32 [T, k]
+ * (expert indices ordered by logit descending, ties to the lower index) and
+ * topk_w fp32 [T, k] (renormalised weights, same order).  Either may be NULL.
+ * Both are DEVICE pointers. */
+int ling_moe_forward_ex(ling_moe_t *h, const void *x, int T, void *out,
+                        int32_t *topk_idx, float *topk_w, void *stream);
+
+/* End-to-end call on HOST buffers: copies x_host [T, H] bf16 to the device,
+ * runs the layer, copies the result to out_host [T, H] bf16 and waits for the
+ * stream.  Pinned (page-locked) host buffers give asynchronous copies.
+ * Errors: as ling_moe_forward, plus DEVICE_TIMEOUT if the call's own device
+ * wait gave up. */
+int ling_moe_forward_host(ling_moe_t *h, const void *x_host, int T, void *out_host,
+                          void *stream);
+
+/* Synchronise `stream` and return the handle's sticky device error
+ * (OK or DEVICE_TIMEOUT), or CUDA if the synchronisation itself failed. */
+int ling_moe_status(ling_moe_t *h, void *stream);
+
+/* Human-readable description of the active configuration and kernel path
+ * (shape, per-path kernels, grid size).  Owned by the handle. */
+const char *ling_moe_describe(const ling_moe_t *h);
+
+/* Number of kernel launches this handle has enqueued since creation. */
+int64_t ling_moe_launch_count(const ling_moe_t *h);
+
+/* Message of the last error on the calling host thread ("" if none). */
+const char *ling_moe_last_error(void);
+
+/* Free everything the handle owns.  NULL is a no-op.  The caller must make
+ * sure no enqueued work still uses the handle. */
+void ling_moe_destroy(ling_moe_t *h);
+
+/* ---- test hooks (not needed in normal use) ----
+ * skip_arrive_cta >= 0 makes that CTA of the next decode launch skip its
+ * arrival at the grid barrier, so that the other CTAs' bounded waits run out;
+ * wait_limit_ns bounds every device-side wait (0 keeps the default, 2 s).
+ * Used to test that a wait that runs out returns an error status instead of
+ * hanging. */
+int ling_moe_test_set_wait(ling_moe_t *h, int skip_arrive_cta, uint64_t wait_limit_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LING_MOE_H */

@@ -1,0 +1,110 @@
+"""The C-ABI library: it loads, exports every declared symbol, and rejects bad
+arguments on the host before touching the GPU (runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import weight_only_int4_fp32_b200 as lm
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+HEADER = os.path.join(os.path.dirname(HERE), "include", "ling_moe.h")
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ling_moe_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_list():
+    assert declared_symbols() == sorted(lm.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported():
+    L = ctypes.CDLL(lm.library_path())
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+
+
+def test_binding_structs_match_header_layout():
+    assert ctypes.sizeof(lm.ling_moe_config_t) == 6 * 4
+    assert ctypes.sizeof(lm.ling_moe_weights_t) == 11 * ctypes.sizeof(ctypes.c_void_p)
+    assert [f for f, _ in lm.ling_moe_weights_t._fields_] == [
+        "router_w", "router_bias", "gate_q", "gate_s", "up_q", "up_s", "down_q", "down_s",
+        "sh_gate", "sh_up", "sh_down"]
+
+
+def _cfg(**kw):
+    d = dict(hidden=2560, inter=768, num_experts=512, top_k=8, group_size=32, max_tokens=4)
+    d.update(kw)
+    return lm.ling_moe_config_t(**d)
+
+
+def _weights(ptr=0x100000):
+    return lm.ling_moe_weights_t(*([ptr] * 11))
+
+
+def _create_rc(cfg, w):
+    h = ctypes.c_void_p()
+    rc = lm.lib.ling_moe_create(ctypes.byref(cfg) if cfg is not None else None,
+                                ctypes.byref(w) if w is not None else None, ctypes.byref(h))
+    return rc, h.value
+
+
+def test_create_rejects_null_arguments():
+    rc, h = _create_rc(None, _weights())
+    assert rc == lm.LING_MOE_ERR_INVALID_ARG and h is None
+    rc, h = _create_rc(_cfg(), None)
+    assert rc == lm.LING_MOE_ERR_INVALID_ARG
+    assert lm.lib.ling_moe_create(ctypes.byref(_cfg()), ctypes.byref(_weights()), None) == \
+        lm.LING_MOE_ERR_INVALID_ARG
+    w = _weights()
+    w.gate_q = None
+    rc, _ = _create_rc(_cfg(), w)
+    assert rc == lm.LING_MOE_ERR_INVALID_ARG
+    assert "NULL" in lm.ling_moe_last_error()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(top_k=9, num_experts=16), lm.LING_MOE_ERR_UNSUPPORTED),
+    (dict(top_k=9, num_experts=8), lm.LING_MOE_ERR_INVALID_ARG),
+    (dict(num_experts=513), lm.LING_MOE_ERR_UNSUPPORTED),
+    (dict(hidden=2048), lm.LING_MOE_ERR_UNSUPPORTED),
+    (dict(inter=1024), lm.LING_MOE_ERR_UNSUPPORTED),
+    (dict(group_size=64), lm.LING_MOE_ERR_UNSUPPORTED),
+    (dict(hidden=2561), lm.LING_MOE_ERR_INVALID_ARG),
+    (dict(max_tokens=0), lm.LING_MOE_ERR_INVALID_ARG),
+    (dict(top_k=0), lm.LING_MOE_ERR_INVALID_ARG),
+    (dict(num_experts=-1), lm.LING_MOE_ERR_INVALID_ARG),
+])
+def test_create_rejects_unsupported_shapes(kw, code):
+    rc, h = _create_rc(_cfg(**kw), _weights())
+    assert rc == code, lm.ling_moe_last_error()
+    assert h is None
+
+
+def test_create_rejects_misaligned_weights():
+    w = _weights()
+    w.down_s = 0x100008
+    rc, _ = _create_rc(_cfg(), w)
+    assert rc == lm.LING_MOE_ERR_INVALID_ARG
+    assert "aligned" in lm.ling_moe_last_error()
+
+
+def test_null_handle_is_rejected_everywhere():
+    assert lm.lib.ling_moe_forward(None, 16, 1, 32, None) == lm.LING_MOE_ERR_INVALID_ARG
+    assert lm.lib.ling_moe_forward_ex(None, 16, 1, 32, None, None, None) == lm.LING_MOE_ERR_INVALID_ARG
+    assert lm.lib.ling_moe_forward_host(None, 16, 1, 32, None) == lm.LING_MOE_ERR_INVALID_ARG
+    assert lm.lib.ling_moe_status(None, None) == lm.LING_MOE_ERR_INVALID_ARG
+    assert lm.lib.ling_moe_test_set_wait(None, 0, 0) == lm.LING_MOE_ERR_INVALID_ARG
+    assert lm.ling_moe_describe(None) == ""
+    assert lm.ling_moe_launch_count(None) == 0
+    lm.ling_moe_destroy(None)  # no-op
+
+
+def test_python_errors_carry_the_code():
+    with pytest.raises(lm.LingMoEError) as ei:
+        lm.ling_moe_create(_cfg(top_k=9, num_experts=16), _weights())
+    assert ei.value.code == lm.LING_MOE_ERR_UNSUPPORTED

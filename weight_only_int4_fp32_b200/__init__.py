@@ -1,0 +1,216 @@
+"""Python binding of libling_moe.so, the B200 W4 g32 MoE-layer library.
+
+Argument marshalling only: every step of the layer runs in the library's
+CUDA kernels.  The functions below carry the C ABI's names and arguments
+(pointers are integers, streams are raw cudaStream_t values); `MoELayer`
+wraps them for torch tensors.  The library must have been built
+(`python -m weight_only_int4_fp32_b200.build`); importing this package
+without it raises instead of falling back to anything else.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "LING_MOE_OK", "LING_MOE_ERR_INVALID_ARG", "LING_MOE_ERR_CUDA", "LING_MOE_ERR_OOM",
+    "LING_MOE_ERR_UNSUPPORTED", "LING_MOE_ERR_DEVICE_TIMEOUT", "LingMoEError",
+    "ling_moe_config_t", "ling_moe_weights_t", "library_path", "lib",
+    "ling_moe_create", "ling_moe_forward", "ling_moe_forward_ex", "ling_moe_forward_host",
+    "ling_moe_status", "ling_moe_describe", "ling_moe_launch_count", "ling_moe_last_error",
+    "ling_moe_destroy", "ling_moe_test_set_wait", "MoELayer", "EXPORTED",
+]
+
+LING_MOE_OK = 0
+LING_MOE_ERR_INVALID_ARG = -1
+LING_MOE_ERR_CUDA = -2
+LING_MOE_ERR_OOM = -3
+LING_MOE_ERR_UNSUPPORTED = -4
+LING_MOE_ERR_DEVICE_TIMEOUT = -5
+
+# every symbol include/ling_moe.h declares
+EXPORTED = (
+    "ling_moe_create", "ling_moe_forward", "ling_moe_forward_ex", "ling_moe_forward_host",
+    "ling_moe_status", "ling_moe_describe", "ling_moe_launch_count", "ling_moe_last_error",
+    "ling_moe_destroy", "ling_moe_test_set_wait",
+)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def library_path() -> str:
+    return os.environ.get("LING_MOE_LIB", os.path.join(_HERE, "libling_moe.so"))
+
+
+class LingMoEError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"ling_moe error {code}: {msg}")
+        self.code = code
+
+
+class ling_moe_config_t(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int), ("inter", ctypes.c_int), ("num_experts", ctypes.c_int),
+                ("top_k", ctypes.c_int), ("group_size", ctypes.c_int), ("max_tokens", ctypes.c_int)]
+
+
+class ling_moe_weights_t(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "router_w", "router_bias", "gate_q", "gate_s", "up_q", "up_s", "down_q", "down_s",
+        "sh_gate", "sh_up", "sh_down")]
+
+
+def _load():
+    path = library_path()
+    if not os.path.exists(path):
+        raise ImportError(
+            f"libling_moe.so not found at {path}: build it with "
+            "`python -m weight_only_int4_fp32_b200.build` (there is no fallback path)")
+    L = ctypes.CDLL(path)
+    vp, ci, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    sig = {
+        "ling_moe_create": (ci, [ctypes.POINTER(ling_moe_config_t), ctypes.POINTER(ling_moe_weights_t),
+                                 ctypes.POINTER(vp)]),
+        "ling_moe_forward": (ci, [vp, vp, ci, vp, vp]),
+        "ling_moe_forward_ex": (ci, [vp, vp, ci, vp, vp, vp, vp]),
+        "ling_moe_forward_host": (ci, [vp, vp, ci, vp, vp]),
+        "ling_moe_status": (ci, [vp, vp]),
+        "ling_moe_describe": (ctypes.c_char_p, [vp]),
+        "ling_moe_launch_count": (i64, [vp]),
+        "ling_moe_last_error": (ctypes.c_char_p, []),
+        "ling_moe_destroy": (None, [vp]),
+        "ling_moe_test_set_wait": (ci, [vp, ci, ctypes.c_uint64]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    return L
+
+
+lib = _load()
+
+
+def ling_moe_last_error() -> str:
+    return lib.ling_moe_last_error().decode()
+
+
+def _check(rc: int) -> int:
+    if rc != LING_MOE_OK:
+        raise LingMoEError(rc, ling_moe_last_error())
+    return rc
+
+
+def ling_moe_create(cfg: ling_moe_config_t, weights: ling_moe_weights_t) -> int:
+    h = ctypes.c_void_p()
+    _check(lib.ling_moe_create(ctypes.byref(cfg), ctypes.byref(weights), ctypes.byref(h)))
+    return h.value
+
+
+def ling_moe_forward(h: int, x: int, T: int, out: int, stream: int = 0) -> int:
+    return _check(lib.ling_moe_forward(h, x, T, out, stream))
+
+
+def ling_moe_forward_ex(h: int, x: int, T: int, out: int, topk_idx: int, topk_w: int,
+                        stream: int = 0) -> int:
+    return _check(lib.ling_moe_forward_ex(h, x, T, out, topk_idx, topk_w, stream))
+
+
+def ling_moe_forward_host(h: int, x_host: int, T: int, out_host: int, stream: int = 0) -> int:
+    return _check(lib.ling_moe_forward_host(h, x_host, T, out_host, stream))
+
+
+def ling_moe_status(h: int, stream: int = 0) -> int:
+    """Returns the status code (does not raise on DEVICE_TIMEOUT)."""
+    return lib.ling_moe_status(h, stream)
+
+
+def ling_moe_describe(h: int) -> str:
+    return lib.ling_moe_describe(h).decode()
+
+
+def ling_moe_launch_count(h: int) -> int:
+    return lib.ling_moe_launch_count(h)
+
+
+def ling_moe_destroy(h: int) -> None:
+    lib.ling_moe_destroy(h)
+
+
+def ling_moe_test_set_wait(h: int, skip_arrive_cta: int, wait_limit_ns: int) -> int:
+    return _check(lib.ling_moe_test_set_wait(h, skip_arrive_cta, wait_limit_ns))
+
+
+class MoELayer:
+    """One MoE layer on the current CUDA device, built from torch tensors.
+
+    `weights` maps the canonical names (router_w, router_bias, gate_q, gate_s,
+    up_q, up_s, down_q, down_s, sh_gate, sh_up, sh_down) to contiguous CUDA
+    tensors; they are copied, so they may be freed after construction.
+    """
+
+    def __init__(self, weights: dict, top_k: int = 8, max_tokens: int = 1, group_size: int = 32):
+        import torch  # device memory and streams only
+        rw = weights["router_w"]
+        E, H = rw.shape
+        I = weights["sh_gate"].shape[0]
+        for k, v in weights.items():
+            if v is not None and (not v.is_cuda or not v.is_contiguous()):
+                raise ValueError(f"{k} must be a contiguous CUDA tensor")
+        cfg = ling_moe_config_t(H, I, E, top_k, group_size, max_tokens)
+        ptr = lambda n: (weights[n].data_ptr() if weights.get(n) is not None else None)
+        w = ling_moe_weights_t(*(ptr(n) for n, _ in ling_moe_weights_t._fields_))
+        self.E, self.H, self.I, self.k, self.max_tokens = E, H, I, top_k, max_tokens
+        self.handle = ling_moe_create(cfg, w)
+        self._torch = torch
+
+    def _stream(self, stream):
+        if stream is None:
+            return self._torch.cuda.current_stream().cuda_stream
+        return getattr(stream, "cuda_stream", stream)
+
+    def forward(self, x, out=None, stream=None, return_routing: bool = False):
+        torch = self._torch
+        if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous() or x.dim() != 2:
+            raise ValueError("x must be a contiguous 2-D bf16 CUDA tensor")
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty_like(x)
+        s = self._stream(stream)
+        if return_routing:
+            idx = torch.empty((T, self.k), dtype=torch.int32, device=x.device)
+            w = torch.empty((T, self.k), dtype=torch.float32, device=x.device)
+            ling_moe_forward_ex(self.handle, x.data_ptr(), T, out.data_ptr(), idx.data_ptr(),
+                                w.data_ptr(), s)
+            return out, idx, w
+        ling_moe_forward(self.handle, x.data_ptr(), T, out.data_ptr(), s)
+        return out
+
+    __call__ = forward
+
+    def forward_host(self, x_host, out_host=None, stream=None):
+        torch = self._torch
+        T = x_host.shape[0]
+        if out_host is None:
+            out_host = torch.empty_like(x_host)
+        ling_moe_forward_host(self.handle, x_host.data_ptr(), T, out_host.data_ptr(), self._stream(stream))
+        return out_host
+
+    def status(self, stream=None) -> int:
+        return ling_moe_status(self.handle, self._stream(stream))
+
+    def describe(self) -> str:
+        return ling_moe_describe(self.handle)
+
+    def launch_count(self) -> int:
+        return ling_moe_launch_count(self.handle)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            ling_moe_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,384 @@
+// C ABI of the W4 g32 MoE-layer library: validation, ownership, dispatch.
+// The layer it computes is documented in include/ling_moe.h.
+#include "ling_moe.h"
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "layout.h"
+#include "decode.h"
+#include "grouped.h"
+#include "repack.h"
+
+using namespace lingmoe;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(e == cudaErrorMemoryAllocation ? LING_MOE_ERR_OOM : LING_MOE_ERR_CUDA, "%s: %s (%s)",
+              what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;  // 2 s
+
+}  // namespace
+
+struct ling_moe {
+  ling_moe_config_t cfg{};
+  int device = 0;
+  int num_sms = 0;
+  int decode_ctas = 0;
+  int decode_T = 0;  // tokens the decode workspace holds
+  std::vector<void*> allocs;
+  // owned weights
+  __nv_bfloat16* router_w = nullptr;
+  float* router_bias = nullptr;
+  uint8_t* gu = nullptr;
+  uint8_t* dn = nullptr;
+  __nv_bfloat16* sh_gate = nullptr;
+  __nv_bfloat16* sh_up = nullptr;
+  __nv_bfloat16* sh_down = nullptr;
+  // decode workspace
+  float* logits = nullptr;
+  float* h_s = nullptr;
+  float* h_pair = nullptr;
+  int32_t* topk_idx = nullptr;
+  float* topk_w = nullptr;
+  unsigned long long* bar = nullptr;
+  unsigned int* err = nullptr;
+  // grouped-path workspace
+  GroupedWorkspace gws{};
+  // host entry point staging
+  __nv_bfloat16* x_stage = nullptr;
+  __nv_bfloat16* out_stage = nullptr;
+  std::string desc;
+  std::atomic<int64_t> launches{0};
+  int skip_arrive_cta = -1;
+  unsigned long long wait_limit_ns = kDefaultWaitNs;
+
+  cudaError_t alloc(void** p, size_t bytes) {
+    *p = nullptr;
+    if (bytes == 0) return cudaSuccess;
+    cudaError_t e = cudaMalloc(p, bytes);
+    if (e == cudaSuccess) allocs.push_back(*p);
+    return e;
+  }
+  void release() {
+    for (void* p : allocs) cudaFree(p);
+    allocs.clear();
+  }
+};
+
+namespace {
+
+int validate_cfg(const ling_moe_config_t* c) {
+  if (c->hidden <= 0 || c->inter <= 0 || c->num_experts <= 0 || c->top_k <= 0 ||
+      c->group_size <= 0 || c->max_tokens <= 0)
+    return fail(LING_MOE_ERR_INVALID_ARG, "config fields must be positive");
+  if (c->top_k > c->num_experts)
+    return fail(LING_MOE_ERR_INVALID_ARG, "top_k (%d) exceeds num_experts (%d)", c->top_k,
+                c->num_experts);
+  if (c->hidden % c->group_size || c->inter % c->group_size)
+    return fail(LING_MOE_ERR_INVALID_ARG, "hidden and inter must be multiples of group_size");
+  if (c->hidden != kH || c->inter != kI)
+    return fail(LING_MOE_ERR_UNSUPPORTED, "kernels are built for hidden=%d inter=%d (got %d, %d)",
+                kH, kI, c->hidden, c->inter);
+  if (c->group_size != kGroup)
+    return fail(LING_MOE_ERR_UNSUPPORTED, "group_size must be %d", kGroup);
+  if (c->top_k > kMaxTopK) return fail(LING_MOE_ERR_UNSUPPORTED, "top_k must be <= %d", kMaxTopK);
+  if (c->num_experts > kMaxExperts)
+    return fail(LING_MOE_ERR_UNSUPPORTED, "num_experts must be <= %d", kMaxExperts);
+  return LING_MOE_OK;
+}
+
+int validate_weights(const ling_moe_weights_t* w) {
+  const void* req[] = {w->router_w, w->gate_q, w->gate_s, w->up_q, w->up_s,
+                       w->down_q,   w->down_s, w->sh_gate, w->sh_up, w->sh_down};
+  for (const void* p : req)
+    if (!p) return fail(LING_MOE_ERR_INVALID_ARG, "a required weight pointer is NULL");
+  for (const void* p : req)
+    if (!aligned16(p)) return fail(LING_MOE_ERR_INVALID_ARG, "weight pointers must be 16-byte aligned");
+  if (w->router_bias && !aligned16(w->router_bias))
+    return fail(LING_MOE_ERR_INVALID_ARG, "router_bias must be 16-byte aligned");
+  return LING_MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ling_moe_last_error(void) { return g_last_error.c_str(); }
+
+int ling_moe_create(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, ling_moe_t** out) {
+  if (!out) return fail(LING_MOE_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (!cfg || !w) return fail(LING_MOE_ERR_INVALID_ARG, "cfg or weights is NULL");
+  int rc = validate_cfg(cfg);
+  if (rc) return rc;
+  rc = validate_weights(w);
+  if (rc) return rc;
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  cudaDeviceProp prop;
+  e = cudaGetDeviceProperties(&prop, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+  if (prop.major != 10)
+    return fail(LING_MOE_ERR_UNSUPPORTED, "needs an sm_100 GPU (got sm_%d%d)", prop.major, prop.minor);
+  if (!prop.cooperativeLaunch) return fail(LING_MOE_ERR_UNSUPPORTED, "cooperative launch unsupported");
+  if (prop.multiProcessorCount < 80)
+    return fail(LING_MOE_ERR_UNSUPPORTED, "needs at least 80 SMs (got %d)", prop.multiProcessorCount);
+
+  e = setup_decode();
+  if (e != cudaSuccess) return cuda_fail(e, "decode kernel attributes");
+  if (decode_max_ctas_per_sm() < 1)
+    return fail(LING_MOE_ERR_UNSUPPORTED, "decode kernel does not fit on an SM");
+  e = setup_grouped();
+  if (e != cudaSuccess) return cuda_fail(e, "grouped kernel attributes");
+
+  ling_moe* h = new ling_moe();
+  h->cfg = *cfg;
+  h->device = dev;
+  h->num_sms = prop.multiProcessorCount;
+  h->decode_ctas = prop.multiProcessorCount;
+  h->decode_T = cfg->max_tokens < kMaxDecodeT ? cfg->max_tokens : kMaxDecodeT;
+
+  const int E = cfg->num_experts, K = cfg->top_k;
+  const size_t bf = sizeof(__nv_bfloat16);
+  struct A { void** p; size_t n; } plan[] = {
+      {(void**)&h->router_w, (size_t)E * kH * bf},
+      {(void**)&h->router_bias, w->router_bias ? (size_t)E * sizeof(float) : 0},
+      {(void**)&h->gu, (size_t)E * kGuExpertBytes},
+      {(void**)&h->dn, (size_t)E * kDnExpertBytes},
+      {(void**)&h->sh_gate, (size_t)kI * kH * bf},
+      {(void**)&h->sh_up, (size_t)kI * kH * bf},
+      {(void**)&h->sh_down, (size_t)kH * kI * bf},
+      {(void**)&h->logits, (size_t)h->decode_T * E * sizeof(float)},
+      {(void**)&h->h_s, (size_t)h->decode_T * kI * sizeof(float)},
+      {(void**)&h->h_pair, (size_t)h->decode_T * K * kI * sizeof(float)},
+      {(void**)&h->topk_idx, (size_t)h->decode_T * K * sizeof(int32_t)},
+      {(void**)&h->topk_w, (size_t)h->decode_T * K * sizeof(float)},
+      {(void**)&h->bar, 4 * sizeof(unsigned long long)},
+      {(void**)&h->err, 4 * sizeof(unsigned int)},
+      {(void**)&h->x_stage, (size_t)cfg->max_tokens * kH * bf},
+      {(void**)&h->out_stage, (size_t)cfg->max_tokens * kH * bf},
+  };
+  for (auto& a : plan) {
+    e = h->alloc(a.p, a.n);
+    if (e != cudaSuccess) {
+      rc = cuda_fail(e, "cudaMalloc");
+      h->release();
+      delete h;
+      return rc;
+    }
+  }
+  if (cfg->max_tokens > kMaxDecodeT) {
+    e = grouped_alloc(&h->gws, E, K, cfg->max_tokens,
+                      [h](void** p, size_t n) { return h->alloc(p, n); });
+    if (e != cudaSuccess) {
+      rc = cuda_fail(e, "cudaMalloc (grouped workspace)");
+      h->release();
+      delete h;
+      return rc;
+    }
+  }
+
+  cudaStream_t s = nullptr;
+  e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(h->router_w, w->router_w, (size_t)E * kH * bf, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && w->router_bias)
+    e = cudaMemcpyAsync(h->router_bias, w->router_bias, (size_t)E * sizeof(float), cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(h->sh_gate, w->sh_gate, (size_t)kI * kH * bf, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(h->sh_up, w->sh_up, (size_t)kI * kH * bf, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(h->sh_down, w->sh_down, (size_t)kH * kI * bf, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->bar, 0, 4 * sizeof(unsigned long long), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->err, 0, 4 * sizeof(unsigned int), s);
+  if (e == cudaSuccess)
+    e = launch_repack(w->gate_q, w->up_q, w->gate_s, w->up_s, w->down_q, w->down_s, h->gu, h->dn, E, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (s) cudaStreamDestroy(s);
+  if (e != cudaSuccess) {
+    rc = cuda_fail(e, "create: copy/repack");
+    h->release();
+    delete h;
+    return rc;
+  }
+
+  char buf[1024];
+  snprintf(buf, sizeof(buf),
+           "ling_moe sm_%d%d %d SMs | H=%d I=%d E=%d k=%d g=%d max_tokens=%d bias=%s | "
+           "decode path (1<=T<=%d): 1 cooperative launch grid=%dx%d smem=%zuB, W4 g32 GEMV "
+           "dequant-in-register, fp32 accumulate | grouped path (T>%d): %s",
+           prop.major, prop.minor, h->num_sms, kH, kI, E, K, kGroup, cfg->max_tokens,
+           w->router_bias ? "yes" : "no", kMaxDecodeT, h->decode_ctas, kDecodeThreads,
+           decode_smem_bytes(), kMaxDecodeT, grouped_describe());
+  h->desc = buf;
+  *out = h;
+  return LING_MOE_OK;
+}
+
+static int forward_impl(ling_moe_t* h, const void* x, int T, void* out, int32_t* topk_idx,
+                        float* topk_w, void* stream_v) {
+  if (!h) return fail(LING_MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (T < 0 || T > h->cfg.max_tokens)
+    return fail(LING_MOE_ERR_INVALID_ARG, "T=%d outside [0, max_tokens=%d]", T, h->cfg.max_tokens);
+  if (T == 0) return LING_MOE_OK;
+  if (!x || !out) return fail(LING_MOE_ERR_INVALID_ARG, "x or out is NULL");
+  if (!aligned16(x) || !aligned16(out))
+    return fail(LING_MOE_ERR_INVALID_ARG, "x and out must be 16-byte aligned");
+  const size_t nbytes = (size_t)T * kH * sizeof(__nv_bfloat16);
+  if (overlaps(x, nbytes, out, nbytes)) return fail(LING_MOE_ERR_INVALID_ARG, "out overlaps x");
+  if ((topk_idx && (reinterpret_cast<uintptr_t>(topk_idx) & 3)) ||
+      (topk_w && (reinterpret_cast<uintptr_t>(topk_w) & 3)))
+    return fail(LING_MOE_ERR_INVALID_ARG, "topk outputs must be 4-byte aligned");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  cudaError_t e;
+  if (T <= kMaxDecodeT) {
+    DecodeParams p{};
+    p.x = static_cast<const __nv_bfloat16*>(x);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.T = T;
+    p.E = h->cfg.num_experts;
+    p.k = h->cfg.top_k;
+    p.router_w = h->router_w;
+    p.router_bias = h->router_bias;
+    p.gu = h->gu;
+    p.dn = h->dn;
+    p.sh_gate = h->sh_gate;
+    p.sh_up = h->sh_up;
+    p.sh_down = h->sh_down;
+    p.logits = h->logits;
+    p.h_s = h->h_s;
+    p.h_pair = h->h_pair;
+    p.topk_idx_ws = h->topk_idx;
+    p.topk_w_ws = h->topk_w;
+    p.topk_idx_out = topk_idx;
+    p.topk_w_out = topk_w;
+    p.bar = h->bar;
+    p.err = h->err;
+    p.skip_arrive_cta = h->skip_arrive_cta;
+    p.wait_limit_ns = h->wait_limit_ns;
+    h->skip_arrive_cta = -1;  // one launch only
+    e = launch_decode(p, h->decode_ctas, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    h->launches.fetch_add(1);
+    return LING_MOE_OK;
+  }
+  GroupedParams gp{};
+  gp.x = static_cast<const __nv_bfloat16*>(x);
+  gp.out = static_cast<__nv_bfloat16*>(out);
+  gp.T = T;
+  gp.E = h->cfg.num_experts;
+  gp.k = h->cfg.top_k;
+  gp.router_w = h->router_w;
+  gp.router_bias = h->router_bias;
+  gp.gu = h->gu;
+  gp.dn = h->dn;
+  gp.sh_gate = h->sh_gate;
+  gp.sh_up = h->sh_up;
+  gp.sh_down = h->sh_down;
+  gp.topk_idx_out = topk_idx;
+  gp.topk_w_out = topk_w;
+  gp.num_sms = h->num_sms;
+  int nl = 0;
+  e = launch_grouped(gp, h->gws, stream, &nl);
+  h->launches.fetch_add(nl);
+  if (e != cudaSuccess) return cuda_fail(e, "grouped launch");
+  return LING_MOE_OK;
+}
+
+int ling_moe_forward(ling_moe_t* h, const void* x, int T, void* out, void* stream) {
+  return forward_impl(h, x, T, out, nullptr, nullptr, stream);
+}
+
+int ling_moe_forward_ex(ling_moe_t* h, const void* x, int T, void* out, int32_t* topk_idx,
+                        float* topk_w, void* stream) {
+  return forward_impl(h, x, T, out, topk_idx, topk_w, stream);
+}
+
+int ling_moe_forward_host(ling_moe_t* h, const void* x_host, int T, void* out_host, void* stream_v) {
+  if (!h) return fail(LING_MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (T < 0 || T > h->cfg.max_tokens)
+    return fail(LING_MOE_ERR_INVALID_ARG, "T=%d outside [0, max_tokens=%d]", T, h->cfg.max_tokens);
+  if (T == 0) return LING_MOE_OK;
+  if (!x_host || !out_host) return fail(LING_MOE_ERR_INVALID_ARG, "x_host or out_host is NULL");
+  const size_t nbytes = (size_t)T * kH * sizeof(__nv_bfloat16);
+  if (overlaps(x_host, nbytes, out_host, nbytes))
+    return fail(LING_MOE_ERR_INVALID_ARG, "out_host overlaps x_host");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  cudaError_t e = cudaMemcpyAsync(h->x_stage, x_host, nbytes, cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "host->device copy");
+  int rc = forward_impl(h, h->x_stage, T, h->out_stage, nullptr, nullptr, stream_v);
+  if (rc) return rc;
+  e = cudaMemcpyAsync(out_host, h->out_stage, nbytes, cudaMemcpyDeviceToHost, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "device->host copy");
+  e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  return LING_MOE_OK;
+}
+
+int ling_moe_status(ling_moe_t* h, void* stream_v) {
+  if (!h) return fail(LING_MOE_ERR_INVALID_ARG, "handle is NULL");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  unsigned int err = 0;
+  e = cudaMemcpy(&err, h->err, sizeof(err), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  if (err) {
+    // A wait gave up: the barrier counters are no longer whole generations.
+    // Reset them and the error word so the handle can run again.
+    cudaMemset(h->bar, 0, 4 * sizeof(unsigned long long));
+    cudaMemset(h->err, 0, 4 * sizeof(unsigned int));
+    cudaDeviceSynchronize();
+    return fail(LING_MOE_ERR_DEVICE_TIMEOUT, "a bounded device-side wait gave up (error word %u)", err);
+  }
+  return LING_MOE_OK;
+}
+
+const char* ling_moe_describe(const ling_moe_t* h) { return h ? h->desc.c_str() : ""; }
+
+int64_t ling_moe_launch_count(const ling_moe_t* h) { return h ? h->launches.load() : 0; }
+
+void ling_moe_destroy(ling_moe_t* h) {
+  if (!h) return;
+  h->release();
+  delete h;
+}
+
+int ling_moe_test_set_wait(ling_moe_t* h, int skip_arrive_cta, uint64_t wait_limit_ns) {
+  if (!h) return fail(LING_MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (skip_arrive_cta >= h->decode_ctas)
+    return fail(LING_MOE_ERR_INVALID_ARG, "skip_arrive_cta out of range");
+  h->skip_arrive_cta = skip_arrive_cta < 0 ? -1 : skip_arrive_cta;
+  h->wait_limit_ns = wait_limit_ns ? wait_limit_ns : kDefaultWaitNs;
+  return LING_MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,44 @@
+// Host-visible interface of the decode / verify kernel (1 <= T <= kMaxDecodeT).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace lingmoe {
+
+constexpr int kMaxDecodeT = 4;     // tokens per call handled by the decode kernel
+constexpr int kDecodeWarps = 12;
+constexpr int kDecodeThreads = kDecodeWarps * 32;
+
+struct DecodeParams {
+  const __nv_bfloat16* x;        // [T, H]
+  __nv_bfloat16* out;            // [T, H]
+  int T, E, k;
+  const __nv_bfloat16* router_w; // [E, H]
+  const float* router_bias;      // [E] or nullptr
+  const uint8_t* gu;             // repacked routed gate/up
+  const uint8_t* dn;             // repacked routed down
+  const __nv_bfloat16* sh_gate;  // [I, H]
+  const __nv_bfloat16* sh_up;    // [I, H]
+  const __nv_bfloat16* sh_down;  // [H, I]
+  float* logits;                 // workspace [T, E]
+  float* h_s;                    // workspace [T, I]
+  float* h_pair;                 // workspace [T*k, I]
+  int32_t* topk_idx_ws;          // workspace [T, k]
+  float* topk_w_ws;              // workspace [T, k]
+  int32_t* topk_idx_out;         // optional caller output [T, k]
+  float* topk_w_out;             // optional caller output [T, k]
+  unsigned long long* bar;       // 3 monotonically increasing barrier counters
+  unsigned int* err;             // sticky device error word
+  int skip_arrive_cta;           // test hook: this CTA never arrives (-1: none)
+  unsigned long long wait_limit_ns;
+};
+
+size_t decode_smem_bytes();
+cudaError_t setup_decode();
+int decode_max_ctas_per_sm();
+cudaError_t launch_decode(const DecodeParams& p, int nctas, cudaStream_t stream);
+
+}  // namespace lingmoe
