@@ -137,11 +137,12 @@ const char *ling_moe_last_error(void);
 void ling_moe_destroy(ling_moe_t *h);
 
 /* ---- test hooks (not needed in normal use) ----
- * skip_arrive_cta >= 0 makes that CTA of the next decode launch skip its
- * arrival at the grid barrier, so that the other CTAs' bounded waits run out;
- * wait_limit_ns bounds every device-side wait (0 keeps the default, 2 s).
- * Used to test that a wait that runs out returns an error status instead of
- * hanging. */
+ * skip_arrive_cta >= 0 makes that CTA of the next decode launch withhold the
+ * router logits it computes, so that every CTA's bounded wait for them runs
+ * out; wait_limit_ns bounds every device-side wait (0 keeps the default, 2 s).
+ * Used to test that a wait that runs out ends the launch with an error status
+ * (reported by ling_moe_status) instead of hanging, and that the next launch
+ * runs normally. */
 int ling_moe_test_set_wait(ling_moe_t *h, int skip_arrive_cta, uint64_t wait_limit_ns);
 
 #ifdef __cplusplus

@@ -63,13 +63,11 @@ struct ling_moe {
   __nv_bfloat16* sh_gate = nullptr;
   __nv_bfloat16* sh_up = nullptr;
   __nv_bfloat16* sh_down = nullptr;
-  // decode workspace
+  // decode workspace: epoch-tagged exchange buffers and the sync words
   float* logits = nullptr;
   float* h_s = nullptr;
   float* h_pair = nullptr;
-  int32_t* topk_idx = nullptr;
-  float* topk_w = nullptr;
-  unsigned long long* bar = nullptr;
+  unsigned int* sync = nullptr;
   unsigned int* err = nullptr;
   // grouped-path workspace
   GroupedWorkspace gws{};
@@ -182,9 +180,7 @@ int ling_moe_create(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, l
       {(void**)&h->logits, (size_t)h->decode_T * E * sizeof(float)},
       {(void**)&h->h_s, (size_t)h->decode_T * kI * sizeof(float)},
       {(void**)&h->h_pair, (size_t)h->decode_T * K * kI * sizeof(float)},
-      {(void**)&h->topk_idx, (size_t)h->decode_T * K * sizeof(int32_t)},
-      {(void**)&h->topk_w, (size_t)h->decode_T * K * sizeof(float)},
-      {(void**)&h->bar, 4 * sizeof(unsigned long long)},
+      {(void**)&h->sync, 4 * sizeof(unsigned int)},
       {(void**)&h->err, 4 * sizeof(unsigned int)},
       {(void**)&h->x_stage, (size_t)cfg->max_tokens * kH * bf},
       {(void**)&h->out_stage, (size_t)cfg->max_tokens * kH * bf},
@@ -217,7 +213,7 @@ int ling_moe_create(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, l
   if (e == cudaSuccess) e = cudaMemcpyAsync(h->sh_gate, w->sh_gate, (size_t)kI * kH * bf, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(h->sh_up, w->sh_up, (size_t)kI * kH * bf, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(h->sh_down, w->sh_down, (size_t)kH * kI * bf, cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(h->bar, 0, 4 * sizeof(unsigned long long), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->sync, 0, 4 * sizeof(unsigned int), s);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->err, 0, 4 * sizeof(unsigned int), s);
   if (e == cudaSuccess)
     e = launch_repack(w->gate_q, w->up_q, w->gate_s, w->up_s, w->down_q, w->down_s, h->gu, h->dn, E, s);
@@ -237,7 +233,7 @@ int ling_moe_create(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, l
            "dequant-in-register, fp32 accumulate | grouped path (T>%d): %s",
            prop.major, prop.minor, h->num_sms, kH, kI, E, K, kGroup, cfg->max_tokens,
            w->router_bias ? "yes" : "no", kMaxDecodeT, h->decode_ctas, kDecodeThreads,
-           decode_smem_bytes(), kMaxDecodeT, grouped_describe());
+           decode_smem_bytes(1), kMaxDecodeT, grouped_describe());
   h->desc = buf;
   *out = h;
   return LING_MOE_OK;
@@ -276,11 +272,9 @@ static int forward_impl(ling_moe_t* h, const void* x, int T, void* out, int32_t*
     p.logits = h->logits;
     p.h_s = h->h_s;
     p.h_pair = h->h_pair;
-    p.topk_idx_ws = h->topk_idx;
-    p.topk_w_ws = h->topk_w;
     p.topk_idx_out = topk_idx;
     p.topk_w_out = topk_w;
-    p.bar = h->bar;
+    p.sync = h->sync;
     p.err = h->err;
     p.skip_arrive_cta = h->skip_arrive_cta;
     p.wait_limit_ns = h->wait_limit_ns;
@@ -352,10 +346,11 @@ int ling_moe_status(ling_moe_t* h, void* stream_v) {
   e = cudaMemcpy(&err, h->err, sizeof(err), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "read device error word");
   if (err) {
-    // A wait gave up: the barrier counters are no longer whole generations.
-    // Reset them and the error word so the handle can run again.
-    cudaMemset(h->bar, 0, 4 * sizeof(unsigned long long));
+    // A wait gave up.  Every CTA still counted itself out and the last one
+    // reset the arrival counters, so the next launch starts clean; clear the
+    // error word (and the counters, in case a launch never ran to its end).
     cudaMemset(h->err, 0, 4 * sizeof(unsigned int));
+    cudaMemset(h->sync, 0, 4 * sizeof(unsigned int));
     cudaDeviceSynchronize();
     return fail(LING_MOE_ERR_DEVICE_TIMEOUT, "a bounded device-side wait gave up (error word %u)", err);
   }

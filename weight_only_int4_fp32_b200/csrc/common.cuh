@@ -198,7 +198,9 @@ __device__ __forceinline__ void warp_topk(const float* logits, int E, int k, int
       for (int j = 0; j < kPer; ++j)
         if (e == lane + 32 * j) key[j] = 0ull;
       idx[r] = e;
-      val[r] = ldcg_f32(logits + e);
+      // the value is in the key: undo the order-preserving transform
+      const uint32_t hk = (uint32_t)(best >> 32);
+      val[r] = __uint_as_float((hk & 0x80000000u) ? (hk & 0x7FFFFFFFu) : ~hk);
     }
   }
   if (lane == 0) {
@@ -238,6 +240,396 @@ __device__ __forceinline__ int xoff(int c) { return 4 * (c + c / 80); }
 __device__ __forceinline__ float scale_of(uint2 s4, int jj) {
   const uint32_t w = (jj < 2) ? s4.x : s4.y;
   return (jj & 1) ? bf16hi(w) : bf16lo(w);
+}
+
+// ---------------------------------------------------------------- mbarrier + bulk copy
+// Non-multicast TMA bulk copies (global -> this CTA's shared memory) completing
+// on an mbarrier.  Addresses 16-byte aligned, sizes multiples of 16.
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared.b64 [%0], %1;" :: "r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared.b64 _, [%0], %1;" :: "r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+// Bounded wait for phase `parity` of the barrier; false (and the sticky error
+// word set) if it did not complete within limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned long long limit_ns,
+                                          unsigned int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) {
+      atomicOr(err, 2u);
+      return false;
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ uint4 lds128(const void* p) { return *reinterpret_cast<const uint4*>(p); }
+__device__ __forceinline__ float4 ldsf4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+
+// ---------------------------------------------------------------- mixed-precision FMA
+// d = a * b + c with a, b taken from one half (lo = 0, hi = 1) of packed
+// 16-bit pairs and c, d in fp32; the product of two 16-bit values is exact in
+// fp32, so only the accumulation rounds.
+#define LING_MIXED_FMA_ASM(TYPE, A, B)                                   \
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"                                  \
+      "mov.b32 {al, ah}, %1;\n\t"                                           \
+      "mov.b32 {bl, bh}, %2;\n\t"                                           \
+      "fma.rn.f32." TYPE " %0, " A ", " B ", %3;\n\t}"                       \
+      : "=f"(d) : "r"(a2), "r"(b2), "f"(c))
+template <int AH, int BH>
+__device__ __forceinline__ float fma_bf16h(uint32_t a2, uint32_t b2, float c) {
+  float d;
+  if constexpr (AH == 0 && BH == 0) LING_MIXED_FMA_ASM("bf16", "al", "bl");
+  else if constexpr (AH == 0 && BH == 1) LING_MIXED_FMA_ASM("bf16", "al", "bh");
+  else if constexpr (AH == 1 && BH == 0) LING_MIXED_FMA_ASM("bf16", "ah", "bl");
+  else LING_MIXED_FMA_ASM("bf16", "ah", "bh");
+  return d;
+}
+template <int AH, int BH>
+__device__ __forceinline__ float fma_f16h(uint32_t a2, uint32_t b2, float c) {
+  float d;
+  if constexpr (AH == 0 && BH == 0) LING_MIXED_FMA_ASM("f16", "al", "bl");
+  else if constexpr (AH == 0 && BH == 1) LING_MIXED_FMA_ASM("f16", "al", "bh");
+  else if constexpr (AH == 1 && BH == 0) LING_MIXED_FMA_ASM("f16", "ah", "bl");
+  else LING_MIXED_FMA_ASM("f16", "ah", "bh");
+  return d;
+}
+
+// 8 bf16 weights (one 16-byte chunk) dot 8 bf16 activations, fp32 accumulate.
+__device__ __forceinline__ float dot8_bf16_bf16(uint4 w, uint4 x, float acc) {
+  acc = fma_bf16h<0, 0>(w.x, x.x, acc);
+  acc = fma_bf16h<1, 1>(w.x, x.x, acc);
+  acc = fma_bf16h<0, 0>(w.y, x.y, acc);
+  acc = fma_bf16h<1, 1>(w.y, x.y, acc);
+  acc = fma_bf16h<0, 0>(w.z, x.z, acc);
+  acc = fma_bf16h<1, 1>(w.z, x.z, acc);
+  acc = fma_bf16h<0, 0>(w.w, x.w, acc);
+  acc = fma_bf16h<1, 1>(w.w, x.w, acc);
+  return acc;
+}
+
+// int4 -> fp16 with one LOP3 per two codes.  For a 32-bit word holding 8
+// offset-binary nibbles n_0..n_7 (n = q + 8, nibble i at bits 4i..4i+3,
+// element i of the word), (w & 0x000F000F) | 0x64006400 is the fp16 pair
+// (1024 + n_0, 1024 + n_4) and (w & 0x00F000F0) | 0x64006400 is
+// (1024 + 16 n_1, 1024 + 16 n_5); the same on w >> 8 gives elements 2, 6
+// and 3, 7.  Even elements carry 1024 + n, odd ones 1024 + 16 n, so for a
+// group of 32 codes with activations x (fp16):
+//   sum_k q_k x_k = (A_even - 1032 S_even) + (A_odd - 1152 S_odd) / 16
+// with A the fp32 FMA sums of the fp16 products and S the sums of x over the
+// even / odd positions.  Each fp16 x fp16 product is exact in fp32.
+struct Pairs4 { uint32_t p0, p1, p2, p3; };
+__device__ __forceinline__ Pairs4 dequant_f16x2(uint32_t w) {
+  Pairs4 r;
+  const uint32_t w8 = w >> 8;
+  asm("lop3.b32 %0, %1, 0x000F000F, 0x64006400, 0xEA;" : "=r"(r.p0) : "r"(w));
+  asm("lop3.b32 %0, %1, 0x00F000F0, 0x64006400, 0xEA;" : "=r"(r.p1) : "r"(w));
+  asm("lop3.b32 %0, %1, 0x000F000F, 0x64006400, 0xEA;" : "=r"(r.p2) : "r"(w8));
+  asm("lop3.b32 %0, %1, 0x00F000F0, 0x64006400, 0xEA;" : "=r"(r.p3) : "r"(w8));
+  return r;
+}
+constexpr float kEvenBias = -1032.0f;
+constexpr float kOddBias = -1152.0f;
+// acc_e += even products, acc_o += odd products of one word (8 codes) with
+// the 8 fp16 activations x = (x0..x7) packed in a uint4.
+__device__ __forceinline__ void dot8_q_f16(const Pairs4& P, uint4 x, float& ae, float& ao) {
+  ae = fma_f16h<0, 0>(P.p0, x.x, ae);  // e0 * x0
+  ae = fma_f16h<1, 0>(P.p0, x.z, ae);  // e4 * x4
+  ae = fma_f16h<0, 0>(P.p2, x.y, ae);  // e2 * x2
+  ae = fma_f16h<1, 0>(P.p2, x.w, ae);  // e6 * x6
+  ao = fma_f16h<0, 1>(P.p1, x.x, ao);  // e1 * x1
+  ao = fma_f16h<1, 1>(P.p1, x.z, ao);  // e5 * x5
+  ao = fma_f16h<0, 1>(P.p3, x.y, ao);  // e3 * x3
+  ao = fma_f16h<1, 1>(P.p3, x.w, ao);  // e7 * x7
+}
+
+// ---------------------------------------------------------------- compact top-k
+// One warp: top-k of logits[0..E) (E <= 512) by (value desc, index asc), with
+// 32-bit order-preserving keys and warp-wide reductions; the renormalised
+// softmax weights of the kept logits.  out_i/out_w/val_s are shared memory.
+__device__ __forceinline__ uint32_t f32_order_key(float v) {
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float f32_from_order_key(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+__device__ __forceinline__ void warp_topk_compact(const float* logits, int E, int k, int* out_i,
+                                                  float* out_w) {
+  const int lane = threadIdx.x & 31;
+  constexpr int kPer = kMaxExperts / 32;
+  uint32_t key[kPer];
+  uint32_t taken = 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int e = lane + 32 * j;
+    key[j] = (e < E) ? f32_order_key(ldcg_f32(logits + e)) : 0u;
+    if (e >= E) taken |= 1u << j;
+  }
+  float m0 = 0.f;
+#pragma unroll 1
+  for (int r = 0; r < k; ++r) {
+    uint32_t lm = 0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) lm = (!(taken >> j & 1u) && key[j] > lm) ? key[j] : lm;
+    const uint32_t m = __reduce_max_sync(0xffffffffu, lm);
+    uint32_t ec = 0xFFFFFFFFu;
+#pragma unroll
+    for (int j = kPer - 1; j >= 0; --j)
+      if (!(taken >> j & 1u) && key[j] == m) ec = (uint32_t)(lane + 32 * j);
+    const uint32_t e = __reduce_min_sync(0xffffffffu, ec);
+    if ((int)(e & 31u) == lane) taken |= 1u << (e >> 5);
+    const float v = f32_from_order_key(m);
+    if (r == 0) m0 = v;
+    if (lane == 0) {
+      out_i[r] = (int)e;
+      out_w[r] = expf(v - m0);
+    }
+  }
+  __syncwarp();
+  if (lane == 0) {
+    float s = 0.f;
+    for (int r = 0; r < k; ++r) s += out_w[r];
+    const float inv = 1.0f / s;
+    for (int r = 0; r < k; ++r) out_w[r] *= inv;
+  }
+  __syncwarp();
+}
+
+// One warp: top-k of the logits staged in shared memory, by (value desc,
+// index asc); each lane keeps its current best so that only the lane that
+// lost its best rescans.  out_w receives the renormalised softmax weights.
+__device__ __forceinline__ void warp_topk_smem(const float* lg, int E, int k, int* out_i, float* out_w) {
+  const int lane = threadIdx.x & 31;
+  constexpr int kPer = kMaxExperts / 32;
+  uint32_t taken = 0;
+  uint32_t best = 0;
+  int beste = 0x7FFFFFFF;
+  auto rescan = [&]() {
+    best = 0;
+    beste = 0x7FFFFFFF;
+#pragma unroll 4
+    for (int j = 0; j < kPer; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E && !(taken >> j & 1u)) {
+        const uint32_t key = f32_order_key(lg[e]);
+        if (key > best) { best = key; beste = e; }
+      }
+    }
+  };
+  rescan();
+  float m0 = 0.f;
+#pragma unroll 1
+  for (int r = 0; r < k; ++r) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, best);
+    const uint32_t e = __reduce_min_sync(0xffffffffu, best == m ? (uint32_t)beste : 0xFFFFFFFFu);
+    const float v = f32_from_order_key(m);
+    if (r == 0) m0 = v;
+    if (lane == 0) {
+      out_i[r] = (int)e;
+      out_w[r] = expf(v - m0);
+    }
+    if ((int)(e & 31u) == lane) {
+      taken |= 1u << (e >> 5);
+      rescan();
+    }
+  }
+  __syncwarp();
+  if (lane == 0) {
+    float s = 0.f;
+    for (int r = 0; r < k; ++r) s += out_w[r];
+    const float inv = 1.0f / s;
+    for (int r = 0; r < k; ++r) out_w[r] *= inv;
+  }
+  __syncwarp();
+}
+
+// One warp: top-k (k <= 8) of the logits staged in shared memory (E <= 512),
+// by (value desc, index asc).  Each lane sorts its 16 candidates in
+// registers; k rounds of warp-wide max/min reductions then pop the global
+// best from the head of one lane's list.  out_w receives the renormalised
+// softmax weights of the kept logits.
+__device__ __forceinline__ void warp_topk_sorted(const float* lg, int E, int k, int* out_i, float* out_w) {
+  const int lane = threadIdx.x & 31;
+  constexpr int kPer = kMaxExperts / 32;
+  uint32_t key[kPer];
+  int idx[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int e = lane + 32 * j;
+    key[j] = (e < E) ? f32_order_key(lg[e]) : 0u;
+    idx[j] = (e < E) ? e : 0x7FFFFFFF;
+  }
+  // odd-even transposition sort, descending by (key, -idx)
+#pragma unroll
+  for (int pass = 0; pass < kPer; ++pass) {
+#pragma unroll
+    for (int j = pass & 1; j + 1 < kPer; j += 2) {
+      const bool sw = key[j + 1] > key[j] || (key[j + 1] == key[j] && idx[j + 1] < idx[j]);
+      const uint32_t ka = key[j], kb = key[j + 1];
+      const int ia = idx[j], ib = idx[j + 1];
+      key[j] = sw ? kb : ka;
+      key[j + 1] = sw ? ka : kb;
+      idx[j] = sw ? ib : ia;
+      idx[j + 1] = sw ? ia : ib;
+    }
+  }
+  float m0 = 0.f;
+#pragma unroll 1
+  for (int r = 0; r < k; ++r) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, key[0]);
+    const uint32_t e = __reduce_min_sync(0xffffffffu, key[0] == m ? (uint32_t)idx[0] : 0xFFFFFFFFu);
+    const float v = f32_from_order_key(m);
+    if (r == 0) m0 = v;
+    if (lane == 0) {
+      out_i[r] = e < (uint32_t)E ? (int)e : 0;  // only a NaN logit could select past the end
+      out_w[r] = expf(v - m0);
+    }
+    if ((uint32_t)idx[0] == e) {  // pop the head
+#pragma unroll
+      for (int j = 0; j + 1 < kPer; ++j) {
+        key[j] = key[j + 1];
+        idx[j] = idx[j + 1];
+      }
+      key[kPer - 1] = 0u;
+      idx[kPer - 1] = 0x7FFFFFFF;
+    }
+  }
+  __syncwarp();
+  if (lane == 0) {
+    float s = 0.f;
+    for (int r = 0; r < k; ++r) s += out_w[r];
+    const float inv = 1.0f / s;
+    for (int r = 0; r < k; ++r) out_w[r] *= inv;
+  }
+  __syncwarp();
+}
+
+// One warp: top-k (k <= 8) of E <= 512 logits, by (value desc, index asc).
+// 64-bit keys (order-preserving value bits, then the complemented index)
+// make every key distinct.  Each lane sorts its 16 keys with a bitonic
+// network; a 5-level butterfly then merges sorted top-8 lists between lanes
+// (each level keeps the top 8 of the lane's and its partner's lists), after
+// which every lane holds the global top-8.  Lane r < k writes slot r and its
+// renormalised softmax weight.  No sequential selection rounds.
+__device__ __forceinline__ void cx_desc(unsigned long long& a, unsigned long long& b) {
+  const unsigned long long hi = a > b ? a : b;
+  const unsigned long long lo = a > b ? b : a;
+  a = hi;
+  b = lo;
+}
+__device__ __forceinline__ void warp_topk_bitonic(const float* lg, int E, int k, int* out_i, float* out_w) {
+  const int lane = threadIdx.x & 31;
+  constexpr int kPer = kMaxExperts / 32;  // 16
+  unsigned long long v[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int e = lane + 32 * j;
+    v[j] = (e < E) ? (((unsigned long long)f32_order_key(lg[e]) << 32) | (0xFFFFFFFFu - (uint32_t)e)) : 0ull;
+  }
+  // bitonic sort of 16, descending
+#pragma unroll
+  for (int size = 2; size <= kPer; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int j = i ^ stride;
+        if (j > i) {
+          if ((i & size) == 0) cx_desc(v[i], v[j]);
+          else cx_desc(v[j], v[i]);
+        }
+      }
+    }
+  }
+  // butterfly merge of the sorted top-8 lists
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    unsigned long long o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = __shfl_xor_sync(0xffffffffu, v[7 - i], d);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = v[i] > o[i] ? v[i] : o[i];
+#pragma unroll
+    for (int stride = 4; stride > 0; stride >>= 1) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int j = i ^ stride;
+        if (j > i) cx_desc(v[i], v[j]);
+      }
+    }
+  }
+  unsigned long long mine = v[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i)
+    if (lane == i) mine = v[i];
+  const float vmax = f32_from_order_key((uint32_t)(v[0] >> 32));
+  const float vr = f32_from_order_key((uint32_t)(mine >> 32));
+  const float ex = (lane < k) ? expf(vr - vmax) : 0.f;
+  float s = ex;
+#pragma unroll
+  for (int o = 4; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane < k) {
+    const uint32_t e = 0xFFFFFFFFu - (uint32_t)(mine & 0xFFFFFFFFull);
+    out_i[lane] = e < (uint32_t)E ? (int)e : 0;  // only a NaN logit could select past the end
+    out_w[lane] = ex / s;
+  }
+  __syncwarp();
+}
+
+// Two-accumulator variants (even / odd elements) to halve dependent chains.
+__device__ __forceinline__ void dot8_bf16_bf16_2(uint4 w, uint4 x, float& a, float& b) {
+  a = fma_bf16h<0, 0>(w.x, x.x, a);
+  b = fma_bf16h<1, 1>(w.x, x.x, b);
+  a = fma_bf16h<0, 0>(w.y, x.y, a);
+  b = fma_bf16h<1, 1>(w.y, x.y, b);
+  a = fma_bf16h<0, 0>(w.z, x.z, a);
+  b = fma_bf16h<1, 1>(w.z, x.z, b);
+  a = fma_bf16h<0, 0>(w.w, x.w, a);
+  b = fma_bf16h<1, 1>(w.w, x.w, b);
+}
+__device__ __forceinline__ void dot8_f_2(const float f[8], float4 x0, float4 x1, float& a, float& b) {
+  a = fmaf(f[0], x0.x, a);
+  b = fmaf(f[1], x0.y, b);
+  a = fmaf(f[2], x0.z, a);
+  b = fmaf(f[3], x0.w, b);
+  a = fmaf(f[4], x1.x, a);
+  b = fmaf(f[5], x1.y, b);
+  a = fmaf(f[6], x1.z, a);
+  b = fmaf(f[7], x1.w, b);
+}
+__device__ __forceinline__ void dot8_bf16_2(uint4 w, float4 x0, float4 x1, float& a, float& b) {
+  a = fmaf(bf16lo(w.x), x0.x, a);
+  b = fmaf(bf16hi(w.x), x0.y, b);
+  a = fmaf(bf16lo(w.y), x0.z, a);
+  b = fmaf(bf16hi(w.y), x0.w, b);
+  a = fmaf(bf16lo(w.z), x1.x, a);
+  b = fmaf(bf16hi(w.z), x1.y, b);
+  a = fmaf(bf16lo(w.w), x1.z, a);
+  b = fmaf(bf16hi(w.w), x1.w, b);
 }
 
 }  // namespace lingmoe

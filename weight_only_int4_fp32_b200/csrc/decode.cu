@@ -1,19 +1,24 @@
 // Decode / verify path (1 <= T <= kMaxDecodeT) of the W4 g32 MoE layer.
 //
 // One persistent launch per call, one CTA per SM, co-resident (cooperative
-// launch).  The work is a chain router -> top-k -> routed gate/up -> down,
-// so the CTAs meet at three bounded grid barriers:
+// launch), specialised at compile time for the token count T.  The work is a
+// chain router -> top-k -> routed gate/up -> down, so the CTAs meet at
+// bounded grid barriers:
 //
-//   phase 1  router logits (bf16 GEMV, fp32)            -> barrier A
-//   phase 2  shared-expert gate/up + SiLU*up (bf16)     -> barrier B
-//   phase 3  wait A; every CTA selects the top-k itself; routed gate/up
-//            (W4 g32, dequantised in registers) + SiLU*up -> barrier C
-//   phase 4  wait B, C; routed down (W4 g32) weighted by the routing weights,
-//            shared down (bf16), summed in a fixed order, one bf16 rounding.
+//   phase 1+2  router logits (bf16 GEMV, fp32) and shared-expert
+//              gate/up + SiLU*up (bf16)                        -> barriers A, B
+//   phase 3    wait A; every CTA selects the top-k itself; routed gate/up
+//              (W4 g32, dequantised in registers) + SiLU*up     -> barrier C
+//   phase 4    routed down (W4 g32) weighted by the routing weights and
+//              shared down (bf16), summed in a fixed order, one bf16 rounding.
 //
-// Bytes that do not depend on the routing (shared expert) are prefetched into
-// L2 at the start, and the routed down weights as soon as the routing is
-// known, so HBM keeps streaming across the barriers.
+// Weight bytes move HBM -> shared memory by non-multicast TMA bulk copies,
+// one private buffer and mbarrier per warp; each warp issues the copy of its
+// next item before it waits, and the compute loops read the staged bytes with
+// conflict-free 16-byte shared loads.  Bytes that do not depend on the
+// routing (shared expert) are requested first; routed down weights are
+// prefetched into L2 as soon as the routing is known and copied into shared
+// memory while the CTA waits at the last grid barrier.
 //
 // Layer definition: vLLM recipe page "inclusionAI/Ling-3.0-flash" (Overview;
 // "Single-GPU int4": symmetric W4, group 32, routed experts only) and the
@@ -24,177 +29,282 @@
 
 namespace lingmoe {
 
-// ---------------------------------------------------------------- smem plan
-constexpr int kMaxPairs = kMaxDecodeT * kMaxTopK;      // 32
-constexpr int kMaxBlkPerCta = 8;                       // down row-blocks per CTA (>= 640 / nctas)
+// Optional phase timestamps (compile with -DLING_MOE_TRACE): thread 0 of
+// every CTA records %globaltimer at each phase boundary.
+#ifdef LING_MOE_TRACE
+__device__ unsigned long long g_trace[1024][16];
+#define LING_TRACE(slot) \
+  do { if (threadIdx.x == 0) g_trace[blockIdx.x][slot] = globaltimer_ns(); } while (0)
+#else
+#define LING_TRACE(slot) do { } while (0)
+#endif
+
+constexpr int kWarps = kDecodeWarps;
+constexpr int kBufA = kGuUnitBytes;                 // per-warp buffer, phases 1-3
+constexpr int kDnBatch = 4;                         // routed down units per copy batch
+constexpr int kBufB = kDnBatch * kDnUnitBytes;      // per-warp buffer, phase 4
+constexpr int kShDnBytes = 4 * kI * 2;              // 4 shared-down rows
+constexpr int kMaxBlkPerCta = 8;                    // down row-blocks per CTA (>= 640 / nctas)
+constexpr int kRowBytes = kH * 2;                   // one bf16 row of H
+static_assert(kBufB >= kShDnBytes, "phase-4 buffer holds a shared-down block");
+static_assert(kBufA >= 2 * kRowBytes, "phase-1/2 buffer holds a gate and an up row");
 
 struct __align__(16) SmemHeader {
+  uint64_t mbar[kWarps][2];
+  uint64_t xbar;
+  uint32_t xmax[kMaxDecodeT];
+  float xscale[kMaxDecodeT];
+  int xinf;
+  int pad0[3];
   int topi[kMaxDecodeT][kMaxTopK];
   float topw[kMaxDecodeT][kMaxTopK];
+  int uniq_e[kMaxDecodeT * kMaxTopK];
+  int uniq_cnt[kMaxDecodeT * kMaxTopK];
+  int uniq_pair[kMaxDecodeT * kMaxTopK][kMaxDecodeT];
   int nuniq;
-  int uniq_e[kMaxPairs];
-  int uniq_cnt[kMaxPairs];
-  int uniq_pair[kMaxPairs][kMaxDecodeT];
   int flag;
+  int abort;
+  int pad[3];
+};
+static_assert(sizeof(SmemHeader) % 16 == 0, "header keeps the body 16-byte aligned");
+
+// x is kept twice: the bf16 input as staged (router and shared rows read it
+// with mixed-precision FMAs) and an fp16 copy scaled by 2^-sigma per token
+// (routed gate/up), laid out in 4 K-quarters of 1296 bytes so that the
+// quarters of a unit fall in different banks.
+constexpr int kXbTok = kH * 2;                   // bytes per token, bf16
+constexpr int kXhQuarter = (kH / 4) * 2 + 16;    // 1296 bytes
+constexpr int kXhTok = 4 * kXhQuarter;           // 5184 bytes
+
+// Shared-memory plan (byte offsets into the body).  Region A (phases 1-3)
+// and region B (phase 4) overlap: B is used only after the CTA's own phase 3.
+template <int T>
+struct Plan {
+  static constexpr int P = T * kMaxTopK;
+  static constexpr size_t xb = 0;                                           // [T][kXbTok]
+  static constexpr size_t xh = xb + (size_t)T * kXbTok;                     // [T][kXhTok]
+  static constexpr size_t cg = xh + (size_t)T * kXhTok;                     // float2 [T][kXGroups]
+  static constexpr size_t bufA = cg + (size_t)T * kXGroups * 8;             // [warps][kBufA]
+  static constexpr size_t endA = bufA + (size_t)kWarps * kBufA;
+  static constexpr size_t hp = 0;                                           // float [P][kHpStride]
+  static constexpr size_t chp = hp + (size_t)P * kHpStride * 4;             // float [P][kHGroups]
+  static constexpr size_t hs = chp + (size_t)P * kHGroups * 4;              // float [T][kHsTok]
+  static constexpr size_t part = hs + (size_t)T * kHsTok * 4;               // float [blk][P + T][4]
+  static constexpr size_t bufB = part + (size_t)kMaxBlkPerCta * (P + T) * 16;
+  static constexpr size_t endB = bufB + (size_t)kWarps * kBufB;
+  static constexpr size_t body = endA > endB ? endA : endB;
+  static constexpr size_t bytes = sizeof(SmemHeader) + body;
+  static_assert(xh % 16 == 0 && cg % 16 == 0 && bufA % 16 == 0 && bufB % 16 == 0 && chp % 16 == 0 &&
+                hs % 16 == 0 && part % 16 == 0, "16-byte aligned regions");
+  static_assert(bytes <= 227 * 1024, "decode smem over budget");
 };
 
-constexpr size_t kPhase13Floats = (size_t)kMaxDecodeT * kXTok + kMaxDecodeT * kXGroups;
-constexpr size_t kPhase4Floats = (size_t)kMaxPairs * kHpStride + kMaxPairs * kHGroups +
-                                 (size_t)kMaxDecodeT * kHsTok +
-                                 (size_t)kMaxBlkPerCta * (kMaxPairs + kMaxDecodeT) * 4;
-constexpr size_t kBodyFloats = kPhase13Floats > kPhase4Floats ? kPhase13Floats : kPhase4Floats;
-constexpr size_t kDecodeSmemBytes = sizeof(SmemHeader) + kBodyFloats * sizeof(float);
+size_t decode_smem_bytes(int T) {
+  switch (T) {
+    case 1: return Plan<1>::bytes;
+    case 2: return Plan<2>::bytes;
+    case 3: return Plan<3>::bytes;
+    default: return Plan<4>::bytes;
+  }
+}
 
-size_t decode_smem_bytes() { return kDecodeSmemBytes; }
+__device__ __forceinline__ bool aborted(const SmemHeader& hd) {
+  return *reinterpret_cast<const volatile int*>(&hd.abort) != 0;
+}
 
-// ---------------------------------------------------------------- helpers
-// ---------------------------------------------------------------- kernel
-__global__ void __launch_bounds__(kDecodeThreads, 1)
-moe_decode_kernel(const DecodeParams p) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+// ---------------------------------------------------------------- arrival counters
+__device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned int* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Publish: the calling thread's earlier stores (and, after a warp or CTA
+// barrier, those of the other threads) become visible before the count.
+__device__ __forceinline__ void arrive(unsigned int* ctr) {
+  __threadfence();
+  atomicAdd(ctr, 1u);
+}
+// Bounded poll until *ctr >= target.  On time-out sets the error word and the
+// CTA's abort flag; returns false.
+__device__ __forceinline__ bool wait_count(const unsigned int* ctr, uint32_t target,
+                                           unsigned long long limit_ns, unsigned int* err, int* abort) {
+  if (ld_acquire_u32(ctr) >= target) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (ld_acquire_u32(ctr) < target) {
+    if (*reinterpret_cast<volatile int*>(abort) || globaltimer_ns() - t0 > limit_ns) {
+      atomicOr(err, 1u);
+      *reinterpret_cast<volatile int*>(abort) = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+template <int T>
+__global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const DecodeParams p) {
+  using PL = Plan<T>;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
   SmemHeader& hd = *reinterpret_cast<SmemHeader*>(smem_raw);
-  float* body = reinterpret_cast<float*>(smem_raw + sizeof(SmemHeader));
+  unsigned char* body = smem_raw + sizeof(SmemHeader);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int cta = blockIdx.x, ncta = gridDim.x;
-  const int T = p.T, E = p.E, K = p.k;
+  const int E = p.E, K = p.k;
+  LING_TRACE(0);
 
-  // barrier generations (read before this CTA arrives anywhere)
-  const unsigned long long genA = ld_acquire_u64(p.bar + 0) / ncta;
-  const unsigned long long genB = ld_acquire_u64(p.bar + 1) / ncta;
-  const unsigned long long genC = ld_acquire_u64(p.bar + 2) / ncta;
-  const bool skip = (cta == p.skip_arrive_cta);
+  const bool withhold = (cta == p.skip_arrive_cta);
 
   // this CTA's slices
   const int r0 = (int)((long long)cta * E / ncta), r1 = (int)((long long)(cta + 1) * E / ncta);
   const int s0 = cta * kI / ncta, s1 = (cta + 1) * kI / ncta;
   const int b0 = cta * kDnUnits / ncta, b1 = (cta + 1) * kDnUnits / ncta;
   const int nblk = b1 - b0;
+  const int nr = r1 - r0, n12 = nr + (s1 - s0);
 
-  // L2 prefetch of routing-independent bytes: shared gate/up rows, shared down rows
-  if (warp == kDecodeWarps - 1) {
-    const uint32_t row_bytes = kH * 2;
-    for (int i = s0 + lane; i < s1; i += 32) {
-      prefetch_l2_bulk(p.sh_gate + (size_t)i * kH, row_bytes);
-      prefetch_l2_bulk(p.sh_up + (size_t)i * kH, row_bytes);
+  uint64_t* barA = &hd.mbar[warp][0];
+  uint64_t* barB = &hd.mbar[warp][1];
+  uint32_t pha = 0, phb = 0;
+  unsigned char* bufA = body + PL::bufA + (size_t)warp * kBufA;
+  unsigned char* bufB = body + PL::bufB + (size_t)warp * kBufB;
+  unsigned char* xb = body + PL::xb;
+  unsigned char* xh = body + PL::xh;
+  float2* cg = reinterpret_cast<float2*>(body + PL::cg);
+  if (tid < kMaxDecodeT) {
+    hd.xmax[tid] = 0u;
+    hd.xscale[tid] = 1.0f;
+  }
+  if (tid == 0) {
+    hd.abort = 0;
+    hd.xinf = 0;
+    mbar_init(&hd.xbar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&hd.xbar, T * kXbTok);
+    bulk_g2s(xb, p.x, T * kXbTok, &hd.xbar);
+  }
+  if (lane == 0) {
+    mbar_init(barA, 1);
+    mbar_init(barB, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();  // barriers initialised before anyone waits on them
+
+  // phase-1/2 item `it`: router row (it < nr) or shared gate+up rows
+  auto issue12 = [&](int it) {
+    if (lane == 0) {
+      if (it < nr) {
+        mbar_arrive_expect_tx(barA, kRowBytes);
+        bulk_g2s(bufA, p.router_w + (size_t)(r0 + it) * kH, kRowBytes, barA);
+      } else {
+        const int i = s0 + it - nr;
+        mbar_arrive_expect_tx(barA, 2 * kRowBytes);
+        bulk_g2s(bufA, p.sh_gate + (size_t)i * kH, kRowBytes, barA);
+        bulk_g2s(bufA + kRowBytes, p.sh_up + (size_t)i * kH, kRowBytes, barA);
+      }
     }
-    if (lane == 0 && nblk > 0)
-      prefetch_l2_bulk(p.sh_down + (size_t)b0 * 4 * kI, (uint32_t)nblk * 4 * kI * 2);
-  }
+  };
+  if (warp < n12) issue12(warp);
 
-  // ---- stage x (fp32 planes) and the group sums
-  float* xs = body;
-  float* cx = body + (size_t)kMaxDecodeT * kXTok;
-  for (int v = tid; v < T * kXChunks; v += kDecodeThreads) {
-    const int t = v / kXChunks, c = v - t * kXChunks;
-    const uint4 w = *reinterpret_cast<const uint4*>(p.x + (size_t)t * kH + 8 * c);
-    float* d = xs + (size_t)t * kXTok + xoff(c);
-    *reinterpret_cast<float4*>(d) = make_float4(bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y));
-    *reinterpret_cast<float4*>(d + kXPlane) =
-        make_float4(bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w));
-  }
-  __syncthreads();
-  for (int v = tid; v < T * kXGroups; v += kDecodeThreads) {
-    const int t = v / kXGroups, G = v - t * kXGroups;
-    const float* xt = xs + (size_t)t * kXTok;
-    float s = 0.f;
-    for (int i = 0; i < 4; ++i) {
-      const int c = 4 * G + i;
-      const float4 a = *reinterpret_cast<const float4*>(xt + xoff(c));
-      const float4 b = *reinterpret_cast<const float4*>(xt + kXPlane + xoff(c));
-      s += a.x + a.y + a.z + a.w + b.x + b.y + b.z + b.w;
-    }
-    cx[t * kXGroups + G] = kBiasCoef * s;
-  }
-  __syncthreads();
+  // L2 prefetch of the shared down rows this CTA will need
+  if (warp == kWarps - 1 && lane == 0 && nblk > 0)
+    prefetch_l2_bulk(p.sh_down + (size_t)b0 * 4 * kI, (uint32_t)nblk * kShDnBytes);
 
-  // ---- phase 1: router logits for rows [r0, r1)
-  for (int e = r0 + warp; e < r1; e += kDecodeWarps) {
-    const __nv_bfloat16* wr = p.router_w + (size_t)e * kH;
-    uint4 w[kXChunks / 32];
+  // x (bf16) lands in shared memory; every warp waits for it once
+  if (!mbar_wait(&hd.xbar, 0, p.wait_limit_ns, p.err)) hd.abort = 1;
+  LING_TRACE(1);
+
+  // ---- phases 1+2: router rows (published at once) and shared gate/up rows
+  for (int it = warp; it < n12; it += kWarps) {
+    if (it != warp) issue12(it);
+    if (!mbar_wait(barA, pha, p.wait_limit_ns, p.err)) { hd.abort = 1; break; }
+    pha ^= 1;
+    const bool router = it < nr;
+    float a0[T], a1[T];
+    {
+      float g0[T], g1[T], g2[T], g3[T], u0_[T], u1_[T], u2_[T], u3_[T];
 #pragma unroll
-    for (int m = 0; m < kXChunks / 32; ++m) w[m] = ldg_stream(wr + 8 * (lane + 32 * m));
-    const float bias = p.router_bias ? p.router_bias[e] : 0.f;
-    float acc[kMaxDecodeT];
+      for (int t = 0; t < T; ++t) g0[t] = g1[t] = g2[t] = g3[t] = u0_[t] = u1_[t] = u2_[t] = u3_[t] = 0.f;
 #pragma unroll
-    for (int t = 0; t < kMaxDecodeT; ++t) acc[t] = 0.f;
+      for (int m = 0; m < kXChunks / 32; m += 2) {
+        const int c0 = lane + 32 * m, c1 = c0 + 32;
+        const uint4 w00 = lds128(bufA + 16 * c0), w01 = lds128(bufA + 16 * c1);
+        const uint4 w10 = router ? w00 : lds128(bufA + kRowBytes + 16 * c0);
+        const uint4 w11 = router ? w01 : lds128(bufA + kRowBytes + 16 * c1);
 #pragma unroll
-    for (int m = 0; m < kXChunks / 32; ++m) {
-      const int o = xoff(lane + 32 * m);
-#pragma unroll
-      for (int t = 0; t < kMaxDecodeT; ++t) {
-        if (t < T) {
-          const float* xt = xs + (size_t)t * kXTok + o;
-          acc[t] = dot8_bf16(w[m], *reinterpret_cast<const float4*>(xt),
-                             *reinterpret_cast<const float4*>(xt + kXPlane), acc[t]);
+        for (int t = 0; t < T; ++t) {
+          const uint4 xv0 = lds128(xb + t * kXbTok + 16 * c0), xv1 = lds128(xb + t * kXbTok + 16 * c1);
+          dot8_bf16_bf16_2(w00, xv0, g0[t], g1[t]);
+          dot8_bf16_bf16_2(w01, xv1, g2[t], g3[t]);
+          if (!router) {
+            dot8_bf16_bf16_2(w10, xv0, u0_[t], u1_[t]);
+            dot8_bf16_bf16_2(w11, xv1, u2_[t], u3_[t]);
+          }
         }
       }
-    }
 #pragma unroll
-    for (int t = 0; t < kMaxDecodeT; ++t) {
-      if (t < T) {
-        const float v = warp_sum(acc[t]);
-        if (lane == 0) p.logits[(size_t)t * E + e] = v + bias;
+      for (int t = 0; t < T; ++t) {
+        a0[t] = (g0[t] + g1[t]) + (g2[t] + g3[t]);
+        a1[t] = (u0_[t] + u1_[t]) + (u2_[t] + u3_[t]);
       }
     }
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+      const float g = warp_sum(a0[t]);
+      if (router) {
+        if (lane == 0) p.logits[(size_t)t * E + r0 + it] = g + (p.router_bias ? p.router_bias[r0 + it] : 0.f);
+      } else {
+        const float u = warp_sum(a1[t]);
+        if (lane == 0) p.h_s[(size_t)t * kI + s0 + it - nr] = silu_mul(g, u);
+      }
+    }
+    if (lane == 0 && !(router && withhold)) arrive(p.sync + (router ? 0 : 1));
+    __syncwarp();
   }
-  grid_arrive(p.bar + 0, skip);
+  LING_TRACE(2);
 
-  // ---- phase 2: shared expert gate/up rows [s0, s1)
-  for (int i = s0 + warp; i < s1; i += kDecodeWarps) {
-    const __nv_bfloat16* wg = p.sh_gate + (size_t)i * kH;
-    const __nv_bfloat16* wu = p.sh_up + (size_t)i * kH;
-    uint4 g[kXChunks / 32], u[kXChunks / 32];
+  LING_TRACE(10);
+  // ---- routing: every CTA selects the top-k itself from the published logits
+  if (warp < T && !aborted(hd)) {
+    float* lg = reinterpret_cast<float*>(bufA);  // scratch: this warp's buffer is idle here
+    bool ok = true;
+    if (lane == 0) ok = wait_count(p.sync + 0, (uint32_t)E, p.wait_limit_ns, p.err, &hd.abort);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (warp == 0) LING_TRACE(11);
+    if (ok) {
+      const float* src = p.logits + (size_t)warp * E;
 #pragma unroll
-    for (int m = 0; m < kXChunks / 32; ++m) {
-      g[m] = ldg_stream(wg + 8 * (lane + 32 * m));
-      u[m] = ldg_stream(wu + 8 * (lane + 32 * m));
+      for (int j = 0; j < kMaxExperts / 32; ++j)
+        if (lane + 32 * j < E) lg[lane + 32 * j] = ldcg_f32(src + lane + 32 * j);
     }
-    float ag[kMaxDecodeT], au[kMaxDecodeT];
-#pragma unroll
-    for (int t = 0; t < kMaxDecodeT; ++t) ag[t] = au[t] = 0.f;
-#pragma unroll
-    for (int m = 0; m < kXChunks / 32; ++m) {
-      const int o = xoff(lane + 32 * m);
-#pragma unroll
-      for (int t = 0; t < kMaxDecodeT; ++t) {
-        if (t < T) {
-          const float* xt = xs + (size_t)t * kXTok + o;
-          const float4 a = *reinterpret_cast<const float4*>(xt);
-          const float4 b = *reinterpret_cast<const float4*>(xt + kXPlane);
-          ag[t] = dot8_bf16(g[m], a, b, ag[t]);
-          au[t] = dot8_bf16(u[m], a, b, au[t]);
-        }
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < kMaxDecodeT; ++t) {
-      if (t < T) {
-        const float vg = warp_sum(ag[t]);
-        const float vu = warp_sum(au[t]);
-        if (lane == 0) p.h_s[(size_t)t * kI + i] = silu_mul(vg, vu);
-      }
-    }
+    __syncwarp();
+    if (warp == 0) LING_TRACE(12);
+    warp_topk_bitonic(lg, E, K, hd.topi[warp], hd.topw[warp]);
   }
-  grid_arrive(p.bar + 1, skip);
-
-  // ---- phase 3: routing (every CTA, redundantly), then routed gate/up
-  if (!grid_wait(p.bar + 0, (genA + 1) * ncta, p.wait_limit_ns, p.err, &hd.flag)) return;
-  if (warp < T) warp_topk(p.logits + (size_t)warp * E, E, K, hd.topi[warp], hd.topw[warp]);
   __syncthreads();
-  if (warp == 0) {
+  LING_TRACE(3);
+  if (T == 1) {
+    // one token: the selected experts are already distinct
+    if (tid < K) {
+      hd.uniq_e[tid] = hd.topi[0][tid];
+      hd.uniq_cnt[tid] = 1;
+      hd.uniq_pair[tid][0] = tid;
+      if (cta == 0) {
+        if (p.topk_idx_out) p.topk_idx_out[tid] = hd.topi[0][tid];
+        if (p.topk_w_out) p.topk_w_out[tid] = hd.topw[0][tid];
+      }
+    }
+    if (tid == 0) hd.nuniq = K;
+  } else if (warp == 0 && !aborted(hd)) {
     // union of the selected experts, in first-occurrence order (t-major)
     const int npairs = T * K;
     const int pe = (lane < npairs) ? hd.topi[lane / K][lane % K] : -1 - lane;
     bool first = lane < npairs;
-    for (int j = 0; j < 32; ++j) {
+    for (int j = 0; j < npairs; ++j) {
       const int ej = __shfl_sync(0xffffffffu, pe, j);
       if (j < lane && ej == pe) first = false;
     }
     const unsigned fm = __ballot_sync(0xffffffffu, first);
     const int myu = first ? __popc(fm & ((1u << lane) - 1u)) : -1;
     if (first) hd.uniq_e[myu] = pe;
-    // token lists (pair indices t*K+slot, ascending) of each unique expert
     int cnt = 0;
     for (int j = 0; j < npairs; ++j) {
       const int ej = __shfl_sync(0xffffffffu, pe, j);
@@ -204,181 +314,308 @@ moe_decode_kernel(const DecodeParams p) {
     if (lane == 0) hd.nuniq = __popc(fm);
     if (cta == 0 && lane < npairs) {
       const int t = lane / K, s = lane % K;
-      p.topk_idx_ws[lane] = hd.topi[t][s];
-      p.topk_w_ws[lane] = hd.topw[t][s];
       if (p.topk_idx_out) p.topk_idx_out[lane] = hd.topi[t][s];
       if (p.topk_w_out) p.topk_w_out[lane] = hd.topw[t][s];
     }
   }
   __syncthreads();
-  const int U = hd.nuniq;
+  const int U = aborted(hd) ? 0 : hd.nuniq;
+  LING_TRACE(4);
 
-  // prefetch this CTA's routed down units (contiguous per expert) into L2
-  if (warp == kDecodeWarps - 1 && nblk > 0) {
+  // ---- phase 3: routed gate/up units, each copied in two halves
+  const int n3 = U * kGuUnits;
+  const int u0 = (int)((long long)cta * n3 / ncta), u1 = (int)((long long)(cta + 1) * n3 / ncta);
+  auto issue3 = [&](int unit) {
+    if (lane == 0) {
+      const int u = unit / kGuUnits, b = unit - u * kGuUnits;
+      const uint8_t* src = p.gu + ((size_t)hd.uniq_e[u] * kGuUnits + b) * kGuUnitBytes;
+      constexpr int kHalf = kGuScaleOff / 2;
+      mbar_arrive_expect_tx(barA, kHalf + (kGuUnitBytes - kGuScaleOff));
+      bulk_g2s(bufA + kGuScaleOff, src + kGuScaleOff, kGuUnitBytes - kGuScaleOff, barA);
+      bulk_g2s(bufA, src, kHalf, barA);
+      mbar_arrive_expect_tx(barB, kHalf);
+      bulk_g2s(bufA + kHalf, src + kHalf, kHalf, barB);
+    }
+  };
+  if (u0 + warp < u1) issue3(u0 + warp);
+  // routed down units of this CTA (contiguous per expert) into L2
+  if (warp == kWarps - 1 && nblk > 0) {
     for (int u = lane; u < U; u += 32) {
       const uint8_t* src = p.dn + ((size_t)hd.uniq_e[u] * kDnUnits + b0) * kDnUnitBytes;
       prefetch_l2_bulk(src, (uint32_t)nblk * kDnUnitBytes);
     }
   }
+  // fp16 copy of x and the per-group bias constants of the int4 dot products,
+  // built while the first units are in flight: 4 lanes per group of 32.  x is
+  // converted as is (exact for normal bf16 values below 65504); if any value
+  // overflows fp16, the token is redone scaled by 2^-sigma.
+  auto build_xh = [&]() {
+    const int sub = lane & 3, gw = lane >> 2;
+    for (int g0 = warp * 8; g0 < T * kXGroups; g0 += kWarps * 8) {
+      const int g = g0 + gw;
+      float se = 0.f, so = 0.f;
+      if (g < T * kXGroups) {
+        const int t = g / kXGroups, G = g - t * kXGroups, c = 4 * G + sub;
+        const uint4 w = lds128(xb + t * kXbTok + 16 * c);
+        const float inv = 1.0f / hd.xscale[t];
+        const __half2 h0 = __floats2half2_rn(bf16lo(w.x) * inv, bf16hi(w.x) * inv);
+        const __half2 h1 = __floats2half2_rn(bf16lo(w.y) * inv, bf16hi(w.y) * inv);
+        const __half2 h2 = __floats2half2_rn(bf16lo(w.z) * inv, bf16hi(w.z) * inv);
+        const __half2 h3 = __floats2half2_rn(bf16lo(w.w) * inv, bf16hi(w.w) * inv);
+        if (__hisinf(h0.x) | __hisinf(h0.y) | __hisinf(h1.x) | __hisinf(h1.y) | __hisinf(h2.x) |
+            __hisinf(h2.y) | __hisinf(h3.x) | __hisinf(h3.y))
+          hd.xinf = 1;
+        uint4 o;
+        o.x = *reinterpret_cast<const uint32_t*>(&h0);
+        o.y = *reinterpret_cast<const uint32_t*>(&h1);
+        o.z = *reinterpret_cast<const uint32_t*>(&h2);
+        o.w = *reinterpret_cast<const uint32_t*>(&h3);
+        *reinterpret_cast<uint4*>(xh + t * kXhTok + (c / 80) * kXhQuarter + 16 * (c % 80)) = o;
+        const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
+        const float2 f2 = __half22float2(h2), f3 = __half22float2(h3);
+        se = (f0.x + f1.x) + (f2.x + f3.x);
+        so = (f0.y + f1.y) + (f2.y + f3.y);
+      }
+      se += __shfl_xor_sync(0xffffffffu, se, 1);
+      so += __shfl_xor_sync(0xffffffffu, so, 1);
+      se += __shfl_xor_sync(0xffffffffu, se, 2);
+      so += __shfl_xor_sync(0xffffffffu, so, 2);
+      if (sub == 0 && g < T * kXGroups) cg[g] = make_float2(kEvenBias * se, kOddBias * so);
+    }
+  };
+  build_xh();
+  __syncthreads();
+  if (hd.xinf) {
+    // rare: some |x| beyond the fp16 range; scale that token by 2^-sigma
+    for (int v = tid; v < T * kXChunks; v += kDecodeThreads) {
+      const int t = v / kXChunks, c = v - t * kXChunks;
+      const uint4 w = lds128(xb + t * kXbTok + 16 * c);
+      const float mx = fmaxf(fmaxf(fmaxf(fabsf(bf16lo(w.x)), fabsf(bf16hi(w.x))),
+                                   fmaxf(fabsf(bf16lo(w.y)), fabsf(bf16hi(w.y)))),
+                             fmaxf(fmaxf(fabsf(bf16lo(w.z)), fabsf(bf16hi(w.z))),
+                                   fmaxf(fabsf(bf16lo(w.w)), fabsf(bf16hi(w.w)))));
+      atomicMax(&hd.xmax[t], __float_as_uint(fminf(mx, 3.0e38f)));  // monotonic for non-negative floats
+    }
+    __syncthreads();
+    if (tid < T) {
+      const int e = (int)(hd.xmax[tid] >> 23) - 127;
+      const int sigma = e >= 14 ? e - 13 : 0;
+      hd.xscale[tid] = __uint_as_float((uint32_t)(127 + sigma) << 23);
+    }
+    __syncthreads();
+    build_xh();
+    __syncthreads();
+  }
+  LING_TRACE(15);
 
   {
-    const int n3 = U * kGuUnits;
-    const int u0 = (int)((long long)cta * n3 / ncta), u1 = (int)((long long)(cta + 1) * n3 / ncta);
     const int r = lane & 7, q = lane >> 3;
-    for (int unit = u0 + warp; unit < u1; unit += kDecodeWarps) {
+    for (int unit = u0 + warp; unit < u1; unit += kWarps) {
+      if (unit != u0 + warp) issue3(unit);
       const int u = unit / kGuUnits, b = unit - u * kGuUnits;
-      const uint8_t* base = p.gu + ((size_t)hd.uniq_e[u] * kGuUnits + b) * kGuUnitBytes;
-      uint4 wq[kGuChunks];
-      uint2 sc[kGuChunks / 4];
-#pragma unroll
-      for (int j = 0; j < kGuChunks; ++j) wq[j] = ldg_stream(base + j * 512 + 16 * lane);
-#pragma unroll
-      for (int j = 0; j < kGuChunks / 4; ++j) sc[j] = ldg_stream64(base + kGuScaleOff + j * 256 + 8 * lane);
       const int cnt = hd.uniq_cnt[u];
-      // per-token bases: chunk 4G+i of quarter q sits at 324q + 16j + 4i
-      const float* xb[kMaxDecodeT];
-      const float* cb[kMaxDecodeT];
-      float acc[kMaxDecodeT];
+      int xo[T], co[T];
+      float xsc[T];
 #pragma unroll
-      for (int tt = 0; tt < kMaxDecodeT; ++tt) {
+      for (int tt = 0; tt < T; ++tt) {
         const int t = (tt < cnt) ? hd.uniq_pair[u][tt] / K : 0;
-        xb[tt] = xs + (size_t)t * kXTok + 324 * q;
-        cb[tt] = cx + t * kXGroups + q * kGuChunks;
-        acc[tt] = 0.f;
+        xo[tt] = t * kXhTok + q * kXhQuarter;   // group 20q+j at + 64j, word i at + 16i
+        co[tt] = t * kXGroups + q * kGuChunks;
+        xsc[tt] = hd.xscale[t];
       }
+      float acc[T];
 #pragma unroll
-      for (int j = 0; j < kGuChunks; ++j) {
-        float part[kMaxDecodeT];
+      for (int tt = 0; tt < T; ++tt) acc[tt] = 0.f;
+      bool ok = mbar_wait(barA, pha, p.wait_limit_ns, p.err);
+      pha ^= 1;
+      if (warp == 0 && unit == u0) LING_TRACE(13);
+#pragma unroll 1
+      for (int j = 0; j < kGuChunks && ok; ++j) {
+        if (j == kGuChunks / 2) {
+          ok = mbar_wait(barB, phb, p.wait_limit_ns, p.err);
+          if (!ok) break;
+        }
+        const uint4 w = lds128(bufA + j * 512 + 16 * lane);
+        const float s = bf16_to_f32(*reinterpret_cast<const unsigned short*>(
+            bufA + kGuScaleOff + (j >> 2) * 256 + 8 * lane + 2 * (j & 3)));
+        float ae[T], ao[T], be[T], bo[T];
 #pragma unroll
-        for (int tt = 0; tt < kMaxDecodeT; ++tt) part[tt] = (tt < cnt) ? cb[tt][j] : 0.f;
-        const uint32_t wj[4] = {wq[j].x, wq[j].y, wq[j].z, wq[j].w};
+        for (int tt = 0; tt < T; ++tt) {
+          const float2 c2 = (tt < cnt) ? cg[co[tt] + j] : make_float2(0.f, 0.f);
+          ae[tt] = c2.x;
+          ao[tt] = c2.y;
+          be[tt] = 0.f;
+          bo[tt] = 0.f;
+        }
+        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          float f[8];
-          dequant8(wj[i], f);
+          const Pairs4 P = dequant_f16x2(wv[i]);
 #pragma unroll
-          for (int tt = 0; tt < kMaxDecodeT; ++tt) {
+          for (int tt = 0; tt < T; ++tt) {
             if (tt < cnt) {
-              const float* xq = xb[tt] + 16 * j + 4 * i;
-              part[tt] = dot8_f(f, *reinterpret_cast<const float4*>(xq),
-                                *reinterpret_cast<const float4*>(xq + kXPlane), part[tt]);
+              const uint4 xv = lds128(xh + xo[tt] + 64 * j + 16 * i);
+              if (i & 1) dot8_q_f16(P, xv, be[tt], bo[tt]);
+              else dot8_q_f16(P, xv, ae[tt], ao[tt]);
             }
           }
         }
-        const float s = scale_of(sc[j >> 2], j & 3);
 #pragma unroll
-        for (int tt = 0; tt < kMaxDecodeT; ++tt) acc[tt] = fmaf(s, part[tt], acc[tt]);
+        for (int tt = 0; tt < T; ++tt)
+          acc[tt] = fmaf(s, fmaf(0.0625f, ao[tt] + bo[tt], ae[tt] + be[tt]), acc[tt]);
       }
+      phb ^= 1;
+      if (!ok) { hd.abort = 1; break; }
+      __syncwarp();
 #pragma unroll
-      for (int tt = 0; tt < kMaxDecodeT; ++tt) {
+      for (int tt = 0; tt < T; ++tt) {
         if (tt < cnt) {
           float v = acc[tt];
           v += __shfl_xor_sync(0xffffffffu, v, 8);
           v += __shfl_xor_sync(0xffffffffu, v, 16);
+          v *= xsc[tt];
           const float up = __shfl_sync(0xffffffffu, v, (lane & ~7) | ((r + 4) & 7));
-          if (r < 4 && q == tt) {
-            const int pr = hd.uniq_pair[u][tt];
-            p.h_pair[(size_t)pr * kI + 4 * b + r] = silu_mul(kCodeScale * v, kCodeScale * up);
-          }
+          if (r < 4 && q == tt)
+            p.h_pair[(size_t)hd.uniq_pair[u][tt] * kI + 4 * b + r] = silu_mul(v, up);
         }
       }
+      __syncwarp();
+      if (lane == 0) arrive(p.sync + 2);
+      if (warp == 0 && unit == u0) LING_TRACE(14);
     }
   }
-  grid_arrive(p.bar + 2, skip);
+  __syncthreads();
+  LING_TRACE(5);
 
   // ---- phase 4: down projections and the output
-  if (!grid_wait(p.bar + 1, (genB + 1) * ncta, p.wait_limit_ns, p.err, &hd.flag)) return;
-  if (!grid_wait(p.bar + 2, (genC + 1) * ncta, p.wait_limit_ns, p.err, &hd.flag)) return;
-
+  // Region A is free now; start this warp's first phase-4 copy before waiting.
   const int npairs = T * K;
-  float* hp = body;                                           // [pairs][kHpStride]
-  float* chp = hp + (size_t)kMaxPairs * kHpStride;            // [pairs][kHGroups]
-  float* hs = chp + (size_t)kMaxPairs * kHGroups;             // [T][kHsTok]
-  float* part = hs + (size_t)kMaxDecodeT * kHsTok;            // [blk][pairs + T][4]
-  for (int v = tid; v < npairs * (kI / 4); v += kDecodeThreads) {
-    const int pr = v / (kI / 4), c4 = v - pr * (kI / 4);
-    const float4 h = ldcg_f4(reinterpret_cast<const float4*>(p.h_pair + (size_t)pr * kI) + c4);
-    const int e0 = 4 * c4;
-    *reinterpret_cast<float4*>(hp + (size_t)pr * kHpStride + e0 + 4 * (e0 / 96)) = h;
-  }
-  for (int v = tid; v < T * (kI / 4); v += kDecodeThreads) {
-    const int t = v / (kI / 4), c4 = v - t * (kI / 4);
-    const float4 h = ldcg_f4(reinterpret_cast<const float4*>(p.h_s + (size_t)t * kI) + c4);
-    const int c = c4 >> 1, pl = c4 & 1;
-    *reinterpret_cast<float4*>(hs + (size_t)t * kHsTok + pl * kHsPlane + 4 * c) = h;
-  }
-  __syncthreads();
-  for (int v = tid; v < npairs * kHGroups; v += kDecodeThreads) {
-    const int pr = v / kHGroups, G = v - pr * kHGroups;
-    const float* src = hp + (size_t)pr * kHpStride + 32 * G + 4 * (G / 3);
-    float s = 0.f;
-    for (int i = 0; i < 32; ++i) s += src[i];
-    chp[pr * kHGroups + G] = kBiasCoef * s;
-  }
-  __syncthreads();
+  const int nitems = nblk * U;
+  const int nbatch = (nitems + kDnBatch - 1) / kDnBatch;
+  const int nmine_r = warp < nbatch ? (nbatch - warp + kWarps - 1) / kWarps : 0;
+  const int sh_first = kWarps - 1 - warp;
+  const int nmine_s = (!aborted(hd) && sh_first < nblk) ? (nblk - sh_first + kWarps - 1) / kWarps : 0;
+  auto issue4 = [&](int s) {
+    if (lane == 0) {
+      if (s < nmine_r) {
+        const int bi = warp + s * kWarps;
+        const int it0 = bi * kDnBatch, n = min(kDnBatch, nitems - it0);
+        mbar_arrive_expect_tx(barA, (uint32_t)n * kDnUnitBytes);
+        for (int bI = 0; bI < n; ++bI) {
+          const int it = it0 + bI, blk = it / U, u = it - blk * U;
+          bulk_g2s(bufB + bI * kDnUnitBytes,
+                   p.dn + ((size_t)hd.uniq_e[u] * kDnUnits + b0 + blk) * kDnUnitBytes, kDnUnitBytes, barA);
+        }
+      } else {
+        const int blk = sh_first + (s - nmine_r) * kWarps;
+        mbar_arrive_expect_tx(barA, kShDnBytes);
+        bulk_g2s(bufB, p.sh_down + (size_t)(b0 + blk) * 4 * kI, kShDnBytes, barA);
+      }
+    }
+  };
+  const int nseq = nmine_r + nmine_s;
+  if (nseq > 0) issue4(0);
 
-  // routed items (blk, u): 4 output rows x one unique expert, for its tokens
+  float* hp = reinterpret_cast<float*>(body + PL::hp);
+  float* chp = reinterpret_cast<float*>(body + PL::chp);
+  float* hsm = reinterpret_cast<float*>(body + PL::hs);
+  float* part = reinterpret_cast<float*>(body + PL::part);
+  if (tid == 0 && !aborted(hd)) {
+    if (wait_count(p.sync + 1, (uint32_t)kI, p.wait_limit_ns, p.err, &hd.abort))
+      wait_count(p.sync + 2, (uint32_t)(U * kGuUnits), p.wait_limit_ns, p.err, &hd.abort);
+  }
+  __syncthreads();
+  if (!aborted(hd)) {
+    for (int v = tid; v < npairs * (kI / 4); v += kDecodeThreads) {
+      const int pr = v / (kI / 4), c4 = v - pr * (kI / 4);
+      const float4 h = ldcg_f4(reinterpret_cast<const float4*>(p.h_pair + (size_t)pr * kI) + c4);
+      const int e0 = 4 * c4;
+      *reinterpret_cast<float4*>(hp + (size_t)pr * kHpStride + e0 + 4 * (e0 / 96)) = h;
+    }
+    for (int v = tid; v < T * (kI / 4); v += kDecodeThreads) {
+      const int t = v / (kI / 4), c4 = v - t * (kI / 4);
+      const float4 h = ldcg_f4(reinterpret_cast<const float4*>(p.h_s + (size_t)t * kI) + c4);
+      const int c = c4 >> 1, pl = c4 & 1;
+      *reinterpret_cast<float4*>(hsm + (size_t)t * kHsTok + pl * kHsPlane + 4 * c) = h;
+    }
+  }
+  __syncthreads();
+  LING_TRACE(6);
+  {
+    // group sums of h, 8 lanes per group of 32 (conflict-free 16-byte reads)
+    const int sub = lane & 7, gw = lane >> 3;
+    for (int g0 = warp * 4; g0 < npairs * kHGroups; g0 += kWarps * 4) {
+      const int g = g0 + gw;
+      float sum = 0.f;
+      if (g < npairs * kHGroups) {
+        const int pr = g / kHGroups, G = g - pr * kHGroups;
+        const float4 v = ldsf4(hp + (size_t)pr * kHpStride + 32 * G + 4 * (G / 3) + 4 * sub);
+        sum = (v.x + v.y) + (v.z + v.w);
+      }
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+      if (sub == 0 && g < npairs * kHGroups) chp[g] = kBiasCoef * sum;
+    }
+  }
+  __syncthreads();
+  LING_TRACE(7);
+
   {
     const int r = lane & 3, q = lane >> 2;
-    const int nitems = nblk * U;
-    for (int it0 = warp; it0 < nitems; it0 += 4 * kDecodeWarps) {
-      uint4 wq[4][kDnChunks];
-      unsigned short sc[4][kDnChunks];
-#pragma unroll
-      for (int bI = 0; bI < 4; ++bI) {
-        const int it = it0 + bI * kDecodeWarps;
-        if (it < nitems) {
-          const int blk = it / U, u = it - blk * U;
-          const uint8_t* base = p.dn + ((size_t)hd.uniq_e[u] * kDnUnits + b0 + blk) * kDnUnitBytes;
-#pragma unroll
-          for (int j = 0; j < kDnChunks; ++j) {
-            wq[bI][j] = ldg_stream(base + j * 512 + 16 * lane);
-            sc[bI][j] = ldg_stream16(base + kDnScaleOff + j * 64 + 2 * lane);
-          }
-        }
-      }
-#pragma unroll
-      for (int bI = 0; bI < 4; ++bI) {
-        const int it = it0 + bI * kDecodeWarps;
-        if (it < nitems) {
-          const int blk = it / U, u = it - blk * U;
+    const bool run = !aborted(hd);
+    for (int s = 0; s < nseq; ++s) {
+      if (s > 0) issue4(s);
+      if (!mbar_wait(barA, pha, p.wait_limit_ns, p.err)) { hd.abort = 1; break; }
+      pha ^= 1;
+      if (!run) continue;
+      if (s < nmine_r) {
+        const int it0 = (warp + s * kWarps) * kDnBatch, n = min(kDnBatch, nitems - it0);
+#pragma unroll 1
+        for (int bI = 0; bI < n; ++bI) {
+          const int it = it0 + bI, blk = it / U, u = it - blk * U;
+          const unsigned char* base = bufB + bI * kDnUnitBytes;
           const int cnt = hd.uniq_cnt[u];
-          float acc[kMaxDecodeT];
+          int ho[T], co[T];
 #pragma unroll
-          for (int tt = 0; tt < kMaxDecodeT; ++tt) acc[tt] = 0.f;
-          const float* hb[kMaxDecodeT];
-          const float* cb[kMaxDecodeT];
-#pragma unroll
-          for (int tt = 0; tt < kMaxDecodeT; ++tt) {
+          for (int tt = 0; tt < T; ++tt) {
             const int pr = (tt < cnt) ? hd.uniq_pair[u][tt] : 0;
-            hb[tt] = hp + (size_t)pr * kHpStride + 100 * q;
-            cb[tt] = chp + pr * kHGroups + q * kDnChunks;
+            ho[tt] = pr * kHpStride + 100 * q;
+            co[tt] = pr * kHGroups + q * kDnChunks;
           }
+          float acc[T];
+#pragma unroll
+          for (int tt = 0; tt < T; ++tt) acc[tt] = 0.f;
 #pragma unroll
           for (int j = 0; j < kDnChunks; ++j) {
-            float part[kMaxDecodeT];
+            const uint4 w = lds128(base + j * 512 + 16 * lane);
+            const float sj = bf16_to_f32(
+                *reinterpret_cast<const unsigned short*>(base + kDnScaleOff + j * 64 + 2 * lane));
+            float pa[T], pb[T], pc[T], pd[T];
 #pragma unroll
-            for (int tt = 0; tt < kMaxDecodeT; ++tt) part[tt] = (tt < cnt) ? cb[tt][j] : 0.f;
-            const uint32_t wj[4] = {wq[bI][j].x, wq[bI][j].y, wq[bI][j].z, wq[bI][j].w};
+            for (int tt = 0; tt < T; ++tt) {
+              pa[tt] = (tt < cnt) ? chp[co[tt] + j] : 0.f;
+              pb[tt] = pc[tt] = pd[tt] = 0.f;
+            }
+            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               float f[8];
-              dequant8(wj[i], f);
+              dequant8(wv[i], f);
 #pragma unroll
-              for (int tt = 0; tt < kMaxDecodeT; ++tt) {
+              for (int tt = 0; tt < T; ++tt) {
                 if (tt < cnt) {
-                  const float* hq = hb[tt] + 32 * j + 8 * i;
-                  part[tt] = dot8_f(f, *reinterpret_cast<const float4*>(hq),
-                                    *reinterpret_cast<const float4*>(hq + 4), part[tt]);
+                  const float* hq = hp + ho[tt] + 32 * j + 8 * i;
+                  if (i & 1) dot8_f_2(f, ldsf4(hq), ldsf4(hq + 4), pc[tt], pd[tt]);
+                  else dot8_f_2(f, ldsf4(hq), ldsf4(hq + 4), pa[tt], pb[tt]);
                 }
               }
             }
-            const float sj = bf16_to_f32(sc[bI][j]);
 #pragma unroll
-            for (int tt = 0; tt < kMaxDecodeT; ++tt) acc[tt] = fmaf(sj, part[tt], acc[tt]);
+            for (int tt = 0; tt < T; ++tt) acc[tt] = fmaf(sj, (pa[tt] + pb[tt]) + (pc[tt] + pd[tt]), acc[tt]);
           }
 #pragma unroll
-          for (int tt = 0; tt < kMaxDecodeT; ++tt) {
+          for (int tt = 0; tt < T; ++tt) {
             if (tt < cnt) {
               float v = acc[tt];
               v += __shfl_xor_sync(0xffffffffu, v, 4);
@@ -386,87 +623,123 @@ moe_decode_kernel(const DecodeParams p) {
               v += __shfl_xor_sync(0xffffffffu, v, 16);
               if (q == 0) {
                 const int pr = hd.uniq_pair[u][tt];
-                const float wgt = hd.topw[pr / K][pr % K];
-                part[((size_t)blk * (kMaxPairs + kMaxDecodeT) + pr) * 4 + r] = kCodeScale * v * wgt;
+                part[((size_t)blk * (PL::P + T) + pr) * 4 + r] = kCodeScale * v * hd.topw[pr / K][pr % K];
               }
             }
           }
         }
-      }
-    }
-  }
-  // shared items: one 4-row block of the shared down projection, all tokens
-  {
-    const int r = lane & 3, q = lane >> 2;
-    for (int blk = kDecodeWarps - 1 - warp; blk < nblk; blk += kDecodeWarps) {
-      const int n = 4 * (b0 + blk) + r;
-      const __nv_bfloat16* wd = p.sh_down + (size_t)n * kI;
-      uint4 w[kI / 64];
+      } else {
+        const int blk = sh_first + (s - nmine_r) * kWarps;
+        float acc[T];
+        {
+          float a0[T], a1[T], a2[T], a3[T];
 #pragma unroll
-      for (int m = 0; m < kI / 64; ++m) w[m] = ldg_stream(wd + 8 * (q + 8 * m));
-      float acc[kMaxDecodeT];
+          for (int t = 0; t < T; ++t) a0[t] = a1[t] = a2[t] = a3[t] = 0.f;
+#pragma unroll 2
+          for (int m = 0; m < kI / 64; m += 2) {
+            const int c0 = q + 8 * m, c1 = c0 + 8;
+            const uint4 w0 = lds128(bufB + r * (kI * 2) + 16 * c0);
+            const uint4 w1 = lds128(bufB + r * (kI * 2) + 16 * c1);
 #pragma unroll
-      for (int t = 0; t < kMaxDecodeT; ++t) acc[t] = 0.f;
-#pragma unroll
-      for (int m = 0; m < kI / 64; ++m) {
-        const int c = q + 8 * m;
-#pragma unroll
-        for (int t = 0; t < kMaxDecodeT; ++t) {
-          if (t < T) {
-            const float* ht = hs + (size_t)t * kHsTok + 4 * c;
-            acc[t] = dot8_bf16(w[m], *reinterpret_cast<const float4*>(ht),
-                               *reinterpret_cast<const float4*>(ht + kHsPlane), acc[t]);
+            for (int t = 0; t < T; ++t) {
+              const float* ht = hsm + (size_t)t * kHsTok;
+              dot8_bf16_2(w0, ldsf4(ht + 4 * c0), ldsf4(ht + kHsPlane + 4 * c0), a0[t], a1[t]);
+              dot8_bf16_2(w1, ldsf4(ht + 4 * c1), ldsf4(ht + kHsPlane + 4 * c1), a2[t], a3[t]);
+            }
           }
-        }
-      }
 #pragma unroll
-      for (int t = 0; t < kMaxDecodeT; ++t) {
-        if (t < T) {
+          for (int t = 0; t < T; ++t) acc[t] = (a0[t] + a1[t]) + (a2[t] + a3[t]);
+        }
+#pragma unroll
+        for (int t = 0; t < T; ++t) {
           float v = acc[t];
           v += __shfl_xor_sync(0xffffffffu, v, 4);
           v += __shfl_xor_sync(0xffffffffu, v, 8);
           v += __shfl_xor_sync(0xffffffffu, v, 16);
-          if (q == 0) part[((size_t)blk * (kMaxPairs + kMaxDecodeT) + kMaxPairs + t) * 4 + r] = v;
+          if (q == 0) part[((size_t)blk * (PL::P + T) + PL::P + t) * 4 + r] = v;
         }
       }
+      __syncwarp();
     }
   }
   __syncthreads();
-  // fixed-order sum: routed slots 0..k-1, then the shared expert
-  for (int v = tid; v < nblk * T * 4; v += kDecodeThreads) {
-    const int blk = v / (T * 4), rem = v - blk * T * 4, t = rem >> 2, r = rem & 3;
-    const float* pb = part + (size_t)blk * (kMaxPairs + kMaxDecodeT) * 4;
-    float s = 0.f;
-    for (int sl = 0; sl < K; ++sl) s += pb[(t * K + sl) * 4 + r];
-    s += pb[(kMaxPairs + t) * 4 + r];
-    p.out[(size_t)t * kH + 4 * (b0 + blk) + r] = __float2bfloat16_rn(s);
+  LING_TRACE(8);
+  if (!aborted(hd)) {
+    // fixed-order sum: routed slots 0..k-1, then the shared expert
+    for (int v = tid; v < nblk * T * 4; v += kDecodeThreads) {
+      const int blk = v / (T * 4), rem = v - blk * T * 4, t = rem >> 2, r = rem & 3;
+      const float* pb = part + (size_t)blk * (PL::P + T) * 4;
+      float s = 0.f;
+      for (int sl = 0; sl < K; ++sl) s += pb[(t * K + sl) * 4 + r];
+      s += pb[(PL::P + t) * 4 + r];
+      p.out[(size_t)t * kH + 4 * (b0 + blk) + r] = __float2bfloat16_rn(s);
+    }
   }
+  // every CTA (aborted or not) counts itself out; the last one resets the
+  // counters for the next launch on the stream
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    const unsigned prev = atomicAdd(p.sync + 3, 1u);
+    if (prev == (unsigned)ncta - 1u) {
+      atomicExch(p.sync + 0, 0u);
+      atomicExch(p.sync + 1, 0u);
+      atomicExch(p.sync + 2, 0u);
+      atomicExch(p.sync + 3, 0u);
+    }
+  }
+  LING_TRACE(9);
 }
 
-cudaError_t launch_decode(const DecodeParams& p, int nctas, cudaStream_t stream) {
-  static_assert(kDecodeSmemBytes <= 227 * 1024, "decode smem over budget");
+#ifdef LING_MOE_TRACE
+extern "C" int ling_moe_trace_read(unsigned long long* host, int nctas) {
+  return (int)cudaMemcpyFromSymbol(host, g_trace, (size_t)nctas * 16 * sizeof(unsigned long long));
+}
+#endif
+
+template <int T>
+static cudaError_t launch_t(const DecodeParams& p, int nctas, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nctas);
   cfg.blockDim = dim3(kDecodeThreads);
-  cfg.dynamicSmemBytes = kDecodeSmemBytes;
+  cfg.dynamicSmemBytes = Plan<T>::bytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, moe_decode_kernel, p);
+  return cudaLaunchKernelEx(&cfg, moe_decode_kernel<T>, p);
+}
+
+cudaError_t launch_decode(const DecodeParams& p, int nctas, cudaStream_t stream) {
+  switch (p.T) {
+    case 1: return launch_t<1>(p, nctas, stream);
+    case 2: return launch_t<2>(p, nctas, stream);
+    case 3: return launch_t<3>(p, nctas, stream);
+    case 4: return launch_t<4>(p, nctas, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int T>
+static cudaError_t setup_t() {
+  return cudaFuncSetAttribute(moe_decode_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)Plan<T>::bytes);
 }
 
 cudaError_t setup_decode() {
-  return cudaFuncSetAttribute(moe_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)kDecodeSmemBytes);
+  cudaError_t e;
+  if ((e = setup_t<1>()) != cudaSuccess) return e;
+  if ((e = setup_t<2>()) != cudaSuccess) return e;
+  if ((e = setup_t<3>()) != cudaSuccess) return e;
+  return setup_t<4>();
 }
 
 int decode_max_ctas_per_sm() {
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, moe_decode_kernel, kDecodeThreads,
-                                                    kDecodeSmemBytes) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, moe_decode_kernel<4>, kDecodeThreads,
+                                                    Plan<4>::bytes) != cudaSuccess)
     return 0;
   return n;
 }

@@ -12,6 +12,11 @@ constexpr int kMaxDecodeT = 4;     // tokens per call handled by the decode kern
 constexpr int kDecodeWarps = 12;
 constexpr int kDecodeThreads = kDecodeWarps * 32;
 
+// Values exchanged between CTAs inside one launch are published through
+// arrival counters: a producer stores its values, fences, and adds 1 to the
+// counter of its kind; a consumer polls the counter (bounded) until all
+// producers of the launch have arrived, then reads the values once.  The last
+// CTA to finish resets the counters for the next launch.
 struct DecodeParams {
   const __nv_bfloat16* x;        // [T, H]
   __nv_bfloat16* out;            // [T, H]
@@ -26,17 +31,15 @@ struct DecodeParams {
   float* logits;                 // workspace [T, E]
   float* h_s;                    // workspace [T, I]
   float* h_pair;                 // workspace [T*k, I]
-  int32_t* topk_idx_ws;          // workspace [T, k]
-  float* topk_w_ws;              // workspace [T, k]
   int32_t* topk_idx_out;         // optional caller output [T, k]
   float* topk_w_out;             // optional caller output [T, k]
-  unsigned long long* bar;       // 3 monotonically increasing barrier counters
+  unsigned int* sync;            // [0] router rows, [1] shared rows, [2] routed units, [3] CTAs done
   unsigned int* err;             // sticky device error word
-  int skip_arrive_cta;           // test hook: this CTA never arrives (-1: none)
+  int skip_arrive_cta;           // test hook: this CTA withholds its router rows (-1: none)
   unsigned long long wait_limit_ns;
 };
 
-size_t decode_smem_bytes();
+size_t decode_smem_bytes(int T);
 cudaError_t setup_decode();
 int decode_max_ctas_per_sm();
 cudaError_t launch_decode(const DecodeParams& p, int nctas, cudaStream_t stream);
