@@ -4,8 +4,8 @@ Argument marshalling only: every step of the layer runs in the library's
 CUDA kernels.  The functions below carry the C ABI's names and arguments
 (pointers are integers, streams are raw cudaStream_t values); `MoELayer`
 wraps them for torch tensors.  The library must have been built
-(`python -m weight_only_int4_fp32_b200.build`); importing this package
-without it raises instead of falling back to anything else.
+(`python -m weight_only_int4_fp32_b200.build`); the first call into it
+raises if it is missing -- there is nothing else to fall back to.
 """
 from __future__ import annotations
 
@@ -15,7 +15,7 @@ import os
 __all__ = [
     "LING_MOE_OK", "LING_MOE_ERR_INVALID_ARG", "LING_MOE_ERR_CUDA", "LING_MOE_ERR_OOM",
     "LING_MOE_ERR_UNSUPPORTED", "LING_MOE_ERR_DEVICE_TIMEOUT", "LingMoEError",
-    "ling_moe_config_t", "ling_moe_weights_t", "library_path", "lib",
+    "ling_moe_config_t", "ling_moe_weights_t", "library_path", "load_library",
     "ling_moe_create", "ling_moe_forward", "ling_moe_forward_ex", "ling_moe_forward_host",
     "ling_moe_status", "ling_moe_describe", "ling_moe_launch_count", "ling_moe_last_error",
     "ling_moe_destroy", "ling_moe_test_set_wait", "MoELayer", "EXPORTED",
@@ -59,6 +59,17 @@ class ling_moe_weights_t(ctypes.Structure):
         "sh_gate", "sh_up", "sh_down")]
 
 
+_LIB = None
+
+
+def load_library():
+    """Load libling_moe.so once (raises ImportError if it is missing or stale)."""
+    global _LIB
+    if _LIB is None:
+        _LIB = _load()
+    return _LIB
+
+
 def _load():
     path = library_path()
     if not os.path.exists(path):
@@ -81,13 +92,22 @@ def _load():
         "ling_moe_test_set_wait": (ci, [vp, ci, ctypes.c_uint64]),
     }
     for name, (res, args) in sig.items():
-        f = getattr(L, name)
+        try:
+            f = getattr(L, name)
+        except AttributeError as e:
+            raise ImportError(f"{path} lacks {name}: rebuild it "
+                              "(`python -m weight_only_int4_fp32_b200.build`)") from e
         f.restype = res
         f.argtypes = args
     return L
 
 
-lib = _load()
+class _LazyLib:
+    def __getattr__(self, name):
+        return getattr(load_library(), name)
+
+
+lib = _LazyLib()
 
 
 def ling_moe_last_error() -> str:
