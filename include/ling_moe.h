@@ -145,6 +145,35 @@ void ling_moe_destroy(ling_moe_t *h);
  * runs normally. */
 int ling_moe_test_set_wait(ling_moe_t *h, int skip_arrive_cta, uint64_t wait_limit_ns);
 
+/* ---- routing that allocates nothing ----
+ * The pages have no counterpart of this call.  It is for callers that cannot
+ * allocate device memory at the point where they route tokens: code running
+ * under a framework that owns all device memory through its own pool, or a
+ * latency-critical path that must not call cudaMalloc (which can synchronise
+ * the device).  It needs no handle.
+ *
+ * For T tokens x[T, H] (bf16, H = 2560) it computes the router logits
+ * x . router_w[E, H]^T (+ router_bias[E]) in fp32, the top_k experts (ties
+ * to the lower index) and their renormalised softmax weights, into
+ * topk_idx int32 [T, top_k] and topk_w fp32 [T, top_k]: the same values that
+ * ling_moe_forward_ex reports for the same router.  All pointers are DEVICE
+ * pointers; x and router_w 16-byte aligned, the others 4-byte aligned;
+ * router_bias may be NULL.
+ * Limits: 0 <= T <= 4, 1 <= num_experts <= 512, 1 <= top_k <= min(8, num_experts);
+ * anything else returns LING_MOE_ERR_INVALID_ARG (message in
+ * ling_moe_last_error) before anything is launched.
+ * Scratch: a static array of 8,448 bytes in device memory (logits of 4 x 512
+ * experts plus two counters) that every GPU which loads the library holds
+ * until the process exits.  Nothing is allocated, by this call or on its
+ * behalf.  The first call on a device looks up that array's device address
+ * (cudaGetSymbolAddress), so make the first call on each device before any
+ * stream capture on it.  Every call shares the array: the counters start at
+ * zero and each call leaves them at zero, but calls that overlap on the GPU
+ * (two streams, or two host threads) race and must not be issued.
+ * A device-side wait that runs out (2 s) writes -1 indices. */
+int ling_moe_route_noalloc(const void *x, int T, const void *router_w, const float *router_bias,
+                           int num_experts, int top_k, int32_t *topk_idx, float *topk_w, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,61 @@
+"""The routing entry point that allocates nothing, against the normal path.
+
+ling_moe_route_noalloc keeps its scratch in a static device array instead of
+allocating it, for callers that cannot allocate device memory where they
+route tokens.  Its routing must equal what ling_moe_forward_ex reports for the
+same router weights and tokens: the same fp32 accumulation order gives the
+same logits, so indices and weights match exactly (well inside the 1e-5
+weight tolerance of the other tests).  Two calls in a row on each token count
+check that every call leaves the shared scratch ready for the next.
+This file is collected last on purpose, and also runs alone in a fresh
+process (the first call looks up the scratch address itself).
+"""
+import pytest
+import torch
+
+import workloads
+import weight_only_int4_fp32_b200 as lm
+
+pytestmark = pytest.mark.gpu
+
+
+def _route_noalloc(x, router_w, bias, E, k):
+    T = x.shape[0]
+    idx = torch.full((T, k), -7, dtype=torch.int32, device=x.device)
+    w = torch.full((T, k), -1.0, dtype=torch.float32, device=x.device)
+    lm.ling_moe_route_noalloc(x.data_ptr(), T, router_w.data_ptr(), bias.data_ptr() if bias is not None else 0,
+                              E, k, idx.data_ptr(), w.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    return idx, w
+
+
+@pytest.mark.parametrize("E,with_bias", [(512, False), (512, True), (32, False)])
+def test_route_noalloc_matches_forward_ex(E, with_bias):
+    k = 8
+    lw = workloads.layer_weights(E, seed=0, device="cuda")
+    weights = dict(lw.tensors())
+    bias = workloads.zipf_router_bias(E, 1.1).cuda() if with_bias else None
+    weights["router_bias"] = bias
+    layer = lm.MoELayer(weights, top_k=k, max_tokens=4)
+    try:
+        for T in (1, 4, 3):
+            for call in range(2):  # two calls in a row share the static scratch
+                x = workloads.tokens(T, seed=300 + 10 * T + call, device="cuda")
+                _, idx_ref, w_ref = layer.forward(x, return_routing=True)
+                idx, w = _route_noalloc(x, lw.router_w, bias, E, k)
+                torch.cuda.synchronize()
+                assert torch.equal(idx, idx_ref), (E, T, call, idx, idx_ref)
+                assert torch.allclose(w, w_ref, rtol=0, atol=1e-5), (E, T, call)
+    finally:
+        layer.close()
+
+
+def test_route_noalloc_rejects_sizes_beyond_its_scratch():
+    x = torch.zeros((5, 2560), dtype=torch.bfloat16, device="cuda")
+    wr = torch.zeros((16, 2560), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((5, 8), dtype=torch.int32, device="cuda")
+    w = torch.empty((5, 8), dtype=torch.float32, device="cuda")
+    for T, E, k in ((5, 16, 8), (1, 513, 8), (1, 16, 9), (1, 4, 8)):
+        with pytest.raises(lm.LingMoEError) as e:
+            lm.ling_moe_route_noalloc(x.data_ptr(), T, wr.data_ptr(), 0, E, k, idx.data_ptr(), w.data_ptr(), 0)
+        assert e.value.code == lm.LING_MOE_ERR_INVALID_ARG
+        assert "route_noalloc" in lm.ling_moe_last_error()

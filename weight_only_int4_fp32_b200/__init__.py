@@ -18,7 +18,7 @@ __all__ = [
     "ling_moe_config_t", "ling_moe_weights_t", "library_path", "load_library",
     "ling_moe_create", "ling_moe_forward", "ling_moe_forward_ex", "ling_moe_forward_host",
     "ling_moe_status", "ling_moe_describe", "ling_moe_launch_count", "ling_moe_last_error",
-    "ling_moe_destroy", "ling_moe_test_set_wait", "MoELayer", "EXPORTED",
+    "ling_moe_destroy", "ling_moe_test_set_wait", "ling_moe_route_noalloc", "MoELayer", "EXPORTED",
 ]
 
 LING_MOE_OK = 0
@@ -32,7 +32,7 @@ LING_MOE_ERR_DEVICE_TIMEOUT = -5
 EXPORTED = (
     "ling_moe_create", "ling_moe_forward", "ling_moe_forward_ex", "ling_moe_forward_host",
     "ling_moe_status", "ling_moe_describe", "ling_moe_launch_count", "ling_moe_last_error",
-    "ling_moe_destroy", "ling_moe_test_set_wait",
+    "ling_moe_destroy", "ling_moe_test_set_wait", "ling_moe_route_noalloc",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -90,6 +90,7 @@ def _load():
         "ling_moe_last_error": (ctypes.c_char_p, []),
         "ling_moe_destroy": (None, [vp]),
         "ling_moe_test_set_wait": (ci, [vp, ci, ctypes.c_uint64]),
+        "ling_moe_route_noalloc": (ci, [vp, ci, vp, vp, ci, ci, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         try:
@@ -158,6 +159,13 @@ def ling_moe_destroy(h: int) -> None:
 
 def ling_moe_test_set_wait(h: int, skip_arrive_cta: int, wait_limit_ns: int) -> int:
     return _check(lib.ling_moe_test_set_wait(h, skip_arrive_cta, wait_limit_ns))
+
+
+def ling_moe_route_noalloc(x: int, T: int, router_w: int, router_bias, num_experts: int, top_k: int,
+                           topk_idx: int, topk_w: int, stream: int = 0) -> int:
+    """Routing with the library's static scratch; allocates nothing (see ling_moe.h)."""
+    return _check(lib.ling_moe_route_noalloc(x, T, router_w, router_bias or None, num_experts, top_k,
+                                             topk_idx, topk_w, stream))
 
 
 class MoELayer:

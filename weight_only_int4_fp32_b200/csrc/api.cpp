@@ -48,6 +48,10 @@ constexpr unsigned long long kDefaultWaitNs = 2000000000ull;  // 2 s
 
 }  // namespace
 
+namespace lingmoe {
+void set_last_error(const char* msg) { g_last_error = msg; }
+}  // namespace lingmoe
+
 struct ling_moe {
   ling_moe_config_t cfg{};
   int device = 0;

@@ -632,4 +632,10 @@ __device__ __forceinline__ void dot8_bf16_2(uint4 w, float4 x0, float4 x1, float
   b = fmaf(bf16hi(w.w), x1.w, b);
 }
 
+__device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned int* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 }  // namespace lingmoe

@@ -113,11 +113,6 @@ __device__ __forceinline__ bool aborted(const SmemHeader& hd) {
 }
 
 // ---------------------------------------------------------------- arrival counters
-__device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned int* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
 // Publish: the calling thread's earlier stores (and, after a warp or CTA
 // barrier, those of the other threads) become visible before the count.
 __device__ __forceinline__ void arrive(unsigned int* ctr) {
