@@ -199,6 +199,7 @@ int ling_moe_create(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, l
     }
   }
   if (cfg->max_tokens > kMaxDecodeT) {
+    h->gws.err = h->err;
     e = grouped_alloc(&h->gws, E, K, cfg->max_tokens,
                       [h](void** p, size_t n) { return h->alloc(p, n); });
     if (e != cudaSuccess) {
@@ -370,6 +371,25 @@ void ling_moe_destroy(ling_moe_t* h) {
   h->release();
   delete h;
 }
+
+#ifdef LING_MOE_TRACE
+// Trace builds only: copy a grouped-path workspace buffer to the host.
+int ling_moe_debug_ws(ling_moe_t* h, int which, void* dst, size_t bytes) {
+  const void* src = nullptr;
+  switch (which) {
+    case 0: src = h->gws.h16; break;
+    case 1: src = h->gws.y; break;
+    case 2: src = h->gws.perm; break;
+    case 3: src = h->gws.x16; break;
+    case 4: src = h->gws.ntiles; break;
+    case 5: src = h->gws.gu_tiles; break;
+    case 6: src = h->gws.topk_w; break;
+    case 7: src = h->gws.hs; break;
+    default: return LING_MOE_ERR_INVALID_ARG;
+  }
+  return cudaMemcpy(dst, src, bytes, cudaMemcpyDeviceToHost) == cudaSuccess ? 0 : LING_MOE_ERR_CUDA;
+}
+#endif
 
 int ling_moe_test_set_wait(ling_moe_t* h, int skip_arrive_cta, uint64_t wait_limit_ns) {
   if (!h) return fail(LING_MOE_ERR_INVALID_ARG, "handle is NULL");

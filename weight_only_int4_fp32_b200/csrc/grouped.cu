@@ -5,11 +5,11 @@
 //   top-k        per token, ties to the lower index, renormalised softmax
 //   grouping     count per expert, exclusive scan, stable scatter of the
 //                (token, slot) pairs into expert order (pair id ascending)
-//   gate/up      per expert, tiles of up to 16 of its tokens: the expert's
-//                weights are read once per tile and dequantised in registers
-//   down         per expert tile: y[pair] = Wd_e h[pair]
+//   gate/up      per expert, tcgen05 tiles of 128 weight rows x up to 128
+//                of its tokens (grouped_tc.cu)
+//   down         per expert tile: y[position] = w * Wd_e h[position]
 //   shared       SiLU(Wg_s x) * (Wu_s x) for all tokens, then Wd_s h
-//   combine      out[t] = sum_slot w[t,slot] y[t*k+slot] + shared, one bf16
+//   combine      out[t] = sum_slot y[position of (t, slot)] + shared, one bf16
 //                rounding, slots summed in a fixed order
 //
 // Chunked prefill feeds this path (vLLM recipe page "inclusionAI/Ling-3.0-flash",
@@ -18,20 +18,20 @@
 // "Optimalizacio 3": four tokens can activate up to 32 experts).
 #include "common.cuh"
 #include "grouped.h"
+#include "grouped_tc.h"
 
 namespace lingmoe {
 
 constexpr int kTile = 16;                 // tokens per expert tile
 constexpr int kGThreads = 384;
 constexpr int kGWarps = kGThreads / 32;
-constexpr size_t kGuSmem = (size_t)kTile * (kXTok + kXGroups) * sizeof(float) + 64 * sizeof(int);
-constexpr size_t kDnSmem = (size_t)kTile * (kHpStride + kHGroups) * sizeof(float) + 64 * sizeof(int);
 constexpr size_t kOutSmem = (size_t)kTile * kHsTok * sizeof(float);
 constexpr size_t kRouterSmem = (size_t)8 * kXTok * sizeof(float);
 
 const char* grouped_describe() {
-  return "router GEMV tiles + top-k + stable counting sort by expert + per-expert 16-token "
-         "tiles (W4 g32 dequant-in-register, fp32 accumulate) + shared expert + fixed-order combine";
+  return "router GEMV tiles + top-k + stable counting sort by expert + tcgen05 grouped GEMMs "
+         "(M=128 weight rows x N<=128 tokens, int4 dequantised to exact fp16 in shared memory, "
+         "fp32 TMEM accumulators) for routed gate/up and down + shared expert + fixed-order combine";
 }
 
 cudaError_t grouped_alloc(GroupedWorkspace* ws, int E, int k, int max_T, const AllocFn& alloc) {
@@ -45,9 +45,15 @@ cudaError_t grouped_alloc(GroupedWorkspace* ws, int E, int k, int max_T, const A
   if ((e = alloc((void**)&ws->off, (size_t)(E + 1) * sizeof(int32_t))) != cudaSuccess) return e;
   if ((e = alloc((void**)&ws->tile_off, (size_t)(E + 1) * sizeof(int32_t))) != cudaSuccess) return e;
   if ((e = alloc((void**)&ws->perm, P * sizeof(int32_t))) != cudaSuccess) return e;
-  if ((e = alloc((void**)&ws->h_g, P * kI * sizeof(float))) != cudaSuccess) return e;
+  if ((e = alloc((void**)&ws->inv, P * sizeof(int32_t))) != cudaSuccess) return e;
   if ((e = alloc((void**)&ws->y, P * kH * sizeof(float))) != cudaSuccess) return e;
   if ((e = alloc((void**)&ws->hs, (size_t)max_T * kI * sizeof(float))) != cudaSuccess) return e;
+  if ((e = alloc((void**)&ws->x16, (size_t)max_T * kH * sizeof(__half))) != cudaSuccess) return e;
+  if ((e = alloc((void**)&ws->xscale, (size_t)max_T * sizeof(float))) != cudaSuccess) return e;
+  if ((e = alloc((void**)&ws->h16, P * 2 * kI * sizeof(__half))) != cudaSuccess) return e;
+  if ((e = alloc((void**)&ws->gu_tiles, tc_max_tiles_gu((int)P, E) * sizeof(int4))) != cudaSuccess) return e;
+  if ((e = alloc((void**)&ws->dn_tiles, tc_max_tiles_dn((int)P, E) * sizeof(int4))) != cudaSuccess) return e;
+  if ((e = alloc((void**)&ws->ntiles, 4 * sizeof(int32_t))) != cudaSuccess) return e;
   return cudaSuccess;
 }
 
@@ -139,7 +145,7 @@ __global__ void __launch_bounds__(256) grp_topk_kernel(GroupedParams p, const fl
 // ascending pair-id order, so the permutation is deterministic.
 __global__ void __launch_bounds__(256) grp_sort_kernel(const int32_t* ti, int P, int E, int pass,
                                                        int32_t* cnt, const int32_t* off,
-                                                       int32_t* perm) {
+                                                       int32_t* perm, int32_t* inv) {
   const int lane = threadIdx.x & 31;
   const int e = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (e >= E) return;
@@ -148,7 +154,11 @@ __global__ void __launch_bounds__(256) grp_sort_kernel(const int32_t* ti, int P,
     const int pp = base + lane;
     const bool hit = pp < P && ti[pp] == e;
     const unsigned m = __ballot_sync(0xffffffffu, hit);
-    if (pass && hit) perm[pos + __popc(m & ((1u << lane) - 1u))] = pp;
+    if (pass && hit) {
+      const int at = pos + __popc(m & ((1u << lane) - 1u));
+      perm[at] = pp;
+      inv[pp] = at;
+    }
     pos += __popc(m);
   }
   if (!pass && lane == 0) cnt[e] = pos;
@@ -165,175 +175,6 @@ __global__ void grp_scan_kernel(const int32_t* cnt, int E, int32_t* off, int32_t
     }
     off[E] = a;
     tile_off[E] = b;
-  }
-}
-
-// tile -> (expert, first position in perm, number of pairs)
-__device__ __forceinline__ void tile_lookup(const int32_t* tile_off, const int32_t* off, int E, int tile,
-                                            int* e_out, int* pos, int* n) {
-  int lo = 0, hi = E - 1;
-  while (lo < hi) {  // largest e with tile_off[e] <= tile
-    const int mid = (lo + hi + 1) >> 1;
-    if (tile_off[mid] <= tile) lo = mid; else hi = mid - 1;
-  }
-  const int e = lo;
-  const int lt = tile - tile_off[e];
-  *e_out = e;
-  *pos = off[e] + lt * kTile;
-  *n = min(kTile, off[e + 1] - *pos);
-}
-
-// ---------------------------------------------------------------- routed gate/up
-__global__ void __launch_bounds__(kGThreads, 1)
-grp_gateup_kernel(GroupedParams p, GroupedWorkspace ws) {
-  extern __shared__ __align__(16) float sm[];
-  float* xs = sm;
-  float* cx = sm + (size_t)kTile * kXTok;
-  int* s_pair = reinterpret_cast<int*>(cx + kTile * kXGroups);
-  int* s_tok = s_pair + kTile;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int r = lane & 7, q = lane >> 3;
-  const int ntiles = ws.tile_off[p.E];
-  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    int e, pos, n;
-    tile_lookup(ws.tile_off, ws.off, p.E, tile, &e, &pos, &n);
-    __syncthreads();
-    if (threadIdx.x < kTile) {
-      const int m = min((int)threadIdx.x, n - 1);
-      s_pair[threadIdx.x] = ws.perm[pos + m];
-      s_tok[threadIdx.x] = ws.perm[pos + m] / p.k;
-    }
-    __syncthreads();
-    stage_x_rows(p.x, s_tok, n, xs, cx);
-    const float* xq = xs + 324 * q;
-    const float* cq = cx + q * kGuChunks;
-    for (int b = warp; b < kGuUnits; b += kGWarps) {
-      const uint8_t* base = p.gu + ((size_t)e * kGuUnits + b) * kGuUnitBytes;
-      uint4 wq[kGuChunks];
-      uint2 sc[kGuChunks / 4];
-#pragma unroll
-      for (int j = 0; j < kGuChunks; ++j) wq[j] = ldg_stream(base + j * 512 + 16 * lane);
-#pragma unroll
-      for (int j = 0; j < kGuChunks / 4; ++j) sc[j] = ldg_stream64(base + kGuScaleOff + j * 256 + 8 * lane);
-      float acc[kTile];
-#pragma unroll
-      for (int m = 0; m < kTile; ++m) acc[m] = 0.f;
-#pragma unroll
-      for (int j = 0; j < kGuChunks; ++j) {
-        float part[kTile];
-#pragma unroll
-        for (int m = 0; m < kTile; ++m) part[m] = (m < n) ? cq[m * kXGroups + j] : 0.f;
-        const uint32_t wj[4] = {wq[j].x, wq[j].y, wq[j].z, wq[j].w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float f[8];
-          dequant8(wj[i], f);
-#pragma unroll
-          for (int m = 0; m < kTile; ++m) {
-            if (m < n) {
-              const float* xp = xq + m * kXTok + 16 * j + 4 * i;
-              part[m] = dot8_f(f, *reinterpret_cast<const float4*>(xp),
-                               *reinterpret_cast<const float4*>(xp + kXPlane), part[m]);
-            }
-          }
-        }
-        const float s = scale_of(sc[j >> 2], j & 3);
-#pragma unroll
-        for (int m = 0; m < kTile; ++m) acc[m] = fmaf(s, part[m], acc[m]);
-      }
-#pragma unroll
-      for (int m = 0; m < kTile; ++m) {
-        if (m < n) {
-          float v = acc[m];
-          v += __shfl_xor_sync(0xffffffffu, v, 8);
-          v += __shfl_xor_sync(0xffffffffu, v, 16);
-          const float up = __shfl_sync(0xffffffffu, v, (lane & ~7) | ((r + 4) & 7));
-          if (r < 4 && q == (m & 3))
-            ws.h_g[(size_t)s_pair[m] * kI + 4 * b + r] = silu_mul(kCodeScale * v, kCodeScale * up);
-        }
-      }
-    }
-  }
-}
-
-// ---------------------------------------------------------------- routed down
-__global__ void __launch_bounds__(kGThreads, 1)
-grp_down_kernel(GroupedParams p, GroupedWorkspace ws) {
-  extern __shared__ __align__(16) float sm[];
-  float* hp = sm;
-  float* chp = sm + (size_t)kTile * kHpStride;
-  int* s_pair = reinterpret_cast<int*>(chp + kTile * kHGroups);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int r = lane & 3, q = lane >> 2;
-  const int ntiles = ws.tile_off[p.E];
-  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    int e, pos, n;
-    tile_lookup(ws.tile_off, ws.off, p.E, tile, &e, &pos, &n);
-    __syncthreads();
-    if (threadIdx.x < kTile) s_pair[threadIdx.x] = ws.perm[pos + min((int)threadIdx.x, n - 1)];
-    __syncthreads();
-    for (int v = threadIdx.x; v < n * (kI / 4); v += blockDim.x) {
-      const int m = v / (kI / 4), c4 = v - m * (kI / 4);
-      const float4 h = reinterpret_cast<const float4*>(ws.h_g + (size_t)s_pair[m] * kI)[c4];
-      const int e0 = 4 * c4;
-      *reinterpret_cast<float4*>(hp + (size_t)m * kHpStride + e0 + 4 * (e0 / 96)) = h;
-    }
-    __syncthreads();
-    for (int v = threadIdx.x; v < n * kHGroups; v += blockDim.x) {
-      const int m = v / kHGroups, G = v - m * kHGroups;
-      const float* src = hp + (size_t)m * kHpStride + 32 * G + 4 * (G / 3);
-      float s = 0.f;
-      for (int i = 0; i < 32; ++i) s += src[i];
-      chp[m * kHGroups + G] = kBiasCoef * s;
-    }
-    __syncthreads();
-    const float* hq = hp + 100 * q;
-    const float* cq = chp + q * kDnChunks;
-    for (int vb = warp; vb < kDnUnits; vb += kGWarps) {
-      const uint8_t* base = p.dn + ((size_t)e * kDnUnits + vb) * kDnUnitBytes;
-      uint4 wq[kDnChunks];
-      float sc[kDnChunks];
-#pragma unroll
-      for (int j = 0; j < kDnChunks; ++j) {
-        wq[j] = ldg_stream(base + j * 512 + 16 * lane);
-        sc[j] = bf16_to_f32(ldg_stream16(base + kDnScaleOff + j * 64 + 2 * lane));
-      }
-      float acc[kTile];
-#pragma unroll
-      for (int m = 0; m < kTile; ++m) acc[m] = 0.f;
-#pragma unroll
-      for (int j = 0; j < kDnChunks; ++j) {
-        float part[kTile];
-#pragma unroll
-        for (int m = 0; m < kTile; ++m) part[m] = (m < n) ? cq[m * kHGroups + j] : 0.f;
-        const uint32_t wj[4] = {wq[j].x, wq[j].y, wq[j].z, wq[j].w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float f[8];
-          dequant8(wj[i], f);
-#pragma unroll
-          for (int m = 0; m < kTile; ++m) {
-            if (m < n) {
-              const float* h = hq + m * kHpStride + 32 * j + 8 * i;
-              part[m] = dot8_f(f, *reinterpret_cast<const float4*>(h),
-                               *reinterpret_cast<const float4*>(h + 4), part[m]);
-            }
-          }
-        }
-#pragma unroll
-        for (int m = 0; m < kTile; ++m) acc[m] = fmaf(sc[j], part[m], acc[m]);
-      }
-#pragma unroll
-      for (int m = 0; m < kTile; ++m) {
-        if (m < n) {
-          float v = acc[m];
-          v += __shfl_xor_sync(0xffffffffu, v, 4);
-          v += __shfl_xor_sync(0xffffffffu, v, 8);
-          v += __shfl_xor_sync(0xffffffffu, v, 16);
-          if (q == (m & 7)) ws.y[(size_t)s_pair[m] * kH + 4 * vb + r] = kCodeScale * v;
-        }
-      }
-    }
   }
 }
 
@@ -426,10 +267,7 @@ grp_out_kernel(GroupedParams p, GroupedWorkspace ws) {
         if (q == (t & 7)) {
           const int tok = t0 + t;
           float s = 0.f;
-          for (int sl = 0; sl < p.k; ++sl) {
-            const int pr = tok * p.k + sl;
-            s += ws.topk_w[pr] * ws.y[(size_t)pr * kH + nrow];
-          }
+          for (int sl = 0; sl < p.k; ++sl) s += ws.y[(size_t)ws.inv[tok * p.k + sl] * kH + nrow];
           s += v;
           p.out[(size_t)tok * kH + nrow] = __float2bfloat16_rn(s);
         }
@@ -442,10 +280,7 @@ cudaError_t setup_grouped() {
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(grp_router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kRouterSmem)) != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(grp_gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)kGuSmem)) != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(grp_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)kDnSmem)) != cudaSuccess) return e;
+  if ((e = setup_grouped_tc()) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(grp_shared_gu_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)(kTile * kXTok * sizeof(float)))) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(grp_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -456,21 +291,39 @@ cudaError_t setup_grouped() {
 cudaError_t launch_grouped(const GroupedParams& p, const GroupedWorkspace& ws, cudaStream_t s,
                            int* nlaunch) {
   int nl = 0;
-  cudaError_t e;
+  cudaError_t e = cudaSuccess;
   const int P = p.T * p.k;
   grp_router_kernel<<<(p.T + 7) / 8, 256, kRouterSmem, s>>>(p, ws.logits);
   ++nl;
   grp_topk_kernel<<<(p.T + 7) / 8, 256, 0, s>>>(p, ws.logits, ws.topk_idx, ws.topk_w);
   ++nl;
-  grp_sort_kernel<<<(p.E + 7) / 8, 256, 0, s>>>(ws.topk_idx, P, p.E, 0, ws.cnt, ws.off, ws.perm);
+  grp_sort_kernel<<<(p.E + 7) / 8, 256, 0, s>>>(ws.topk_idx, P, p.E, 0, ws.cnt, ws.off, ws.perm, ws.inv);
   ++nl;
   grp_scan_kernel<<<1, 32, 0, s>>>(ws.cnt, p.E, ws.off, ws.tile_off);
   ++nl;
-  grp_sort_kernel<<<(p.E + 7) / 8, 256, 0, s>>>(ws.topk_idx, P, p.E, 1, ws.cnt, ws.off, ws.perm);
+  grp_sort_kernel<<<(p.E + 7) / 8, 256, 0, s>>>(ws.topk_idx, P, p.E, 1, ws.cnt, ws.off, ws.perm, ws.inv);
   ++nl;
-  grp_gateup_kernel<<<p.num_sms, kGThreads, kGuSmem, s>>>(p, ws);
+  if ((e = launch_tc_tiles(ws.cnt, ws.off, p.E, ws.gu_tiles, ws.dn_tiles, ws.ntiles, s)) != cudaSuccess) return e;
   ++nl;
-  grp_down_kernel<<<p.num_sms, kGThreads, kDnSmem, s>>>(p, ws);
+  if ((e = launch_x16(p.x, p.T, ws.x16, ws.xscale, s)) != cudaSuccess) return e;
+  ++nl;
+  TcParams tp{};
+  tp.gu = p.gu;
+  tp.dn = p.dn;
+  tp.x16 = ws.x16;
+  tp.xscale = ws.xscale;
+  tp.h16 = ws.h16;
+  tp.y = ws.y;
+  tp.perm = ws.perm;
+  tp.topk_w = ws.topk_w;
+  tp.k = p.k;
+  tp.gu_tiles = ws.gu_tiles;
+  tp.dn_tiles = ws.dn_tiles;
+  tp.ntiles = ws.ntiles;
+  tp.err = ws.err;
+  if ((e = launch_tc_gemm(0, tp, p.num_sms, s)) != cudaSuccess) return e;
+  ++nl;
+  if ((e = launch_tc_gemm(1, tp, p.num_sms, s)) != cudaSuccess) return e;
   ++nl;
   grp_shared_gu_kernel<<<(p.T + kTile - 1) / kTile, kGThreads, kTile * kXTok * sizeof(float), s>>>(p, ws.hs);
   ++nl;

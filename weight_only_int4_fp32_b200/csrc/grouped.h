@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <functional>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 namespace lingmoe {
@@ -34,9 +35,16 @@ struct GroupedWorkspace {
   int32_t* off = nullptr;       // [E+1] start of each expert's run in perm
   int32_t* tile_off = nullptr;  // [E+1] first token tile of each expert
   int32_t* perm = nullptr;      // [T*k] pair ids (t*k+slot) sorted by (expert, pair id)
-  float* h_g = nullptr;         // [T*k, I] routed SiLU(gate)*up per pair
-  float* y = nullptr;           // [T*k, H] routed expert output per pair (unweighted)
+  int32_t* inv = nullptr;       // [T*k] pair id -> position in perm
+  float* y = nullptr;           // [T*k, H] routed expert output per position, weighted
   float* hs = nullptr;          // [T, I]   shared SiLU(gate)*up
+  __half* x16 = nullptr;        // [T, H]   x in fp16 (tensor-core B operand)
+  float* xscale = nullptr;      // [T]
+  __half* h16 = nullptr;        // [T*k, 2, I] SiLU(gate)*up per position, fp16 hi + lo
+  int4* gu_tiles = nullptr;     // tcgen05 tile lists
+  int4* dn_tiles = nullptr;
+  int32_t* ntiles = nullptr;    // [2]
+  unsigned int* err = nullptr;  // the handle's sticky device error word
 };
 
 using AllocFn = std::function<cudaError_t(void**, size_t)>;
