@@ -291,7 +291,7 @@ def run_ours(args):
         xh = [inputs[nwarm + i].cpu().pin_memory() for i in range(nsteps)]
         oh = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
         for i in range(min(nwarm, 5)):
-            layers[0].forward_host(xh[i], oh)
+            layers[0].forward_host(xh[i % nsteps], oh)
         torch.cuda.synchronize()
         if ws > 1:
             dist.barrier()

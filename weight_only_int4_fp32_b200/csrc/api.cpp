@@ -222,6 +222,8 @@ int ling_moe_create(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, l
   if (e == cudaSuccess) e = cudaMemsetAsync(h->err, 0, 4 * sizeof(unsigned int), s);
   if (e == cudaSuccess)
     e = launch_repack(w->gate_q, w->up_q, w->gate_s, w->up_s, w->down_q, w->down_s, h->gu, h->dn, E, s);
+  if (e == cudaSuccess && cfg->max_tokens > kMaxDecodeT)
+    e = grouped_prepare(&h->gws, E, h->sh_gate, h->sh_up, h->sh_down, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (s) cudaStreamDestroy(s);
   if (e != cudaSuccess) {
@@ -299,9 +301,6 @@ static int forward_impl(ling_moe_t* h, const void* x, int T, void* out, int32_t*
   gp.router_bias = h->router_bias;
   gp.gu = h->gu;
   gp.dn = h->dn;
-  gp.sh_gate = h->sh_gate;
-  gp.sh_up = h->sh_up;
-  gp.sh_down = h->sh_down;
   gp.topk_idx_out = topk_idx;
   gp.topk_w_out = topk_w;
   gp.num_sms = h->num_sms;
@@ -356,6 +355,10 @@ int ling_moe_status(ling_moe_t* h, void* stream_v) {
     // error word (and the counters, in case a launch never ran to its end).
     cudaMemset(h->err, 0, 4 * sizeof(unsigned int));
     cudaMemset(h->sync, 0, 4 * sizeof(unsigned int));
+    if (h->gws.cnt) {  // grouped-path counters that a cut-short call may have left behind
+      cudaMemset(h->gws.cnt, 0, (size_t)h->cfg.num_experts * sizeof(int32_t));
+      cudaMemset(h->gws.fill, 0, (size_t)h->cfg.num_experts * sizeof(int32_t));
+    }
     cudaDeviceSynchronize();
     return fail(LING_MOE_ERR_DEVICE_TIMEOUT, "a bounded device-side wait gave up (error word %u)", err);
   }
@@ -380,11 +383,11 @@ int ling_moe_debug_ws(ling_moe_t* h, int which, void* dst, size_t bytes) {
     case 0: src = h->gws.h16; break;
     case 1: src = h->gws.y; break;
     case 2: src = h->gws.perm; break;
-    case 3: src = h->gws.x16; break;
+    case 3: src = h->gws.xg; break;
     case 4: src = h->gws.ntiles; break;
     case 5: src = h->gws.gu_tiles; break;
     case 6: src = h->gws.topk_w; break;
-    case 7: src = h->gws.hs; break;
+    case 7: src = h->gws.inv; break;
     default: return LING_MOE_ERR_INVALID_ARG;
   }
   return cudaMemcpy(dst, src, bytes, cudaMemcpyDeviceToHost) == cudaSuccess ? 0 : LING_MOE_ERR_CUDA;

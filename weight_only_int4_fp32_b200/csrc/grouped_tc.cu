@@ -1,18 +1,27 @@
 // Tensor-core grouped GEMMs of the token-grouped path (tcgen05, sm_100a).
 //
-// For every routed expert e with m_e tokens (after the stable sort by expert):
+// For every routed expert e with m_e positions (token-expert pairs after the
+// sort by expert), and for the shared expert over all T tokens:
 //   gate/up:  H_e[m_e, 768]  = SiLU(X_e Wg_e^T) * (X_e Wu_e^T)     K = 2560
 //   down:     Y_e[m_e, 2560] = w * (H_e Wd_e^T)                    K = 768
-// as tiles of M = 128 weight rows x N <= 128 tokens.  The weights are the
-// A operand: producer warps dequantise the repacked int4 codes into exact
-// fp16 values q*s (q has at most 4 significant bits and s is a bf16, so the
-// product fits fp16's 11 bits) and write them into 128-byte-swizzled K-major
-// shared-memory tiles.  The activations are the B operand, stored in fp16 in
-// the same per-8-element K order as the dequantised codes (the order a LOP3
-// extracts nibbles in), so no permutation is needed inside the main loop.
-// One elected thread issues tcgen05.mma into a TMEM accumulator; tcgen05.commit
-// releases each pipeline stage and finally signals the epilogue, which reads
-// the accumulator with tcgen05.ld.
+// as tiles of M = 256 weight rows (two M=128 MMAs) x N <= 128 positions.
+//
+// The weights are the A operand.  Routed weights are dequantised by 8
+// producer warps into exact fp16 values q * s * 2^8 (q has at most 4
+// significant bits and s is a bf16, so the product fits fp16's 11 bits) and
+// written into 128-byte-swizzled K-major shared-memory tiles; their int4
+// codes and scales arrive ahead of use through a per-thread cp.async ring.
+// The shared expert's weights are pre-converted fp16 copies that TMA loads
+// directly.  The activations are the B operand, fetched by TMA from buffers
+// in position order: x (fp16, exact after a per-token power-of-two scale) for
+// gate/up and h as two fp16 terms hi + lo (~22 significant bits) for down.
+// Both operands use the same per-8-element K order (the order in which a LOP3
+// extracts nibbles), so nothing is permuted inside the main loop.
+//
+// One thread issues tcgen05.mma into a double-buffered TMEM accumulator
+// (2 x 256 columns); tcgen05.commit releases each pipeline stage, and 4
+// epilogue warps drain a finished accumulator with tcgen05.ld while the next
+// tile is already accumulating.
 //
 // Source of the layer: vLLM recipe page "inclusionAI/Ling-3.0-flash"
 // ("Single-GPU int4": symmetric W4, group 32; "Launching the Server":
@@ -23,25 +32,43 @@
 
 namespace lingmoe {
 
-constexpr int kTcThreads = 160;      // warps 0-3: producers + epilogue, warp 4: MMA issue
-constexpr int kTcStages = 4;
-constexpr int kTcM = 128;            // weight rows per tile
-constexpr int kTcN = 128;            // tokens per tile (max)
-constexpr int kTcK = 64;             // K per stage (one 128-byte swizzle row of fp16)
-constexpr int kStageA = kTcM * kTcK * 2;  // 16 KB
-constexpr int kStageB = kTcN * kTcK * 2;  // 16 KB per B part
-constexpr int kTmemCols = 128;
-// B parts per stage: gate/up reads x (exact in fp16), down reads h as the two
-// fp16 terms hi + lo, so that h keeps ~22 bits through the contraction.
-__host__ __device__ constexpr int tc_bparts(int mode) { return mode == 0 ? 1 : 2; }
-__host__ __device__ constexpr size_t tc_smem(int mode) {
-  return 1024 /*align slack*/ + (size_t)kTcStages * (kStageA + tc_bparts(mode) * kStageB) + 1024;
-}
+// ---------------------------------------------------------------- roles and sizes
+constexpr int kProdWarps = 8;                  // one A row per thread
+constexpr int kEpiWarps = 4;                   // TMEM lane quadrants 0..3
+constexpr int kMmaWarp = kProdWarps + kEpiWarps;  // 12
+constexpr int kTmaWarp = kMmaWarp + 1;            // 13
+constexpr int kTcThreads = (kTmaWarp + 1) * 32;   // 448
+constexpr int kProd = kProdWarps * 32;            // 256
+static_assert(kProd == kTcTileM, "one producer thread per A row");
+static_assert(kProdWarps % 4 == 0, "epilogue warps must start at a multiple of 4");
+
+constexpr int kTcK = 64;                        // K per stage: one 128-byte swizzle row of fp16
+constexpr int kTcStages = 3;
+constexpr int kStageA = kTcTileM * kTcK * 2;    // 32 KB
+constexpr int kStageBPart = kTcTileN * kTcK * 2;  // 16 KB per B part
+constexpr int kBoxRows = 32;                    // B rows per TMA box
+constexpr int kBoxBytes = kBoxRows * kTcK * 2;  // 4 KB
+constexpr int kShBoxRows = 128;                 // shared-expert A rows per TMA box
+constexpr int kTmemCols = 512;                  // 2 buffers x (2 M-halves x 128 columns)
+// raw ring, per stage: int4 codes [2 groups][256 threads] x 16 B, then the
+// 4-byte words holding each group's bf16 scale [2][256] x 4 B
+constexpr int kRawCodes = 2 * kProd * 16;
+constexpr int kRawStage = kRawCodes + 2 * kProd * 4;  // 10 KB
 constexpr unsigned long long kTcWaitNs = 2000000000ull;
 
-// K order inside each group of 8 elements: position p holds element kPerm[p];
-// kInvPerm maps an element to its position.  It is the order in which
-// (w >> 4s) & 0x000F000F yields nibble pairs (e_s, e_{s+4}).
+__host__ __device__ constexpr int tc_bparts(int mode) { return mode == 0 ? 1 : 2; }
+__host__ __device__ constexpr int tc_raw_stages(int mode) { return mode == 0 ? 4 : 2; }
+__host__ __device__ constexpr int tc_nk(int mode) { return (mode == 0 ? kH : kI) / kTcK; }
+__host__ __device__ constexpr size_t tc_bar_off(int mode) {
+  return (size_t)kTcStages * (kStageA + tc_bparts(mode) * kStageBPart) + (size_t)tc_raw_stages(mode) * kRawStage;
+}
+__host__ __device__ constexpr size_t tc_smem(int mode) { return 1024 /*align slack*/ + tc_bar_off(mode) + 256; }
+static_assert(tc_smem(1) <= 232448, "down-projection pipeline exceeds 227 KB of shared memory");
+static_assert(tc_smem(0) <= 232448, "gate/up pipeline exceeds 227 KB of shared memory");
+
+// K order inside each group of 8 elements: element o sits at position
+// perm_pos(o).  It is the order in which (w >> 4s) & 0x000F000F yields nibble
+// pairs (e_s, e_{s+4}).
 __host__ __device__ constexpr int perm_pos(int o) { return (o < 4) ? 2 * o : 2 * (o - 4) + 1; }
 
 // ---------------------------------------------------------------- PTX helpers
@@ -52,7 +79,7 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 }
 __device__ __forceinline__ uint32_t make_idesc(int n) {
   // D = f32, A = B = f16, both K-major, M = 128, N = n
-  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kTcM >> 4) << 24);
+  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 __device__ __forceinline__ void tc_mma(uint32_t tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
@@ -82,6 +109,22 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float v[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
+// 2-D tiled TMA load (no multicast) into this CTA's shared memory.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" :: "r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // bounded wait used by every role; on time-out sets the error word and the
 // CTA's abort flag and returns false
@@ -98,16 +141,18 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, unsigned
   return true;
 }
 
-// Two exact fp16 weights q*s from a nibble pair (1024 + n in each half):
-// v - 1032 = q is exact, and so is q * s (q has at most 4 significant bits,
-// s at most 8).  Folding the bias into one fma would round -1032 * s.
+// ---------------------------------------------------------------- dequantisation
+// Two exact fp16 weights from a nibble pair (1024 + n in each half):
+// v - 1032 = q is exact, and so is q * s' for s' = s * 2^8 (q has at most 4
+// significant bits, s' at most 8).  Folding the bias into one fma would
+// round -1032 * s'.
 __device__ __forceinline__ uint32_t deq_pair(uint32_t v, __half2 s2, __half2 b2) {
   const __half2 q = __hsub2(*reinterpret_cast<const __half2*>(&v), b2);
   const __half2 r = __hmul2(q, s2);
   return *reinterpret_cast<const uint32_t*>(&r);
 }
-// 32 codes (16 bytes, offset-binary nibbles) of one group with scale s ->
-// 32 fp16 in permuted K order, written as 4 x 16 bytes to dst chunks.
+// 32 codes (16 bytes, offset-binary nibbles) of one group with scale s' ->
+// 32 fp16 in permuted K order, as 4 x 16 bytes.
 __device__ __forceinline__ void deq_group(uint4 q, float s, uint4 out[4]) {
   const __half sh = __float2half_rn(s);
   const __half2 s2 = __halves2half2(sh, sh);
@@ -127,100 +172,118 @@ __device__ __forceinline__ void deq_group(uint4 q, float s, uint4 out[4]) {
   }
 }
 
-// ---------------------------------------------------------------- x -> fp16 (permuted)
-// x [T, H] bf16 -> x16 [T, H] fp16 in the permuted K order, scaled by
-// 2^-sigma_t so that max|x_t| stays inside fp16; xscale[t] = 2^sigma_t.
-__global__ void __launch_bounds__(256) x16_kernel(const __nv_bfloat16* __restrict__ x, int T,
-                                                  __half* __restrict__ x16, float* __restrict__ xscale) {
-  const int t = blockIdx.x;
-  if (t >= T) return;
-  __shared__ uint32_t smax;
-  if (threadIdx.x == 0) smax = 0;
-  __syncthreads();
-  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * kH);
-  for (int c = threadIdx.x; c < kH / 8; c += blockDim.x) {
-    const uint4 w = src[c];
-    const float m = fmaxf(fmaxf(fmaxf(fabsf(bf16lo(w.x)), fabsf(bf16hi(w.x))), fmaxf(fabsf(bf16lo(w.y)), fabsf(bf16hi(w.y)))),
-                          fmaxf(fmaxf(fabsf(bf16lo(w.z)), fabsf(bf16hi(w.z))), fmaxf(fabsf(bf16lo(w.w)), fabsf(bf16hi(w.w)))));
-    atomicMax(&smax, __float_as_uint(fminf(m, 3.0e38f)));
+// ---------------------------------------------------------------- shared-expert fp16 copies
+// Power-of-two exponent c with max|w| * 2^c in [2^14, 2^15) (0 for an all-zero
+// matrix), clamped so that 2^c and 2^-c stay normal fp32 numbers.
+__device__ __forceinline__ int sh_exp(unsigned int amax_bits) {
+  if (amax_bits == 0) return 0;
+  const int e = (int)(amax_bits >> 23) - 127;
+  return max(-100, min(100, 14 - e));
+}
+__device__ __forceinline__ float pow2f(int c) { return __uint_as_float((uint32_t)(127 + c) << 23); }
+
+__global__ void __launch_bounds__(256) sh_amax_kernel(const __nv_bfloat16* g, const __nv_bfloat16* u,
+                                                      const __nv_bfloat16* d, unsigned int* amax) {
+  const int m = blockIdx.y;  // 0 gate, 1 up, 2 down (all kI * kH elements)
+  const __nv_bfloat16* w = m == 0 ? g : (m == 1 ? u : d);
+  const uint4* w4 = reinterpret_cast<const uint4*>(w);
+  float a = 0.f;
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < kI * kH / 8; c += gridDim.x * blockDim.x) {
+    const uint4 v = w4[c];
+    a = fmaxf(a, fmaxf(fmaxf(fmaxf(fabsf(bf16lo(v.x)), fabsf(bf16hi(v.x))), fmaxf(fabsf(bf16lo(v.y)), fabsf(bf16hi(v.y)))),
+                       fmaxf(fmaxf(fabsf(bf16lo(v.z)), fabsf(bf16hi(v.z))), fmaxf(fabsf(bf16lo(v.w)), fabsf(bf16hi(v.w))))));
   }
-  __syncthreads();
-  const int e = (int)(smax >> 23) - 127;
-  const int sigma = e >= 14 ? e - 13 : 0;
-  const float inv = __uint_as_float((uint32_t)(127 - sigma) << 23);
-  if (threadIdx.x == 0) xscale[t] = __uint_as_float((uint32_t)(127 + sigma) << 23);
-  uint4* dst = reinterpret_cast<uint4*>(x16 + (size_t)t * kH);
-  for (int c = threadIdx.x; c < kH / 8; c += blockDim.x) {
-    const uint4 w = src[c];
-    const float f[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
-                        bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(&amax[m], __float_as_uint(fminf(a, 3.0e38f)));
+}
+
+// One thread per 8 consecutive K elements: scale by 2^c, convert to fp16,
+// store in the permuted K order.  Gate/up rows are interleaved (2i gate, 2i+1 up).
+__global__ void __launch_bounds__(256) sh_convert_kernel(const __nv_bfloat16* g, const __nv_bfloat16* u,
+                                                         const __nv_bfloat16* d, const unsigned int* amax,
+                                                         __half* shgu16, __half* shdn16, float* sh_scale) {
+  const int m = blockIdx.y;
+  const int c = sh_exp(amax[m]);
+  if (blockIdx.x == 0 && threadIdx.x == 0) sh_scale[m] = pow2f(-c);
+  const float f = pow2f(c);
+  const __nv_bfloat16* w = m == 0 ? g : (m == 1 ? u : d);
+  const int K = m < 2 ? kH : kI;
+  for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < kI * kH / 8; v += gridDim.x * blockDim.x) {
+    const int row = (v * 8) / K, k0 = (v * 8) % K;
+    const uint4 x = reinterpret_cast<const uint4*>(w)[v];
+    const float e[8] = {bf16lo(x.x), bf16hi(x.x), bf16lo(x.y), bf16hi(x.y),
+                        bf16lo(x.z), bf16hi(x.z), bf16lo(x.w), bf16hi(x.w)};
     __half h[8];
 #pragma unroll
-    for (int o = 0; o < 8; ++o) h[perm_pos(o)] = __float2half_rn(f[o] * inv);
-    dst[c] = *reinterpret_cast<const uint4*>(h);
+    for (int o = 0; o < 8; ++o) h[perm_pos(o)] = __float2half_rn(e[o] * f);
+    __half* dst = m < 2 ? shgu16 + (size_t)(2 * row + m) * kH + k0 : shdn16 + (size_t)row * kI + k0;
+    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(h);
   }
 }
 
-// ---------------------------------------------------------------- tile lists
-// One thread: tiles (expert, m-tile, first token position, tokens) in expert
-// order, for both GEMMs.
-__global__ void tc_tiles_kernel(const int32_t* cnt, const int32_t* off, int E, int4* gu_tiles, int4* dn_tiles,
-                                int32_t* ntiles) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  int ng = 0, nd = 0;
-  for (int e = 0; e < E; ++e) {
-    const int m = cnt[e];
-    for (int n0 = 0; n0 < m; n0 += kTcN) {
-      const int n = min(kTcN, m - n0);
-      for (int mt = 0; mt < kI * 2 / kTcM; ++mt) gu_tiles[ng++] = make_int4(e, mt, off[e] + n0, n);
-      for (int mt = 0; mt < kH / kTcM; ++mt) dn_tiles[nd++] = make_int4(e, mt, off[e] + n0, n);
-    }
-  }
-  ntiles[0] = ng;
-  ntiles[1] = nd;
+cudaError_t launch_tc_prep_shared(const __nv_bfloat16* g, const __nv_bfloat16* u, const __nv_bfloat16* d,
+                                  __half* shgu16, __half* shdn16, float* sh_scale, unsigned int* amax_scratch,
+                                  cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(amax_scratch, 0, 3 * sizeof(unsigned int), s);
+  if (e != cudaSuccess) return e;
+  sh_amax_kernel<<<dim3(148, 3), 256, 0, s>>>(g, u, d, amax_scratch);
+  sh_convert_kernel<<<dim3(296, 3), 256, 0, s>>>(g, u, d, amax_scratch, shgu16, shdn16, sh_scale);
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- the GEMM
-// MODE 0: gate/up (A = gate/up rows interleaved: tile row 2j = gate, 2j+1 = up
-// of intermediate row 64*mt + j; B = x16 rows of the tile's tokens; output h16
-// [positions, 768] fp16 in permuted K order).
-// MODE 1: down (A = down rows 128*mt..+127; B = the hi and lo halves of the
-// h16 rows, both accumulated into one TMEM tile; output y [positions, 2560]
-// fp32 scaled by the pair's routing weight).
+// MODE 0, gate/up: A row r of tile (e, mt) is gate (r even) or up (r odd) of
+// intermediate row i = 128 mt + r/2; B = x rows of the tile's positions; the
+// epilogue writes h = SiLU(g) * u per position as fp16 hi + lo.
+// MODE 1, down: A row r is output row 256 mt + r; B = the hi and lo halves of
+// h, both accumulated into one TMEM tile; the epilogue writes y = w (Wd h).
+//
+// Roles: warps 0-7 dequantise A, warps 8-11 drain TMEM, warp 12 issues the
+// MMAs (one thread), warp 13 issues the TMA loads (one thread).  Every role
+// walks the same sequence of tiles (blockIdx.x, + gridDim.x, ...) and stages.
 template <int MODE>
-__global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(TcParams p) {
+__global__ void __launch_bounds__(kTcThreads, 1)
+tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmA,
+                  const TcParams p) {
+  constexpr int NB = tc_bparts(MODE);
+  constexpr int R = tc_raw_stages(MODE);
+  constexpr int NK = tc_nk(MODE);
+  constexpr int S = kTcStages;
   extern __shared__ __align__(1024) unsigned char smem_raw_tc[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw_tc) + 1023) & ~uintptr_t(1023));
   unsigned char* sA = smem;
-  constexpr int NB = tc_bparts(MODE);
-  unsigned char* sB = smem + kTcStages * kStageA;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kTcStages * NB * kStageB);
-  uint64_t* empty = full + kTcStages;
-  uint64_t* accf = empty + kTcStages;
-  uint64_t* acce = accf + 1;
-  uint64_t* drain = acce + 1;
+  unsigned char* sB = smem + S * kStageA;
+  unsigned char* sRaw = sB + S * NB * kStageBPart;
+  uint64_t* full_a = reinterpret_cast<uint64_t*>(smem + tc_bar_off(MODE));
+  uint64_t* full_b = full_a + S;
+  uint64_t* empty = full_b + S;
+  uint64_t* accf = empty + S;
+  uint64_t* acce = accf + 2;
+  uint64_t* drain = acce + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int KTOT = MODE == 0 ? kH : kI;
-  constexpr int NK = KTOT / kTcK;
   const int4* tiles = MODE == 0 ? p.gu_tiles : p.dn_tiles;
   const int ntiles = p.ntiles[MODE];
+  const int ntl = ntiles > (int)blockIdx.x ? (ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
   if (tid == 0) {
-    for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&full[s], 128);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full_a[s], kProd);
+      mbar_init(&full_b[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(accf, 1);
-    mbar_init(acce, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accf[b], 1);
+      mbar_init(&acce[b], kEpiWarps * 32);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  :: "r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -230,175 +293,287 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_grouped_kernel(TcParams p) {
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  int g = 0;     // global stage counter (same sequence in every role)
-  int tj = 0;    // tiles done by this CTA
-  for (int ti = blockIdx.x; ti < ntiles; ti += gridDim.x, ++tj) {
-    const int4 tl = tiles[ti];
-    const int e = tl.x, mt = tl.y, pos0 = tl.z, nrow = tl.w;
-    const int nmma = (nrow + 15) & ~15;  // N of the MMA: multiple of 16, >= 16
-    if (warp < 4) {
-      // ------------------------------------------------ producers
-      const int r = tid;  // A row and B row handled by this thread
-      // A source for row r
-      const uint8_t* abase;
-      int alane;
-      if (MODE == 0) {
-        const int i = 64 * mt + (r >> 1);          // intermediate row
-        const int rin = (r & 1) ? 4 + (i & 3) : (i & 3);  // row within the unit (gate 0-3, up 4-7)
-        abase = p.gu + ((size_t)e * kGuUnits + (i >> 2)) * kGuUnitBytes;
-        alane = rin;                                 // + 8 * quarter, below
-      } else {
-        const int n = kTcM * mt + r;                 // output row
-        abase = p.dn + ((size_t)e * kDnUnits + (n >> 2)) * kDnUnitBytes;
-        alane = n & 3;                               // + 4 * slice, below
+  if (warp < kProdWarps) {
+    // ------------------------------------------------ producers: A row r
+    const int r = tid;
+    const int total = ntl * NK;
+    const uint32_t raw0 = smem_u32(sRaw);
+    // cp.async the codes and the scale word of groups 2kk, 2kk+1 of row r for
+    // stage q into raw slot q % R (one commit group per stage, empty or not)
+    auto issue = [&](int q) {
+      if (q < total) {
+        const int j = q / NK, kk = q - j * NK;
+        const int4 tl = tiles[blockIdx.x + j * gridDim.x];
+        if (tl.x < p.E) {
+          const uint32_t slot = raw0 + (q % R) * kRawStage;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int G = 2 * kk + h;
+            const uint8_t* codes;
+            const uint8_t* sword;
+            if (MODE == 0) {
+              const int i = (kTcTileM / 2) * tl.y + (r >> 1);
+              const int rin = (r & 1) ? 4 + (i & 3) : (i & 3);
+              const uint8_t* abase = p.gu + ((size_t)tl.x * kGuUnits + (i >> 2)) * kGuUnitBytes;
+              const int quarter = G / kGuChunks, jj = G - quarter * kGuChunks, ln = rin + 8 * quarter;
+              codes = abase + jj * 512 + 16 * ln;
+              sword = abase + kGuScaleOff + (jj >> 2) * 256 + 8 * ln + 4 * ((jj & 3) >> 1);
+            } else {
+              const int n = kTcTileM * tl.y + r;
+              const uint8_t* abase = p.dn + ((size_t)tl.x * kDnUnits + (n >> 2)) * kDnUnitBytes;
+              const int slice = G / kDnChunks, jj = G - slice * kDnChunks, ln = (n & 3) + 4 * slice;
+              codes = abase + jj * 512 + 16 * ln;
+              sword = abase + kDnScaleOff + jj * 64 + 4 * (ln >> 1);
+            }
+            cp_async16(slot + h * (kProd * 16) + r * 16, codes);
+            cp_async4(slot + kRawCodes + h * (kProd * 4) + r * 4, sword);
+          }
+        }
       }
-      // B source for row r (token or position)
-      const bool bvalid = r < nrow;
-      const unsigned char* bsrc;
-      if (MODE == 0) {
-        const int tok = bvalid ? p.perm[pos0 + r] / p.k : 0;
-        bsrc = reinterpret_cast<const unsigned char*>(p.x16 + (size_t)tok * kH);
-      } else {
-        bsrc = reinterpret_cast<const unsigned char*>(p.h16 + (size_t)(pos0 + (bvalid ? r : 0)) * 2 * kI);
+      cp_async_commit();
+    };
+#pragma unroll 1
+    for (int q = 0; q < R - 1; ++q) issue(q);
+    int jc = -1;
+    int4 tl = make_int4(0, 0, 0, 0);
+#pragma unroll 1
+    for (int g = 0; g < total; ++g) {
+      issue(g + R - 1);
+      cp_async_wait<R - 1>();
+      const int j = g / NK, kk = g - j * NK;
+      if (j != jc) {
+        tl = tiles[blockIdx.x + j * gridDim.x];
+        jc = j;
       }
-      for (int kk = 0; kk < NK; ++kk, ++g) {
-        const int s = g % kTcStages;
-        if (!tc_wait(&empty[s], ((g / kTcStages) & 1) ^ 1, p.err, abort_flag)) break;
-        // two groups of 32 codes: groups 2kk, 2kk+1 of this row
+      const int s = g % S;
+      if (!tc_wait(&empty[s], ((g / S) & 1) ^ 1, p.err, abort_flag)) break;
+      if (tl.x < p.E) {
+        const unsigned char* slot = sRaw + (g % R) * kRawStage;
         uint4 outv[8];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int G = 2 * kk + h;
-          uint4 q;
-          float sc;
+          int hi_half;
           if (MODE == 0) {
-            const int quarter = G / kGuChunks, j = G - quarter * kGuChunks, ln = alane + 8 * quarter;
-            q = *reinterpret_cast<const uint4*>(abase + j * 512 + 16 * ln);
-            sc = bf16_to_f32(*reinterpret_cast<const unsigned short*>(abase + kGuScaleOff + (j >> 2) * 256 + 8 * ln + 2 * (j & 3)));
+            hi_half = (G % kGuChunks) & 1;
           } else {
-            const int slice = G / kDnChunks, j = G - slice * kDnChunks, ln = alane + 4 * slice;
-            q = *reinterpret_cast<const uint4*>(abase + j * 512 + 16 * ln);
-            sc = bf16_to_f32(*reinterpret_cast<const unsigned short*>(abase + kDnScaleOff + j * 64 + 2 * ln));
+            const int n = kTcTileM * tl.y + r;
+            hi_half = ((n & 3) + 4 * (G / kDnChunks)) & 1;
           }
+          const uint4 q = *reinterpret_cast<const uint4*>(slot + h * (kProd * 16) + r * 16);
+          const uint32_t wv = *reinterpret_cast<const uint32_t*>(slot + kRawCodes + h * (kProd * 4) + r * 4);
+          const float sc = __uint_as_float(hi_half ? (wv & 0xFFFF0000u) : (wv << 16)) * (float)(1 << kTcScaleShift);
           deq_group(q, sc, outv + 4 * h);
         }
         unsigned char* a = sA + s * kStageA + r * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(a + ((c ^ (r & 7)) << 4)) = outv[c];
-#pragma unroll
-        for (int part = 0; part < NB; ++part) {
-          unsigned char* b = sB + (s * NB + part) * kStageB + r * 128;
-          const uint4* bs = reinterpret_cast<const uint4*>(bsrc + part * 2 * kI + kk * 128);
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(b + ((c ^ (r & 7)) << 4)) = bvalid ? bs[c] : make_uint4(0, 0, 0, 0);
-        }
         fence_async_smem();
-        mbar_arrive(&full[s]);
       }
-      // ------------------------------------------------ epilogue
-      if (!tc_wait(accf, tj & 1, p.err, abort_flag)) break;
+      mbar_arrive(&full_a[s]);
+    }
+    cp_async_wait_all();
+  } else if (warp < kMmaWarp) {
+    // ------------------------------------------------ epilogue: TMEM lanes 32 qd .. 32 qd + 31
+    const int qd = warp & 3;
+    const int l = 32 * qd + lane;  // accumulator row within an M-half
+#pragma unroll 1
+    for (int j = 0; j < ntl; ++j) {
+      const int b = j & 1;
+      if (!tc_wait(&accf[b], (j >> 1) & 1, p.err, abort_flag)) break;
       tc_fence_after();
-      const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-      for (int c0 = 0; c0 < nmma; c0 += 16) {
-        float v[16];
-        tmem_ld16(trow + c0, v);
-        if (MODE == 0) {
-          const int rr = warp * 32 + lane, j = rr >> 1, i = 64 * mt + j;
-          const int ip = (i & ~7) + perm_pos(i & 7);
-#pragma unroll
-          for (int cc = 0; cc < 16; ++cc) {
-            const float other = __shfl_xor_sync(0xffffffffu, v[cc], 1);
-            const int col = c0 + cc;
-            if (!(lane & 1) && col < nrow) {
-              const int pos = pos0 + col;
-              const float xs = p.xscale[p.perm[pos] / p.k];
-              const float hv = silu_mul(v[cc] * xs, other * xs);
-              const __half hi = __float2half_rn(hv);
-              p.h16[(size_t)pos * 2 * kI + ip] = hi;
-              p.h16[(size_t)pos * 2 * kI + kI + ip] = __float2half_rn(hv - __half2float(hi));
-            }
+      const int4 tl = tiles[blockIdx.x + j * gridDim.x];
+      const int mt = tl.y, pos0 = tl.z, n = tl.w, nmma = (n + 15) & ~15;
+      const bool shared = tl.x >= p.E;
+#pragma unroll 1
+      for (int mh = 0; mh < 2; ++mh) {
+        const uint32_t tb = tmem + ((uint32_t)(32 * qd) << 16) + (uint32_t)(b * 256 + mh * 128);
+#pragma unroll 1
+        for (int c0 = 0; c0 < nmma; c0 += 16) {
+          float v[16];
+          tmem_ld16(tb + c0, v);
+          // per-column factor: lane L < 16 fetches it for column c0 + L
+          float fac = 0.f;
+          const int cl = c0 + (lane & 15);
+          if (cl < n) {
+            const int pos = pos0 + cl;
+            if (MODE == 0) fac = p.xscale[shared ? pos - p.P : p.perm[pos] / p.k];
+            else fac = shared ? 1.f : p.topk_w[p.perm[pos]];
           }
-        } else {
-          const int n = kTcM * mt + warp * 32 + lane;
+          if (MODE == 0) {
+            const int rr = mh * 128 + l, i = (kTcTileM / 2) * mt + (rr >> 1);
+            const int ip = (i & ~7) + perm_pos(i & 7);
+            const float cg = shared ? p.sh_scale[0] : 1.f / (float)(1 << kTcScaleShift);
+            const float cu = shared ? p.sh_scale[1] : 1.f / (float)(1 << kTcScaleShift);
 #pragma unroll
-          for (int cc = 0; cc < 16; ++cc) {
-            const int col = c0 + cc;
-            if (col < nrow) {
-              const int pos = pos0 + col;
-              p.y[(size_t)pos * kH + n] = v[cc] * p.topk_w[p.perm[pos]];
+            for (int cc = 0; cc < 16; ++cc) {
+              const float other = __shfl_xor_sync(0xffffffffu, v[cc], 1);
+              const float f = __shfl_sync(0xffffffffu, fac, cc);
+              const int col = c0 + cc;
+              if (!(lane & 1) && col < n) {
+                const float hv = silu_mul(v[cc] * f * cg, other * f * cu) * (1.f / (float)(1 << kTcScaleShift));
+                const __half hi = __float2half_rn(hv);
+                __half* dst = p.h16 + (size_t)(pos0 + col) * (2 * kI) + ip;
+                dst[0] = hi;
+                dst[kI] = __float2half_rn(hv - __half2float(hi));
+              }
+            }
+          } else {
+            const int nrow = kTcTileM * mt + mh * 128 + l;
+            const float cf = shared ? p.sh_scale[2] * (float)(1 << kTcScaleShift) : 1.f;
+#pragma unroll
+            for (int cc = 0; cc < 16; ++cc) {
+              const float f = __shfl_sync(0xffffffffu, fac, cc);
+              const int col = c0 + cc;
+              if (col < n) p.y[(size_t)(pos0 + col) * kH + nrow] = v[cc] * f * cf;
             }
           }
         }
       }
       tc_fence_before();
-      mbar_arrive(acce);
-    } else {
-      // ------------------------------------------------ MMA issue (one thread)
+      mbar_arrive(&acce[b]);
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------ MMA issue (one thread)
+    if (lane == 0) {
+      int g = 0;
       bool ok = true;
-      if (lane == 0) {
-        if (tj > 0) ok = tc_wait(acce, (tj - 1) & 1, p.err, abort_flag);
+#pragma unroll 1
+      for (int j = 0; j < ntl && ok; ++j) {
+        const int b = j & 1;
+        const int4 tl = tiles[blockIdx.x + j * gridDim.x];
+        const int nmma = (tl.w + 15) & ~15;
+        if (j >= 2 && !tc_wait(&acce[b], ((j >> 1) - 1) & 1, p.err, abort_flag)) break;
         tc_fence_after();
         const uint32_t idesc = make_idesc(nmma);
-        for (int kk = 0; kk < NK && ok; ++kk, ++g) {
-          const int s = g % kTcStages;
-          if (!tc_wait(&full[s], (g / kTcStages) & 1, p.err, abort_flag)) { ok = false; break; }
+        const uint32_t dcol = tmem + (uint32_t)(b * 256);
+#pragma unroll 1
+        for (int kk = 0; kk < NK; ++kk, ++g) {
+          const int s = g % S;
+          const uint32_t ph = (g / S) & 1;
+          if (!tc_wait(&full_a[s], ph, p.err, abort_flag) || !tc_wait(&full_b[s], ph, p.err, abort_flag)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + s * kStageA), b0 = smem_u32(sB + s * NB * kStageB);
+          const uint32_t a0 = smem_u32(sA + s * kStageA), b0 = smem_u32(sB + s * NB * kStageBPart);
 #pragma unroll
           for (int k4 = 0; k4 < kTcK / 16; ++k4)
 #pragma unroll
-            for (int part = 0; part < NB; ++part)
-              tc_mma(tmem, sw128_desc(a0 + 32 * k4), sw128_desc(b0 + part * kStageB + 32 * k4), idesc,
-                     (kk | k4 | part) ? 1u : 0u);
+            for (int mh = 0; mh < 2; ++mh)
+#pragma unroll
+              for (int part = 0; part < NB; ++part)
+                tc_mma(dcol + mh * 128, sw128_desc(a0 + mh * (kStageA / 2) + 32 * k4),
+                       sw128_desc(b0 + part * kStageBPart + 32 * k4), idesc, (kk | k4 | part) ? 1u : 0u);
           tc_commit(&empty[s]);
         }
-        if (ok) tc_commit(accf);
+        if (ok) tc_commit(&accf[b]);
       }
-      g = __shfl_sync(0xffffffffu, g, 0);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
+      // no MMA may still be writing TMEM when it is freed
+      tc_commit(drain);
+      mbar_wait(drain, 0, kTcWaitNs, p.err);
     }
-    if (*reinterpret_cast<volatile int*>(abort_flag)) break;
-  }
-  // teardown: no MMA may still be writing TMEM when it is freed
-  if (warp == 4 && lane == 0) {
-    tc_commit(drain);
-    const unsigned long long t0 = globaltimer_ns();
-    while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kTcWaitNs) {
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ TMA issue (one thread)
+    if (lane == 0) {
+      int g = 0;
+      bool ok = true;
+#pragma unroll 1
+      for (int j = 0; j < ntl && ok; ++j) {
+        const int4 tl = tiles[blockIdx.x + j * gridDim.x];
+        const int nmma = (tl.w + 15) & ~15, nbox = (nmma + kBoxRows - 1) / kBoxRows;
+        const bool shared = tl.x >= p.E;
+        const uint32_t bytes = (uint32_t)(NB * nbox * kBoxBytes + (shared ? kStageA : 0));
+#pragma unroll 1
+        for (int kk = 0; kk < NK; ++kk, ++g) {
+          const int s = g % S;
+          if (!tc_wait(&empty[s], ((g / S) & 1) ^ 1, p.err, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full_b[s], bytes);
+          const uint32_t bdst = smem_u32(sB + s * NB * kStageBPart);
+#pragma unroll
+          for (int part = 0; part < NB; ++part)
+            for (int bx = 0; bx < nbox; ++bx)
+              tma_load_2d(bdst + part * kStageBPart + bx * kBoxBytes, &tmB, part * kI + kk * kTcK,
+                          tl.z + bx * kBoxRows, &full_b[s]);
+          if (shared) {
+            const uint32_t adst = smem_u32(sA + s * kStageA);
+            for (int hf = 0; hf < kTcTileM / kShBoxRows; ++hf)
+              tma_load_2d(adst + hf * (kShBoxRows * 128), &tmA, kk * kTcK, kTcTileM * tl.y + hf * kShBoxRows,
+                          &full_b[s]);
+          }
+        }
+      }
+      // after an abort, loads may still be landing: wait for every armed stage
+      for (int q = g - S > 0 ? g - S : 0; q < g; ++q) mbar_wait(&full_b[q % S], (q / S) & 1, kTcWaitNs, p.err);
     }
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kTmemCols) : "memory");
   }
 }
 
-size_t tc_smem_bytes() { return tc_smem(1); }
-
+// ---------------------------------------------------------------- host
 cudaError_t setup_grouped_tc() {
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(tc_grouped_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_smem(0))) != cudaSuccess)
+  if ((e = cudaFuncSetAttribute(tc_grouped_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)tc_smem(0))) != cudaSuccess)
     return e;
   return cudaFuncSetAttribute(tc_grouped_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_smem(1));
 }
 
-cudaError_t launch_x16(const __nv_bfloat16* x, int T, __half* x16, float* xscale, cudaStream_t s) {
-  x16_kernel<<<T, 256, 0, s>>>(x, T, x16, xscale);
-  return cudaGetLastError();
+namespace {
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
 }
 
-cudaError_t launch_tc_tiles(const int32_t* cnt, const int32_t* off, int E, int4* gu_tiles, int4* dn_tiles,
-                            int32_t* ntiles, cudaStream_t s) {
-  tc_tiles_kernel<<<1, 32, 0, s>>>(cnt, off, E, gu_tiles, dn_tiles, ntiles);
-  return cudaGetLastError();
+// fp16 matrix [rows, cols] row-major; boxes of 64 columns (128 B) x box_rows,
+// 128-byte swizzle, zero fill outside the matrix
+cudaError_t encode_2d(CUtensorMap* m, const __half* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * sizeof(__half)};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+}  // namespace
+
+cudaError_t tc_encode_maps(TcMaps* m, const __half* xg, const __half* h16, int rows, const __half* shgu16,
+                           const __half* shdn16) {
+  cudaError_t e;
+  if ((e = encode_2d(&m->b_x, xg, rows, kH, kBoxRows)) != cudaSuccess) return e;
+  if ((e = encode_2d(&m->b_h, h16, rows, 2 * kI, kBoxRows)) != cudaSuccess) return e;
+  if ((e = encode_2d(&m->a_shgu, shgu16, 2 * kI, kH, kShBoxRows)) != cudaSuccess) return e;
+  return encode_2d(&m->a_shdn, shdn16, kH, kI, kShBoxRows);
 }
 
-cudaError_t launch_tc_gemm(int mode, const TcParams& p, int nctas, cudaStream_t s) {
-  if (mode == 0) tc_grouped_kernel<0><<<nctas, kTcThreads, tc_smem(0), s>>>(p);
-  else tc_grouped_kernel<1><<<nctas, kTcThreads, tc_smem(1), s>>>(p);
+cudaError_t launch_tc_gemm(int mode, const TcMaps& m, const TcParams& p, int nctas, cudaStream_t s) {
+  if (mode == 0) tc_grouped_kernel<0><<<nctas, kTcThreads, tc_smem(0), s>>>(m.b_x, m.a_shgu, p);
+  else tc_grouped_kernel<1><<<nctas, kTcThreads, tc_smem(1), s>>>(m.b_h, m.a_shdn, p);
   return cudaGetLastError();
 }
 

@@ -3,36 +3,63 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>  // CUtensorMap (types only; the encoder is fetched at run time)
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "layout.h"
+
 namespace lingmoe {
 
+constexpr int kTcTileM = 256;                  // weight rows per CTA tile
+constexpr int kTcTileN = 128;                  // positions per CTA tile (max)
+constexpr int kTcMTilesGu = 2 * kI / kTcTileM;  // 6: gate/up rows interleaved
+constexpr int kTcMTilesDn = kH / kTcTileM;      // 10
+// Routed weights enter the MMA as q * s * 2^kTcScaleShift and h as h *
+// 2^-kTcScaleShift, which keeps both inside fp16's normal range for scales in
+// [2^-22, 32] and |h| < 2^23.
+constexpr int kTcScaleShift = 8;
+
+// Tile record: (expert or E for the shared expert, m-tile, first position, positions).
 struct TcParams {
   const uint8_t* gu;        // repacked routed gate/up
   const uint8_t* dn;        // repacked routed down
-  const __half* x16;        // [T, H] fp16, permuted K order, scaled by 1/xscale
-  const float* xscale;      // [T]
-  __half* h16;              // [positions, 2, I] fp16 hi and lo terms, permuted K order
-  float* y;                 // [positions, H] fp32, weighted by the routing weight
-  const int32_t* perm;      // position -> pair id (t*k + slot)
-  const float* topk_w;      // [pairs]
-  int k;
-  const int4* gu_tiles;     // (expert, m-tile, first position, tokens)
+  const float* xscale;      // [T] 2^sigma_t: x16 rows hold x * 2^-sigma_t
+  __half* h16;              // [rows, 2, I] h * 2^-8 as fp16 hi + lo, permuted K order
+  float* y;                 // [rows, H] expert output per position, times the routing weight
+  const int32_t* perm;      // position (< P) -> pair id t*k + slot
+  const float* topk_w;      // [P] routing weight per pair id
+  const float* sh_scale;    // [3] 2^-c of the fp16 shared-expert copies (gate, up, down)
+  int k, E, P;              // shared-expert tiles carry expert E and positions P + t
+  const int4* gu_tiles;
   const int4* dn_tiles;
   const int32_t* ntiles;    // [0] gate/up tiles, [1] down tiles
   unsigned int* err;        // sticky device error word
 };
 
-size_t tc_smem_bytes();
+// TMA descriptors: the B operands (x rows by position, h rows by position)
+// and the fp16 copies of the shared expert, all 128-byte swizzled.
+struct TcMaps {
+  CUtensorMap b_x;     // xg  [rows, H]     box 64 x 32
+  CUtensorMap b_h;     // h16 [rows, 2I]    box 64 x 32
+  CUtensorMap a_shgu;  // shgu16 [2I, H]    box 64 x 128
+  CUtensorMap a_shdn;  // shdn16 [H, I]     box 64 x 128
+};
+
 cudaError_t setup_grouped_tc();
-cudaError_t launch_x16(const __nv_bfloat16* x, int T, __half* x16, float* xscale, cudaStream_t s);
-cudaError_t launch_tc_tiles(const int32_t* cnt, const int32_t* off, int E, int4* gu_tiles, int4* dn_tiles,
-                            int32_t* ntiles, cudaStream_t s);
-cudaError_t launch_tc_gemm(int mode, const TcParams& p, int nctas, cudaStream_t s);
-// upper bounds on the tile counts for P token-expert pairs over E experts
-inline size_t tc_max_tiles_gu(int P, int E) { return ((size_t)P / 128 + (size_t)E + 1) * 12; }
-inline size_t tc_max_tiles_dn(int P, int E) { return ((size_t)P / 128 + (size_t)E + 1) * 20; }
+cudaError_t tc_encode_maps(TcMaps* m, const __half* xg, const __half* h16, int rows, const __half* shgu16,
+                           const __half* shdn16);
+// fp16 copies of the shared expert in the permuted K order, gate/up rows
+// interleaved, each matrix scaled by a power of two 2^c so that max |w| * 2^c
+// lies in [2^14, 2^15); sh_scale receives 2^-c.  amax_scratch: 3 words.
+cudaError_t launch_tc_prep_shared(const __nv_bfloat16* g, const __nv_bfloat16* u, const __nv_bfloat16* d,
+                                  __half* shgu16, __half* shdn16, float* sh_scale, unsigned int* amax_scratch,
+                                  cudaStream_t s);
+cudaError_t launch_tc_gemm(int mode, const TcMaps& m, const TcParams& p, int nctas, cudaStream_t s);
+// upper bound on the number of N-tiles (each expands into kTcMTiles* tiles)
+inline size_t tc_max_ntiles(int P, int T, int E) {
+  return (size_t)P / kTcTileN + (size_t)E + (size_t)T / kTcTileN + 2;
+}
 
 }  // namespace lingmoe
