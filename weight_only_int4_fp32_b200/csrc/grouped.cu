@@ -407,6 +407,9 @@ cudaError_t launch_grouped(const GroupedParams& p, const GroupedWorkspace& ws, c
   tp.dn_tiles = ws.dn_tiles;
   tp.ntiles = ws.ntiles;
   tp.err = ws.err;
+  tp.xg = ws.xg;
+  tp.shgu16 = ws.shgu16;
+  tp.shdn16 = ws.shdn16;
   if ((e = launch_tc_gemm(0, ws.maps, tp, p.num_sms, s)) != cudaSuccess) return e;
   ++nl;
   if ((e = launch_tc_gemm(1, ws.maps, tp, p.num_sms, s)) != cudaSuccess) return e;

@@ -62,7 +62,12 @@ __host__ __device__ constexpr int tc_nk(int mode) { return (mode == 0 ? kH : kI)
 __host__ __device__ constexpr size_t tc_bar_off(int mode) {
   return (size_t)kTcStages * (kStageA + tc_bparts(mode) * kStageBPart) + (size_t)tc_raw_stages(mode) * kRawStage;
 }
-__host__ __device__ constexpr size_t tc_smem(int mode) { return 1024 /*align slack*/ + tc_bar_off(mode) + 256; }
+// after the barriers: per epilogue warp, per TMEM buffer, 128 column factors
+constexpr int kFacOff = 256;
+constexpr int kFacBytes = kEpiWarps * 2 * kTcTileN * 4;
+__host__ __device__ constexpr size_t tc_smem(int mode) {
+  return 1024 /*align slack*/ + tc_bar_off(mode) + kFacOff + kFacBytes;
+}
 static_assert(tc_smem(1) <= 232448, "down-projection pipeline exceeds 227 KB of shared memory");
 static_assert(tc_smem(0) <= 232448, "gate/up pipeline exceeds 227 KB of shared memory");
 
@@ -109,6 +114,27 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float v[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
+__device__ __forceinline__ void tmem_ld16x2(uint32_t ta, uint32_t tb, float va[16], float vb[16]) {
+  uint32_t r[16], q[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(ta));
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(q[0]), "=r"(q[1]), "=r"(q[2]), "=r"(q[3]), "=r"(q[4]), "=r"(q[5]), "=r"(q[6]), "=r"(q[7]),
+        "=r"(q[8]), "=r"(q[9]), "=r"(q[10]), "=r"(q[11]), "=r"(q[12]), "=r"(q[13]), "=r"(q[14]), "=r"(q[15])
+      : "r"(tb));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    va[i] = __uint_as_float(r[i]);
+    vb[i] = __uint_as_float(q[i]);
+  }
+}
+// SiLU(g) * u with the fast exponential and division (relative error ~1e-6)
+__device__ __forceinline__ float tc_silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 // 2-D tiled TMA load (no multicast) into this CTA's shared memory.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   asm volatile(
@@ -198,7 +224,8 @@ __global__ void __launch_bounds__(256) sh_amax_kernel(const __nv_bfloat16* g, co
 }
 
 // One thread per 8 consecutive K elements: scale by 2^c, convert to fp16,
-// store in the permuted K order.  Gate/up rows are interleaved (2i gate, 2i+1 up).
+// store in the permuted K order.  Gate/up rows are laid out per block of 128
+// intermediate rows i: 128 gate rows, then the 128 up rows of the same i.
 __global__ void __launch_bounds__(256) sh_convert_kernel(const __nv_bfloat16* g, const __nv_bfloat16* u,
                                                          const __nv_bfloat16* d, const unsigned int* amax,
                                                          __half* shgu16, __half* shdn16, float* sh_scale) {
@@ -216,7 +243,8 @@ __global__ void __launch_bounds__(256) sh_convert_kernel(const __nv_bfloat16* g,
     __half h[8];
 #pragma unroll
     for (int o = 0; o < 8; ++o) h[perm_pos(o)] = __float2half_rn(e[o] * f);
-    __half* dst = m < 2 ? shgu16 + (size_t)(2 * row + m) * kH + k0 : shdn16 + (size_t)row * kI + k0;
+    const int grow = 2 * (row & ~127) + 128 * m + (row & 127);
+    __half* dst = m < 2 ? shgu16 + (size_t)grow * kH + k0 : shdn16 + (size_t)row * kI + k0;
     *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(h);
   }
 }
@@ -231,10 +259,43 @@ cudaError_t launch_tc_prep_shared(const __nv_bfloat16* g, const __nv_bfloat16* u
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- L2 prefetch of a tile
+// Everything one tile reads is contiguous: its 256 weight rows (routed units
+// or fp16 shared rows) and its B rows (positions pos0 .. pos0 + n - 1).
+// Issued for the next tile while the current one runs, so that the cp.async
+// and TMA loads of the main loop find their data in L2.
+template <int MODE>
+__device__ __forceinline__ void prefetch_tile(const TcParams& p, int4 tl, const __half* xg, const __half* h16,
+                                              const __half* shgu16, const __half* shdn16) {
+  const unsigned char* a;
+  size_t abytes;
+  if (tl.x < p.E) {
+    if (MODE == 0) {
+      a = p.gu + ((size_t)tl.x * kGuUnits + (size_t)tl.y * (kTcTileM / 8)) * kGuUnitBytes;
+      abytes = (size_t)(kTcTileM / 8) * kGuUnitBytes;
+    } else {
+      a = p.dn + ((size_t)tl.x * kDnUnits + (size_t)tl.y * (kTcTileM / 4)) * kDnUnitBytes;
+      abytes = (size_t)(kTcTileM / 4) * kDnUnitBytes;
+    }
+  } else {
+    const int K = MODE == 0 ? kH : kI;
+    a = reinterpret_cast<const unsigned char*>((MODE == 0 ? shgu16 : shdn16) + (size_t)tl.y * kTcTileM * K);
+    abytes = (size_t)kTcTileM * K * sizeof(__half);
+  }
+  const size_t rowb = (MODE == 0 ? kH : 2 * kI) * sizeof(__half);
+  const unsigned char* b = reinterpret_cast<const unsigned char*>(MODE == 0 ? xg : h16) + (size_t)tl.z * rowb;
+  const size_t bbytes = (size_t)tl.w * rowb;
+  constexpr size_t kPiece = 32768;
+  for (size_t o = 0; o < abytes; o += kPiece) prefetch_l2_bulk(a + o, (uint32_t)min(kPiece, abytes - o));
+  for (size_t o = 0; o < bbytes; o += kPiece) prefetch_l2_bulk(b + o, (uint32_t)min(kPiece, bbytes - o));
+}
+
 // ---------------------------------------------------------------- the GEMM
-// MODE 0, gate/up: A row r of tile (e, mt) is gate (r even) or up (r odd) of
-// intermediate row i = 128 mt + r/2; B = x rows of the tile's positions; the
-// epilogue writes h = SiLU(g) * u per position as fp16 hi + lo.
+// MODE 0, gate/up: A row r of tile (e, mt) is the gate row (r < 128) or the
+// up row (r >= 128) of intermediate row i = 128 mt + r % 128, so the two
+// M-halves of the accumulator hold g and u for the same i in the same TMEM
+// lane; B = x rows of the tile's positions; the epilogue writes
+// h = SiLU(g) * u per position as fp16 hi + lo.
 // MODE 1, down: A row r is output row 256 mt + r; B = the hi and lo halves of
 // h, both accumulated into one TMEM tile; the epilogue writes y = w (Wd h).
 //
@@ -263,6 +324,7 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
   uint64_t* drain = acce + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  float* fac_s = reinterpret_cast<float*>(smem + tc_bar_off(MODE) + kFacOff);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int4* tiles = MODE == 0 ? p.gu_tiles : p.dn_tiles;
@@ -271,13 +333,13 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full_a[s], kProd);
+      mbar_init(&full_a[s], kProdWarps);
       mbar_init(&full_b[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accf[b], 1);
-      mbar_init(&acce[b], kEpiWarps * 32);
+      mbar_init(&acce[b], kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -300,10 +362,16 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
     const uint32_t raw0 = smem_u32(sRaw);
     // cp.async the codes and the scale word of groups 2kk, 2kk+1 of row r for
     // stage q into raw slot q % R (one commit group per stage, empty or not)
+    int jn = -1;
+    int4 tln = make_int4(0, 0, 0, 0);
     auto issue = [&](int q) {
       if (q < total) {
         const int j = q / NK, kk = q - j * NK;
-        const int4 tl = tiles[blockIdx.x + j * gridDim.x];
+        if (j != jn) {
+          tln = tiles[blockIdx.x + j * gridDim.x];
+          jn = j;
+        }
+        const int4 tl = tln;
         if (tl.x < p.E) {
           const uint32_t slot = raw0 + (q % R) * kRawStage;
 #pragma unroll
@@ -312,8 +380,8 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
             const uint8_t* codes;
             const uint8_t* sword;
             if (MODE == 0) {
-              const int i = (kTcTileM / 2) * tl.y + (r >> 1);
-              const int rin = (r & 1) ? 4 + (i & 3) : (i & 3);
+              const int i = (kTcTileM / 2) * tl.y + (r & 127);
+              const int rin = (r >> 7) ? 4 + (i & 3) : (i & 3);
               const uint8_t* abase = p.gu + ((size_t)tl.x * kGuUnits + (i >> 2)) * kGuUnitBytes;
               const int quarter = G / kGuChunks, jj = G - quarter * kGuChunks, ln = rin + 8 * quarter;
               codes = abase + jj * 512 + 16 * ln;
@@ -346,7 +414,9 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
         jc = j;
       }
       const int s = g % S;
-      if (!tc_wait(&empty[s], ((g / S) & 1) ^ 1, p.err, abort_flag)) break;
+      bool ok = true;
+      if (lane == 0) ok = tc_wait(&empty[s], ((g / S) & 1) ^ 1, p.err, abort_flag);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       if (tl.x < p.E) {
         const unsigned char* slot = sRaw + (g % R) * kRawStage;
         uint4 outv[8];
@@ -370,68 +440,83 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
         for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(a + ((c ^ (r & 7)) << 4)) = outv[c];
         fence_async_smem();
       }
-      mbar_arrive(&full_a[s]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full_a[s]);
     }
     cp_async_wait_all();
   } else if (warp < kMmaWarp) {
     // ------------------------------------------------ epilogue: TMEM lanes 32 qd .. 32 qd + 31
     const int qd = warp & 3;
     const int l = 32 * qd + lane;  // accumulator row within an M-half
+    float* facw = fac_s + (warp - kProdWarps) * (2 * kTcTileN);
 #pragma unroll 1
     for (int j = 0; j < ntl; ++j) {
       const int b = j & 1;
-      if (!tc_wait(&accf[b], (j >> 1) & 1, p.err, abort_flag)) break;
-      tc_fence_after();
       const int4 tl = tiles[blockIdx.x + j * gridDim.x];
       const int mt = tl.y, pos0 = tl.z, n = tl.w, nmma = (n + 15) & ~15;
       const bool shared = tl.x >= p.E;
-#pragma unroll 1
-      for (int mh = 0; mh < 2; ++mh) {
-        const uint32_t tb = tmem + ((uint32_t)(32 * qd) << 16) + (uint32_t)(b * 256 + mh * 128);
+      // per-column factors, fetched while the tile is still accumulating:
+      // gate/up the token's 2^sigma, down the pair's routing weight
+      float* fb = facw + b * kTcTileN;
+      for (int c = lane; c < n; c += 32) {
+        const int pos = pos0 + c;
+        float f;
+        if (MODE == 0) f = p.xscale[shared ? pos - p.P : p.perm[pos] / p.k];
+        else f = shared ? p.sh_scale[2] * (float)(1 << kTcScaleShift) : p.topk_w[p.perm[pos]];
+        fb[c] = f;
+      }
+      __syncwarp();
+      bool ok = true;
+      if (lane == 0) ok = tc_wait(&accf[b], (j >> 1) & 1, p.err, abort_flag);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem + ((uint32_t)(32 * qd) << 16) + (uint32_t)(b * 256);
+      if (MODE == 0) {
+        const int i = (kTcTileM / 2) * mt + l;
+        const int ip = (i & ~7) + perm_pos(i & 7);
+        const float cg = shared ? p.sh_scale[0] : 1.f / (float)(1 << kTcScaleShift);
+        const float cu = shared ? p.sh_scale[1] : 1.f / (float)(1 << kTcScaleShift);
+        __half* hrow = p.h16 + (size_t)pos0 * (2 * kI) + ip;
 #pragma unroll 1
         for (int c0 = 0; c0 < nmma; c0 += 16) {
-          float v[16];
-          tmem_ld16(tb + c0, v);
-          // per-column factor: lane L < 16 fetches it for column c0 + L
-          float fac = 0.f;
-          const int cl = c0 + (lane & 15);
-          if (cl < n) {
-            const int pos = pos0 + cl;
-            if (MODE == 0) fac = p.xscale[shared ? pos - p.P : p.perm[pos] / p.k];
-            else fac = shared ? 1.f : p.topk_w[p.perm[pos]];
-          }
-          if (MODE == 0) {
-            const int rr = mh * 128 + l, i = (kTcTileM / 2) * mt + (rr >> 1);
-            const int ip = (i & ~7) + perm_pos(i & 7);
-            const float cg = shared ? p.sh_scale[0] : 1.f / (float)(1 << kTcScaleShift);
-            const float cu = shared ? p.sh_scale[1] : 1.f / (float)(1 << kTcScaleShift);
+          float g[16], u[16];
+          tmem_ld16x2(tb + c0, tb + 128 + c0, g, u);
 #pragma unroll
-            for (int cc = 0; cc < 16; ++cc) {
-              const float other = __shfl_xor_sync(0xffffffffu, v[cc], 1);
-              const float f = __shfl_sync(0xffffffffu, fac, cc);
-              const int col = c0 + cc;
-              if (!(lane & 1) && col < n) {
-                const float hv = silu_mul(v[cc] * f * cg, other * f * cu) * (1.f / (float)(1 << kTcScaleShift));
-                const __half hi = __float2half_rn(hv);
-                __half* dst = p.h16 + (size_t)(pos0 + col) * (2 * kI) + ip;
-                dst[0] = hi;
-                dst[kI] = __float2half_rn(hv - __half2float(hi));
-              }
+          for (int cc = 0; cc < 16; ++cc) {
+            const int col = c0 + cc;
+            if (col < n) {
+              const float f = fb[col];
+              const float hv = tc_silu_mul(g[cc] * f * cg, u[cc] * f * cu) * (1.f / (float)(1 << kTcScaleShift));
+              const __half hi = __float2half_rn(hv);
+              hrow[(size_t)col * (2 * kI)] = hi;
+              hrow[(size_t)col * (2 * kI) + kI] = __float2half_rn(hv - __half2float(hi));
             }
-          } else {
-            const int nrow = kTcTileM * mt + mh * 128 + l;
-            const float cf = shared ? p.sh_scale[2] * (float)(1 << kTcScaleShift) : 1.f;
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int mh = 0; mh < 2; ++mh) {
+          float* yrow = p.y + (size_t)pos0 * kH + kTcTileM * mt + mh * 128 + l;
+#pragma unroll 1
+          for (int c0 = 0; c0 < nmma; c0 += 32) {
+            float v0[16], v1[16];
+            tmem_ld16x2(tb + mh * 128 + c0, tb + mh * 128 + c0 + 16, v0, v1);
 #pragma unroll
             for (int cc = 0; cc < 16; ++cc) {
-              const float f = __shfl_sync(0xffffffffu, fac, cc);
               const int col = c0 + cc;
-              if (col < n) p.y[(size_t)(pos0 + col) * kH + nrow] = v[cc] * f * cf;
+              if (col < n) yrow[(size_t)col * kH] = v0[cc] * fb[col];
+            }
+#pragma unroll
+            for (int cc = 0; cc < 16; ++cc) {
+              const int col = c0 + 16 + cc;
+              if (col < n) yrow[(size_t)col * kH] = v1[cc] * fb[col];
             }
           }
         }
       }
       tc_fence_before();
-      mbar_arrive(&acce[b]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[b]);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------ MMA issue (one thread)
@@ -479,9 +564,12 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
     if (lane == 0) {
       int g = 0;
       bool ok = true;
+      if (ntl > 0) prefetch_tile<MODE>(p, tiles[blockIdx.x], p.xg, p.h16, p.shgu16, p.shdn16);
 #pragma unroll 1
       for (int j = 0; j < ntl && ok; ++j) {
         const int4 tl = tiles[blockIdx.x + j * gridDim.x];
+        if (j + 1 < ntl)
+          prefetch_tile<MODE>(p, tiles[blockIdx.x + (j + 1) * gridDim.x], p.xg, p.h16, p.shgu16, p.shdn16);
         const int nmma = (tl.w + 15) & ~15, nbox = (nmma + kBoxRows - 1) / kBoxRows;
         const bool shared = tl.x >= p.E;
         const uint32_t bytes = (uint32_t)(NB * nbox * kBoxBytes + (shared ? kStageA : 0));

@@ -36,6 +36,9 @@ struct TcParams {
   const int4* dn_tiles;
   const int32_t* ntiles;    // [0] gate/up tiles, [1] down tiles
   unsigned int* err;        // sticky device error word
+  const __half* xg;         // the buffers behind the tensor maps (for L2 prefetch)
+  const __half* shgu16;
+  const __half* shdn16;
 };
 
 // TMA descriptors: the B operands (x rows by position, h rows by position)
