@@ -159,66 +159,6 @@ __device__ __forceinline__ float dot8_f(const float f[8], float4 a, float4 b, fl
   return acc;
 }
 
-// ---------------------------------------------------------------- top-k
-// Order-preserving key: larger logit first, then smaller index.
-__device__ __forceinline__ unsigned long long topk_key(float v, int idx) {
-  uint32_t u = __float_as_uint(v);
-  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-  return ((unsigned long long)u << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)idx);
-}
-
-// One warp: top-k of logits[0..E) by (value desc, index asc) and the
-// renormalised softmax weights of the kept logits.
-__device__ __forceinline__ void warp_topk(const float* logits, int E, int k, int* out_i, float* out_w) {
-  const int lane = threadIdx.x & 31;
-  constexpr int kPer = kMaxExperts / 32;
-  unsigned long long key[kPer];
-#pragma unroll
-  for (int j = 0; j < kPer; ++j) {
-    const int e = lane + 32 * j;
-    key[j] = (e < E) ? topk_key(ldcg_f32(logits + e), e) : 0ull;
-  }
-  float val[kMaxTopK];
-  int idx[kMaxTopK];
-#pragma unroll
-  for (int r = 0; r < kMaxTopK; ++r) {
-    val[r] = 0.f;
-    idx[r] = 0;
-    if (r < k) {
-      unsigned long long best = 0ull;
-#pragma unroll
-      for (int j = 0; j < kPer; ++j) best = key[j] > best ? key[j] : best;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
-        best = other > best ? other : best;
-      }
-      const int e = (int)(0xFFFFFFFFu - (uint32_t)(best & 0xFFFFFFFFull));
-#pragma unroll
-      for (int j = 0; j < kPer; ++j)
-        if (e == lane + 32 * j) key[j] = 0ull;
-      idx[r] = e;
-      // the value is in the key: undo the order-preserving transform
-      const uint32_t hk = (uint32_t)(best >> 32);
-      val[r] = __uint_as_float((hk & 0x80000000u) ? (hk & 0x7FFFFFFFu) : ~hk);
-    }
-  }
-  if (lane == 0) {
-    const float m = val[0];
-    float sum = 0.f;
-    float ex[kMaxTopK];
-#pragma unroll
-    for (int r = 0; r < kMaxTopK; ++r) {
-      ex[r] = (r < k) ? expf(val[r] - m) : 0.f;
-      sum += ex[r];
-    }
-    const float inv = 1.0f / sum;
-#pragma unroll
-    for (int r = 0; r < kMaxTopK; ++r)
-      if (r < k) { out_i[r] = idx[r]; out_w[r] = ex[r] * inv; }
-  }
-}
-
 // ---------------------------------------------------------------- smem layouts
 // x as fp32 in two planes of 4-float chunks (chunk c = elements 8c..8c+7;
 // plane 0 holds 8c..8c+3, plane 1 holds 8c+4..8c+7), one pad chunk after
@@ -263,13 +203,17 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
       :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
+// The thread sleeps (up to kMbarSuspendNs) until the phase completes instead
+// of returning at once, so waiting warps leave the issue slots to the warps
+// that compute.
+constexpr uint32_t kMbarSuspendNs = 20000;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(kMbarSuspendNs) : "memory");
   return ok != 0;
 }
 // Bounded wait for phase `parity` of the barrier; false (and the sticky error
@@ -366,10 +310,8 @@ __device__ __forceinline__ void dot8_q_f16(const Pairs4& P, uint4 x, float& ae, 
   ao = fma_f16h<1, 1>(P.p3, x.w, ao);  // e7 * x7
 }
 
-// ---------------------------------------------------------------- compact top-k
-// One warp: top-k of logits[0..E) (E <= 512) by (value desc, index asc), with
-// 32-bit order-preserving keys and warp-wide reductions; the renormalised
-// softmax weights of the kept logits.  out_i/out_w/val_s are shared memory.
+// ---------------------------------------------------------------- top-k
+// Order-preserving 32-bit key of a float: larger float, larger key.
 __device__ __forceinline__ uint32_t f32_order_key(float v) {
   const uint32_t u = __float_as_uint(v);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
@@ -377,224 +319,73 @@ __device__ __forceinline__ uint32_t f32_order_key(float v) {
 __device__ __forceinline__ float f32_from_order_key(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
-__device__ __forceinline__ void warp_topk_compact(const float* logits, int E, int k, int* out_i,
-                                                  float* out_w) {
-  const int lane = threadIdx.x & 31;
-  constexpr int kPer = kMaxExperts / 32;
-  uint32_t key[kPer];
-  uint32_t taken = 0;
-#pragma unroll
-  for (int j = 0; j < kPer; ++j) {
-    const int e = lane + 32 * j;
-    key[j] = (e < E) ? f32_order_key(ldcg_f32(logits + e)) : 0u;
-    if (e >= E) taken |= 1u << j;
-  }
-  float m0 = 0.f;
-#pragma unroll 1
-  for (int r = 0; r < k; ++r) {
-    uint32_t lm = 0;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) lm = (!(taken >> j & 1u) && key[j] > lm) ? key[j] : lm;
-    const uint32_t m = __reduce_max_sync(0xffffffffu, lm);
-    uint32_t ec = 0xFFFFFFFFu;
-#pragma unroll
-    for (int j = kPer - 1; j >= 0; --j)
-      if (!(taken >> j & 1u) && key[j] == m) ec = (uint32_t)(lane + 32 * j);
-    const uint32_t e = __reduce_min_sync(0xffffffffu, ec);
-    if ((int)(e & 31u) == lane) taken |= 1u << (e >> 5);
-    const float v = f32_from_order_key(m);
-    if (r == 0) m0 = v;
-    if (lane == 0) {
-      out_i[r] = (int)e;
-      out_w[r] = expf(v - m0);
-    }
-  }
-  __syncwarp();
-  if (lane == 0) {
-    float s = 0.f;
-    for (int r = 0; r < k; ++r) s += out_w[r];
-    const float inv = 1.0f / s;
-    for (int r = 0; r < k; ++r) out_w[r] *= inv;
-  }
-  __syncwarp();
-}
 
-// One warp: top-k of the logits staged in shared memory, by (value desc,
-// index asc); each lane keeps its current best so that only the lane that
-// lost its best rescans.  out_w receives the renormalised softmax weights.
-__device__ __forceinline__ void warp_topk_smem(const float* lg, int E, int k, int* out_i, float* out_w) {
-  const int lane = threadIdx.x & 31;
-  constexpr int kPer = kMaxExperts / 32;
-  uint32_t taken = 0;
-  uint32_t best = 0;
-  int beste = 0x7FFFFFFF;
-  auto rescan = [&]() {
-    best = 0;
-    beste = 0x7FFFFFFF;
-#pragma unroll 4
-    for (int j = 0; j < kPer; ++j) {
-      const int e = lane + 32 * j;
-      if (e < E && !(taken >> j & 1u)) {
-        const uint32_t key = f32_order_key(lg[e]);
-        if (key > best) { best = key; beste = e; }
-      }
-    }
-  };
-  rescan();
-  float m0 = 0.f;
-#pragma unroll 1
-  for (int r = 0; r < k; ++r) {
-    const uint32_t m = __reduce_max_sync(0xffffffffu, best);
-    const uint32_t e = __reduce_min_sync(0xffffffffu, best == m ? (uint32_t)beste : 0xFFFFFFFFu);
-    const float v = f32_from_order_key(m);
-    if (r == 0) m0 = v;
-    if (lane == 0) {
-      out_i[r] = (int)e;
-      out_w[r] = expf(v - m0);
-    }
-    if ((int)(e & 31u) == lane) {
-      taken |= 1u << (e >> 5);
-      rescan();
-    }
-  }
-  __syncwarp();
-  if (lane == 0) {
-    float s = 0.f;
-    for (int r = 0; r < k; ++r) s += out_w[r];
-    const float inv = 1.0f / s;
-    for (int r = 0; r < k; ++r) out_w[r] *= inv;
-  }
-  __syncwarp();
-}
-
-// One warp: top-k (k <= 8) of the logits staged in shared memory (E <= 512),
-// by (value desc, index asc).  Each lane sorts its 16 candidates in
-// registers; k rounds of warp-wide max/min reductions then pop the global
-// best from the head of one lane's list.  out_w receives the renormalised
-// softmax weights of the kept logits.
-__device__ __forceinline__ void warp_topk_sorted(const float* lg, int E, int k, int* out_i, float* out_w) {
-  const int lane = threadIdx.x & 31;
-  constexpr int kPer = kMaxExperts / 32;
-  uint32_t key[kPer];
-  int idx[kPer];
+// One warp: top-k (k <= 8) of lg[0..E) (E <= 512) by (value desc, index asc)
+// and the renormalised softmax weights of the kept logits.
+// Lane l holds entries l, l + 32, ... as order keys (0 marks a removed or
+// absent entry).  Each lane keeps its best entry (largest key, lowest index
+// among equal keys) from a 4-level comparison tree.  A round takes the
+// warp-wide largest key with redux.sync, then the lowest index among the
+// lanes holding it (a second redux.sync on 0xFFFF - index); the owner
+// removes the entry and rebuilds its tree.  Lane r keeps the result of
+// round r.  Lane r < k writes slot r and exp(l_r - l_0) / sum_s exp(l_s - l_0).
+__device__ __forceinline__ void lane_best16(const uint32_t key[16], uint32_t& bk, int& bj) {
+  uint32_t k8[8];
+  int j8[8];
 #pragma unroll
-  for (int j = 0; j < kPer; ++j) {
+  for (int i = 0; i < 8; ++i) {
+    const bool hi = key[2 * i + 1] > key[2 * i];
+    k8[i] = hi ? key[2 * i + 1] : key[2 * i];
+    j8[i] = hi ? 2 * i + 1 : 2 * i;
+  }
+#pragma unroll
+  for (int w = 4; w >= 1; w >>= 1) {
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const bool hi = k8[2 * i + 1] > k8[2 * i];
+      k8[i] = hi ? k8[2 * i + 1] : k8[2 * i];
+      j8[i] = hi ? j8[2 * i + 1] : j8[2 * i];
+    }
+  }
+  bk = k8[0];
+  bj = j8[0];
+}
+__device__ __forceinline__ void warp_topk_fast(const float* lg, int E, int k, int* out_i, float* out_w) {
+  const int lane = threadIdx.x & 31;
+  uint32_t key[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
     const int e = lane + 32 * j;
     key[j] = (e < E) ? f32_order_key(lg[e]) : 0u;
-    idx[j] = (e < E) ? e : 0x7FFFFFFF;
   }
-  // odd-even transposition sort, descending by (key, -idx)
-#pragma unroll
-  for (int pass = 0; pass < kPer; ++pass) {
-#pragma unroll
-    for (int j = pass & 1; j + 1 < kPer; j += 2) {
-      const bool sw = key[j + 1] > key[j] || (key[j + 1] == key[j] && idx[j + 1] < idx[j]);
-      const uint32_t ka = key[j], kb = key[j + 1];
-      const int ia = idx[j], ib = idx[j + 1];
-      key[j] = sw ? kb : ka;
-      key[j + 1] = sw ? ka : kb;
-      idx[j] = sw ? ib : ia;
-      idx[j + 1] = sw ? ia : ib;
-    }
-  }
-  float m0 = 0.f;
+  uint32_t bk;
+  int bj;
+  lane_best16(key, bk, bj);
+  uint32_t mine_k = 0u;
+  int mine_i = 0;
 #pragma unroll 1
   for (int r = 0; r < k; ++r) {
-    const uint32_t m = __reduce_max_sync(0xffffffffu, key[0]);
-    const uint32_t e = __reduce_min_sync(0xffffffffu, key[0] == m ? (uint32_t)idx[0] : 0xFFFFFFFFu);
-    const float v = f32_from_order_key(m);
-    if (r == 0) m0 = v;
-    if (lane == 0) {
-      out_i[r] = e < (uint32_t)E ? (int)e : 0;  // only a NaN logit could select past the end
-      out_w[r] = expf(v - m0);
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    const uint32_t cand = (bk == m) ? 0xFFFFu - (uint32_t)(lane + 32 * bj) : 0u;
+    const uint32_t c = __reduce_max_sync(0xffffffffu, cand);
+    const int idx = (int)(0xFFFFu - c);
+    if (lane == r) {
+      mine_k = m;
+      mine_i = idx;
     }
-    if ((uint32_t)idx[0] == e) {  // pop the head
+    const int kj = (lane == (idx & 31)) ? (idx >> 5) : -1;  // the owner's entry
 #pragma unroll
-      for (int j = 0; j + 1 < kPer; ++j) {
-        key[j] = key[j + 1];
-        idx[j] = idx[j + 1];
-      }
-      key[kPer - 1] = 0u;
-      idx[kPer - 1] = 0x7FFFFFFF;
-    }
+    for (int j = 0; j < 16; ++j) key[j] = (j == kj) ? 0u : key[j];
+    if (kj >= 0) lane_best16(key, bk, bj);
   }
-  __syncwarp();
-  if (lane == 0) {
-    float s = 0.f;
-    for (int r = 0; r < k; ++r) s += out_w[r];
-    const float inv = 1.0f / s;
-    for (int r = 0; r < k; ++r) out_w[r] *= inv;
-  }
-  __syncwarp();
-}
-
-// One warp: top-k (k <= 8) of E <= 512 logits, by (value desc, index asc).
-// 64-bit keys (order-preserving value bits, then the complemented index)
-// make every key distinct.  Each lane sorts its 16 keys with a bitonic
-// network; a 5-level butterfly then merges sorted top-8 lists between lanes
-// (each level keeps the top 8 of the lane's and its partner's lists), after
-// which every lane holds the global top-8.  Lane r < k writes slot r and its
-// renormalised softmax weight.  No sequential selection rounds.
-__device__ __forceinline__ void cx_desc(unsigned long long& a, unsigned long long& b) {
-  const unsigned long long hi = a > b ? a : b;
-  const unsigned long long lo = a > b ? b : a;
-  a = hi;
-  b = lo;
-}
-__device__ __forceinline__ void warp_topk_bitonic(const float* lg, int E, int k, int* out_i, float* out_w) {
-  const int lane = threadIdx.x & 31;
-  constexpr int kPer = kMaxExperts / 32;  // 16
-  unsigned long long v[kPer];
-#pragma unroll
-  for (int j = 0; j < kPer; ++j) {
-    const int e = lane + 32 * j;
-    v[j] = (e < E) ? (((unsigned long long)f32_order_key(lg[e]) << 32) | (0xFFFFFFFFu - (uint32_t)e)) : 0ull;
-  }
-  // bitonic sort of 16, descending
-#pragma unroll
-  for (int size = 2; size <= kPer; size <<= 1) {
-#pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-#pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int j = i ^ stride;
-        if (j > i) {
-          if ((i & size) == 0) cx_desc(v[i], v[j]);
-          else cx_desc(v[j], v[i]);
-        }
-      }
-    }
-  }
-  // butterfly merge of the sorted top-8 lists
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    unsigned long long o[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) o[i] = __shfl_xor_sync(0xffffffffu, v[7 - i], d);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = v[i] > o[i] ? v[i] : o[i];
-#pragma unroll
-    for (int stride = 4; stride > 0; stride >>= 1) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int j = i ^ stride;
-        if (j > i) cx_desc(v[i], v[j]);
-      }
-    }
-  }
-  unsigned long long mine = v[0];
-#pragma unroll
-  for (int i = 1; i < 8; ++i)
-    if (lane == i) mine = v[i];
-  const float vmax = f32_from_order_key((uint32_t)(v[0] >> 32));
-  const float vr = f32_from_order_key((uint32_t)(mine >> 32));
+  const float vmax = f32_from_order_key(__shfl_sync(0xffffffffu, mine_k, 0));
+  const float vr = f32_from_order_key(mine_k);
   const float ex = (lane < k) ? expf(vr - vmax) : 0.f;
   float s = ex;
 #pragma unroll
   for (int o = 4; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if (lane < k) {
-    const uint32_t e = 0xFFFFFFFFu - (uint32_t)(mine & 0xFFFFFFFFull);
-    out_i[lane] = e < (uint32_t)E ? (int)e : 0;  // only a NaN logit could select past the end
+    out_i[lane] = mine_i < E ? mine_i : 0;  // only a NaN logit could select past the end
     out_w[lane] = ex / s;
   }
   __syncwarp();

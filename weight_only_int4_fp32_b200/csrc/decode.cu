@@ -16,9 +16,13 @@
 // one private buffer and mbarrier per warp; each warp issues the copy of its
 // next item before it waits, and the compute loops read the staged bytes with
 // conflict-free 16-byte shared loads.  Bytes that do not depend on the
-// routing (shared expert) are requested first; routed down weights are
-// prefetched into L2 as soon as the routing is known and copied into shared
-// memory while the CTA waits at the last grid barrier.
+// routing (shared expert) are requested first.  A routed gate/up unit is
+// copied in four pieces with one mbarrier each, so its dot products start
+// when the first piece lands.  For one token the CTA's routed down units are
+// copied into a dedicated shared-memory region as soon as the routing is
+// known (they land during the gate/up phase); otherwise they are prefetched
+// into L2 then and copied in batches while the CTA waits at the last grid
+// barrier.
 //
 // Layer definition: vLLM recipe page "inclusionAI/Ling-3.0-flash" (Overview;
 // "Single-GPU int4": symmetric W4, group 32, routed experts only) and the
@@ -32,7 +36,17 @@ namespace lingmoe {
 // Optional phase timestamps (compile with -DLING_MOE_TRACE): thread 0 of
 // every CTA records %globaltimer at each phase boundary.
 #ifdef LING_MOE_TRACE
+__device__ float g_sink;
+__device__ __forceinline__ void g_clk_sink(float v) { if (v == 12345.f) g_sink = v; }
 __device__ unsigned long long g_trace[1024][16];
+__device__ long long g_clk[16];
+#define LING_CLK(slot) \
+  do { if (blockIdx.x == 0 && threadIdx.x == 0) g_clk[slot] = clock64(); } while (0)
+#else
+#define LING_CLK(slot) do { } while (0)
+__device__ __forceinline__ void g_clk_sink(float) {}
+#endif
+#ifdef LING_MOE_TRACE
 #define LING_TRACE(slot) \
   do { if (threadIdx.x == 0) g_trace[blockIdx.x][slot] = globaltimer_ns(); } while (0)
 #else
@@ -45,13 +59,17 @@ constexpr int kDnBatch = 4;                         // routed down units per cop
 constexpr int kBufB = kDnBatch * kDnUnitBytes;      // per-warp buffer, phase 4
 constexpr int kShDnBytes = 4 * kI * 2;              // 4 shared-down rows
 constexpr int kMaxBlkPerCta = 8;                    // down row-blocks per CTA (>= 640 / nctas)
+constexpr int kDnPrefBlk = 5;                       // T = 1: routed down units kept in shared memory
+                                                    // when the CTA has <= 5 row-blocks (>= 128 CTAs)
+constexpr int kGuPiece = kGuScaleOff / 4;           // 2560 B: 5 chunks of a gate/up unit
 constexpr int kRowBytes = kH * 2;                   // one bf16 row of H
 static_assert(kBufB >= kShDnBytes, "phase-4 buffer holds a shared-down block");
 static_assert(kBufA >= 2 * kRowBytes, "phase-1/2 buffer holds a gate and an up row");
 
 struct __align__(16) SmemHeader {
-  uint64_t mbar[kWarps][2];
+  uint64_t mbar[kWarps][4];
   uint64_t xbar;
+  uint64_t dbar;
   uint32_t xmax[kMaxDecodeT];
   float xscale[kMaxDecodeT];
   int xinf;
@@ -62,7 +80,7 @@ struct __align__(16) SmemHeader {
   int uniq_cnt[kMaxDecodeT * kMaxTopK];
   int uniq_pair[kMaxDecodeT * kMaxTopK][kMaxDecodeT];
   int nuniq;
-  int flag;
+  int dcopies;  // T = 1: routed down copies into the dedicated region were issued
   int abort;
   int pad[3];
 };
@@ -92,10 +110,13 @@ struct Plan {
   static constexpr size_t part = hs + (size_t)T * kHsTok * 4;               // float [blk][P + T][4]
   static constexpr size_t bufB = part + (size_t)kMaxBlkPerCta * (P + T) * 16;
   static constexpr size_t endB = bufB + (size_t)kWarps * kBufB;
-  static constexpr size_t body = endA > endB ? endA : endB;
+  static constexpr size_t endAB = endA > endB ? endA : endB;
+  // T = 1: the CTA's routed down units, [expert slot][row-block] x 1728 B
+  static constexpr size_t dn = endAB;
+  static constexpr size_t body = dn + (T == 1 ? (size_t)kMaxTopK * kDnPrefBlk * kDnUnitBytes : 0);
   static constexpr size_t bytes = sizeof(SmemHeader) + body;
   static_assert(xh % 16 == 0 && cg % 16 == 0 && bufA % 16 == 0 && bufB % 16 == 0 && chp % 16 == 0 &&
-                hs % 16 == 0 && part % 16 == 0, "16-byte aligned regions");
+                hs % 16 == 0 && part % 16 == 0 && dn % 16 == 0, "16-byte aligned regions");
   static_assert(bytes <= 227 * 1024, "decode smem over budget");
 };
 
@@ -156,9 +177,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   const int nblk = b1 - b0;
   const int nr = r1 - r0, n12 = nr + (s1 - s0);
 
-  uint64_t* barA = &hd.mbar[warp][0];
-  uint64_t* barB = &hd.mbar[warp][1];
-  uint32_t pha = 0, phb = 0;
+  uint64_t* barA = &hd.mbar[warp][0];  // phases 1-2 items, piece 0 of a gate/up unit, phase-4 copies
+  uint32_t pha = 0, phq = 0;           // phq: parity of pieces 1-3 (always used together)
+  const bool use_d = (T == 1) && nblk <= kDnPrefBlk;
   unsigned char* bufA = body + PL::bufA + (size_t)warp * kBufA;
   unsigned char* bufB = body + PL::bufB + (size_t)warp * kBufB;
   unsigned char* xb = body + PL::xb;
@@ -171,14 +192,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   if (tid == 0) {
     hd.abort = 0;
     hd.xinf = 0;
+    hd.dcopies = 0;
     mbar_init(&hd.xbar, 1);
+    mbar_init(&hd.dbar, 1);
     fence_mbar_init();
     mbar_arrive_expect_tx(&hd.xbar, T * kXbTok);
     bulk_g2s(xb, p.x, T * kXbTok, &hd.xbar);
   }
   if (lane == 0) {
-    mbar_init(barA, 1);
-    mbar_init(barB, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&hd.mbar[warp][i], 1);
     fence_mbar_init();
   }
   __syncthreads();  // barriers initialised before anyone waits on them
@@ -206,142 +228,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   // x (bf16) lands in shared memory; every warp waits for it once
   if (!mbar_wait(&hd.xbar, 0, p.wait_limit_ns, p.err)) hd.abort = 1;
   LING_TRACE(1);
-
-  // ---- phases 1+2: router rows (published at once) and shared gate/up rows
-  for (int it = warp; it < n12; it += kWarps) {
-    if (it != warp) issue12(it);
-    if (!mbar_wait(barA, pha, p.wait_limit_ns, p.err)) { hd.abort = 1; break; }
-    pha ^= 1;
-    const bool router = it < nr;
-    float a0[T], a1[T];
-    {
-      float g0[T], g1[T], g2[T], g3[T], u0_[T], u1_[T], u2_[T], u3_[T];
-#pragma unroll
-      for (int t = 0; t < T; ++t) g0[t] = g1[t] = g2[t] = g3[t] = u0_[t] = u1_[t] = u2_[t] = u3_[t] = 0.f;
-#pragma unroll
-      for (int m = 0; m < kXChunks / 32; m += 2) {
-        const int c0 = lane + 32 * m, c1 = c0 + 32;
-        const uint4 w00 = lds128(bufA + 16 * c0), w01 = lds128(bufA + 16 * c1);
-        const uint4 w10 = router ? w00 : lds128(bufA + kRowBytes + 16 * c0);
-        const uint4 w11 = router ? w01 : lds128(bufA + kRowBytes + 16 * c1);
-#pragma unroll
-        for (int t = 0; t < T; ++t) {
-          const uint4 xv0 = lds128(xb + t * kXbTok + 16 * c0), xv1 = lds128(xb + t * kXbTok + 16 * c1);
-          dot8_bf16_bf16_2(w00, xv0, g0[t], g1[t]);
-          dot8_bf16_bf16_2(w01, xv1, g2[t], g3[t]);
-          if (!router) {
-            dot8_bf16_bf16_2(w10, xv0, u0_[t], u1_[t]);
-            dot8_bf16_bf16_2(w11, xv1, u2_[t], u3_[t]);
-          }
-        }
-      }
-#pragma unroll
-      for (int t = 0; t < T; ++t) {
-        a0[t] = (g0[t] + g1[t]) + (g2[t] + g3[t]);
-        a1[t] = (u0_[t] + u1_[t]) + (u2_[t] + u3_[t]);
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < T; ++t) {
-      const float g = warp_sum(a0[t]);
-      if (router) {
-        if (lane == 0) p.logits[(size_t)t * E + r0 + it] = g + (p.router_bias ? p.router_bias[r0 + it] : 0.f);
-      } else {
-        const float u = warp_sum(a1[t]);
-        if (lane == 0) p.h_s[(size_t)t * kI + s0 + it - nr] = silu_mul(g, u);
-      }
-    }
-    if (lane == 0 && !(router && withhold)) arrive(p.sync + (router ? 0 : 1));
-    __syncwarp();
-  }
-  LING_TRACE(2);
-
-  LING_TRACE(10);
-  // ---- routing: every CTA selects the top-k itself from the published logits
-  if (warp < T && !aborted(hd)) {
-    float* lg = reinterpret_cast<float*>(bufA);  // scratch: this warp's buffer is idle here
-    bool ok = true;
-    if (lane == 0) ok = wait_count(p.sync + 0, (uint32_t)E, p.wait_limit_ns, p.err, &hd.abort);
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (warp == 0) LING_TRACE(11);
-    if (ok) {
-      const float* src = p.logits + (size_t)warp * E;
-#pragma unroll
-      for (int j = 0; j < kMaxExperts / 32; ++j)
-        if (lane + 32 * j < E) lg[lane + 32 * j] = ldcg_f32(src + lane + 32 * j);
-    }
-    __syncwarp();
-    if (warp == 0) LING_TRACE(12);
-    warp_topk_bitonic(lg, E, K, hd.topi[warp], hd.topw[warp]);
-  }
-  __syncthreads();
-  LING_TRACE(3);
-  if (T == 1) {
-    // one token: the selected experts are already distinct
-    if (tid < K) {
-      hd.uniq_e[tid] = hd.topi[0][tid];
-      hd.uniq_cnt[tid] = 1;
-      hd.uniq_pair[tid][0] = tid;
-      if (cta == 0) {
-        if (p.topk_idx_out) p.topk_idx_out[tid] = hd.topi[0][tid];
-        if (p.topk_w_out) p.topk_w_out[tid] = hd.topw[0][tid];
-      }
-    }
-    if (tid == 0) hd.nuniq = K;
-  } else if (warp == 0 && !aborted(hd)) {
-    // union of the selected experts, in first-occurrence order (t-major)
-    const int npairs = T * K;
-    const int pe = (lane < npairs) ? hd.topi[lane / K][lane % K] : -1 - lane;
-    bool first = lane < npairs;
-    for (int j = 0; j < npairs; ++j) {
-      const int ej = __shfl_sync(0xffffffffu, pe, j);
-      if (j < lane && ej == pe) first = false;
-    }
-    const unsigned fm = __ballot_sync(0xffffffffu, first);
-    const int myu = first ? __popc(fm & ((1u << lane) - 1u)) : -1;
-    if (first) hd.uniq_e[myu] = pe;
-    int cnt = 0;
-    for (int j = 0; j < npairs; ++j) {
-      const int ej = __shfl_sync(0xffffffffu, pe, j);
-      if (first && ej == pe) hd.uniq_pair[myu][cnt++] = j;
-    }
-    if (first) hd.uniq_cnt[myu] = cnt;
-    if (lane == 0) hd.nuniq = __popc(fm);
-    if (cta == 0 && lane < npairs) {
-      const int t = lane / K, s = lane % K;
-      if (p.topk_idx_out) p.topk_idx_out[lane] = hd.topi[t][s];
-      if (p.topk_w_out) p.topk_w_out[lane] = hd.topw[t][s];
-    }
-  }
-  __syncthreads();
-  const int U = aborted(hd) ? 0 : hd.nuniq;
-  LING_TRACE(4);
-
-  // ---- phase 3: routed gate/up units, each copied in two halves
-  const int n3 = U * kGuUnits;
-  const int u0 = (int)((long long)cta * n3 / ncta), u1 = (int)((long long)(cta + 1) * n3 / ncta);
-  auto issue3 = [&](int unit) {
-    if (lane == 0) {
-      const int u = unit / kGuUnits, b = unit - u * kGuUnits;
-      const uint8_t* src = p.gu + ((size_t)hd.uniq_e[u] * kGuUnits + b) * kGuUnitBytes;
-      constexpr int kHalf = kGuScaleOff / 2;
-      mbar_arrive_expect_tx(barA, kHalf + (kGuUnitBytes - kGuScaleOff));
-      bulk_g2s(bufA + kGuScaleOff, src + kGuScaleOff, kGuUnitBytes - kGuScaleOff, barA);
-      bulk_g2s(bufA, src, kHalf, barA);
-      mbar_arrive_expect_tx(barB, kHalf);
-      bulk_g2s(bufA + kHalf, src + kHalf, kHalf, barB);
-    }
-  };
-  if (u0 + warp < u1) issue3(u0 + warp);
-  // routed down units of this CTA (contiguous per expert) into L2
-  if (warp == kWarps - 1 && nblk > 0) {
-    for (int u = lane; u < U; u += 32) {
-      const uint8_t* src = p.dn + ((size_t)hd.uniq_e[u] * kDnUnits + b0) * kDnUnitBytes;
-      prefetch_l2_bulk(src, (uint32_t)nblk * kDnUnitBytes);
-    }
-  }
   // fp16 copy of x and the per-group bias constants of the int4 dot products,
-  // built while the first units are in flight: 4 lanes per group of 32.  x is
+  // built as soon as x lands (the first weight rows are still in flight):
+  // 4 lanes per group of 32.  x is
   // converted as is (exact for normal bf16 values below 65504); if any value
   // overflows fp16, the token is redone scaled by 2^-sigma.
   auto build_xh = [&]() {
@@ -403,6 +292,166 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   }
   LING_TRACE(15);
 
+  // ---- phases 1+2: router rows (published at once) and shared gate/up rows
+  for (int it = warp; it < n12; it += kWarps) {
+    if (it != warp) issue12(it);
+    if (!mbar_wait(barA, pha, p.wait_limit_ns, p.err)) { hd.abort = 1; break; }
+    pha ^= 1;
+    const bool router = it < nr;
+    float a0[T], a1[T];
+    {
+      float g0[T], g1[T], g2[T], g3[T], u0_[T], u1_[T], u2_[T], u3_[T];
+#pragma unroll
+      for (int t = 0; t < T; ++t) g0[t] = g1[t] = g2[t] = g3[t] = u0_[t] = u1_[t] = u2_[t] = u3_[t] = 0.f;
+#pragma unroll
+      for (int m = 0; m < kXChunks / 32; m += 2) {
+        const int c0 = lane + 32 * m, c1 = c0 + 32;
+        const uint4 w00 = lds128(bufA + 16 * c0), w01 = lds128(bufA + 16 * c1);
+        const uint4 w10 = router ? w00 : lds128(bufA + kRowBytes + 16 * c0);
+        const uint4 w11 = router ? w01 : lds128(bufA + kRowBytes + 16 * c1);
+#pragma unroll
+        for (int t = 0; t < T; ++t) {
+          const uint4 xv0 = lds128(xb + t * kXbTok + 16 * c0), xv1 = lds128(xb + t * kXbTok + 16 * c1);
+          dot8_bf16_bf16_2(w00, xv0, g0[t], g1[t]);
+          dot8_bf16_bf16_2(w01, xv1, g2[t], g3[t]);
+          if (!router) {
+            dot8_bf16_bf16_2(w10, xv0, u0_[t], u1_[t]);
+            dot8_bf16_bf16_2(w11, xv1, u2_[t], u3_[t]);
+          }
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < T; ++t) {
+        a0[t] = (g0[t] + g1[t]) + (g2[t] + g3[t]);
+        a1[t] = (u0_[t] + u1_[t]) + (u2_[t] + u3_[t]);
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+      const float g = warp_sum(a0[t]);
+      if (router) {
+        if (lane == 0) p.logits[(size_t)t * E + r0 + it] = g + (p.router_bias ? p.router_bias[r0 + it] : 0.f);
+      } else {
+        const float u = warp_sum(a1[t]);
+        if (lane == 0) p.h_s[(size_t)t * kI + s0 + it - nr] = silu_mul(g, u);
+      }
+    }
+    if (lane == 0 && !(router && withhold)) arrive(p.sync + (router ? 0 : 1));
+    __syncwarp();
+  }
+  LING_TRACE(2);
+
+  LING_TRACE(10);
+  // All warps leave phases 1-2 together, so that the selecting warps run
+  // alone: with other warps still streaming shared-memory dot products, the
+  // shuffle/reduction-bound selection was measured ~3x slower.  The shared
+  // rows finish before the router counter completes, so this costs nothing.
+  __syncthreads();
+  // ---- routing: every CTA selects the top-k itself from the published logits
+  if (warp < T && !aborted(hd)) {
+    float* lg = reinterpret_cast<float*>(bufA);  // scratch: this warp's buffer is idle here
+    bool ok = true;
+    if (lane == 0) ok = wait_count(p.sync + 0, (uint32_t)E, p.wait_limit_ns, p.err, &hd.abort);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (warp == 0) LING_TRACE(11);
+    if (warp == 0) LING_CLK(0);
+    if (ok) {
+      // all 16 loads in flight before the first shared store (the compiler
+      // cannot tell the two pointers apart and would otherwise serialise them)
+      const float* src = p.logits + (size_t)warp * E;
+      float v[kMaxExperts / 32];
+#pragma unroll
+      for (int j = 0; j < kMaxExperts / 32; ++j) v[j] = (lane + 32 * j < E) ? ldcg_f32(src + lane + 32 * j) : 0.f;
+#pragma unroll
+      for (int j = 0; j < kMaxExperts / 32; ++j)
+        if (lane + 32 * j < E) lg[lane + 32 * j] = v[j];
+    }
+    __syncwarp();
+    if (warp == 0) LING_TRACE(12);
+    if (warp == 0) { LING_CLK(1); if (lane == 0) g_clk_sink(lg[0] + lg[E - 1]); LING_CLK(2); }
+    warp_topk_fast(lg, E, K, hd.topi[warp], hd.topw[warp]);
+    if (warp == 0) LING_CLK(3);
+    if (warp == 0) LING_TRACE(4);
+  }
+  __syncthreads();
+  LING_TRACE(3);
+  if (T == 1) {
+    // one token: the selected experts are already distinct
+    if (tid < K) {
+      hd.uniq_e[tid] = hd.topi[0][tid];
+      hd.uniq_cnt[tid] = 1;
+      hd.uniq_pair[tid][0] = tid;
+      if (cta == 0) {
+        if (p.topk_idx_out) p.topk_idx_out[tid] = hd.topi[0][tid];
+        if (p.topk_w_out) p.topk_w_out[tid] = hd.topw[0][tid];
+      }
+    }
+    if (tid == 0) hd.nuniq = K;
+  } else if (warp == 0 && !aborted(hd)) {
+    // union of the selected experts, in first-occurrence order (t-major)
+    const int npairs = T * K;
+    const int pe = (lane < npairs) ? hd.topi[lane / K][lane % K] : -1 - lane;
+    bool first = lane < npairs;
+    for (int j = 0; j < npairs; ++j) {
+      const int ej = __shfl_sync(0xffffffffu, pe, j);
+      if (j < lane && ej == pe) first = false;
+    }
+    const unsigned fm = __ballot_sync(0xffffffffu, first);
+    const int myu = first ? __popc(fm & ((1u << lane) - 1u)) : -1;
+    if (first) hd.uniq_e[myu] = pe;
+    int cnt = 0;
+    for (int j = 0; j < npairs; ++j) {
+      const int ej = __shfl_sync(0xffffffffu, pe, j);
+      if (first && ej == pe) hd.uniq_pair[myu][cnt++] = j;
+    }
+    if (first) hd.uniq_cnt[myu] = cnt;
+    if (lane == 0) hd.nuniq = __popc(fm);
+    if (cta == 0 && lane < npairs) {
+      const int t = lane / K, s = lane % K;
+      if (p.topk_idx_out) p.topk_idx_out[lane] = hd.topi[t][s];
+      if (p.topk_w_out) p.topk_w_out[lane] = hd.topw[t][s];
+    }
+  }
+  __syncthreads();
+  const int U = aborted(hd) ? 0 : hd.nuniq;
+
+  // ---- phase 3: routed gate/up units, each copied in four pieces (the scales
+  // travel with piece 0)
+  const int n3 = U * kGuUnits;
+  const int u0 = (int)((long long)cta * n3 / ncta), u1 = (int)((long long)(cta + 1) * n3 / ncta);
+  auto issue3 = [&](int unit) {
+    if (lane == 0) {
+      const int u = unit / kGuUnits, b = unit - u * kGuUnits;
+      const uint8_t* src = p.gu + ((size_t)hd.uniq_e[u] * kGuUnits + b) * kGuUnitBytes;
+      mbar_arrive_expect_tx(barA, kGuPiece + (kGuUnitBytes - kGuScaleOff));
+      bulk_g2s(bufA + kGuScaleOff, src + kGuScaleOff, kGuUnitBytes - kGuScaleOff, barA);
+      bulk_g2s(bufA, src, kGuPiece, barA);
+      for (int pc = 1; pc < 4; ++pc) {
+        mbar_arrive_expect_tx(&hd.mbar[warp][pc], kGuPiece);
+        bulk_g2s(bufA + pc * kGuPiece, src + pc * kGuPiece, kGuPiece, &hd.mbar[warp][pc]);
+      }
+    }
+  };
+  if (u0 + warp < u1) issue3(u0 + warp);
+  if (use_d) {
+    // T = 1: this CTA's routed down units, one contiguous copy per expert
+    if (warp == kWarps - 1 && U > 0 && !aborted(hd)) {
+      const uint32_t per = (uint32_t)nblk * kDnUnitBytes;
+      if (lane == 0) mbar_arrive_expect_tx(&hd.dbar, per * (uint32_t)U);
+      __syncwarp();
+      if (lane < U)
+        bulk_g2s(body + PL::dn + (size_t)lane * per,
+                 p.dn + ((size_t)hd.uniq_e[lane] * kDnUnits + b0) * kDnUnitBytes, per, &hd.dbar);
+      if (lane == 0) hd.dcopies = 1;
+    }
+  } else if (warp == kWarps - 1 && nblk > 0) {
+    // routed down units of this CTA (contiguous per expert) into L2
+    for (int u = lane; u < U; u += 32) {
+      const uint8_t* src = p.dn + ((size_t)hd.uniq_e[u] * kDnUnits + b0) * kDnUnitBytes;
+      prefetch_l2_bulk(src, (uint32_t)nblk * kDnUnitBytes);
+    }
+  }
+
   {
     const int r = lane & 7, q = lane >> 3;
     for (int unit = u0 + warp; unit < u1; unit += kWarps) {
@@ -423,43 +472,50 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       for (int tt = 0; tt < T; ++tt) acc[tt] = 0.f;
       bool ok = mbar_wait(barA, pha, p.wait_limit_ns, p.err);
       pha ^= 1;
-      if (warp == 0 && unit == u0) LING_TRACE(13);
+      if (warp == 0 && unit == u0) { LING_TRACE(13); LING_CLK(6); }
+      // four pieces of 5 chunks; the chunks of a piece are unrolled so that
+      // their loads and FMA chains overlap
 #pragma unroll 1
-      for (int j = 0; j < kGuChunks && ok; ++j) {
-        if (j == kGuChunks / 2) {
-          ok = mbar_wait(barB, phb, p.wait_limit_ns, p.err);
+      for (int pc = 0; pc < 4 && ok; ++pc) {
+        if (pc > 0) {
+          ok = mbar_wait(&hd.mbar[warp][pc], phq, p.wait_limit_ns, p.err);
           if (!ok) break;
+          if (warp == 0 && unit == u0) LING_CLK(6 + pc);
         }
-        const uint4 w = lds128(bufA + j * 512 + 16 * lane);
-        const float s = bf16_to_f32(*reinterpret_cast<const unsigned short*>(
-            bufA + kGuScaleOff + (j >> 2) * 256 + 8 * lane + 2 * (j & 3)));
-        float ae[T], ao[T], be[T], bo[T];
 #pragma unroll
-        for (int tt = 0; tt < T; ++tt) {
-          const float2 c2 = (tt < cnt) ? cg[co[tt] + j] : make_float2(0.f, 0.f);
-          ae[tt] = c2.x;
-          ao[tt] = c2.y;
-          be[tt] = 0.f;
-          bo[tt] = 0.f;
-        }
-        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const Pairs4 P = dequant_f16x2(wv[i]);
+        for (int jj = 0; jj < kGuChunks / 4; ++jj) {
+          const int j = pc * (kGuChunks / 4) + jj;
+          const uint4 w = lds128(bufA + j * 512 + 16 * lane);
+          const float s = bf16_to_f32(*reinterpret_cast<const unsigned short*>(
+              bufA + kGuScaleOff + (j >> 2) * 256 + 8 * lane + 2 * (j & 3)));
+          float ae[T], ao[T], be[T], bo[T];
 #pragma unroll
           for (int tt = 0; tt < T; ++tt) {
-            if (tt < cnt) {
-              const uint4 xv = lds128(xh + xo[tt] + 64 * j + 16 * i);
-              if (i & 1) dot8_q_f16(P, xv, be[tt], bo[tt]);
-              else dot8_q_f16(P, xv, ae[tt], ao[tt]);
+            const float2 c2 = (tt < cnt) ? cg[co[tt] + j] : make_float2(0.f, 0.f);
+            ae[tt] = c2.x;
+            ao[tt] = c2.y;
+            be[tt] = 0.f;
+            bo[tt] = 0.f;
+          }
+          const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const Pairs4 P = dequant_f16x2(wv[i]);
+#pragma unroll
+            for (int tt = 0; tt < T; ++tt) {
+              if (tt < cnt) {
+                const uint4 xv = lds128(xh + xo[tt] + 64 * j + 16 * i);
+                if (i & 1) dot8_q_f16(P, xv, be[tt], bo[tt]);
+                else dot8_q_f16(P, xv, ae[tt], ao[tt]);
+              }
             }
           }
-        }
 #pragma unroll
-        for (int tt = 0; tt < T; ++tt)
-          acc[tt] = fmaf(s, fmaf(0.0625f, ao[tt] + bo[tt], ae[tt] + be[tt]), acc[tt]);
+          for (int tt = 0; tt < T; ++tt)
+            acc[tt] = fmaf(s, fmaf(0.0625f, ao[tt] + bo[tt], ae[tt] + be[tt]), acc[tt]);
+        }
       }
-      phb ^= 1;
+      phq ^= 1;
       if (!ok) { hd.abort = 1; break; }
       __syncwarp();
 #pragma unroll
@@ -476,7 +532,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       }
       __syncwarp();
       if (lane == 0) arrive(p.sync + 2);
-      if (warp == 0 && unit == u0) LING_TRACE(14);
+      if (warp == 0 && unit == u0) { LING_TRACE(14); LING_CLK(10); }
     }
   }
   __syncthreads();
@@ -486,7 +542,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   // Region A is free now; start this warp's first phase-4 copy before waiting.
   const int npairs = T * K;
   const int nitems = nblk * U;
-  const int nbatch = (nitems + kDnBatch - 1) / kDnBatch;
+  const int nbatch = use_d ? 0 : (nitems + kDnBatch - 1) / kDnBatch;
   const int nmine_r = warp < nbatch ? (nbatch - warp + kWarps - 1) / kWarps : 0;
   const int sh_first = kWarps - 1 - warp;
   const int nmine_s = (!aborted(hd) && sh_first < nblk) ? (nblk - sh_first + kWarps - 1) / kWarps : 0;
@@ -556,6 +612,74 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   __syncthreads();
   LING_TRACE(7);
 
+  // one routed down unit (4 output rows of expert slot u, row-block blk):
+  // partial sums per pair into part[], weighted by the routing weight
+  auto down_item = [&](const unsigned char* base, int blk, int u) {
+    const int r = lane & 3, q = lane >> 2;
+    const int cnt = hd.uniq_cnt[u];
+    int ho[T], co[T];
+#pragma unroll
+    for (int tt = 0; tt < T; ++tt) {
+      const int pr = (tt < cnt) ? hd.uniq_pair[u][tt] : 0;
+      ho[tt] = pr * kHpStride + 100 * q;
+      co[tt] = pr * kHGroups + q * kDnChunks;
+    }
+    float acc[T];
+#pragma unroll
+    for (int tt = 0; tt < T; ++tt) acc[tt] = 0.f;
+#pragma unroll
+    for (int j = 0; j < kDnChunks; ++j) {
+      const uint4 w = lds128(base + j * 512 + 16 * lane);
+      const float sj = bf16_to_f32(
+          *reinterpret_cast<const unsigned short*>(base + kDnScaleOff + j * 64 + 2 * lane));
+      float pa[T], pb[T], pc[T], pd[T];
+#pragma unroll
+      for (int tt = 0; tt < T; ++tt) {
+        pa[tt] = (tt < cnt) ? chp[co[tt] + j] : 0.f;
+        pb[tt] = pc[tt] = pd[tt] = 0.f;
+      }
+      const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float f[8];
+        dequant8(wv[i], f);
+#pragma unroll
+        for (int tt = 0; tt < T; ++tt) {
+          if (tt < cnt) {
+            const float* hq = hp + ho[tt] + 32 * j + 8 * i;
+            if (i & 1) dot8_f_2(f, ldsf4(hq), ldsf4(hq + 4), pc[tt], pd[tt]);
+            else dot8_f_2(f, ldsf4(hq), ldsf4(hq + 4), pa[tt], pb[tt]);
+          }
+        }
+      }
+#pragma unroll
+      for (int tt = 0; tt < T; ++tt) acc[tt] = fmaf(sj, (pa[tt] + pb[tt]) + (pc[tt] + pd[tt]), acc[tt]);
+    }
+#pragma unroll
+    for (int tt = 0; tt < T; ++tt) {
+      if (tt < cnt) {
+        float v = acc[tt];
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        if (q == 0) {
+          const int pr = hd.uniq_pair[u][tt];
+          part[((size_t)blk * (PL::P + T) + pr) * 4 + r] = kCodeScale * v * hd.topw[pr / K][pr % K];
+        }
+      }
+    }
+  };
+  if (use_d && !aborted(hd) && warp < nitems) {
+    // T = 1: routed units straight from the dedicated region
+    if (!mbar_wait(&hd.dbar, 0, p.wait_limit_ns, p.err)) {
+      hd.abort = 1;
+    } else {
+      for (int it = warp; it < nitems; it += kWarps) {
+        const int blk = it / U, u = it - blk * U;
+        down_item(body + PL::dn + ((size_t)u * nblk + blk) * kDnUnitBytes, blk, u);
+      }
+    }
+  }
   {
     const int r = lane & 3, q = lane >> 2;
     const bool run = !aborted(hd);
@@ -569,59 +693,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
 #pragma unroll 1
         for (int bI = 0; bI < n; ++bI) {
           const int it = it0 + bI, blk = it / U, u = it - blk * U;
-          const unsigned char* base = bufB + bI * kDnUnitBytes;
-          const int cnt = hd.uniq_cnt[u];
-          int ho[T], co[T];
-#pragma unroll
-          for (int tt = 0; tt < T; ++tt) {
-            const int pr = (tt < cnt) ? hd.uniq_pair[u][tt] : 0;
-            ho[tt] = pr * kHpStride + 100 * q;
-            co[tt] = pr * kHGroups + q * kDnChunks;
-          }
-          float acc[T];
-#pragma unroll
-          for (int tt = 0; tt < T; ++tt) acc[tt] = 0.f;
-#pragma unroll
-          for (int j = 0; j < kDnChunks; ++j) {
-            const uint4 w = lds128(base + j * 512 + 16 * lane);
-            const float sj = bf16_to_f32(
-                *reinterpret_cast<const unsigned short*>(base + kDnScaleOff + j * 64 + 2 * lane));
-            float pa[T], pb[T], pc[T], pd[T];
-#pragma unroll
-            for (int tt = 0; tt < T; ++tt) {
-              pa[tt] = (tt < cnt) ? chp[co[tt] + j] : 0.f;
-              pb[tt] = pc[tt] = pd[tt] = 0.f;
-            }
-            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              float f[8];
-              dequant8(wv[i], f);
-#pragma unroll
-              for (int tt = 0; tt < T; ++tt) {
-                if (tt < cnt) {
-                  const float* hq = hp + ho[tt] + 32 * j + 8 * i;
-                  if (i & 1) dot8_f_2(f, ldsf4(hq), ldsf4(hq + 4), pc[tt], pd[tt]);
-                  else dot8_f_2(f, ldsf4(hq), ldsf4(hq + 4), pa[tt], pb[tt]);
-                }
-              }
-            }
-#pragma unroll
-            for (int tt = 0; tt < T; ++tt) acc[tt] = fmaf(sj, (pa[tt] + pb[tt]) + (pc[tt] + pd[tt]), acc[tt]);
-          }
-#pragma unroll
-          for (int tt = 0; tt < T; ++tt) {
-            if (tt < cnt) {
-              float v = acc[tt];
-              v += __shfl_xor_sync(0xffffffffu, v, 4);
-              v += __shfl_xor_sync(0xffffffffu, v, 8);
-              v += __shfl_xor_sync(0xffffffffu, v, 16);
-              if (q == 0) {
-                const int pr = hd.uniq_pair[u][tt];
-                part[((size_t)blk * (PL::P + T) + pr) * 4 + r] = kCodeScale * v * hd.topw[pr / K][pr % K];
-              }
-            }
-          }
+          down_item(bufB + bI * kDnUnitBytes, blk, u);
         }
       } else {
         const int blk = sh_first + (s - nmine_r) * kWarps;
@@ -673,6 +745,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   // every CTA (aborted or not) counts itself out; the last one resets the
   // counters for the next launch on the stream
   __syncthreads();
+  if (tid == 0 && hd.dcopies) mbar_wait(&hd.dbar, 0, p.wait_limit_ns, p.err);  // no copy left in flight
   if (tid == 0) {
     __threadfence();
     const unsigned prev = atomicAdd(p.sync + 3, 1u);
@@ -687,6 +760,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
 }
 
 #ifdef LING_MOE_TRACE
+extern "C" int ling_moe_clk_read(long long* host) { return (int)cudaMemcpyFromSymbol(host, g_clk, sizeof(g_clk)); }
 extern "C" int ling_moe_trace_read(unsigned long long* host, int nctas) {
   return (int)cudaMemcpyFromSymbol(host, g_trace, (size_t)nctas * 16 * sizeof(unsigned long long));
 }

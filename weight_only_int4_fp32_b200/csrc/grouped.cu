@@ -1,8 +1,9 @@
 // Token-grouped path (T > kMaxDecodeT): prefill chunks and large verify
 // batches of the W4 g32 MoE layer.
 //
-//   route        logits[t, e] = x_t . Wr_e (+ b_e) in fp32 on CUDA cores, then
-//                top-k per token (ties to the lower index) and the renormalised
+//   route        logits[t, e] = x_t . Wr_e (+ b_e) in fp32 on CUDA cores, tiles
+//                of <= 16 tokens x 64 experts
+//   top-k        per token (ties to the lower index) and the renormalised
 //                softmax weights; pairs per expert counted on the fly
 //   plan         exclusive scan of the counts, tile lists for both GEMMs
 //                (N-tiles of <= 128 positions, the costly ones first)
@@ -28,12 +29,13 @@ constexpr int kRtThreads = 256;
 constexpr int kRtWarps = kRtThreads / 32;
 constexpr int kRtPass = 8;      // tokens per pass (register tile: 8 experts x 8 tokens per lane)
 constexpr int kRtMaxTok = 16;   // tokens per CTA
-constexpr size_t kRtSmem = (size_t)kRtPass * kXTok * sizeof(float) + (size_t)kRtPass * kMaxExperts * sizeof(float);
+constexpr int kRtExperts = 8 * kRtWarps;  // experts per CTA: 8 per warp
+constexpr size_t kRtSmem = (size_t)kRtPass * kXTok * sizeof(float);
 constexpr int kPlanThreads = 1024;
 constexpr int kRowThreads = kH / 8;  // 320: one thread per 8 columns of a row
 
 const char* grouped_describe() {
-  return "fp32 router GEMM + fused top-k + counting scatter by expert + tcgen05 grouped GEMMs "
+  return "fp32 router GEMM + top-k + counting scatter by expert + tcgen05 grouped GEMMs "
          "(M=256 weight rows x N<=128 positions; routed int4 dequantised to exact fp16 in shared memory, "
          "shared expert as fp16 tiles via TMA; activations via TMA; fp32 accumulators in double-buffered TMEM) "
          "+ fixed-order combine";
@@ -46,6 +48,7 @@ cudaError_t grouped_alloc(GroupedWorkspace* ws, int E, int k, int max_T, const A
   const size_t nt = tc_max_ntiles((int)P, max_T, E);
   cudaError_t e;
   struct A { void** p; size_t n; } plan[] = {
+      {(void**)&ws->logits, (size_t)max_T * E * sizeof(float)},
       {(void**)&ws->topk_idx, P * sizeof(int32_t)},
       {(void**)&ws->topk_w, P * sizeof(float)},
       {(void**)&ws->cnt, (size_t)E * sizeof(int32_t)},
@@ -99,15 +102,17 @@ __device__ void stage_x_rows(const __nv_bfloat16* x, const int* toks, int n, flo
 }
 
 // ---------------------------------------------------------------- route
-// Logits of NT <= 8 staged tokens for all experts.  A warp takes 8 experts
-// at a time; each lane accumulates 8 experts x NT tokens over its K-chunks
-// (every 8th chunk of 8 columns), then a reduce-scatter across the warp
-// leaves lane l with the sums for expert 8w + l/4 and tokens 2(l%4), +1.
+// Logits of NT <= 8 staged tokens (rows t0 ..) for the CTA's experts.  A warp
+// takes 8 experts; each lane accumulates 8 experts x NT tokens over its
+// K-chunks (every 32nd chunk of 8 columns), then a reduce-scatter across the
+// warp leaves lane l with the sums for expert e0 + l/4 and tokens 2(l%4), +1.
 template <int NT>
-__device__ __forceinline__ void route_logits(const float* xs, const GroupedParams& p, float* lg) {
+__device__ __forceinline__ void route_logits(const float* xs, const GroupedParams& p, int t0, int ebase,
+                                             float* logits) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll 1
-  for (int e0 = 8 * warp; e0 < p.E; e0 += 8 * kRtWarps) {
+  {
+    const int e0 = ebase + 8 * warp;
+    if (e0 >= p.E) return;
     float acc[64];
 #pragma unroll
     for (int i = 0; i < 64; ++i) acc[i] = 0.f;
@@ -155,25 +160,21 @@ __device__ __forceinline__ void route_logits(const float* xs, const GroupedParam
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int t = 2 * (lane & 3) + u;
-        if (t < NT) lg[t * kMaxExperts + e] = acc[u] + bias;
+        if (t < NT) logits[(size_t)(t0 + t) * p.E + e] = acc[u] + bias;
       }
     }
   }
 }
 
-// One CTA: tokens [t0, t0 + tpc) in passes of <= 8; per pass the logits go
-// to shared memory and warp w selects the top-k of token w.
-__global__ void __launch_bounds__(kRtThreads, 1) grp_route_kernel(GroupedParams p, int tpc, int32_t* ti, float* tw,
-                                                                 int32_t* cnt) {
-  extern __shared__ __align__(16) float sm_rt[];
-  float* xs = sm_rt;
-  float* lg = sm_rt + kRtPass * kXTok;
+// CTA (x, y): tokens [x tpc, x tpc + tpc) in passes of <= 8, experts
+// [64 y, 64 y + 64).  Splitting the experts keeps every SM streaming router
+// rows at small T too.
+__global__ void __launch_bounds__(kRtThreads, 1) grp_route_kernel(GroupedParams p, int tpc, float* logits) {
+  extern __shared__ __align__(16) float xs[];
   __shared__ int toks[kRtPass];
-  __shared__ int s_idx[kRtPass][kMaxTopK];
-  __shared__ float s_w[kRtPass][kMaxTopK];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t_begin = blockIdx.x * tpc, t_end = min(p.T, t_begin + tpc);
   const int ntok = t_end - t_begin;
+  const int ebase = blockIdx.y * kRtExperts;
   if (ntok <= 0) return;
   const int npass = (ntok + kRtPass - 1) / kRtPass;
   const int per = (ntok + npass - 1) / npass;
@@ -185,30 +186,40 @@ __global__ void __launch_bounds__(kRtThreads, 1) grp_route_kernel(GroupedParams 
     stage_x_rows(p.x, toks, nt, xs);
     __syncthreads();
     switch (nt) {
-      case 1: route_logits<1>(xs, p, lg); break;
-      case 2: route_logits<2>(xs, p, lg); break;
-      case 3: route_logits<3>(xs, p, lg); break;
-      case 4: route_logits<4>(xs, p, lg); break;
-      case 5: route_logits<5>(xs, p, lg); break;
-      case 6: route_logits<6>(xs, p, lg); break;
-      case 7: route_logits<7>(xs, p, lg); break;
-      default: route_logits<8>(xs, p, lg); break;
+      case 1: route_logits<1>(xs, p, t0, ebase, logits); break;
+      case 2: route_logits<2>(xs, p, t0, ebase, logits); break;
+      case 3: route_logits<3>(xs, p, t0, ebase, logits); break;
+      case 4: route_logits<4>(xs, p, t0, ebase, logits); break;
+      case 5: route_logits<5>(xs, p, t0, ebase, logits); break;
+      case 6: route_logits<6>(xs, p, t0, ebase, logits); break;
+      case 7: route_logits<7>(xs, p, t0, ebase, logits); break;
+      default: route_logits<8>(xs, p, t0, ebase, logits); break;
     }
     __syncthreads();
-    if (warp < nt) {
-      const int t = t0 + warp;
-      warp_topk_bitonic(lg + warp * kMaxExperts, p.E, p.k, s_idx[warp], s_w[warp]);
-      if (lane < p.k) {
-        const int e = s_idx[warp][lane];
-        const float w = s_w[warp][lane];
-        ti[t * p.k + lane] = e;
-        tw[t * p.k + lane] = w;
-        if (p.topk_idx_out) p.topk_idx_out[t * p.k + lane] = e;
-        if (p.topk_w_out) p.topk_w_out[t * p.k + lane] = w;
-        atomicAdd(&cnt[e], 1);
-      }
-    }
-    __syncthreads();
+  }
+}
+
+// One warp per token: top-k of its logits, the renormalised weights, and
+// one count per selected expert.
+__global__ void __launch_bounds__(256) grp_topk_kernel(GroupedParams p, const float* logits, int32_t* ti,
+                                                       float* tw, int32_t* cnt) {
+  __shared__ float lg[8][kMaxExperts];
+  __shared__ int s_idx[8][kMaxTopK];
+  __shared__ float s_w[8][kMaxTopK];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t = blockIdx.x * 8 + warp;
+  if (t >= p.T) return;
+  for (int e = lane; e < p.E; e += 32) lg[warp][e] = logits[(size_t)t * p.E + e];
+  __syncwarp();
+  warp_topk_fast(lg[warp], p.E, p.k, s_idx[warp], s_w[warp]);
+  if (lane < p.k) {
+    const int e = s_idx[warp][lane];
+    const float w = s_w[warp][lane];
+    ti[t * p.k + lane] = e;
+    tw[t * p.k + lane] = w;
+    if (p.topk_idx_out) p.topk_idx_out[t * p.k + lane] = e;
+    if (p.topk_w_out) p.topk_w_out[t * p.k + lane] = w;
+    atomicAdd(&cnt[e], 1);
   }
 }
 
@@ -383,8 +394,12 @@ cudaError_t launch_grouped(const GroupedParams& p, const GroupedWorkspace& ws, c
   int nl = 0;
   cudaError_t e = cudaSuccess;
   const int P = p.T * p.k;
-  const int tpc = std::min(kRtMaxTok, (p.T + p.num_sms - 1) / p.num_sms);
-  grp_route_kernel<<<(p.T + tpc - 1) / tpc, kRtThreads, kRtSmem, s>>>(p, tpc, ws.topk_idx, ws.topk_w, ws.cnt);
+  const int eblocks = (p.E + kRtExperts - 1) / kRtExperts;
+  const int tpc = std::max(1, std::min(kRtMaxTok, (p.T * eblocks + 2 * p.num_sms - 1) / (2 * p.num_sms)));
+  grp_route_kernel<<<dim3((p.T + tpc - 1) / tpc, (p.E + kRtExperts - 1) / kRtExperts), kRtThreads, kRtSmem, s>>>(
+      p, tpc, ws.logits);
+  ++nl;
+  grp_topk_kernel<<<(p.T + 7) / 8, 256, 0, s>>>(p, ws.logits, ws.topk_idx, ws.topk_w, ws.cnt);
   ++nl;
   grp_plan_kernel<<<1, kPlanThreads, 0, s>>>(p.T, p.E, ws.cnt, ws.fill, ws.off, ws.gu_tiles, ws.dn_tiles, ws.ntiles);
   ++nl;

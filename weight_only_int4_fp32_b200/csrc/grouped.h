@@ -30,6 +30,7 @@ struct GroupedParams {
 struct GroupedWorkspace {
   int max_T = 0;
   size_t rows = 0;              // max_T * (k + 1) positions
+  float* logits = nullptr;      // [T, E] router logits
   int32_t* topk_idx = nullptr;  // [T*k]
   float* topk_w = nullptr;      // [T*k]
   int32_t* cnt = nullptr;       // [E] pairs per expert (left at zero after each call)

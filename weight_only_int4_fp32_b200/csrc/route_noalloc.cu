@@ -102,7 +102,7 @@ route_noalloc_kernel(const __nv_bfloat16* __restrict__ x, int T, const __nv_bflo
     __syncthreads();
     if (warp < T) {
       if (ok) {
-        warp_topk_bitonic(lg[warp], E, K, si[warp], sw[warp]);
+        warp_topk_fast(lg[warp], E, K, si[warp], sw[warp]);
         if (lane < K) {
           topk_idx[warp * K + lane] = si[warp][lane];
           topk_w[warp * K + lane] = sw[warp][lane];
