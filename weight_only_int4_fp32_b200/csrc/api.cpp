@@ -67,11 +67,11 @@ struct ling_moe {
   __nv_bfloat16* sh_gate = nullptr;
   __nv_bfloat16* sh_up = nullptr;
   __nv_bfloat16* sh_down = nullptr;
-  // decode workspace: epoch-tagged exchange buffers and the sync words
+  // decode workspace: exchange buffers and the arrival counters
   float* logits = nullptr;
   float* h_s = nullptr;
   float* h_pair = nullptr;
-  unsigned int* sync = nullptr;
+  unsigned long long* sync = nullptr;  // monotonic arrival counters of the decode kernel
   unsigned int* err = nullptr;
   // grouped-path workspace
   GroupedWorkspace gws{};
@@ -184,7 +184,7 @@ int ling_moe_create(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, l
       {(void**)&h->logits, (size_t)h->decode_T * E * sizeof(float)},
       {(void**)&h->h_s, (size_t)h->decode_T * kI * sizeof(float)},
       {(void**)&h->h_pair, (size_t)h->decode_T * K * kI * sizeof(float)},
-      {(void**)&h->sync, 4 * sizeof(unsigned int)},
+      {(void**)&h->sync, 4 * sizeof(unsigned long long)},
       {(void**)&h->err, 4 * sizeof(unsigned int)},
       {(void**)&h->x_stage, (size_t)cfg->max_tokens * kH * bf},
       {(void**)&h->out_stage, (size_t)cfg->max_tokens * kH * bf},
@@ -218,7 +218,7 @@ int ling_moe_create(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, l
   if (e == cudaSuccess) e = cudaMemcpyAsync(h->sh_gate, w->sh_gate, (size_t)kI * kH * bf, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(h->sh_up, w->sh_up, (size_t)kI * kH * bf, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(h->sh_down, w->sh_down, (size_t)kH * kI * bf, cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(h->sync, 0, 4 * sizeof(unsigned int), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->sync, 0, 4 * sizeof(unsigned long long), s);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->err, 0, 4 * sizeof(unsigned int), s);
   if (e == cudaSuccess)
     e = launch_repack(w->gate_q, w->up_q, w->gate_s, w->up_s, w->down_q, w->down_s, h->gu, h->dn, E, s);
@@ -350,11 +350,11 @@ int ling_moe_status(ling_moe_t* h, void* stream_v) {
   e = cudaMemcpy(&err, h->err, sizeof(err), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "read device error word");
   if (err) {
-    // A wait gave up.  Every CTA still counted itself out and the last one
-    // reset the arrival counters, so the next launch starts clean; clear the
-    // error word (and the counters, in case a launch never ran to its end).
+    // A wait gave up, so some arrivals of that launch never happened and the
+    // monotonic counters no longer match the launch index: clear them (no
+    // launch is in flight after the synchronize) and the error word.
     cudaMemset(h->err, 0, 4 * sizeof(unsigned int));
-    cudaMemset(h->sync, 0, 4 * sizeof(unsigned int));
+    cudaMemset(h->sync, 0, 4 * sizeof(unsigned long long));
     if (h->gws.cnt) {  // grouped-path counters that a cut-short call may have left behind
       cudaMemset(h->gws.cnt, 0, (size_t)h->cfg.num_experts * sizeof(int32_t));
       cudaMemset(h->gws.fill, 0, (size_t)h->cfg.num_experts * sizeof(int32_t));

@@ -19,10 +19,10 @@
 // routing (shared expert) are requested first.  A routed gate/up unit is
 // copied in four pieces with one mbarrier each, so its dot products start
 // when the first piece lands.  For one token the CTA's routed down units are
-// copied into a dedicated shared-memory region as soon as the routing is
-// known (they land during the gate/up phase); otherwise they are prefetched
-// into L2 then and copied in batches while the CTA waits at the last grid
-// barrier.
+// copied into a dedicated shared-memory region as soon as the CTA's own
+// gate/up work is done (they land while the grid exchanges h); otherwise
+// they are prefetched into L2 once the routing is known and copied in
+// batches while the CTA waits at the last grid barrier.
 //
 // Layer definition: vLLM recipe page "inclusionAI/Ling-3.0-flash" (Overview;
 // "Single-GPU int4": symmetric W4, group 32, routed experts only) and the
@@ -66,7 +66,7 @@ constexpr int kRowBytes = kH * 2;                   // one bf16 row of H
 static_assert(kBufB >= kShDnBytes, "phase-4 buffer holds a shared-down block");
 static_assert(kBufA >= 2 * kRowBytes, "phase-1/2 buffer holds a gate and an up row");
 
-struct __align__(16) SmemHeader {
+struct __align__(128) SmemHeader {  // 128-byte multiple: the body starts on a full line
   uint64_t mbar[kWarps][4];
   uint64_t xbar;
   uint64_t dbar;
@@ -81,10 +81,11 @@ struct __align__(16) SmemHeader {
   int uniq_pair[kMaxDecodeT * kMaxTopK][kMaxDecodeT];
   int nuniq;
   int dcopies;  // T = 1: routed down copies into the dedicated region were issued
+  unsigned long long epoch;  // launch index (see the arrival counters)
   int abort;
   int pad[3];
 };
-static_assert(sizeof(SmemHeader) % 16 == 0, "header keeps the body 16-byte aligned");
+static_assert(sizeof(SmemHeader) % 128 == 0, "header keeps the body 128-byte aligned");
 
 // x is kept twice: the bf16 input as staged (router and shared rows read it
 // with mixed-precision FMAs) and an fp16 copy scaled by 2^-sigma per token
@@ -136,17 +137,19 @@ __device__ __forceinline__ bool aborted(const SmemHeader& hd) {
 // ---------------------------------------------------------------- arrival counters
 // Publish: the calling thread's earlier stores (and, after a warp or CTA
 // barrier, those of the other threads) become visible before the count.
-__device__ __forceinline__ void arrive(unsigned int* ctr) {
+// The counters only grow (64-bit): launch L waits for (L + 1) x its per-launch
+// total, so nothing has to be reset between launches.
+__device__ __forceinline__ void arrive(unsigned long long* ctr) {
   __threadfence();
-  atomicAdd(ctr, 1u);
+  atomicAdd(ctr, 1ull);
 }
 // Bounded poll until *ctr >= target.  On time-out sets the error word and the
 // CTA's abort flag; returns false.
-__device__ __forceinline__ bool wait_count(const unsigned int* ctr, uint32_t target,
+__device__ __forceinline__ bool wait_count(const unsigned long long* ctr, unsigned long long target,
                                            unsigned long long limit_ns, unsigned int* err, int* abort) {
-  if (ld_acquire_u32(ctr) >= target) return true;
+  if (ld_acquire_u64(ctr) >= target) return true;
   const unsigned long long t0 = globaltimer_ns();
-  while (ld_acquire_u32(ctr) < target) {
+  while (ld_acquire_u64(ctr) < target) {
     if (*reinterpret_cast<volatile int*>(abort) || globaltimer_ns() - t0 > limit_ns) {
       atomicOr(err, 1u);
       *reinterpret_cast<volatile int*>(abort) = 1;
@@ -159,7 +162,7 @@ __device__ __forceinline__ bool wait_count(const unsigned int* ctr, uint32_t tar
 template <int T>
 __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const DecodeParams p) {
   using PL = Plan<T>;
-  extern __shared__ __align__(128) unsigned char smem_raw[];
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   SmemHeader& hd = *reinterpret_cast<SmemHeader*>(smem_raw);
   unsigned char* body = smem_raw + sizeof(SmemHeader);
 
@@ -189,6 +192,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     hd.xmax[tid] = 0u;
     hd.xscale[tid] = 1.0f;
   }
+  // Launch index of this call: every CTA of the earlier launches on the
+  // stream has counted itself out, and no CTA of this one can before all
+  // have passed the router barrier (which comes after this read).
+  // (the load is issued here; its value is first needed at the routing)
+  const unsigned long long done_ctas = (tid == 0) ? ld_acquire_u64(p.sync + 3) : 0ull;
   if (tid == 0) {
     hd.abort = 0;
     hd.xinf = 0;
@@ -346,12 +354,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   // alone: with other warps still streaming shared-memory dot products, the
   // shuffle/reduction-bound selection was measured ~3x slower.  The shared
   // rows finish before the router counter completes, so this costs nothing.
+  if (tid == 0) hd.epoch = done_ctas / (unsigned long long)ncta;
   __syncthreads();
   // ---- routing: every CTA selects the top-k itself from the published logits
   if (warp < T && !aborted(hd)) {
     float* lg = reinterpret_cast<float*>(bufA);  // scratch: this warp's buffer is idle here
     bool ok = true;
-    if (lane == 0) ok = wait_count(p.sync + 0, (uint32_t)E, p.wait_limit_ns, p.err, &hd.abort);
+    if (lane == 0) ok = wait_count(p.sync + 0, (hd.epoch + 1) * (unsigned long long)E, p.wait_limit_ns, p.err, &hd.abort);
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (warp == 0) LING_TRACE(11);
     if (warp == 0) LING_CLK(0);
@@ -433,18 +442,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     }
   };
   if (u0 + warp < u1) issue3(u0 + warp);
-  if (use_d) {
-    // T = 1: this CTA's routed down units, one contiguous copy per expert
-    if (warp == kWarps - 1 && U > 0 && !aborted(hd)) {
-      const uint32_t per = (uint32_t)nblk * kDnUnitBytes;
-      if (lane == 0) mbar_arrive_expect_tx(&hd.dbar, per * (uint32_t)U);
-      __syncwarp();
-      if (lane < U)
-        bulk_g2s(body + PL::dn + (size_t)lane * per,
-                 p.dn + ((size_t)hd.uniq_e[lane] * kDnUnits + b0) * kDnUnitBytes, per, &hd.dbar);
-      if (lane == 0) hd.dcopies = 1;
-    }
-  } else if (warp == kWarps - 1 && nblk > 0) {
+  if (!use_d && warp == kWarps - 1 && nblk > 0) {
     // routed down units of this CTA (contiguous per expert) into L2
     for (int u = lane; u < U; u += 32) {
       const uint8_t* src = p.dn + ((size_t)hd.uniq_e[u] * kDnUnits + b0) * kDnUnitBytes;
@@ -531,11 +529,23 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         }
       }
       __syncwarp();
-      if (lane == 0) arrive(p.sync + 2);
       if (warp == 0 && unit == u0) { LING_TRACE(14); LING_CLK(10); }
     }
   }
   __syncthreads();
+  if (tid == 0) arrive(p.sync + 2);  // this CTA's h values are published
+  if (use_d && warp == kWarps - 1 && U > 0 && !aborted(hd)) {
+    // T = 1: this CTA's routed down units, one contiguous copy per expert,
+    // requested now so that they stream in during the h exchange (during the
+    // gate/up phase they would only share its bandwidth)
+    const uint32_t per = (uint32_t)nblk * kDnUnitBytes;
+    if (lane == 0) mbar_arrive_expect_tx(&hd.dbar, per * (uint32_t)U);
+    __syncwarp();
+    if (lane < U)
+      bulk_g2s(body + PL::dn + (size_t)lane * per,
+               p.dn + ((size_t)hd.uniq_e[lane] * kDnUnits + b0) * kDnUnitBytes, per, &hd.dbar);
+    if (lane == 0) hd.dcopies = 1;
+  }
   LING_TRACE(5);
 
   // ---- phase 4: down projections and the output
@@ -572,22 +582,38 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   float* hsm = reinterpret_cast<float*>(body + PL::hs);
   float* part = reinterpret_cast<float*>(body + PL::part);
   if (tid == 0 && !aborted(hd)) {
-    if (wait_count(p.sync + 1, (uint32_t)kI, p.wait_limit_ns, p.err, &hd.abort))
-      wait_count(p.sync + 2, (uint32_t)(U * kGuUnits), p.wait_limit_ns, p.err, &hd.abort);
+    const unsigned long long ep1 = hd.epoch + 1;
+    if (wait_count(p.sync + 1, ep1 * (unsigned long long)kI, p.wait_limit_ns, p.err, &hd.abort))
+      wait_count(p.sync + 2, ep1 * (unsigned long long)ncta, p.wait_limit_ns, p.err, &hd.abort);
   }
   __syncthreads();
   if (!aborted(hd)) {
-    for (int v = tid; v < npairs * (kI / 4); v += kDecodeThreads) {
-      const int pr = v / (kI / 4), c4 = v - pr * (kI / 4);
-      const float4 h = ldcg_f4(reinterpret_cast<const float4*>(p.h_pair + (size_t)pr * kI) + c4);
-      const int e0 = 4 * c4;
-      *reinterpret_cast<float4*>(hp + (size_t)pr * kHpStride + e0 + 4 * (e0 / 96)) = h;
-    }
-    for (int v = tid; v < T * (kI / 4); v += kDecodeThreads) {
-      const int t = v / (kI / 4), c4 = v - t * (kI / 4);
-      const float4 h = ldcg_f4(reinterpret_cast<const float4*>(p.h_s + (size_t)t * kI) + c4);
-      const int c = c4 >> 1, pl = c4 & 1;
-      *reinterpret_cast<float4*>(hsm + (size_t)t * kHsTok + pl * kHsPlane + 4 * c) = h;
+    // routed h (per pair) then shared h (per token), in batches whose loads
+    // are all in flight before the first shared store
+    constexpr int kB = 5;
+    const int nh = npairs * (kI / 4), nall = nh + T * (kI / 4);
+    for (int v0 = tid; v0 < nall; v0 += kB * kDecodeThreads) {
+      float4 hv[kB];
+#pragma unroll
+      for (int b = 0; b < kB; ++b) {
+        const int v = v0 + b * kDecodeThreads;
+        if (v < nh) {
+          hv[b] = ldcg_f4(reinterpret_cast<const float4*>(p.h_pair) + v);
+        } else if (v < nall) {
+          hv[b] = ldcg_f4(reinterpret_cast<const float4*>(p.h_s) + (v - nh));
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < kB; ++b) {
+        const int v = v0 + b * kDecodeThreads;
+        if (v < nh) {
+          const int pr = v / (kI / 4), c4 = v - pr * (kI / 4), e0 = 4 * c4;
+          *reinterpret_cast<float4*>(hp + (size_t)pr * kHpStride + e0 + 4 * (e0 / 96)) = hv[b];
+        } else if (v < nall) {
+          const int t = (v - nh) / (kI / 4), c4 = (v - nh) - t * (kI / 4), c = c4 >> 1, pl = c4 & 1;
+          *reinterpret_cast<float4*>(hsm + (size_t)t * kHsTok + pl * kHsPlane + 4 * c) = hv[b];
+        }
+      }
     }
   }
   __syncthreads();
@@ -742,20 +768,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       p.out[(size_t)t * kH + 4 * (b0 + blk) + r] = __float2bfloat16_rn(s);
     }
   }
-  // every CTA (aborted or not) counts itself out; the last one resets the
-  // counters for the next launch on the stream
+  // every CTA (aborted or not) counts itself out: the next launch's index
   __syncthreads();
   if (tid == 0 && hd.dcopies) mbar_wait(&hd.dbar, 0, p.wait_limit_ns, p.err);  // no copy left in flight
-  if (tid == 0) {
-    __threadfence();
-    const unsigned prev = atomicAdd(p.sync + 3, 1u);
-    if (prev == (unsigned)ncta - 1u) {
-      atomicExch(p.sync + 0, 0u);
-      atomicExch(p.sync + 1, 0u);
-      atomicExch(p.sync + 2, 0u);
-      atomicExch(p.sync + 3, 0u);
-    }
-  }
+  if (tid == 0) atomicAdd(p.sync + 3, 1ull);  // read by later launches only: no fence needed
   LING_TRACE(9);
 }
 

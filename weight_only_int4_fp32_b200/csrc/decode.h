@@ -33,7 +33,8 @@ struct DecodeParams {
   float* h_pair;                 // workspace [T*k, I]
   int32_t* topk_idx_out;         // optional caller output [T, k]
   float* topk_w_out;             // optional caller output [T, k]
-  unsigned int* sync;            // [0] router rows, [1] shared rows, [2] routed units, [3] CTAs done
+  unsigned long long* sync;      // monotonic: [0] router rows, [1] shared rows, [2] CTAs past the
+                                 // routed gate/up, [3] CTAs done (launch index x CTAs)
   unsigned int* err;             // sticky device error word
   int skip_arrive_cta;           // test hook: this CTA withholds its router rows (-1: none)
   unsigned long long wait_limit_ns;
