@@ -295,6 +295,32 @@ __device__ __forceinline__ Pairs4 dequant_f16x2(uint32_t w) {
   asm("lop3.b32 %0, %1, 0x00F000F0, 0x64006400, 0xEA;" : "=r"(r.p3) : "r"(w8));
   return r;
 }
+// Exact codes from a fragment word (offset-binary nibbles): the pair of
+// nibbles (0, 4) as fp16 (q0, q4) = (1024 + n) - 1032, and the pair (1, 5)
+// as 16 q = (1024 + 16 n) - 1152; w >> 8 gives the pairs (2, 6) and (3, 7).
+__device__ __forceinline__ uint32_t deq_q_even(uint32_t w) {
+  uint32_t v, r;
+  asm("lop3.b32 %0, %1, 0x000F000F, 0x64006400, 0xEA;" : "=r"(v) : "r"(w));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(0x64086408u));  // 1032
+  return r;
+}
+__device__ __forceinline__ uint32_t deq_q_odd16(uint32_t w) {
+  uint32_t v, r;
+  asm("lop3.b32 %0, %1, 0x00F000F0, 0x64006400, 0xEA;" : "=r"(v) : "r"(w));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(0x64806480u));  // 1152
+  return r;
+}
+// D = A B + C for one m16n8k16 tile: A 16x16 fp16 (row-major fragment),
+// B 16x8 fp16 (column-major fragment), C and D fp32.
+__device__ __forceinline__ void mma_16816(float& d0, float& d1, float& d2, float& d3, uint32_t a0, uint32_t a1,
+                                          uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1, float c0, float c1,
+                                          float c2, float c3) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%10, %11, %12, %13};"
+      : "=f"(d0), "=f"(d1), "=f"(d2), "=f"(d3)
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(c2), "f"(c3));
+}
+
 constexpr float kEvenBias = -1032.0f;
 constexpr float kOddBias = -1152.0f;
 // acc_e += even products, acc_o += odd products of one word (8 codes) with

@@ -54,14 +54,15 @@ __device__ __forceinline__ void g_clk_sink(float) {}
 #endif
 
 constexpr int kWarps = kDecodeWarps;
-constexpr int kBufA = kGuUnitBytes;                 // per-warp buffer, phases 1-3
+constexpr int kBufA = kGuHalfBytes;                 // per-warp buffer, phases 1-3 (one K half of a unit)
 constexpr int kDnBatch = 4;                         // routed down units per copy batch
 constexpr int kBufB = kDnBatch * kDnUnitBytes;      // per-warp buffer, phase 4
 constexpr int kShDnBytes = 4 * kI * 2;              // 4 shared-down rows
 constexpr int kMaxBlkPerCta = 8;                    // down row-blocks per CTA (>= 640 / nctas)
 constexpr int kDnPrefBlk = 5;                       // T = 1: routed down units kept in shared memory
                                                     // when the CTA has <= 5 row-blocks (>= 128 CTAs)
-constexpr int kGuPiece = kGuScaleOff / 4;           // 2560 B: 5 chunks of a gate/up unit
+constexpr int kGuPiece = kGuHalfCodes / 4;          // 2560 B: 5 chunks of a gate/up half-unit
+constexpr int kPairs = kDecodeWarps / 2;            // phase-3 warp pairs (one K half each)
 constexpr int kRowBytes = kH * 2;                   // one bf16 row of H
 static_assert(kBufB >= kShDnBytes, "phase-4 buffer holds a shared-down block");
 static_assert(kBufA >= 2 * kRowBytes, "phase-1/2 buffer holds a gate and an up row");
@@ -88,12 +89,13 @@ struct __align__(128) SmemHeader {  // 128-byte multiple: the body starts on a f
 static_assert(sizeof(SmemHeader) % 128 == 0, "header keeps the body 128-byte aligned");
 
 // x is kept twice: the bf16 input as staged (router and shared rows read it
-// with mixed-precision FMAs) and an fp16 copy scaled by 2^-sigma per token
-// (routed gate/up), laid out in 4 K-quarters of 1296 bytes so that the
-// quarters of a unit fall in different banks.
+// with mixed-precision FMAs) and an fp16 copy scaled by 2^-sigma per token in
+// MMA B-fragment order for the routed gate/up: per chunk of 64 K, per lane
+// class m = lane % 4, per K block w, the pair (x[c], x[c+1]) and the pair
+// (x[c+8], x[c+9]) / 16 with c = 16 kb + 2 m (the /16 matches the 16 q form
+// in which the upper half of a block's codes is dequantised).
 constexpr int kXbTok = kH * 2;                   // bytes per token, bf16
-constexpr int kXhQuarter = (kH / 4) * 2 + 16;    // 1296 bytes
-constexpr int kXhTok = 4 * kXhQuarter;           // 5184 bytes
+constexpr int kXfTok = (kH / 64) * 128;          // 5120 bytes per token
 
 // Shared-memory plan (byte offsets into the body).  Region A (phases 1-3)
 // and region B (phase 4) overlap: B is used only after the CTA's own phase 3.
@@ -101,9 +103,9 @@ template <int T>
 struct Plan {
   static constexpr int P = T * kMaxTopK;
   static constexpr size_t xb = 0;                                           // [T][kXbTok]
-  static constexpr size_t xh = xb + (size_t)T * kXbTok;                     // [T][kXhTok]
-  static constexpr size_t cg = xh + (size_t)T * kXhTok;                     // float2 [T][kXGroups]
-  static constexpr size_t bufA = cg + (size_t)T * kXGroups * 8;             // [warps][kBufA]
+  static constexpr size_t xf = xb + (size_t)T * kXbTok;                     // [T][kXfTok]
+  static constexpr size_t comb = xf + (size_t)T * kXfTok;                   // float [pairs][2][32][4]
+  static constexpr size_t bufA = comb + (size_t)kPairs * 2 * 32 * 16;       // [warps][kBufA]
   static constexpr size_t endA = bufA + (size_t)kWarps * kBufA;
   static constexpr size_t hp = 0;                                           // float [P][kHpStride]
   static constexpr size_t chp = hp + (size_t)P * kHpStride * 4;             // float [P][kHGroups]
@@ -116,7 +118,7 @@ struct Plan {
   static constexpr size_t dn = endAB;
   static constexpr size_t body = dn + (T == 1 ? (size_t)kMaxTopK * kDnPrefBlk * kDnUnitBytes : 0);
   static constexpr size_t bytes = sizeof(SmemHeader) + body;
-  static_assert(xh % 16 == 0 && cg % 16 == 0 && bufA % 16 == 0 && bufB % 16 == 0 && chp % 16 == 0 &&
+  static_assert(xf % 16 == 0 && comb % 16 == 0 && bufA % 16 == 0 && bufB % 16 == 0 && chp % 16 == 0 &&
                 hs % 16 == 0 && part % 16 == 0 && dn % 16 == 0, "16-byte aligned regions");
   static_assert(bytes <= 227 * 1024, "decode smem over budget");
 };
@@ -186,8 +188,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   unsigned char* bufA = body + PL::bufA + (size_t)warp * kBufA;
   unsigned char* bufB = body + PL::bufB + (size_t)warp * kBufB;
   unsigned char* xb = body + PL::xb;
-  unsigned char* xh = body + PL::xh;
-  float2* cg = reinterpret_cast<float2*>(body + PL::cg);
+  unsigned char* xf = body + PL::xf;
   if (tid < kMaxDecodeT) {
     hd.xmax[tid] = 0u;
     hd.xscale[tid] = 1.0f;
@@ -236,43 +237,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   // x (bf16) lands in shared memory; every warp waits for it once
   if (!mbar_wait(&hd.xbar, 0, p.wait_limit_ns, p.err)) hd.abort = 1;
   LING_TRACE(1);
-  // fp16 copy of x and the per-group bias constants of the int4 dot products,
-  // built as soon as x lands (the first weight rows are still in flight):
-  // 4 lanes per group of 32.  x is
-  // converted as is (exact for normal bf16 values below 65504); if any value
-  // overflows fp16, the token is redone scaled by 2^-sigma.
+  // fp16 copy of x in B-fragment order, built as soon as x lands (the first
+  // weight rows are still in flight).  x is converted as is (exact for normal
+  // bf16 values below 65504); if any value overflows fp16, the token is redone
+  // scaled by 2^-sigma.
   auto build_xh = [&]() {
-    const int sub = lane & 3, gw = lane >> 2;
-    for (int g0 = warp * 8; g0 < T * kXGroups; g0 += kWarps * 8) {
-      const int g = g0 + gw;
-      float se = 0.f, so = 0.f;
-      if (g < T * kXGroups) {
-        const int t = g / kXGroups, G = g - t * kXGroups, c = 4 * G + sub;
-        const uint4 w = lds128(xb + t * kXbTok + 16 * c);
-        const float inv = 1.0f / hd.xscale[t];
-        const __half2 h0 = __floats2half2_rn(bf16lo(w.x) * inv, bf16hi(w.x) * inv);
-        const __half2 h1 = __floats2half2_rn(bf16lo(w.y) * inv, bf16hi(w.y) * inv);
-        const __half2 h2 = __floats2half2_rn(bf16lo(w.z) * inv, bf16hi(w.z) * inv);
-        const __half2 h3 = __floats2half2_rn(bf16lo(w.w) * inv, bf16hi(w.w) * inv);
-        if (__hisinf(h0.x) | __hisinf(h0.y) | __hisinf(h1.x) | __hisinf(h1.y) | __hisinf(h2.x) |
-            __hisinf(h2.y) | __hisinf(h3.x) | __hisinf(h3.y))
-          hd.xinf = 1;
-        uint4 o;
-        o.x = *reinterpret_cast<const uint32_t*>(&h0);
-        o.y = *reinterpret_cast<const uint32_t*>(&h1);
-        o.z = *reinterpret_cast<const uint32_t*>(&h2);
-        o.w = *reinterpret_cast<const uint32_t*>(&h3);
-        *reinterpret_cast<uint4*>(xh + t * kXhTok + (c / 80) * kXhQuarter + 16 * (c % 80)) = o;
-        const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
-        const float2 f2 = __half22float2(h2), f3 = __half22float2(h3);
-        se = (f0.x + f1.x) + (f2.x + f3.x);
-        so = (f0.y + f1.y) + (f2.y + f3.y);
-      }
-      se += __shfl_xor_sync(0xffffffffu, se, 1);
-      so += __shfl_xor_sync(0xffffffffu, so, 1);
-      se += __shfl_xor_sync(0xffffffffu, se, 2);
-      so += __shfl_xor_sync(0xffffffffu, so, 2);
-      if (sub == 0 && g < T * kXGroups) cg[g] = make_float2(kEvenBias * se, kOddBias * so);
+    for (int v = tid; v < T * (kH / 4); v += kDecodeThreads) {
+      const int t = v / (kH / 4), r = v - t * (kH / 4), kb = r >> 2, m = r & 3;
+      const int c = 16 * kb + 2 * m;
+      const uint32_t lo = *reinterpret_cast<const uint32_t*>(xb + t * kXbTok + 2 * c);
+      const uint32_t hi = *reinterpret_cast<const uint32_t*>(xb + t * kXbTok + 2 * (c + 8));
+      const float inv = 1.0f / hd.xscale[t];
+      const __half2 h0 = __floats2half2_rn(bf16lo(lo) * inv, bf16hi(lo) * inv);
+      const __half2 h1 = __floats2half2_rn(bf16lo(hi) * inv * 0.0625f, bf16hi(hi) * inv * 0.0625f);
+      if (__hisinf(h0.x) | __hisinf(h0.y) | __hisinf(__float2half_rn(bf16lo(hi) * inv)) |
+          __hisinf(__float2half_rn(bf16hi(hi) * inv)))
+        hd.xinf = 1;
+      *reinterpret_cast<uint2*>(xf + t * kXfTok + (kb >> 2) * 128 + m * 32 + (kb & 3) * 8) =
+          make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
     }
   };
   build_xh();
@@ -424,24 +406,30 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   __syncthreads();
   const int U = aborted(hd) ? 0 : hd.nuniq;
 
-  // ---- phase 3: routed gate/up units, each copied in four pieces (the scales
-  // travel with piece 0)
+  // ---- phase 3: routed gate/up, whole units [u0, u1) of 8 intermediate rows
+  // (gate and up).  Warp pair p takes units u0 + p, u0 + p + kPairs, ...; warp
+  // 2p computes the first K half, warp 2p+1 the second, each copied in four
+  // pieces (the half's scales travel with piece 0).  Per 16-K block one
+  // fragment word per lane is dequantised to the exact codes q (LOP3 + HSUB2)
+  // and fed to one m16n8k16 MMA whose columns are the expert's tokens; per
+  // 32-K group the fp32 result is scaled by the group's bf16 scale.
   const int n3 = U * kGuUnits;
   const int u0 = (int)((long long)cta * n3 / ncta), u1 = (int)((long long)(cta + 1) * n3 / ncta);
+  const int pair = warp >> 1, half = warp & 1;
   auto issue3 = [&](int unit) {
     if (lane == 0) {
       const int u = unit / kGuUnits, b = unit - u * kGuUnits;
       const uint8_t* src = p.gu + ((size_t)hd.uniq_e[u] * kGuUnits + b) * kGuUnitBytes;
-      mbar_arrive_expect_tx(barA, kGuPiece + (kGuUnitBytes - kGuScaleOff));
-      bulk_g2s(bufA + kGuScaleOff, src + kGuScaleOff, kGuUnitBytes - kGuScaleOff, barA);
-      bulk_g2s(bufA, src, kGuPiece, barA);
+      mbar_arrive_expect_tx(barA, kGuPiece + kGuHalfScales);
+      bulk_g2s(bufA + kGuHalfCodes, src + kGuScaleOff + half * kGuHalfScales, kGuHalfScales, barA);
+      bulk_g2s(bufA, src + half * kGuHalfCodes, kGuPiece, barA);
       for (int pc = 1; pc < 4; ++pc) {
         mbar_arrive_expect_tx(&hd.mbar[warp][pc], kGuPiece);
-        bulk_g2s(bufA + pc * kGuPiece, src + pc * kGuPiece, kGuPiece, &hd.mbar[warp][pc]);
+        bulk_g2s(bufA + pc * kGuPiece, src + half * kGuHalfCodes + pc * kGuPiece, kGuPiece, &hd.mbar[warp][pc]);
       }
     }
   };
-  if (u0 + warp < u1) issue3(u0 + warp);
+  if (u0 + pair < u1 && !aborted(hd)) issue3(u0 + pair);
   if (!use_d && warp == kWarps - 1 && nblk > 0) {
     // routed down units of this CTA (contiguous per expert) into L2
     for (int u = lane; u < U; u += 32) {
@@ -451,28 +439,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   }
 
   {
-    const int r = lane & 7, q = lane >> 3;
-    for (int unit = u0 + warp; unit < u1; unit += kWarps) {
-      if (unit != u0 + warp) issue3(unit);
+    float* comb = reinterpret_cast<float*>(body + PL::comb) + (size_t)pair * (2 * 32 * 4);
+    const int n = lane >> 2, m = lane & 3;  // B column (token of the expert) / lane class
+    int par = 0;
+    bool issued = u0 + pair < u1 && !aborted(hd);
+    for (int unit = u0 + pair; unit < u1; unit += kPairs, par ^= 1) {
+      if (unit != u0 + pair) {
+        issued = !aborted(hd);
+        if (issued) issue3(unit);
+      }
       const int u = unit / kGuUnits, b = unit - u * kGuUnits;
       const int cnt = hd.uniq_cnt[u];
-      int xo[T], co[T];
-      float xsc[T];
-#pragma unroll
-      for (int tt = 0; tt < T; ++tt) {
-        const int t = (tt < cnt) ? hd.uniq_pair[u][tt] / K : 0;
-        xo[tt] = t * kXhTok + q * kXhQuarter;   // group 20q+j at + 64j, word i at + 16i
-        co[tt] = t * kXGroups + q * kGuChunks;
-        xsc[tt] = hd.xscale[t];
-      }
-      float acc[T];
-#pragma unroll
-      for (int tt = 0; tt < T; ++tt) acc[tt] = 0.f;
-      bool ok = mbar_wait(barA, pha, p.wait_limit_ns, p.err);
-      pha ^= 1;
+      const bool bval = n < cnt;
+      const unsigned char* xrow = xf + (bval ? hd.uniq_pair[u][n] / K : 0) * kXfTok + m * 32 +
+                                  half * (kGuChunks / 2) * 128;
+      float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+      bool ok = issued && mbar_wait(barA, pha, p.wait_limit_ns, p.err);
+      if (issued) pha ^= 1;
       if (warp == 0 && unit == u0) { LING_TRACE(13); LING_CLK(6); }
-      // four pieces of 5 chunks; the chunks of a piece are unrolled so that
-      // their loads and FMA chains overlap
 #pragma unroll 1
       for (int pc = 0; pc < 4 && ok; ++pc) {
         if (pc > 0) {
@@ -481,54 +465,59 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
           if (warp == 0 && unit == u0) LING_CLK(6 + pc);
         }
 #pragma unroll
-        for (int jj = 0; jj < kGuChunks / 4; ++jj) {
-          const int j = pc * (kGuChunks / 4) + jj;
-          const uint4 w = lds128(bufA + j * 512 + 16 * lane);
-          const float s = bf16_to_f32(*reinterpret_cast<const unsigned short*>(
-              bufA + kGuScaleOff + (j >> 2) * 256 + 8 * lane + 2 * (j & 3)));
-          float ae[T], ao[T], be[T], bo[T];
+        for (int jj = 0; jj < kGuChunks / 8; ++jj) {
+          const int jl = pc * (kGuChunks / 8) + jj;  // chunk within the half
+          const uint4 wv = lds128(bufA + jl * 512 + 16 * lane);
+          const uint4 xa = bval ? lds128(xrow + jl * 128) : make_uint4(0, 0, 0, 0);
+          const uint4 xc = bval ? lds128(xrow + jl * 128 + 16) : make_uint4(0, 0, 0, 0);
+          const uint32_t s01 = *reinterpret_cast<const uint32_t*>(bufA + kGuHalfCodes + (2 * jl) * 32 + 4 * n);
+          const uint32_t s23 = *reinterpret_cast<const uint32_t*>(bufA + kGuHalfCodes + (2 * jl + 1) * 32 + 4 * n);
+          const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
+          const uint32_t bx[8] = {xa.x, xa.y, xa.z, xa.w, xc.x, xc.y, xc.z, xc.w};
+          float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
 #pragma unroll
-          for (int tt = 0; tt < T; ++tt) {
-            const float2 c2 = (tt < cnt) ? cg[co[tt] + j] : make_float2(0.f, 0.f);
-            ae[tt] = c2.x;
-            ao[tt] = c2.y;
-            be[tt] = 0.f;
-            bo[tt] = 0.f;
-          }
-          const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const Pairs4 P = dequant_f16x2(wv[i]);
-#pragma unroll
-            for (int tt = 0; tt < T; ++tt) {
-              if (tt < cnt) {
-                const uint4 xv = lds128(xh + xo[tt] + 64 * j + 16 * i);
-                if (i & 1) dot8_q_f16(P, xv, be[tt], bo[tt]);
-                else dot8_q_f16(P, xv, ae[tt], ao[tt]);
-              }
+          for (int w = 0; w < 4; ++w) {
+            const uint32_t a0 = deq_q_even(wd[w]), a2 = deq_q_odd16(wd[w]);
+            const uint32_t a1 = deq_q_even(wd[w] >> 8), a3 = deq_q_odd16(wd[w] >> 8);
+            if (w & 1) {
+              mma_16816(d0, d1, d2, d3, a0, a1, a2, a3, bx[2 * w], bx[2 * w + 1], d0, d1, d2, d3);
+              const uint32_t sw = (w == 1) ? s01 : s23;
+              const float sg = bf16lo(sw), su = bf16hi(sw);
+              acc0 = fmaf(sg, d0, acc0);
+              acc1 = fmaf(sg, d1, acc1);
+              acc2 = fmaf(su, d2, acc2);
+              acc3 = fmaf(su, d3, acc3);
+            } else {
+              mma_16816(d0, d1, d2, d3, a0, a1, a2, a3, bx[2 * w], bx[2 * w + 1], 0.f, 0.f, 0.f, 0.f);
             }
           }
-#pragma unroll
-          for (int tt = 0; tt < T; ++tt)
-            acc[tt] = fmaf(s, fmaf(0.0625f, ao[tt] + bo[tt], ae[tt] + be[tt]), acc[tt]);
         }
       }
-      phq ^= 1;
-      if (!ok) { hd.abort = 1; break; }
-      __syncwarp();
+      if (issued) phq ^= 1;
+      if (!ok && issued) hd.abort = 1;
+      // combine the two K halves: the second half's partials go through
+      // shared memory (double-buffered by unit parity, one barrier per unit)
+      float* cb = comb + par * (32 * 4) + lane * 4;
+      if (half == 1) *reinterpret_cast<float4*>(cb) = make_float4(acc0, acc1, acc2, acc3);
+      asm volatile("bar.sync %0, %1;" :: "r"(1 + pair), "r"(64) : "memory");
+      if (half == 0 && !aborted(hd)) {
+        const float4 o = *reinterpret_cast<const float4*>(cb);
+        acc0 += o.x;
+        acc1 += o.y;
+        acc2 += o.z;
+        acc3 += o.w;
+        const int i = 8 * b + n;  // intermediate row of this lane
 #pragma unroll
-      for (int tt = 0; tt < T; ++tt) {
-        if (tt < cnt) {
-          float v = acc[tt];
-          v += __shfl_xor_sync(0xffffffffu, v, 8);
-          v += __shfl_xor_sync(0xffffffffu, v, 16);
-          v *= xsc[tt];
-          const float up = __shfl_sync(0xffffffffu, v, (lane & ~7) | ((r + 4) & 7));
-          if (r < 4 && q == tt)
-            p.h_pair[(size_t)hd.uniq_pair[u][tt] * kI + 4 * b + r] = silu_mul(v, up);
+        for (int cc = 0; cc < 2; ++cc) {
+          const int col = 2 * m + cc;  // the expert's token column
+          if (col < cnt) {
+            const int pr = hd.uniq_pair[u][col];
+            const float xs = hd.xscale[pr / K];
+            const float g = (cc ? acc1 : acc0) * xs, up = (cc ? acc3 : acc2) * xs;
+            p.h_pair[(size_t)pr * kI + i] = silu_mul(g, up);
+          }
         }
       }
-      __syncwarp();
       if (warp == 0 && unit == u0) { LING_TRACE(14); LING_CLK(10); }
     }
   }

@@ -319,8 +319,8 @@ __global__ void __launch_bounds__(kPlanThreads) grp_plan_kernel(int T, int E, in
 // One CTA per token: each of its k pairs takes the next position in its
 // expert's run; x_t is scaled by 2^-sigma_t (max |x_t| * 2^-sigma_t in
 // [2^14, 2^15), so fp16 holds every bf16 value of a normal-range row exactly),
-// converted to fp16 in the permuted K order and written to its k positions
-// and to the shared-expert row P + t.
+// converted to fp16 and written to its k positions and to the shared-expert
+// row P + t.
 __global__ void __launch_bounds__(kRowThreads) grp_scatter_kernel(const __nv_bfloat16* x, int k, int P,
                                                                   const int32_t* ti, const int32_t* off,
                                                                   int32_t* fill, int32_t* perm, int32_t* inv,
@@ -354,10 +354,7 @@ __global__ void __launch_bounds__(kRowThreads) grp_scatter_kernel(const __nv_bfl
   if (c == 0) xscale[t] = __uint_as_float((uint32_t)(127 + sigma) << 23);
   __half h[8];
 #pragma unroll
-  for (int o = 0; o < 8; ++o) {
-    const int at = (o < 4) ? 2 * o : 2 * (o - 4) + 1;  // permuted K order within 8
-    h[at] = __float2half_rn(f[o] * inv_s);
-  }
+  for (int o = 0; o < 8; ++o) h[o] = __float2half_rn(f[o] * inv_s);
   const uint4 hv = *reinterpret_cast<const uint4*>(h);
   for (int i = 0; i <= k; ++i) *reinterpret_cast<uint4*>(xg + (size_t)spos[i] * kH + 8 * c) = hv;
 }

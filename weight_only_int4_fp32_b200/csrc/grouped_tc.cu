@@ -15,8 +15,10 @@
 // directly.  The activations are the B operand, fetched by TMA from buffers
 // in position order: x (fp16, exact after a per-token power-of-two scale) for
 // gate/up and h as two fp16 terms hi + lo (~22 significant bits) for down.
-// Both operands use the same per-8-element K order (the order in which a LOP3
-// extracts nibbles), so nothing is permuted inside the main loop.
+// Gate/up tiles are in natural K order: a producer gathers one row's 16-K
+// block from the four MMA-fragment words that hold it.  Down tiles and h use
+// the per-8-element order in which a LOP3 extracts nibbles from a 32-code
+// group.  Either way A and B agree, so nothing is permuted in the main loop.
 //
 // One thread issues tcgen05.mma into a double-buffered TMEM accumulator
 // (2 x 256 columns); tcgen05.commit releases each pipeline stage, and 4
@@ -50,8 +52,9 @@ constexpr int kBoxRows = 32;                    // B rows per TMA box
 constexpr int kBoxBytes = kBoxRows * kTcK * 2;  // 4 KB
 constexpr int kShBoxRows = 128;                 // shared-expert A rows per TMA box
 constexpr int kTmemCols = 512;                  // 2 buffers x (2 M-halves x 128 columns)
-// raw ring, per stage: int4 codes [2 groups][256 threads] x 16 B, then the
-// 4-byte words holding each group's bf16 scale [2][256] x 4 B
+// raw ring, per stage.  Gate/up: int4 codes [4 fragment lanes][256 threads]
+// x 8 B, then [256] x 4 B (gate, up) scale words.  Down: codes [2 groups]
+// [256 threads] x 16 B, then [2][256] x 4 B words holding each group's scale.
 constexpr int kRawCodes = 2 * kProd * 16;
 constexpr int kRawStage = kRawCodes + 2 * kProd * 4;  // 10 KB
 constexpr unsigned long long kTcWaitNs = 2000000000ull;
@@ -144,6 +147,9 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst), "l"(src) : "memory");
 }
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" :: "r"(dst), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" :: "r"(dst), "l"(src) : "memory");
 }
@@ -223,9 +229,10 @@ __global__ void __launch_bounds__(256) sh_amax_kernel(const __nv_bfloat16* g, co
   if ((threadIdx.x & 31) == 0) atomicMax(&amax[m], __float_as_uint(fminf(a, 3.0e38f)));
 }
 
-// One thread per 8 consecutive K elements: scale by 2^c, convert to fp16,
-// store in the permuted K order.  Gate/up rows are laid out per block of 128
-// intermediate rows i: 128 gate rows, then the 128 up rows of the same i.
+// One thread per 8 consecutive K elements: scale by 2^c, convert to fp16.
+// Gate/up keep the natural K order (the order of the routed gate/up tiles);
+// down takes the permuted order of h.  Gate/up rows are laid out per block of
+// 128 intermediate rows i: 128 gate rows, then the 128 up rows of the same i.
 __global__ void __launch_bounds__(256) sh_convert_kernel(const __nv_bfloat16* g, const __nv_bfloat16* u,
                                                          const __nv_bfloat16* d, const unsigned int* amax,
                                                          __half* shgu16, __half* shdn16, float* sh_scale) {
@@ -242,7 +249,7 @@ __global__ void __launch_bounds__(256) sh_convert_kernel(const __nv_bfloat16* g,
                         bf16lo(x.z), bf16hi(x.z), bf16lo(x.w), bf16hi(x.w)};
     __half h[8];
 #pragma unroll
-    for (int o = 0; o < 8; ++o) h[perm_pos(o)] = __float2half_rn(e[o] * f);
+    for (int o = 0; o < 8; ++o) h[m < 2 ? o : perm_pos(o)] = __float2half_rn(e[o] * f);
     const int grow = 2 * (row & ~127) + 128 * m + (row & 127);
     __half* dst = m < 2 ? shgu16 + (size_t)grow * kH + k0 : shdn16 + (size_t)row * kI + k0;
     *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(h);
@@ -271,8 +278,8 @@ __device__ __forceinline__ void prefetch_tile(const TcParams& p, int4 tl, const 
   size_t abytes;
   if (tl.x < p.E) {
     if (MODE == 0) {
-      a = p.gu + ((size_t)tl.x * kGuUnits + (size_t)tl.y * (kTcTileM / 8)) * kGuUnitBytes;
-      abytes = (size_t)(kTcTileM / 8) * kGuUnitBytes;
+      a = p.gu + ((size_t)tl.x * kGuUnits + (size_t)tl.y * (kTcTileM / 16)) * kGuUnitBytes;
+      abytes = (size_t)(kTcTileM / 16) * kGuUnitBytes;
     } else {
       a = p.dn + ((size_t)tl.x * kDnUnits + (size_t)tl.y * (kTcTileM / 4)) * kDnUnitBytes;
       abytes = (size_t)(kTcTileM / 4) * kDnUnitBytes;
@@ -374,27 +381,27 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
         const int4 tl = tln;
         if (tl.x < p.E) {
           const uint32_t slot = raw0 + (q % R) * kRawStage;
+          if (MODE == 0) {
+            // row i (gate and up), K blocks 2 kh, 2 kh + 1 of chunk kk: 8 bytes
+            // from each of the four fragment lanes 4 (i % 8) + m, and the
+            // (gate, up) scale word of group 2 kk + kh
+            const int il = r & 127, kh = r >> 7;
+            const int i = (kTcTileM / 2) * tl.y + il;
+            const uint8_t* ub = p.gu + ((size_t)tl.x * kGuUnits + (i >> 3)) * kGuUnitBytes;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int G = 2 * kk + h;
-            const uint8_t* codes;
-            const uint8_t* sword;
-            if (MODE == 0) {
-              const int i = (kTcTileM / 2) * tl.y + (r & 127);
-              const int rin = (r >> 7) ? 4 + (i & 3) : (i & 3);
-              const uint8_t* abase = p.gu + ((size_t)tl.x * kGuUnits + (i >> 2)) * kGuUnitBytes;
-              const int quarter = G / kGuChunks, jj = G - quarter * kGuChunks, ln = rin + 8 * quarter;
-              codes = abase + jj * 512 + 16 * ln;
-              sword = abase + kGuScaleOff + (jj >> 2) * 256 + 8 * ln + 4 * ((jj & 3) >> 1);
-            } else {
+            for (int m = 0; m < 4; ++m)
+              cp_async8(slot + m * (kProd * 8) + r * 8, ub + kk * 512 + 16 * (4 * (i & 7) + m) + 8 * kh);
+            cp_async4(slot + 4 * (kProd * 8) + r * 4, ub + kGuScaleOff + (2 * kk + kh) * 32 + 4 * (i & 7));
+          } else {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int G = 2 * kk + h;
               const int n = kTcTileM * tl.y + r;
               const uint8_t* abase = p.dn + ((size_t)tl.x * kDnUnits + (n >> 2)) * kDnUnitBytes;
               const int slice = G / kDnChunks, jj = G - slice * kDnChunks, ln = (n & 3) + 4 * slice;
-              codes = abase + jj * 512 + 16 * ln;
-              sword = abase + kDnScaleOff + jj * 64 + 4 * (ln >> 1);
+              cp_async16(slot + h * (kProd * 16) + r * 16, abase + jj * 512 + 16 * ln);
+              cp_async4(slot + kRawCodes + h * (kProd * 4) + r * 4, abase + kDnScaleOff + jj * 64 + 4 * (ln >> 1));
             }
-            cp_async16(slot + h * (kProd * 16) + r * 16, codes);
-            cp_async4(slot + kRawCodes + h * (kProd * 4) + r * 4, sword);
           }
         }
       }
@@ -419,25 +426,59 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       if (tl.x < p.E) {
         const unsigned char* slot = sRaw + (g % R) * kRawStage;
-        uint4 outv[8];
+        if (MODE == 0) {
+          // exact fp16 q * s * 2^8 for gate row il and up row 128 + il, K blocks
+          // 2 kh and 2 kh + 1 of this stage (natural K order)
+          const int il = r & 127, kh = r >> 7;
+          const uint32_t sw = *reinterpret_cast<const uint32_t*>(slot + 4 * (kProd * 8) + r * 4);
+          const float sgf = __uint_as_float(sw << 16) * (float)(1 << kTcScaleShift);
+          const float suf = __uint_as_float(sw & 0xFFFF0000u) * (float)(1 << kTcScaleShift);
+          const __half2 sg = __float2half2_rn(sgf), sg16 = __float2half2_rn(sgf * 0.0625f);
+          const __half2 su = __float2half2_rn(suf), su16 = __float2half2_rn(suf * 0.0625f);
+          const __half2 be = __float2half2_rn(1032.0f), bo = __float2half2_rn(1152.0f);
+          uint2 cw[4];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int G = 2 * kk + h;
-          int hi_half;
-          if (MODE == 0) {
-            hi_half = (G % kGuChunks) & 1;
-          } else {
-            const int n = kTcTileM * tl.y + r;
-            hi_half = ((n & 3) + 4 * (G / kDnChunks)) & 1;
+          for (int m = 0; m < 4; ++m) cw[m] = *reinterpret_cast<const uint2*>(slot + m * (kProd * 8) + r * 8);
+          unsigned char* ag = sA + s * kStageA + il * 128;
+          unsigned char* au = sA + s * kStageA + (128 + il) * 128;
+#pragma unroll
+          for (int ww = 0; ww < 2; ++ww) {
+            uint32_t glo[4], ghi[4], ulo[4], uhi[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+              const uint32_t w = ww ? cw[m].y : cw[m].x;
+              uint32_t v0, v1, v2, v3;
+              asm("lop3.b32 %0, %1, 0x000F000F, 0x64006400, 0xEA;" : "=r"(v0) : "r"(w));
+              asm("lop3.b32 %0, %1, 0x00F000F0, 0x64006400, 0xEA;" : "=r"(v1) : "r"(w));
+              asm("lop3.b32 %0, %1, 0x000F000F, 0x64006400, 0xEA;" : "=r"(v2) : "r"(w >> 8));
+              asm("lop3.b32 %0, %1, 0x00F000F0, 0x64006400, 0xEA;" : "=r"(v3) : "r"(w >> 8));
+              glo[m] = deq_pair(v0, sg, be);    // gate c, c+1:  (1024 + n - 1032) s
+              ghi[m] = deq_pair(v1, sg16, bo);  // gate c+8, c+9: (1024 + 16 n - 1152) s / 16
+              ulo[m] = deq_pair(v2, su, be);
+              uhi[m] = deq_pair(v3, su16, bo);
+            }
+            const int cl = 4 * kh + 2 * ww, ch = cl + 1;
+            *reinterpret_cast<uint4*>(ag + ((cl ^ (il & 7)) << 4)) = make_uint4(glo[0], glo[1], glo[2], glo[3]);
+            *reinterpret_cast<uint4*>(ag + ((ch ^ (il & 7)) << 4)) = make_uint4(ghi[0], ghi[1], ghi[2], ghi[3]);
+            *reinterpret_cast<uint4*>(au + ((cl ^ (il & 7)) << 4)) = make_uint4(ulo[0], ulo[1], ulo[2], ulo[3]);
+            *reinterpret_cast<uint4*>(au + ((ch ^ (il & 7)) << 4)) = make_uint4(uhi[0], uhi[1], uhi[2], uhi[3]);
           }
-          const uint4 q = *reinterpret_cast<const uint4*>(slot + h * (kProd * 16) + r * 16);
-          const uint32_t wv = *reinterpret_cast<const uint32_t*>(slot + kRawCodes + h * (kProd * 4) + r * 4);
-          const float sc = __uint_as_float(hi_half ? (wv & 0xFFFF0000u) : (wv << 16)) * (float)(1 << kTcScaleShift);
-          deq_group(q, sc, outv + 4 * h);
-        }
-        unsigned char* a = sA + s * kStageA + r * 128;
+        } else {
+          uint4 outv[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(a + ((c ^ (r & 7)) << 4)) = outv[c];
+          for (int h = 0; h < 2; ++h) {
+            const int G = 2 * kk + h;
+            const int n = kTcTileM * tl.y + r;
+            const int hi_half = ((n & 3) + 4 * (G / kDnChunks)) & 1;
+            const uint4 q = *reinterpret_cast<const uint4*>(slot + h * (kProd * 16) + r * 16);
+            const uint32_t wv = *reinterpret_cast<const uint32_t*>(slot + kRawCodes + h * (kProd * 4) + r * 4);
+            const float sc = __uint_as_float(hi_half ? (wv & 0xFFFF0000u) : (wv << 16)) * (float)(1 << kTcScaleShift);
+            deq_group(q, sc, outv + 4 * h);
+          }
+          unsigned char* a = sA + s * kStageA + r * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(a + ((c ^ (r & 7)) << 4)) = outv[c];
+        }
         fence_async_smem();
       }
       __syncwarp();

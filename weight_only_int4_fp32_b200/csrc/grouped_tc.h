@@ -53,8 +53,9 @@ struct TcMaps {
 cudaError_t setup_grouped_tc();
 cudaError_t tc_encode_maps(TcMaps* m, const __half* xg, const __half* h16, int rows, const __half* shgu16,
                            const __half* shdn16);
-// fp16 copies of the shared expert in the permuted K order, gate/up rows
-// interleaved, each matrix scaled by a power of two 2^c so that max |w| * 2^c
+// fp16 copies of the shared expert (gate/up in natural K order, 128 gate rows
+// then the 128 up rows of the same intermediate rows per block; down in the
+// permuted K order of h), each matrix scaled by a power of two 2^c so that max |w| * 2^c
 // lies in [2^14, 2^15); sh_scale receives 2^-c.  amax_scratch: 3 words.
 cudaError_t launch_tc_prep_shared(const __nv_bfloat16* g, const __nv_bfloat16* u, const __nv_bfloat16* d,
                                   __half* shgu16, __half* shdn16, float* sh_scale, unsigned int* amax_scratch,

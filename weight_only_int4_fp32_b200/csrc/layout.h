@@ -15,18 +15,27 @@ constexpr int kMaxTopK = 8;
 constexpr int kMaxExperts = 512;
 
 // ---------------------------------------------------------------- repacked layouts
-// Routed gate/up, per expert: kGuUnits units, one per block of 4 intermediate
-// rows i = 4b..4b+3.  A unit holds 8 rows (gate i0..i3, up i0..i3) split into
-// 4 K-quarters; lane l of a warp owns row (l & 7) and quarter (l >> 3).
-// Chunk j (0..kGuChunks-1) is 32 lanes x 16 B; lane l's 16 B are the 32 int4
-// codes of group G = quarter * kGuChunks + j of its row, as offset-binary
-// nibbles (code + 8), low nibble = even K index.  The 4*kGuChunks bf16 scales
-// of each lane follow, as kGuChunks/4 blocks of [32 lanes x 4 scales].
-constexpr int kGuUnits = kI / 4;                  // 192
-constexpr int kGuChunks = kH / 128;               // 20 groups per lane
-constexpr int kGuScaleOff = kGuChunks * 512;      // 10240
-constexpr int kGuUnitBytes = kGuScaleOff + kGuChunks * 64;  // 11520
+// Routed gate/up, per expert: kGuUnits units, one per block of 8 intermediate
+// rows i = 8b..8b+7, each unit holding the 16 rows (gate i, up i) x K.  K is
+// cut into blocks of 16; a block is 32 words, and word t (lane t of a warp)
+// holds exactly the int4 codes of lane t's A fragment of an m16n8k16 MMA
+// whose rows are (gate i_t, up i_t), i_t = 8b + t/4, and whose columns are
+// c, c+1, c+8, c+9 with c = 16 kb + 2 (t % 4):
+//   nibble 0: gate c    nibble 4: gate c+1    nibble 1: gate c+8   nibble 5: gate c+9
+//   nibble 2: up c      nibble 6: up c+1      nibble 3: up c+8     nibble 7: up c+9
+// as offset-binary codes (q + 8).  A chunk of 512 B covers 64 K (4 blocks):
+// lane t's 16 bytes are its words for blocks 4j .. 4j+3.  The bf16 scales
+// follow the kGuChunks chunks as [group][i (8)][gate, up].  The first and
+// second halves of K (chunks 0..19 with groups 0..39, and the rest) are
+// what the decode path streams as one work item each.
+constexpr int kGuUnits = kI / 8;                  // 96
+constexpr int kGuChunks = kH / 64;                // 40 chunks of 64 K
+constexpr int kGuScaleOff = kGuChunks * 512;      // 20480
+constexpr int kGuUnitBytes = kGuScaleOff + (kH / kGroup) * 32;  // 23040
 constexpr size_t kGuExpertBytes = (size_t)kGuUnits * kGuUnitBytes;  // 2211840
+constexpr int kGuHalfCodes = kGuScaleOff / 2;     // 10240: codes of one K half
+constexpr int kGuHalfScales = (kH / kGroup) * 16; // 1280: scales of one K half
+constexpr int kGuHalfBytes = kGuHalfCodes + kGuHalfScales;  // 11520
 
 // Routed down, per expert: kDnUnits units, one per block of 4 output rows
 // n = 4v..4v+3; lane l owns row (l & 3) and K-slice (l >> 2) of 3 groups.
@@ -38,7 +47,7 @@ constexpr int kDnScaleOff = kDnChunks * 512;      // 1536
 constexpr int kDnUnitBytes = kDnScaleOff + kDnChunks * 64;  // 1728
 constexpr size_t kDnExpertBytes = (size_t)kDnUnits * kDnUnitBytes;  // 1105920
 
-static_assert(kGuChunks % 4 == 0, "gate/up scales are loaded 4 at a time");
+static_assert(kGuChunks % 2 == 0, "gate/up units split into two K halves");
 static_assert(kH % 256 == 0 && kI % 256 == 0, "shape must tile by 256");
 
 }  // namespace lingmoe

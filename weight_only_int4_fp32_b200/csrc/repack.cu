@@ -16,41 +16,47 @@ __device__ __forceinline__ uint4 flip_sign_nibbles(uint4 v) {
   return v;
 }
 
-// gate/up: one thread per 16-byte chunk slot and per 8-byte scale slot.
+// gate/up: one thread per 32-bit fragment word and per (group, row pair)
+// scale slot.  A word gathers two bytes of the gate row and two of the up row
+// (each byte: K even in the low nibble, K odd in the high one).
+__device__ __forceinline__ uint32_t nib(uint32_t byte, int hi) { return (byte >> (4 * hi)) & 0xFu; }
 __global__ void repack_gu_kernel(const uint8_t* __restrict__ gate_q, const uint8_t* __restrict__ up_q,
                                  const uint16_t* __restrict__ gate_s, const uint16_t* __restrict__ up_s,
                                  uint8_t* __restrict__ gu, int E) {
-  const long long nchunk = (long long)E * kGuUnits * kGuChunks * 32;
-  const long long nscale = (long long)E * kGuUnits * (kGuChunks / 4) * 32;
-  for (long long g = blockIdx.x * (long long)blockDim.x + threadIdx.x; g < nchunk + nscale;
+  constexpr int kBlocks = kH / 16;                    // K blocks per row
+  const long long nword = (long long)E * kGuUnits * kBlocks * 32;
+  const long long nscale = (long long)E * kGuUnits * (kH / kGroup) * 8;
+  for (long long g = blockIdx.x * (long long)blockDim.x + threadIdx.x; g < nword + nscale;
        g += (long long)gridDim.x * blockDim.x) {
-    if (g < nchunk) {
-      const int lane = (int)(g & 31);
+    if (g < nword) {
+      const int t = (int)(g & 31);
       const long long rest = g >> 5;
-      const int j = (int)(rest % kGuChunks);
-      const long long eu = rest / kGuChunks;  // e * kGuUnits + b
+      const int kb = (int)(rest % kBlocks);
+      const long long eu = rest / kBlocks;            // e * kGuUnits + b
       const int b = (int)(eu % kGuUnits);
       const long long e = eu / kGuUnits;
-      const int r = lane & 7, q = lane >> 3;
-      const int row = 4 * b + (r & 3);
-      const int G = q * kGuChunks + j;
-      const uint8_t* src = (r < 4 ? gate_q : up_q) + ((e * kI + row) * (kH / 2) + 16 * G);
-      const uint4 v = *reinterpret_cast<const uint4*>(src);
-      *reinterpret_cast<uint4*>(gu + eu * kGuUnitBytes + j * 512 + 16 * lane) = flip_sign_nibbles(v);
+      const int i = 8 * b + (t >> 2);
+      const int c = 16 * kb + 2 * (t & 3);
+      const uint8_t* gr = gate_q + (e * kI + i) * (kH / 2);
+      const uint8_t* ur = up_q + (e * kI + i) * (kH / 2);
+      const uint32_t g0 = gr[c / 2], g1 = gr[(c + 8) / 2], u0 = ur[c / 2], u1 = ur[(c + 8) / 2];
+      uint32_t w = nib(g0, 0) | nib(g1, 0) << 4 | nib(u0, 0) << 8 | nib(u1, 0) << 12 |
+                   nib(g0, 1) << 16 | nib(g1, 1) << 20 | nib(u0, 1) << 24 | nib(u1, 1) << 28;
+      w ^= 0x88888888u;  // two's complement -> offset binary
+      const int j = kb >> 2, wi = kb & 3;
+      *reinterpret_cast<uint32_t*>(gu + eu * kGuUnitBytes + j * 512 + 16 * t + 4 * wi) = w;
     } else {
-      const long long g2 = g - nchunk;
-      const int lane = (int)(g2 & 31);
-      const long long rest = g2 >> 5;
-      const int bb = (int)(rest % (kGuChunks / 4));
-      const long long eu = rest / (kGuChunks / 4);
+      const long long g2 = g - nword;
+      const int r8 = (int)(g2 & 7);
+      const long long rest = g2 >> 3;
+      const int grp = (int)(rest % (kH / kGroup));
+      const long long eu = rest / (kH / kGroup);
       const int b = (int)(eu % kGuUnits);
       const long long e = eu / kGuUnits;
-      const int r = lane & 7, q = lane >> 3;
-      const int row = 4 * b + (r & 3);
-      const int G = q * kGuChunks + 4 * bb;
-      const uint16_t* src = (r < 4 ? gate_s : up_s) + ((e * kI + row) * (kH / kGroup) + G);
-      const uint2 v = *reinterpret_cast<const uint2*>(src);
-      *reinterpret_cast<uint2*>(gu + eu * kGuUnitBytes + kGuScaleOff + bb * 256 + 8 * lane) = v;
+      const int i = 8 * b + r8;
+      const uint32_t sg = gate_s[(e * kI + i) * (kH / kGroup) + grp];
+      const uint32_t su = up_s[(e * kI + i) * (kH / kGroup) + grp];
+      *reinterpret_cast<uint32_t*>(gu + eu * kGuUnitBytes + kGuScaleOff + grp * 32 + 4 * r8) = sg | (su << 16);
     }
   }
 }
