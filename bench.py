@@ -129,6 +129,19 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(x, device=None):
+    """Max of a float over all ranks of the process group (x itself without one).
+
+    Every rank must call it, in the same order (it is a collective)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ------------------------------------------------------------------ reference arm (the oracle)
 
 def cpu_oracle_rate(workload: str, seconds: float = 15.0, max_tokens: int = 64):
@@ -228,19 +241,24 @@ def build_layers(workload, device):
     return layers, E, T
 
 
-def make_inputs(workload, n, T, device):
+REPLICA_SEED_STRIDE = 1_000_003  # rank r > 0 draws its token stream from seeds shifted by r times this
+
+
+def make_inputs(workload, n, T, device, rank=0):
+    """The first n inputs of the workload's token stream; replica rank r > 0 runs its own stream."""
     import torch
     import workloads
     wl = workloads.WORKLOADS[workload]
+    off = rank * REPLICA_SEED_STRIDE
     if workload.startswith("decode") or workload.startswith("reduced"):
         seeds = [1 + t for t in range(n)] if workload.startswith("decode") else list(range(n))
-        return [workloads.tokens(1, seed=s, device=device) for s in seeds]
+        return [workloads.tokens(1, seed=s + off, device=device) for s in seeds]
     if workload.startswith("verify"):
-        return [workloads.tokens(4, seed=10000 + i, device=device) for i in range(n)]
+        return [workloads.tokens(4, seed=10000 + i + off, device=device) for i in range(n)]
     if workload.startswith("stack"):
-        return [torch.stack([workloads.tokens(1, seed=workloads.stack_token_seed(t, l), device=device)[0]
+        return [torch.stack([workloads.tokens(1, seed=workloads.stack_token_seed(t, l) + off, device=device)[0]
                              for l in range(wl["layers"])]) for t in range(n)]
-    return [workloads.tokens(T, seed=wl["token_seed"] + i, device=device) for i in range(n)]
+    return [workloads.tokens(T, seed=wl["token_seed"] + i + off, device=device) for i in range(n)]
 
 
 def run_ours(args):
@@ -254,7 +272,7 @@ def run_ours(args):
     import weight_only_int4_fp32_b200 as lm
     layers, E, T = build_layers(args.workload, dev)
     nsteps, nwarm = args.steps, args.warmup
-    inputs = make_inputs(args.workload, nsteps + nwarm, T, dev)
+    inputs = make_inputs(args.workload, nsteps + nwarm, T, dev, rank=rank)
     stack = args.workload.startswith("stack")
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
@@ -303,11 +321,7 @@ def run_ours(args):
         dist.barrier()
     launches = sum(l.launch_count() for l in layers) - n0
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    kern_ms = sum(step_ms)
-    if ws > 1:
-        tt = torch.tensor([kern_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        kern_ms = float(tt.item())
+    kern_ms = max_over_ranks(sum(step_ms), dev)
     status = [l.status() for l in layers]
     if any(s != lm.LING_MOE_OK for s in status):
         raise RuntimeError(f"device status {status}")
@@ -326,11 +340,8 @@ def run_ours(args):
         for i in range(nsteps):
             flush.fill_(float(i))
             layers[0].forward_host(xh[i], oh)
-        te = time.perf_counter() - te
-        tt = torch.tensor([te], device=dev)
-        if ws > 1:
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e = {"value": ws * nsteps * T / float(tt.item()), "unit": "tokens/s",
+        te = max_over_ranks(time.perf_counter() - te, dev)
+        e2e = {"value": ws * nsteps * T / te, "unit": "tokens/s",
                "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2,
                "note": "ling_moe_forward_host per step: pinned H2D copy + layer + D2H copy + "
                        "stream sync; the L2 flush fill runs between steps inside this wall clock"}
