@@ -16,17 +16,6 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
   return v;
 }
-__device__ __forceinline__ uint2 ldg_stream64(const void* p) {
-  uint2 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
-               : "=r"(v.x), "=r"(v.y) : "l"(p));
-  return v;
-}
-__device__ __forceinline__ unsigned short ldg_stream16(const void* p) {
-  unsigned short v;
-  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
-  return v;
-}
 // Data written earlier in the same launch by other CTAs: read from L2.
 __device__ __forceinline__ float ldcg_f32(const float* p) { return __ldcg(p); }
 __device__ __forceinline__ float4 ldcg_f4(const float4* p) { return __ldcg(p); }
@@ -40,35 +29,6 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) 
 // ---------------------------------------------------------------- conversions
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
-__device__ __forceinline__ float bf16_to_f32(unsigned short v) {
-  return __uint_as_float(((uint32_t)v) << 16);
-}
-
-// int4 -> fp32 without a conversion instruction: with the code stored as an
-// offset-binary nibble n = q + 8 in 0..15, the bit pattern 0x3F000000 | n<<16
-// is the float 0.5 + n/256 exactly.  One byte permute per element places the
-// nibble (already masked to the low half of its byte) into bits 16..19 under
-// the exponent byte 0x3F.  So for a group of 32 codes and inputs x:
-//   sum_k q_k x_k = 256 * (sum_k f_k x_k - (136/256) * sum_k x_k)
-// which the kernels evaluate as an fp32 FMA chain started at
-// c_G = -0.53125 * sum_k x_k, multiplied by 256 once per row at the end.
-// Each product f_k * x_k is exact in fp32 (f has 8 significant bits, x a
-// bf16-or-fp32 activation), so only the running sums round.
-__device__ __forceinline__ void dequant8(uint32_t w, float f[8]) {
-  const uint32_t lo = w & 0x0F0F0F0Fu;
-  const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;
-  const uint32_t m = 0x3F000000u;
-  f[0] = __uint_as_float(__byte_perm(lo, m, 0x7054));
-  f[1] = __uint_as_float(__byte_perm(hi, m, 0x7054));
-  f[2] = __uint_as_float(__byte_perm(lo, m, 0x7154));
-  f[3] = __uint_as_float(__byte_perm(hi, m, 0x7154));
-  f[4] = __uint_as_float(__byte_perm(lo, m, 0x7254));
-  f[5] = __uint_as_float(__byte_perm(hi, m, 0x7254));
-  f[6] = __uint_as_float(__byte_perm(lo, m, 0x7354));
-  f[7] = __uint_as_float(__byte_perm(hi, m, 0x7354));
-}
-constexpr float kBiasCoef = -0.53125f;  // -(136/256)
-constexpr float kCodeScale = 256.0f;
 
 __device__ __forceinline__ float silu_mul(float g, float u) {
   // SiLU(g) * u = g / (1 + e^-g) * u
@@ -98,67 +58,6 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
   return t;
 }
 
-// All threads of the CTA call this after their writes; thread 0 arrives.
-__device__ __forceinline__ void grid_arrive(unsigned long long* ctr, bool skip) {
-  __syncthreads();
-  if (threadIdx.x == 0 && !skip) {
-    __threadfence();
-    atomicAdd(ctr, 1ull);
-  }
-}
-
-// All threads call; returns false (for every thread) if the wait gave up.
-__device__ __forceinline__ bool grid_wait(const unsigned long long* ctr, unsigned long long target,
-                                          unsigned long long limit_ns, unsigned int* err,
-                                          int* s_flag) {
-  if (threadIdx.x == 0) {
-    int ok = 1;
-    if (ld_acquire_u64(ctr) < target) {
-      const unsigned long long t0 = globaltimer_ns();
-      while (ld_acquire_u64(ctr) < target) {
-        if (globaltimer_ns() - t0 > limit_ns) {
-          atomicOr(err, 1u);
-          ok = 0;
-          break;
-        }
-      }
-    }
-    __threadfence();
-    *s_flag = ok;
-  }
-  __syncthreads();
-  const int ok = *s_flag;
-  __syncthreads();
-  return ok != 0;
-}
-
-// ---------------------------------------------------------------- dot helpers
-// bf16 chunk (8 weights) dot the matching 8 fp32 activations.
-__device__ __forceinline__ float dot8_bf16(uint4 w, float4 a, float4 b, float acc) {
-  acc = fmaf(bf16lo(w.x), a.x, acc);
-  acc = fmaf(bf16hi(w.x), a.y, acc);
-  acc = fmaf(bf16lo(w.y), a.z, acc);
-  acc = fmaf(bf16hi(w.y), a.w, acc);
-  acc = fmaf(bf16lo(w.z), b.x, acc);
-  acc = fmaf(bf16hi(w.z), b.y, acc);
-  acc = fmaf(bf16lo(w.w), b.z, acc);
-  acc = fmaf(bf16hi(w.w), b.w, acc);
-  return acc;
-}
-
-// 8 dequantised codes (0.5 + n/256 form) dot 8 activations.
-__device__ __forceinline__ float dot8_f(const float f[8], float4 a, float4 b, float acc) {
-  acc = fmaf(f[0], a.x, acc);
-  acc = fmaf(f[1], a.y, acc);
-  acc = fmaf(f[2], a.z, acc);
-  acc = fmaf(f[3], a.w, acc);
-  acc = fmaf(f[4], b.x, acc);
-  acc = fmaf(f[5], b.y, acc);
-  acc = fmaf(f[6], b.z, acc);
-  acc = fmaf(f[7], b.w, acc);
-  return acc;
-}
-
 // ---------------------------------------------------------------- smem layouts
 // x as fp32 in two planes of 4-float chunks (chunk c = elements 8c..8c+7;
 // plane 0 holds 8c..8c+3, plane 1 holds 8c+4..8c+7), one pad chunk after
@@ -167,20 +66,11 @@ __device__ __forceinline__ float dot8_f(const float f[8], float4 a, float4 b, fl
 constexpr int kXChunks = kH / 8;                       // 320
 constexpr int kXPlane = (kXChunks + kXChunks / 80) * 4;  // 1296 floats
 constexpr int kXTok = 2 * kXPlane;                     // 2592 floats
-constexpr int kXGroups = kH / kGroup;                  // 80
-// Routed intermediate activations h (fp32), padded by 4 floats per 96.
-constexpr int kHpStride = kI + 4 * (kI / 96);          // 800 floats
-constexpr int kHGroups = kI / kGroup;                  // 24
 // Shared-expert h in two planes of 4-float chunks.
 constexpr int kHsPlane = (kI / 8) * 4;                 // 384 floats
 constexpr int kHsTok = 2 * kHsPlane;
 // fp32 x of token t, chunk c (8 elements) -> the two float4 planes.
 __device__ __forceinline__ int xoff(int c) { return 4 * (c + c / 80); }
-
-__device__ __forceinline__ float scale_of(uint2 s4, int jj) {
-  const uint32_t w = (jj < 2) ? s4.x : s4.y;
-  return (jj & 1) ? bf16hi(w) : bf16lo(w);
-}
 
 // ---------------------------------------------------------------- mbarrier + bulk copy
 // Non-multicast TMA bulk copies (global -> this CTA's shared memory) completing
@@ -230,6 +120,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
   }
   return true;
 }
+// The same, with one answer for the whole warp (for waits in front of
+// warp-wide instructions: mma.sync, full-mask shuffles).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, unsigned long long limit_ns,
+                                               unsigned int* err) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit_ns, err));
+}
 __device__ __forceinline__ uint4 lds128(const void* p) { return *reinterpret_cast<const uint4*>(p); }
 __device__ __forceinline__ float4 ldsf4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
@@ -251,49 +147,6 @@ __device__ __forceinline__ float fma_bf16h(uint32_t a2, uint32_t b2, float c) {
   else if constexpr (AH == 1 && BH == 0) LING_MIXED_FMA_ASM("bf16", "ah", "bl");
   else LING_MIXED_FMA_ASM("bf16", "ah", "bh");
   return d;
-}
-template <int AH, int BH>
-__device__ __forceinline__ float fma_f16h(uint32_t a2, uint32_t b2, float c) {
-  float d;
-  if constexpr (AH == 0 && BH == 0) LING_MIXED_FMA_ASM("f16", "al", "bl");
-  else if constexpr (AH == 0 && BH == 1) LING_MIXED_FMA_ASM("f16", "al", "bh");
-  else if constexpr (AH == 1 && BH == 0) LING_MIXED_FMA_ASM("f16", "ah", "bl");
-  else LING_MIXED_FMA_ASM("f16", "ah", "bh");
-  return d;
-}
-
-// 8 bf16 weights (one 16-byte chunk) dot 8 bf16 activations, fp32 accumulate.
-__device__ __forceinline__ float dot8_bf16_bf16(uint4 w, uint4 x, float acc) {
-  acc = fma_bf16h<0, 0>(w.x, x.x, acc);
-  acc = fma_bf16h<1, 1>(w.x, x.x, acc);
-  acc = fma_bf16h<0, 0>(w.y, x.y, acc);
-  acc = fma_bf16h<1, 1>(w.y, x.y, acc);
-  acc = fma_bf16h<0, 0>(w.z, x.z, acc);
-  acc = fma_bf16h<1, 1>(w.z, x.z, acc);
-  acc = fma_bf16h<0, 0>(w.w, x.w, acc);
-  acc = fma_bf16h<1, 1>(w.w, x.w, acc);
-  return acc;
-}
-
-// int4 -> fp16 with one LOP3 per two codes.  For a 32-bit word holding 8
-// offset-binary nibbles n_0..n_7 (n = q + 8, nibble i at bits 4i..4i+3,
-// element i of the word), (w & 0x000F000F) | 0x64006400 is the fp16 pair
-// (1024 + n_0, 1024 + n_4) and (w & 0x00F000F0) | 0x64006400 is
-// (1024 + 16 n_1, 1024 + 16 n_5); the same on w >> 8 gives elements 2, 6
-// and 3, 7.  Even elements carry 1024 + n, odd ones 1024 + 16 n, so for a
-// group of 32 codes with activations x (fp16):
-//   sum_k q_k x_k = (A_even - 1032 S_even) + (A_odd - 1152 S_odd) / 16
-// with A the fp32 FMA sums of the fp16 products and S the sums of x over the
-// even / odd positions.  Each fp16 x fp16 product is exact in fp32.
-struct Pairs4 { uint32_t p0, p1, p2, p3; };
-__device__ __forceinline__ Pairs4 dequant_f16x2(uint32_t w) {
-  Pairs4 r;
-  const uint32_t w8 = w >> 8;
-  asm("lop3.b32 %0, %1, 0x000F000F, 0x64006400, 0xEA;" : "=r"(r.p0) : "r"(w));
-  asm("lop3.b32 %0, %1, 0x00F000F0, 0x64006400, 0xEA;" : "=r"(r.p1) : "r"(w));
-  asm("lop3.b32 %0, %1, 0x000F000F, 0x64006400, 0xEA;" : "=r"(r.p2) : "r"(w8));
-  asm("lop3.b32 %0, %1, 0x00F000F0, 0x64006400, 0xEA;" : "=r"(r.p3) : "r"(w8));
-  return r;
 }
 // Exact codes from a fragment word (offset-binary nibbles): the pair of
 // nibbles (0, 4) as fp16 (q0, q4) = (1024 + n) - 1032, and the pair (1, 5)
@@ -321,19 +174,73 @@ __device__ __forceinline__ void mma_16816(float& d0, float& d1, float& d2, float
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(c2), "f"(c3));
 }
 
-constexpr float kEvenBias = -1032.0f;
-constexpr float kOddBias = -1152.0f;
-// acc_e += even products, acc_o += odd products of one word (8 codes) with
-// the 8 fp16 activations x = (x0..x7) packed in a uint4.
-__device__ __forceinline__ void dot8_q_f16(const Pairs4& P, uint4 x, float& ae, float& ao) {
-  ae = fma_f16h<0, 0>(P.p0, x.x, ae);  // e0 * x0
-  ae = fma_f16h<1, 0>(P.p0, x.z, ae);  // e4 * x4
-  ae = fma_f16h<0, 0>(P.p2, x.y, ae);  // e2 * x2
-  ae = fma_f16h<1, 0>(P.p2, x.w, ae);  // e6 * x6
-  ao = fma_f16h<0, 1>(P.p1, x.x, ao);  // e1 * x1
-  ao = fma_f16h<1, 1>(P.p1, x.z, ao);  // e5 * x5
-  ao = fma_f16h<0, 1>(P.p3, x.y, ao);  // e3 * x3
-  ao = fma_f16h<1, 1>(P.p3, x.w, ao);  // e7 * x7
+// Exact codes of the pair of nibbles (1, 5) without the factor 16:
+// (1024 + 16 n) / 16 - 72 = n - 8 = q, one rounding of an exact value.
+__device__ __forceinline__ uint32_t deq_q_odd(uint32_t w) {
+  uint32_t v, r;
+  asm("lop3.b32 %0, %1, 0x00F000F0, 0x64006400, 0xEA;" : "=r"(v) : "r"(w));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(v), "r"(0x2C002C00u), "r"(0xD480D480u));  // 1/16, -72
+  return r;
+}
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// ---------------------------------------------------------------- routed down on mma.sync
+// The down units (layout.h) are the B operand of m16n8k16 MMAs whose 8
+// columns are a unit's output rows.  The A operand is h: rows 0..7 of the A
+// tile are up to 8 tokens' h * 2^-8 as fp16 (hi), rows 8..15 the remainders
+// lo = fp16(h * 2^-8 - hi) of the same tokens, so one MMA takes both terms
+// (~22 significant bits of h) and the accumulator rows g and g + 8 add up.
+// A token's fragments in shared memory: for chunk j (128 K), group-in-chunk
+// gg and K block b, lane class c = lane % 4 owns the 16 bytes
+// (hi[k], hi[k+1]), (lo[k], lo[k+1]), (hi[k+8], hi[k+9]), (lo[k+8], lo[k+9])
+// with k = 128 j + 32 gg + 16 b + 2 c, at byte ((8 j + 2 gg + b) * 4 + c) * 16.
+constexpr int kHShift = 8;                       // h is scaled by 2^-8 before the split
+constexpr int kHfTokBytes = kDnChunks * 512;     // 3072
+constexpr int kHfStride = kHfTokBytes + 64;      // consecutive tokens in opposite bank halves
+__device__ __forceinline__ int hf_off(int k) {   // byte of (hi[k], hi[k+1]) for even k
+  const int G = k >> 5, b = (k >> 4) & 1, kk = k & 15;
+  return ((8 * (G >> 2) + 2 * (G & 3) + b) * 4 + ((kk & 7) >> 1)) * 16 + (kk >= 8 ? 8 : 0);
+}
+// (hi pair, lo pair) of two consecutive h values
+__device__ __forceinline__ uint2 h_split2(float h0, float h1) {
+  const float a = h0 * (1.0f / (float)(1 << kHShift)), b = h1 * (1.0f / (float)(1 << kHShift));
+  const __half2 hi = __floats2half2_rn(a, b);
+  const float2 hf = __half22float2(hi);
+  const __half2 lo = __floats2half2_rn(a - hf.x, b - hf.y);
+  return make_uint2(*reinterpret_cast<const uint32_t*>(&hi), *reinterpret_cast<const uint32_t*>(&lo));
+}
+// One down unit (kDnUnitBytes in shared memory) against the h of up to 8
+// tokens.  Lane (g = lane / 4, c = lane % 4) returns token g's sums for the
+// unit's rows 2c and 2c + 1, times 2^-8.  hf points at this lane's token's
+// fragments plus 16 c; act is false for lanes whose token does not exist
+// (their A rows are zero).  Every lane of the warp must call it.
+// Chunks j0 .. j1 - 1 of K only (default: all of K).
+__device__ __forceinline__ void dn_unit_mma(const unsigned char* unit, const unsigned char* hf, bool act, int lane,
+                                            float& r0, float& r1, int j0 = 0, int j1 = kDnChunks) {
+  const int c = lane & 3;
+  float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 2
+  for (int j = j0; j < j1; ++j) {
+    const uint4 w = lds128(unit + j * 512 + 16 * lane);
+    const uint4 s = lds128(unit + kDnScaleOff + j * 64 + 16 * c);
+    const uint32_t wv[4] = {w.x, w.y, w.z, w.w}, sv[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+    for (int gg = 0; gg < 4; ++gg) {
+      uint4 a0 = make_uint4(0u, 0u, 0u, 0u), a1 = a0;
+      if (act) {
+        a0 = lds128(hf + (8 * j + 2 * gg) * 64);
+        a1 = lds128(hf + (8 * j + 2 * gg + 1) * 64);
+      }
+      float d0, d1, d2, d3;
+      mma_16816(d0, d1, d2, d3, a0.x, a0.y, a0.z, a0.w, deq_q_even(wv[gg]), deq_q_odd(wv[gg]), 0.f, 0.f, 0.f, 0.f);
+      mma_16816(d0, d1, d2, d3, a1.x, a1.y, a1.z, a1.w, deq_q_even(wv[gg] >> 8), deq_q_odd(wv[gg] >> 8), d0, d1,
+                d2, d3);
+      acc0 = fmaf(bf16lo(sv[gg]), d0 + d2, acc0);
+      acc1 = fmaf(bf16hi(sv[gg]), d1 + d3, acc1);
+    }
+  }
+  r0 = acc0;
+  r1 = acc1;
 }
 
 // ---------------------------------------------------------------- top-k
@@ -427,16 +334,6 @@ __device__ __forceinline__ void dot8_bf16_bf16_2(uint4 w, uint4 x, float& a, flo
   b = fma_bf16h<1, 1>(w.z, x.z, b);
   a = fma_bf16h<0, 0>(w.w, x.w, a);
   b = fma_bf16h<1, 1>(w.w, x.w, b);
-}
-__device__ __forceinline__ void dot8_f_2(const float f[8], float4 x0, float4 x1, float& a, float& b) {
-  a = fmaf(f[0], x0.x, a);
-  b = fmaf(f[1], x0.y, b);
-  a = fmaf(f[2], x0.z, a);
-  b = fmaf(f[3], x0.w, b);
-  a = fmaf(f[4], x1.x, a);
-  b = fmaf(f[5], x1.y, b);
-  a = fmaf(f[6], x1.z, a);
-  b = fmaf(f[7], x1.w, b);
 }
 __device__ __forceinline__ void dot8_bf16_2(uint4 w, float4 x0, float4 x1, float& a, float& b) {
   a = fmaf(bf16lo(w.x), x0.x, a);

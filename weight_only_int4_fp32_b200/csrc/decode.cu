@@ -9,8 +9,9 @@
 //              gate/up + SiLU*up (bf16)                        -> barriers A, B
 //   phase 3    wait A; every CTA selects the top-k itself; routed gate/up
 //              (W4 g32, dequantised in registers) + SiLU*up     -> barrier C
-//   phase 4    routed down (W4 g32) weighted by the routing weights and
-//              shared down (bf16), summed in a fixed order, one bf16 rounding.
+//   phase 4    routed down (W4 g32, mma.sync with h as fp16 hi + lo) weighted
+//              by the routing weights and shared down (bf16), summed in a
+//              fixed order, one bf16 rounding.
 //
 // Weight bytes move HBM -> shared memory by non-multicast TMA bulk copies,
 // one private buffer and mbarrier per warp; each warp issues the copy of its
@@ -22,7 +23,9 @@
 // copied into a dedicated shared-memory region as soon as the CTA's own
 // gate/up work is done (they land while the grid exchanges h); otherwise
 // they are prefetched into L2 once the routing is known and copied in
-// batches while the CTA waits at the last grid barrier.
+// batches while the CTA waits at the last grid barrier.  A CTA owns whole
+// 8-row down units (the granularity of the routed down layout), so its
+// output rows need no exchange with other CTAs.
 //
 // Layer definition: vLLM recipe page "inclusionAI/Ling-3.0-flash" (Overview;
 // "Single-GPU int4": symmetric W4, group 32, routed experts only) and the
@@ -55,12 +58,12 @@ __device__ __forceinline__ void g_clk_sink(float) {}
 
 constexpr int kWarps = kDecodeWarps;
 constexpr int kBufA = kGuHalfBytes;                 // per-warp buffer, phases 1-3 (one K half of a unit)
-constexpr int kDnBatch = 4;                         // routed down units per copy batch
+constexpr int kDnBatch = 2;                         // routed down units per copy batch
 constexpr int kBufB = kDnBatch * kDnUnitBytes;      // per-warp buffer, phase 4
-constexpr int kShDnBytes = 4 * kI * 2;              // 4 shared-down rows
-constexpr int kMaxBlkPerCta = 8;                    // down row-blocks per CTA (>= 640 / nctas)
-constexpr int kDnPrefBlk = 5;                       // T = 1: routed down units kept in shared memory
-                                                    // when the CTA has <= 5 row-blocks (>= 128 CTAs)
+constexpr int kShDnBytes = 4 * kI * 2;              // 4 shared-down rows (half a row-block)
+constexpr int kMaxBlkPerCta = 4;                    // 8-row down blocks per CTA (>= 320 / nctas, nctas >= 80)
+constexpr int kDnPrefBlk = 3;                       // T = 1: routed down units kept in shared memory
+                                                    // when the CTA has <= 3 row-blocks (>= 107 CTAs)
 constexpr int kGuPiece = kGuHalfCodes / 4;          // 2560 B: 5 chunks of a gate/up half-unit
 constexpr int kPairs = kDecodeWarps / 2;            // phase-3 warp pairs (one K half each)
 constexpr int kRowBytes = kH * 2;                   // one bf16 row of H
@@ -98,7 +101,8 @@ constexpr int kXbTok = kH * 2;                   // bytes per token, bf16
 constexpr int kXfTok = (kH / 64) * 128;          // 5120 bytes per token
 
 // Shared-memory plan (byte offsets into the body).  Region A (phases 1-3)
-// and region B (phase 4) overlap: B is used only after the CTA's own phase 3.
+// and region B (phase 4) overlap: B is used only after the CTA's own phase 3,
+// and so is region D (T = 1), which follows B.
 template <int T>
 struct Plan {
   static constexpr int P = T * kMaxTopK;
@@ -107,19 +111,18 @@ struct Plan {
   static constexpr size_t comb = xf + (size_t)T * kXfTok;                   // float [pairs][2][32][4]
   static constexpr size_t bufA = comb + (size_t)kPairs * 2 * 32 * 16;       // [warps][kBufA]
   static constexpr size_t endA = bufA + (size_t)kWarps * kBufA;
-  static constexpr size_t hp = 0;                                           // float [P][kHpStride]
-  static constexpr size_t chp = hp + (size_t)P * kHpStride * 4;             // float [P][kHGroups]
-  static constexpr size_t hs = chp + (size_t)P * kHGroups * 4;              // float [T][kHsTok]
-  static constexpr size_t part = hs + (size_t)T * kHsTok * 4;               // float [blk][P + T][4]
-  static constexpr size_t bufB = part + (size_t)kMaxBlkPerCta * (P + T) * 16;
+  static constexpr size_t hf = 0;                                           // [P][kHfStride] h as MMA A fragments
+  static constexpr size_t hs = hf + (size_t)P * kHfStride;                  // float [T][kHsTok]
+  static constexpr size_t part = hs + (size_t)T * kHsTok * 4;               // float [blk][P + T][8]
+  static constexpr size_t bufB = part + (size_t)kMaxBlkPerCta * (P + T) * 32;
   static constexpr size_t endB = bufB + (size_t)kWarps * kBufB;
-  static constexpr size_t endAB = endA > endB ? endA : endB;
-  // T = 1: the CTA's routed down units, [expert slot][row-block] x 1728 B
-  static constexpr size_t dn = endAB;
-  static constexpr size_t body = dn + (T == 1 ? (size_t)kMaxTopK * kDnPrefBlk * kDnUnitBytes : 0);
+  // T = 1: the CTA's routed down units, [expert slot][row-block] x kDnUnitBytes
+  static constexpr size_t dn = endB;
+  static constexpr size_t endD = dn + (T == 1 ? (size_t)kMaxTopK * kDnPrefBlk * kDnUnitBytes : 0);
+  static constexpr size_t body = endA > endD ? endA : endD;
   static constexpr size_t bytes = sizeof(SmemHeader) + body;
-  static_assert(xf % 16 == 0 && comb % 16 == 0 && bufA % 16 == 0 && bufB % 16 == 0 && chp % 16 == 0 &&
-                hs % 16 == 0 && part % 16 == 0 && dn % 16 == 0, "16-byte aligned regions");
+  static_assert(xf % 16 == 0 && comb % 16 == 0 && bufA % 16 == 0 && bufB % 16 == 0 && hs % 16 == 0 &&
+                part % 16 == 0 && dn % 16 == 0, "16-byte aligned regions");
   static_assert(bytes <= 227 * 1024, "decode smem over budget");
 };
 
@@ -232,7 +235,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
 
   // L2 prefetch of the shared down rows this CTA will need
   if (warp == kWarps - 1 && lane == 0 && nblk > 0)
-    prefetch_l2_bulk(p.sh_down + (size_t)b0 * 4 * kI, (uint32_t)nblk * kShDnBytes);
+    prefetch_l2_bulk(p.sh_down + (size_t)b0 * kDnUnitRows * kI, (uint32_t)nblk * 2 * kShDnBytes);
 
   // x (bf16) lands in shared memory; every warp waits for it once
   if (!mbar_wait(&hd.xbar, 0, p.wait_limit_ns, p.err)) hd.abort = 1;
@@ -429,7 +432,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       }
     }
   };
-  if (u0 + pair < u1 && !aborted(hd)) issue3(u0 + pair);
+  const bool first_issued = u0 + pair < u1 && __shfl_sync(0xffffffffu, !aborted(hd), 0);  // one view per warp
+  if (first_issued) issue3(u0 + pair);
   if (!use_d && warp == kWarps - 1 && nblk > 0) {
     // routed down units of this CTA (contiguous per expert) into L2
     for (int u = lane; u < U; u += 32) {
@@ -442,10 +446,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     float* comb = reinterpret_cast<float*>(body + PL::comb) + (size_t)pair * (2 * 32 * 4);
     const int n = lane >> 2, m = lane & 3;  // B column (token of the expert) / lane class
     int par = 0;
-    bool issued = u0 + pair < u1 && !aborted(hd);
+    bool issued = first_issued;
     for (int unit = u0 + pair; unit < u1; unit += kPairs, par ^= 1) {
       if (unit != u0 + pair) {
-        issued = !aborted(hd);
+        issued = __shfl_sync(0xffffffffu, !aborted(hd), 0);
         if (issued) issue3(unit);
       }
       const int u = unit / kGuUnits, b = unit - u * kGuUnits;
@@ -454,13 +458,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       const unsigned char* xrow = xf + (bval ? hd.uniq_pair[u][n] / K : 0) * kXfTok + m * 32 +
                                   half * (kGuChunks / 2) * 128;
       float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-      bool ok = issued && mbar_wait(barA, pha, p.wait_limit_ns, p.err);
+      bool ok = issued && mbar_wait_warp(barA, pha, p.wait_limit_ns, p.err);
       if (issued) pha ^= 1;
       if (warp == 0 && unit == u0) { LING_TRACE(13); LING_CLK(6); }
 #pragma unroll 1
       for (int pc = 0; pc < 4 && ok; ++pc) {
         if (pc > 0) {
-          ok = mbar_wait(&hd.mbar[warp][pc], phq, p.wait_limit_ns, p.err);
+          ok = mbar_wait_warp(&hd.mbar[warp][pc], phq, p.wait_limit_ns, p.err);
           if (!ok) break;
           if (warp == 0 && unit == u0) LING_CLK(6 + pc);
         }
@@ -526,7 +530,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   if (use_d && warp == kWarps - 1 && U > 0 && !aborted(hd)) {
     // T = 1: this CTA's routed down units, one contiguous copy per expert,
     // requested now so that they stream in during the h exchange (during the
-    // gate/up phase they would only share its bandwidth)
+    // gate/up phase they would only share its bandwidth).  Region D overlays
+    // the phase 1-3 buffers, read until the barrier above.
+    fence_async_smem();
     const uint32_t per = (uint32_t)nblk * kDnUnitBytes;
     if (lane == 0) mbar_arrive_expect_tx(&hd.dbar, per * (uint32_t)U);
     __syncwarp();
@@ -543,8 +549,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   const int nitems = nblk * U;
   const int nbatch = use_d ? 0 : (nitems + kDnBatch - 1) / kDnBatch;
   const int nmine_r = warp < nbatch ? (nbatch - warp + kWarps - 1) / kWarps : 0;
-  const int sh_first = kWarps - 1 - warp;
-  const int nmine_s = (!aborted(hd) && sh_first < nblk) ? (nblk - sh_first + kWarps - 1) / kWarps : 0;
+  const int sh_first = kWarps - 1 - warp;  // shared down: half-blocks of 4 rows
+  const int nsub = 2 * nblk;
+  const int nmine_s = (!aborted(hd) && sh_first < nsub) ? (nsub - sh_first + kWarps - 1) / kWarps : 0;
   auto issue4 = [&](int s) {
     if (lane == 0) {
       if (s < nmine_r) {
@@ -557,17 +564,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
                    p.dn + ((size_t)hd.uniq_e[u] * kDnUnits + b0 + blk) * kDnUnitBytes, kDnUnitBytes, barA);
         }
       } else {
-        const int blk = sh_first + (s - nmine_r) * kWarps;
+        const int sb = sh_first + (s - nmine_r) * kWarps;
         mbar_arrive_expect_tx(barA, kShDnBytes);
-        bulk_g2s(bufB, p.sh_down + (size_t)(b0 + blk) * 4 * kI, kShDnBytes, barA);
+        bulk_g2s(bufB, p.sh_down + ((size_t)2 * b0 + sb) * 4 * kI, kShDnBytes, barA);
       }
     }
   };
   const int nseq = nmine_r + nmine_s;
+  fence_async_smem();  // region B overlays buffers read through the generic proxy
   if (nseq > 0) issue4(0);
 
-  float* hp = reinterpret_cast<float*>(body + PL::hp);
-  float* chp = reinterpret_cast<float*>(body + PL::chp);
+  unsigned char* hfb = body + PL::hf;
   float* hsm = reinterpret_cast<float*>(body + PL::hs);
   float* part = reinterpret_cast<float*>(body + PL::part);
   if (tid == 0 && !aborted(hd)) {
@@ -596,8 +603,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       for (int b = 0; b < kB; ++b) {
         const int v = v0 + b * kDecodeThreads;
         if (v < nh) {
-          const int pr = v / (kI / 4), c4 = v - pr * (kI / 4), e0 = 4 * c4;
-          *reinterpret_cast<float4*>(hp + (size_t)pr * kHpStride + e0 + 4 * (e0 / 96)) = hv[b];
+          // h * 2^-8 as fp16 hi + lo in MMA A-fragment order
+          const int pr = v / (kI / 4), k = 4 * (v - pr * (kI / 4));
+          unsigned char* dst = hfb + (size_t)pr * kHfStride + hf_off(k);
+          *reinterpret_cast<uint2*>(dst) = h_split2(hv[b].x, hv[b].y);
+          *reinterpret_cast<uint2*>(dst + 16) = h_split2(hv[b].z, hv[b].w);
         } else if (v < nall) {
           const int t = (v - nh) / (kI / 4), c4 = (v - nh) - t * (kI / 4), c = c4 >> 1, pl = c4 & 1;
           *reinterpret_cast<float4*>(hsm + (size_t)t * kHsTok + pl * kHsPlane + 4 * c) = hv[b];
@@ -607,81 +617,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   }
   __syncthreads();
   LING_TRACE(6);
-  {
-    // group sums of h, 8 lanes per group of 32 (conflict-free 16-byte reads)
-    const int sub = lane & 7, gw = lane >> 3;
-    for (int g0 = warp * 4; g0 < npairs * kHGroups; g0 += kWarps * 4) {
-      const int g = g0 + gw;
-      float sum = 0.f;
-      if (g < npairs * kHGroups) {
-        const int pr = g / kHGroups, G = g - pr * kHGroups;
-        const float4 v = ldsf4(hp + (size_t)pr * kHpStride + 32 * G + 4 * (G / 3) + 4 * sub);
-        sum = (v.x + v.y) + (v.z + v.w);
-      }
-      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 4);
-      if (sub == 0 && g < npairs * kHGroups) chp[g] = kBiasCoef * sum;
-    }
-  }
-  __syncthreads();
-  LING_TRACE(7);
-
-  // one routed down unit (4 output rows of expert slot u, row-block blk):
-  // partial sums per pair into part[], weighted by the routing weight
+  // one routed down unit (8 output rows of expert slot u, row-block blk) on
+  // the tensor cores: per pair, the partial sums times the routing weight go
+  // to part[]
   auto down_item = [&](const unsigned char* base, int blk, int u) {
-    const int r = lane & 3, q = lane >> 2;
-    const int cnt = hd.uniq_cnt[u];
-    int ho[T], co[T];
-#pragma unroll
-    for (int tt = 0; tt < T; ++tt) {
-      const int pr = (tt < cnt) ? hd.uniq_pair[u][tt] : 0;
-      ho[tt] = pr * kHpStride + 100 * q;
-      co[tt] = pr * kHGroups + q * kDnChunks;
-    }
-    float acc[T];
-#pragma unroll
-    for (int tt = 0; tt < T; ++tt) acc[tt] = 0.f;
-#pragma unroll
-    for (int j = 0; j < kDnChunks; ++j) {
-      const uint4 w = lds128(base + j * 512 + 16 * lane);
-      const float sj = bf16_to_f32(
-          *reinterpret_cast<const unsigned short*>(base + kDnScaleOff + j * 64 + 2 * lane));
-      float pa[T], pb[T], pc[T], pd[T];
-#pragma unroll
-      for (int tt = 0; tt < T; ++tt) {
-        pa[tt] = (tt < cnt) ? chp[co[tt] + j] : 0.f;
-        pb[tt] = pc[tt] = pd[tt] = 0.f;
-      }
-      const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float f[8];
-        dequant8(wv[i], f);
-#pragma unroll
-        for (int tt = 0; tt < T; ++tt) {
-          if (tt < cnt) {
-            const float* hq = hp + ho[tt] + 32 * j + 8 * i;
-            if (i & 1) dot8_f_2(f, ldsf4(hq), ldsf4(hq + 4), pc[tt], pd[tt]);
-            else dot8_f_2(f, ldsf4(hq), ldsf4(hq + 4), pa[tt], pb[tt]);
-          }
-        }
-      }
-#pragma unroll
-      for (int tt = 0; tt < T; ++tt) acc[tt] = fmaf(sj, (pa[tt] + pb[tt]) + (pc[tt] + pd[tt]), acc[tt]);
-    }
-#pragma unroll
-    for (int tt = 0; tt < T; ++tt) {
-      if (tt < cnt) {
-        float v = acc[tt];
-        v += __shfl_xor_sync(0xffffffffu, v, 4);
-        v += __shfl_xor_sync(0xffffffffu, v, 8);
-        v += __shfl_xor_sync(0xffffffffu, v, 16);
-        if (q == 0) {
-          const int pr = hd.uniq_pair[u][tt];
-          part[((size_t)blk * (PL::P + T) + pr) * 4 + r] = kCodeScale * v * hd.topw[pr / K][pr % K];
-        }
-      }
+    const int g = lane >> 2, c = lane & 3;
+    const bool act = g < hd.uniq_cnt[u];
+    const int pr = act ? hd.uniq_pair[u][g] : 0;
+    float v0, v1;
+    dn_unit_mma(base, hfb + (size_t)pr * kHfStride + 16 * c, act, lane, v0, v1);
+    if (act) {
+      const float f = (float)(1 << kHShift) * hd.topw[pr / K][pr % K];
+      *reinterpret_cast<float2*>(part + ((size_t)blk * (PL::P + T) + pr) * 8 + 2 * c) = make_float2(v0 * f, v1 * f);
     }
   };
   if (use_d && !aborted(hd) && warp < nitems) {
@@ -711,7 +658,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
           down_item(bufB + bI * kDnUnitBytes, blk, u);
         }
       } else {
-        const int blk = sh_first + (s - nmine_r) * kWarps;
+        const int sb = sh_first + (s - nmine_r) * kWarps;
         float acc[T];
         {
           float a0[T], a1[T], a2[T], a3[T];
@@ -738,7 +685,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
           v += __shfl_xor_sync(0xffffffffu, v, 4);
           v += __shfl_xor_sync(0xffffffffu, v, 8);
           v += __shfl_xor_sync(0xffffffffu, v, 16);
-          if (q == 0) part[((size_t)blk * (PL::P + T) + PL::P + t) * 4 + r] = v;
+          if (q == 0) part[((size_t)(sb >> 1) * (PL::P + T) + PL::P + t) * 8 + 4 * (sb & 1) + r] = v;
         }
       }
       __syncwarp();
@@ -748,13 +695,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   LING_TRACE(8);
   if (!aborted(hd)) {
     // fixed-order sum: routed slots 0..k-1, then the shared expert
-    for (int v = tid; v < nblk * T * 4; v += kDecodeThreads) {
-      const int blk = v / (T * 4), rem = v - blk * T * 4, t = rem >> 2, r = rem & 3;
-      const float* pb = part + (size_t)blk * (PL::P + T) * 4;
+    for (int v = tid; v < nblk * T * kDnUnitRows; v += kDecodeThreads) {
+      const int blk = v / (T * kDnUnitRows), rem = v - blk * T * kDnUnitRows, t = rem >> 3, r = rem & 7;
+      const float* pb = part + (size_t)blk * (PL::P + T) * 8;
       float s = 0.f;
-      for (int sl = 0; sl < K; ++sl) s += pb[(t * K + sl) * 4 + r];
-      s += pb[(PL::P + t) * 4 + r];
-      p.out[(size_t)t * kH + 4 * (b0 + blk) + r] = __float2bfloat16_rn(s);
+      for (int sl = 0; sl < K; ++sl) s += pb[(t * K + sl) * 8 + r];
+      s += pb[(PL::P + t) * 8 + r];
+      p.out[(size_t)t * kH + kDnUnitRows * (b0 + blk) + r] = __float2bfloat16_rn(s);
     }
   }
   // every CTA (aborted or not) counts itself out: the next launch's index

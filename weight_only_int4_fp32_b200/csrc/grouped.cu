@@ -9,8 +9,10 @@
 //                (N-tiles of <= 128 positions, the costly ones first)
 //   scatter      each pair gets a position in its expert's run; x is written
 //                in fp16 by position (8 routed copies + 1 shared row per token)
-//   gate/up      tcgen05 tiles over routed experts and the shared expert
-//   down         tcgen05 tiles: y[position] = w * Wd h[position]
+//   gate/up      tcgen05 tiles over the routed experts with more than
+//                kGvMaxTok tokens and the shared expert; a GEMV kernel
+//                (mma.sync on streamed weights) for the experts with fewer
+//   down         the same split: y[position] = w * Wd h[position]
 //   combine      out[t] = sum_slot y[position of (t, slot)] + y[shared row t],
 //                one bf16 rounding, slots summed in a fixed order
 //
@@ -22,6 +24,7 @@
 
 #include "common.cuh"
 #include "grouped.h"
+#include "grouped_gemv.h"
 
 namespace lingmoe {
 
@@ -67,6 +70,8 @@ cudaError_t grouped_alloc(GroupedWorkspace* ws, int E, int k, int max_T, const A
       {(void**)&ws->gu_tiles, nt * kTcMTilesGu * sizeof(int4)},
       {(void**)&ws->dn_tiles, nt * kTcMTilesDn * sizeof(int4)},
       {(void**)&ws->ntiles, 4 * sizeof(int32_t)},
+      {(void**)&ws->small, (size_t)E * sizeof(int4)},
+      {(void**)&ws->nsmall, 4 * sizeof(int32_t)},
   };
   for (auto& a : plan)
     if ((e = alloc(a.p, a.n)) != cudaSuccess) return e;
@@ -225,6 +230,8 @@ __global__ void __launch_bounds__(256) grp_topk_kernel(GroupedParams p, const fl
 
 // ---------------------------------------------------------------- plan
 // One CTA, thread e <= E (e == E is the shared expert over all T tokens).
+// Routed experts with 1..kGvMaxTok tokens go to the GEMV list (small), the
+// others and the shared expert to the tile lists.
 // Position runs: off[e] = exclusive scan of the pair counts.  N-tiles of
 // <= 128 positions: the full ones and each expert's remainder, bucketed by
 // MMA width (16..128 in steps of 16) and listed widest first, so that the
@@ -238,19 +245,21 @@ __device__ __forceinline__ void write_ntile(int idx, int e, int pos0, int n, int
 
 __global__ void __launch_bounds__(kPlanThreads) grp_plan_kernel(int T, int E, int32_t* cnt, int32_t* fill,
                                                                 int32_t* off, int4* gu_tiles, int4* dn_tiles,
-                                                                int32_t* ntiles) {
-  constexpr int NV = 9;  // [0] pairs, [1 + b] N-tiles of width bucket b
+                                                                int32_t* ntiles, int4* small, int32_t* nsmall) {
+  constexpr int NV = 10;  // [0] pairs, [1 + b] N-tiles of width bucket b, [9] GEMV experts
   __shared__ int wtot[kPlanThreads / 32][NV];
   __shared__ int wbase[kPlanThreads / 32][NV];
   __shared__ int total[NV];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int c = t < E ? cnt[t] : (t == E ? T : 0);
-  const int full = c / kTcTileN, rem = c % kTcTileN;
+  const bool gemv = t < E && c > 0 && c <= kGvMaxTok;
+  const int full = gemv ? 0 : c / kTcTileN, rem = gemv ? 0 : c % kTcTileN;
   const int pb = rem > 0 ? (rem + 15) / 16 - 1 : -1;
   int v[NV];
   v[0] = t < E ? c : 0;
 #pragma unroll
   for (int b = 0; b < 8; ++b) v[1 + b] = (b == 7 ? full : 0) + (pb == b ? 1 : 0);
+  v[9] = gemv ? 1 : 0;
   // block exclusive scan of the 9 values
   int incl[NV];
 #pragma unroll
@@ -289,12 +298,14 @@ __global__ void __launch_bounds__(kPlanThreads) grp_plan_kernel(int T, int E, in
     if (t == 0) {
       ntiles[0] = a * kTcMTilesGu;
       ntiles[1] = a * kTcMTilesDn;
+      nsmall[0] = total[9];
     }
   }
   const int P = total[0];
   if (t < E) off[t] = excl[0];
   if (t == E) off[E] = P;
-  if (t <= E) {
+  if (gemv) small[excl[9]] = make_int4(t, excl[0], c, 0);
+  if (t <= E && !gemv) {
     const int pos_base = t < E ? excl[0] : P;
     const int i7 = bstart[7] + excl[8];
     for (int q = 0; q < full; ++q) write_ntile(i7 + q, t, pos_base + kTcTileN * q, kTcTileN, gu_tiles, dn_tiles);
@@ -384,6 +395,7 @@ cudaError_t setup_grouped() {
   if ((e = cudaFuncSetAttribute(grp_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRtSmem)) !=
       cudaSuccess)
     return e;
+  if ((e = setup_grouped_gemv()) != cudaSuccess) return e;
   return setup_grouped_tc();
 }
 
@@ -398,7 +410,8 @@ cudaError_t launch_grouped(const GroupedParams& p, const GroupedWorkspace& ws, c
   ++nl;
   grp_topk_kernel<<<(p.T + 7) / 8, 256, 0, s>>>(p, ws.logits, ws.topk_idx, ws.topk_w, ws.cnt);
   ++nl;
-  grp_plan_kernel<<<1, kPlanThreads, 0, s>>>(p.T, p.E, ws.cnt, ws.fill, ws.off, ws.gu_tiles, ws.dn_tiles, ws.ntiles);
+  grp_plan_kernel<<<1, kPlanThreads, 0, s>>>(p.T, p.E, ws.cnt, ws.fill, ws.off, ws.gu_tiles, ws.dn_tiles, ws.ntiles,
+                                             ws.small, ws.nsmall);
   ++nl;
   grp_scatter_kernel<<<p.T, kRowThreads, 0, s>>>(p.x, p.k, P, ws.topk_idx, ws.off, ws.fill, ws.perm, ws.inv, ws.xg,
                                                  ws.xscale);
@@ -422,7 +435,25 @@ cudaError_t launch_grouped(const GroupedParams& p, const GroupedWorkspace& ws, c
   tp.xg = ws.xg;
   tp.shgu16 = ws.shgu16;
   tp.shdn16 = ws.shdn16;
+  GvParams gv{};
+  gv.gu = p.gu;
+  gv.dn = p.dn;
+  gv.xg = ws.xg;
+  gv.xscale = ws.xscale;
+  gv.perm = ws.perm;
+  gv.topk_w = ws.topk_w;
+  gv.k = p.k;
+  gv.h16 = ws.h16;
+  gv.y = ws.y;
+  gv.small = ws.small;
+  gv.nsmall = ws.nsmall;
+  gv.err = ws.err;
+  gv.wait_limit_ns = 2000000000ull;
+  if ((e = launch_gemv_gu(gv, p.num_sms, s)) != cudaSuccess) return e;
+  ++nl;
   if ((e = launch_tc_gemm(0, ws.maps, tp, p.num_sms, s)) != cudaSuccess) return e;
+  ++nl;
+  if ((e = launch_gemv_dn(gv, p.num_sms, s)) != cudaSuccess) return e;
   ++nl;
   if ((e = launch_tc_gemm(1, ws.maps, tp, p.num_sms, s)) != cudaSuccess) return e;
   ++nl;

@@ -49,6 +49,8 @@ struct GroupedWorkspace {
   int4* gu_tiles = nullptr;     // tcgen05 tile lists
   int4* dn_tiles = nullptr;
   int32_t* ntiles = nullptr;    // [2]
+  int4* small = nullptr;        // [E] experts for the GEMV kernels: (expert, first position, tokens, 0)
+  int32_t* nsmall = nullptr;    // [1] entries in small
   TcMaps maps{};
   unsigned int* err = nullptr;  // the handle's sticky device error word
 };

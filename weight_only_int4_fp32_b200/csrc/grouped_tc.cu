@@ -15,10 +15,8 @@
 // directly.  The activations are the B operand, fetched by TMA from buffers
 // in position order: x (fp16, exact after a per-token power-of-two scale) for
 // gate/up and h as two fp16 terms hi + lo (~22 significant bits) for down.
-// Gate/up tiles are in natural K order: a producer gathers one row's 16-K
-// block from the four MMA-fragment words that hold it.  Down tiles and h use
-// the per-8-element order in which a LOP3 extracts nibbles from a 32-code
-// group.  Either way A and B agree, so nothing is permuted in the main loop.
+// All tiles are in natural K order: a producer gathers one row's K slice
+// from the four MMA-fragment words of the repacked layouts that hold it.
 //
 // One thread issues tcgen05.mma into a double-buffered TMEM accumulator
 // (2 x 256 columns); tcgen05.commit releases each pipeline stage, and 4
@@ -52,11 +50,11 @@ constexpr int kBoxRows = 32;                    // B rows per TMA box
 constexpr int kBoxBytes = kBoxRows * kTcK * 2;  // 4 KB
 constexpr int kShBoxRows = 128;                 // shared-expert A rows per TMA box
 constexpr int kTmemCols = 512;                  // 2 buffers x (2 M-halves x 128 columns)
-// raw ring, per stage.  Gate/up: int4 codes [4 fragment lanes][256 threads]
-// x 8 B, then [256] x 4 B (gate, up) scale words.  Down: codes [2 groups]
-// [256 threads] x 16 B, then [2][256] x 4 B words holding each group's scale.
-constexpr int kRawCodes = 2 * kProd * 16;
-constexpr int kRawStage = kRawCodes + 2 * kProd * 4;  // 10 KB
+// raw ring, per stage: int4 codes [4 fragment lanes][256 threads] x 8 B, then
+// per thread the scale words: gate/up one (gate, up) word of 4 B, down the
+// two 4-byte (row pair) words of the stage's two groups.
+constexpr int kRawCodes = 4 * kProd * 8;
+constexpr int kRawStage = kRawCodes + kProd * 8;  // 10 KB
 constexpr unsigned long long kTcWaitNs = 2000000000ull;
 
 __host__ __device__ constexpr int tc_bparts(int mode) { return mode == 0 ? 1 : 2; }
@@ -74,10 +72,6 @@ __host__ __device__ constexpr size_t tc_smem(int mode) {
 static_assert(tc_smem(1) <= 232448, "down-projection pipeline exceeds 227 KB of shared memory");
 static_assert(tc_smem(0) <= 232448, "gate/up pipeline exceeds 227 KB of shared memory");
 
-// K order inside each group of 8 elements: element o sits at position
-// perm_pos(o).  It is the order in which (w >> 4s) & 0x000F000F yields nibble
-// pairs (e_s, e_{s+4}).
-__host__ __device__ constexpr int perm_pos(int o) { return (o < 4) ? 2 * o : 2 * (o - 4) + 1; }
 
 // ---------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
@@ -102,7 +96,6 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
 }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared.b64 _, [%0];" :: "r"(smem_u32(bar)) : "memory");
 }
@@ -183,26 +176,6 @@ __device__ __forceinline__ uint32_t deq_pair(uint32_t v, __half2 s2, __half2 b2)
   const __half2 r = __hmul2(q, s2);
   return *reinterpret_cast<const uint32_t*>(&r);
 }
-// 32 codes (16 bytes, offset-binary nibbles) of one group with scale s' ->
-// 32 fp16 in permuted K order, as 4 x 16 bytes.
-__device__ __forceinline__ void deq_group(uint4 q, float s, uint4 out[4]) {
-  const __half sh = __float2half_rn(s);
-  const __half2 s2 = __halves2half2(sh, sh);
-  const __half bh = __float2half_rn(1032.0f);
-  const __half2 b2 = __halves2half2(bh, bh);
-  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint32_t p[4];
-#pragma unroll
-    for (int sft = 0; sft < 4; ++sft) {
-      uint32_t v;
-      asm("lop3.b32 %0, %1, 0x000F000F, 0x64006400, 0xEA;" : "=r"(v) : "r"(w[i] >> (4 * sft)));
-      p[sft] = deq_pair(v, s2, b2);  // (e_sft, e_{sft+4}) -> positions 2 sft, 2 sft + 1
-    }
-    out[i] = make_uint4(p[0], p[1], p[2], p[3]);
-  }
-}
 
 // ---------------------------------------------------------------- shared-expert fp16 copies
 // Power-of-two exponent c with max|w| * 2^c in [2^14, 2^15) (0 for an all-zero
@@ -230,9 +203,9 @@ __global__ void __launch_bounds__(256) sh_amax_kernel(const __nv_bfloat16* g, co
 }
 
 // One thread per 8 consecutive K elements: scale by 2^c, convert to fp16.
-// Gate/up keep the natural K order (the order of the routed gate/up tiles);
-// down takes the permuted order of h.  Gate/up rows are laid out per block of
-// 128 intermediate rows i: 128 gate rows, then the 128 up rows of the same i.
+// All keep the natural K order of the routed tiles.  Gate/up rows are laid out
+// per block of 128 intermediate rows i: 128 gate rows, then the 128 up rows of
+// the same i.
 __global__ void __launch_bounds__(256) sh_convert_kernel(const __nv_bfloat16* g, const __nv_bfloat16* u,
                                                          const __nv_bfloat16* d, const unsigned int* amax,
                                                          __half* shgu16, __half* shdn16, float* sh_scale) {
@@ -249,7 +222,7 @@ __global__ void __launch_bounds__(256) sh_convert_kernel(const __nv_bfloat16* g,
                         bf16lo(x.z), bf16hi(x.z), bf16lo(x.w), bf16hi(x.w)};
     __half h[8];
 #pragma unroll
-    for (int o = 0; o < 8; ++o) h[m < 2 ? o : perm_pos(o)] = __float2half_rn(e[o] * f);
+    for (int o = 0; o < 8; ++o) h[o] = __float2half_rn(e[o] * f);
     const int grow = 2 * (row & ~127) + 128 * m + (row & 127);
     __half* dst = m < 2 ? shgu16 + (size_t)grow * kH + k0 : shdn16 + (size_t)row * kI + k0;
     *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(h);
@@ -281,8 +254,8 @@ __device__ __forceinline__ void prefetch_tile(const TcParams& p, int4 tl, const 
       a = p.gu + ((size_t)tl.x * kGuUnits + (size_t)tl.y * (kTcTileM / 16)) * kGuUnitBytes;
       abytes = (size_t)(kTcTileM / 16) * kGuUnitBytes;
     } else {
-      a = p.dn + ((size_t)tl.x * kDnUnits + (size_t)tl.y * (kTcTileM / 4)) * kDnUnitBytes;
-      abytes = (size_t)(kTcTileM / 4) * kDnUnitBytes;
+      a = p.dn + ((size_t)tl.x * kDnUnits + (size_t)tl.y * (kTcTileM / kDnUnitRows)) * kDnUnitBytes;
+      abytes = (size_t)(kTcTileM / kDnUnitRows) * kDnUnitBytes;
     }
   } else {
     const int K = MODE == 0 ? kH : kI;
@@ -391,17 +364,17 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
 #pragma unroll
             for (int m = 0; m < 4; ++m)
               cp_async8(slot + m * (kProd * 8) + r * 8, ub + kk * 512 + 16 * (4 * (i & 7) + m) + 8 * kh);
-            cp_async4(slot + 4 * (kProd * 8) + r * 4, ub + kGuScaleOff + (2 * kk + kh) * 32 + 4 * (i & 7));
+            cp_async4(slot + kRawCodes + r * 4, ub + kGuScaleOff + (2 * kk + kh) * 32 + 4 * (i & 7));
           } else {
+            // output row n, groups G = 2 kk and G + 1: 8 bytes from each of the
+            // four fragment lanes 4 (n % 8) + m, and the two scale words of
+            // the row pair that holds n
+            const int n = kTcTileM * tl.y + r, G = 2 * kk;
+            const uint8_t* ub = p.dn + ((size_t)tl.x * kDnUnits + (n >> 3)) * kDnUnitBytes;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int G = 2 * kk + h;
-              const int n = kTcTileM * tl.y + r;
-              const uint8_t* abase = p.dn + ((size_t)tl.x * kDnUnits + (n >> 2)) * kDnUnitBytes;
-              const int slice = G / kDnChunks, jj = G - slice * kDnChunks, ln = (n & 3) + 4 * slice;
-              cp_async16(slot + h * (kProd * 16) + r * 16, abase + jj * 512 + 16 * ln);
-              cp_async4(slot + kRawCodes + h * (kProd * 4) + r * 4, abase + kDnScaleOff + jj * 64 + 4 * (ln >> 1));
-            }
+            for (int m = 0; m < 4; ++m)
+              cp_async8(slot + m * (kProd * 8) + r * 8, ub + (G >> 2) * 512 + 16 * (4 * (n & 7) + m) + 4 * (G & 3));
+            cp_async8(slot + kRawCodes + r * 8, ub + kDnScaleOff + (G >> 2) * 64 + 16 * ((n & 7) >> 1) + 4 * (G & 3));
           }
         }
       }
@@ -430,7 +403,7 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
           // exact fp16 q * s * 2^8 for gate row il and up row 128 + il, K blocks
           // 2 kh and 2 kh + 1 of this stage (natural K order)
           const int il = r & 127, kh = r >> 7;
-          const uint32_t sw = *reinterpret_cast<const uint32_t*>(slot + 4 * (kProd * 8) + r * 4);
+          const uint32_t sw = *reinterpret_cast<const uint32_t*>(slot + kRawCodes + r * 4);
           const float sgf = __uint_as_float(sw << 16) * (float)(1 << kTcScaleShift);
           const float suf = __uint_as_float(sw & 0xFFFF0000u) * (float)(1 << kTcScaleShift);
           const __half2 sg = __float2half2_rn(sgf), sg16 = __float2half2_rn(sgf * 0.0625f);
@@ -464,20 +437,41 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
             *reinterpret_cast<uint4*>(au + ((ch ^ (il & 7)) << 4)) = make_uint4(uhi[0], uhi[1], uhi[2], uhi[3]);
           }
         } else {
-          uint4 outv[8];
+          // exact fp16 q * s * 2^8 for output row n, groups 2 kk and 2 kk + 1:
+          // the fragment word of lane class m holds K = 2m, 2m+1 (even
+          // extraction), 2m+8, 2m+9 (odd, as 16 q), and the same + 16 in w >> 8
+          const int n = kTcTileM * tl.y + r;
+          const uint2 sw = *reinterpret_cast<const uint2*>(slot + kRawCodes + r * 8);
+          const __half2 be = __float2half2_rn(1032.0f), bo = __float2half2_rn(1152.0f);
+          uint2 cw[4];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int G = 2 * kk + h;
-            const int n = kTcTileM * tl.y + r;
-            const int hi_half = ((n & 3) + 4 * (G / kDnChunks)) & 1;
-            const uint4 q = *reinterpret_cast<const uint4*>(slot + h * (kProd * 16) + r * 16);
-            const uint32_t wv = *reinterpret_cast<const uint32_t*>(slot + kRawCodes + h * (kProd * 4) + r * 4);
-            const float sc = __uint_as_float(hi_half ? (wv & 0xFFFF0000u) : (wv << 16)) * (float)(1 << kTcScaleShift);
-            deq_group(q, sc, outv + 4 * h);
-          }
+          for (int m = 0; m < 4; ++m) cw[m] = *reinterpret_cast<const uint2*>(slot + m * (kProd * 8) + r * 8);
           unsigned char* a = sA + s * kStageA + r * 128;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(a + ((c ^ (r & 7)) << 4)) = outv[c];
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t ws = h ? sw.y : sw.x;
+            const float sf = __uint_as_float((n & 1) ? (ws & 0xFFFF0000u) : (ws << 16)) * (float)(1 << kTcScaleShift);
+            const __half2 s2 = __float2half2_rn(sf), s16 = __float2half2_rn(sf * 0.0625f);
+            uint32_t q0[4], q1[4], q2[4], q3[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+              const uint32_t w = h ? cw[m].y : cw[m].x;
+              uint32_t v0, v1, v2, v3;
+              asm("lop3.b32 %0, %1, 0x000F000F, 0x64006400, 0xEA;" : "=r"(v0) : "r"(w));
+              asm("lop3.b32 %0, %1, 0x00F000F0, 0x64006400, 0xEA;" : "=r"(v1) : "r"(w));
+              asm("lop3.b32 %0, %1, 0x000F000F, 0x64006400, 0xEA;" : "=r"(v2) : "r"(w >> 8));
+              asm("lop3.b32 %0, %1, 0x00F000F0, 0x64006400, 0xEA;" : "=r"(v3) : "r"(w >> 8));
+              q0[m] = deq_pair(v0, s2, be);
+              q1[m] = deq_pair(v1, s16, bo);
+              q2[m] = deq_pair(v2, s2, be);
+              q3[m] = deq_pair(v3, s16, bo);
+            }
+            const int c0 = 4 * h;
+            *reinterpret_cast<uint4*>(a + (((c0 + 0) ^ (r & 7)) << 4)) = make_uint4(q0[0], q0[1], q0[2], q0[3]);
+            *reinterpret_cast<uint4*>(a + (((c0 + 1) ^ (r & 7)) << 4)) = make_uint4(q1[0], q1[1], q1[2], q1[3]);
+            *reinterpret_cast<uint4*>(a + (((c0 + 2) ^ (r & 7)) << 4)) = make_uint4(q2[0], q2[1], q2[2], q2[3]);
+            *reinterpret_cast<uint4*>(a + (((c0 + 3) ^ (r & 7)) << 4)) = make_uint4(q3[0], q3[1], q3[2], q3[3]);
+          }
         }
         fence_async_smem();
       }
@@ -514,10 +508,9 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
       const uint32_t tb = tmem + ((uint32_t)(32 * qd) << 16) + (uint32_t)(b * 256);
       if (MODE == 0) {
         const int i = (kTcTileM / 2) * mt + l;
-        const int ip = (i & ~7) + perm_pos(i & 7);
         const float cg = shared ? p.sh_scale[0] : 1.f / (float)(1 << kTcScaleShift);
         const float cu = shared ? p.sh_scale[1] : 1.f / (float)(1 << kTcScaleShift);
-        __half* hrow = p.h16 + (size_t)pos0 * (2 * kI) + ip;
+        __half* hrow = p.h16 + (size_t)pos0 * (2 * kI) + i;
 #pragma unroll 1
         for (int c0 = 0; c0 < nmma; c0 += 16) {
           float g[16], u[16];

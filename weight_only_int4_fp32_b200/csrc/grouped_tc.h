@@ -26,7 +26,7 @@ struct TcParams {
   const uint8_t* gu;        // repacked routed gate/up
   const uint8_t* dn;        // repacked routed down
   const float* xscale;      // [T] 2^sigma_t: x16 rows hold x * 2^-sigma_t
-  __half* h16;              // [rows, 2, I] h * 2^-8 as fp16 hi + lo, permuted K order
+  __half* h16;              // [rows, 2, I] h * 2^-8 as fp16 hi + lo, natural K order
   float* y;                 // [rows, H] expert output per position, times the routing weight
   const int32_t* perm;      // position (< P) -> pair id t*k + slot
   const float* topk_w;      // [P] routing weight per pair id
@@ -54,8 +54,8 @@ cudaError_t setup_grouped_tc();
 cudaError_t tc_encode_maps(TcMaps* m, const __half* xg, const __half* h16, int rows, const __half* shgu16,
                            const __half* shdn16);
 // fp16 copies of the shared expert (gate/up in natural K order, 128 gate rows
-// then the 128 up rows of the same intermediate rows per block; down in the
-// permuted K order of h), each matrix scaled by a power of two 2^c so that max |w| * 2^c
+// then the 128 up rows of the same intermediate rows per block; down in
+// natural K order too), each matrix scaled by a power of two 2^c so that max |w| * 2^c
 // lies in [2^14, 2^15); sh_scale receives 2^-c.  amax_scratch: 3 words.
 cudaError_t launch_tc_prep_shared(const __nv_bfloat16* g, const __nv_bfloat16* u, const __nv_bfloat16* d,
                                   __half* shgu16, __half* shdn16, float* sh_scale, unsigned int* amax_scratch,

@@ -37,14 +37,25 @@ constexpr int kGuHalfCodes = kGuScaleOff / 2;     // 10240: codes of one K half
 constexpr int kGuHalfScales = (kH / kGroup) * 16; // 1280: scales of one K half
 constexpr int kGuHalfBytes = kGuHalfCodes + kGuHalfScales;  // 11520
 
-// Routed down, per expert: kDnUnits units, one per block of 4 output rows
-// n = 4v..4v+3; lane l owns row (l & 3) and K-slice (l >> 2) of 3 groups.
-// Chunk j (0..2) is 32 lanes x 16 B (group 3*slice + j of the lane's row),
-// then 3 blocks of [32 lanes x bf16 scale].
-constexpr int kDnUnits = kH / 4;                  // 640
-constexpr int kDnChunks = kI / 256;               // 3 groups per lane
-constexpr int kDnScaleOff = kDnChunks * 512;      // 1536
-constexpr int kDnUnitBytes = kDnScaleOff + kDnChunks * 64;  // 1728
+// Routed down, per expert: kDnUnits units, one per block of 8 output rows
+// n = 8v..8v+7 (all 768 K).  K is cut into groups of 32; a group is 32
+// words, and word t holds exactly the int4 codes of lane t's B fragments of
+// the two m16n8k16 MMAs (K blocks 32G and 32G + 16) whose columns are the
+// unit's 8 rows: row n_t = 8v + t/4, K = 32G + c, c + 1, c + 8, c + 9 and the
+// same + 16, with c = 2 (t % 4):
+//   nibble 0: c       nibble 4: c+1       nibble 1: c+8      nibble 5: c+9
+//   nibble 2: c+16    nibble 6: c+17      nibble 3: c+24     nibble 7: c+25
+// as offset-binary codes (q + 8), the nibble order of the gate/up words.  A
+// chunk of 512 B covers 128 K (4 groups): lane t's 16 bytes are its words for
+// groups 4j .. 4j+3.  The scales follow the kDnChunks chunks as 64-byte
+// blocks [c/2 (4)][group within the chunk (4)] of 32-bit words, each the bf16
+// pair (row 8v + c, row 8v + c + 1) of one group: the two output rows whose
+// results lane t's accumulator fragment holds.
+constexpr int kDnUnitRows = 8;
+constexpr int kDnUnits = kH / kDnUnitRows;        // 320
+constexpr int kDnChunks = kI / 128;               // 6 chunks of 128 K
+constexpr int kDnScaleOff = kDnChunks * 512;      // 3072
+constexpr int kDnUnitBytes = kDnScaleOff + kDnChunks * 64;  // 3456
 constexpr size_t kDnExpertBytes = (size_t)kDnUnits * kDnUnitBytes;  // 1105920
 
 static_assert(kGuChunks % 2 == 0, "gate/up units split into two K halves");

@@ -2,19 +2,11 @@
 // layout (two's-complement nibbles, low nibble = even K, row-major [rows, K/2],
 // bf16 scales [rows, K/32]) into the unit layouts the kernels stream.
 // The codes become offset-binary (q + 8) by flipping the top bit of every
-// nibble; nothing else about a 16-byte group changes.
+// nibble, and are regrouped into the MMA-fragment words of layout.h.
 #include "common.cuh"
 #include "repack.h"
 
 namespace lingmoe {
-
-__device__ __forceinline__ uint4 flip_sign_nibbles(uint4 v) {
-  v.x ^= 0x88888888u;
-  v.y ^= 0x88888888u;
-  v.z ^= 0x88888888u;
-  v.w ^= 0x88888888u;
-  return v;
-}
 
 // gate/up: one thread per 32-bit fragment word and per (group, row pair)
 // scale slot.  A word gathers two bytes of the gate row and two of the up row
@@ -61,29 +53,44 @@ __global__ void repack_gu_kernel(const uint8_t* __restrict__ gate_q, const uint8
   }
 }
 
-// down: one thread per 16-byte chunk slot and per 2-byte scale slot.
+// down: one thread per 32-bit fragment word and per (group, row pair) scale
+// word.  A word gathers four bytes of one row: K = 32G + c (+1), c + 8 (+9),
+// c + 16 (+17), c + 24 (+25).
 __global__ void repack_dn_kernel(const uint8_t* __restrict__ down_q, const uint16_t* __restrict__ down_s,
                                  uint8_t* __restrict__ dn, int E) {
-  const long long nslot = (long long)E * kDnUnits * kDnChunks * 32;
-  for (long long g = blockIdx.x * (long long)blockDim.x + threadIdx.x; g < 2 * nslot;
+  constexpr int kGroups = kI / kGroup;                // 24
+  const long long nword = (long long)E * kDnUnits * kGroups * 32;
+  const long long nscale = (long long)E * kDnUnits * kGroups * 4;
+  for (long long g = blockIdx.x * (long long)blockDim.x + threadIdx.x; g < nword + nscale;
        g += (long long)gridDim.x * blockDim.x) {
-    const bool is_scale = g >= nslot;
-    const long long g1 = is_scale ? g - nslot : g;
-    const int lane = (int)(g1 & 31);
-    const long long rest = g1 >> 5;
-    const int j = (int)(rest % kDnChunks);
-    const long long ev = rest / kDnChunks;  // e * kDnUnits + v
-    const int v = (int)(ev % kDnUnits);
-    const long long e = ev / kDnUnits;
-    const int r = lane & 3, q = lane >> 2;
-    const int n = 4 * v + r;
-    const int G = q * kDnChunks + j;
-    if (!is_scale) {
-      const uint4 w = *reinterpret_cast<const uint4*>(down_q + ((e * kH + n) * (kI / 2) + 16 * G));
-      *reinterpret_cast<uint4*>(dn + ev * kDnUnitBytes + j * 512 + 16 * lane) = flip_sign_nibbles(w);
+    if (g < nword) {
+      const int t = (int)(g & 31);
+      const long long rest = g >> 5;
+      const int G = (int)(rest % kGroups);
+      const long long ev = rest / kGroups;            // e * kDnUnits + v
+      const int v = (int)(ev % kDnUnits);
+      const long long e = ev / kDnUnits;
+      const int n = kDnUnitRows * v + (t >> 2);
+      const int c = kGroup * G + 2 * (t & 3);
+      const uint8_t* row = down_q + (e * kH + n) * (kI / 2);
+      const uint32_t b0 = row[c / 2], b1 = row[(c + 8) / 2], b2 = row[(c + 16) / 2], b3 = row[(c + 24) / 2];
+      uint32_t w = nib(b0, 0) | nib(b1, 0) << 4 | nib(b2, 0) << 8 | nib(b3, 0) << 12 |
+                   nib(b0, 1) << 16 | nib(b1, 1) << 20 | nib(b2, 1) << 24 | nib(b3, 1) << 28;
+      w ^= 0x88888888u;  // two's complement -> offset binary
+      *reinterpret_cast<uint32_t*>(dn + ev * kDnUnitBytes + (G >> 2) * 512 + 16 * t + 4 * (G & 3)) = w;
     } else {
-      const uint16_t s = down_s[(e * kH + n) * (kI / kGroup) + G];
-      *reinterpret_cast<uint16_t*>(dn + ev * kDnUnitBytes + kDnScaleOff + j * 64 + 2 * lane) = s;
+      const long long g2 = g - nword;
+      const int cp = (int)(g2 & 3);
+      const long long rest = g2 >> 2;
+      const int G = (int)(rest % kGroups);
+      const long long ev = rest / kGroups;
+      const int v = (int)(ev % kDnUnits);
+      const long long e = ev / kDnUnits;
+      const int n = kDnUnitRows * v + 2 * cp;
+      const uint32_t s0 = down_s[(e * kH + n) * kGroups + G];
+      const uint32_t s1 = down_s[(e * kH + n + 1) * kGroups + G];
+      *reinterpret_cast<uint32_t*>(dn + ev * kDnUnitBytes + kDnScaleOff + (G >> 2) * 64 + 16 * cp + 4 * (G & 3)) =
+          s0 | (s1 << 16);
     }
   }
 }
