@@ -211,12 +211,13 @@ __device__ __forceinline__ uint2 h_split2(float h0, float h1) {
 }
 // One down unit (kDnUnitBytes in shared memory) against the h of up to 8
 // tokens.  Lane (g = lane / 4, c = lane % 4) returns token g's sums for the
-// unit's rows 2c and 2c + 1, times 2^-8.  hf points at this lane's token's
-// fragments plus 16 c; act is false for lanes whose token does not exist
-// (their A rows are zero).  Every lane of the warp must call it.
-// Chunks j0 .. j1 - 1 of K only (default: all of K).
-__device__ __forceinline__ void dn_unit_mma(const unsigned char* unit, const unsigned char* hf, bool act, int lane,
-                                            float& r0, float& r1, int j0 = 0, int j1 = kDnChunks) {
+// unit's rows 2c and 2c + 1, times 2^-8, over chunks j0 .. j1 - 1 of K
+// (default: all of K).  hf points at this lane's token's fragments plus 16 c.
+// A lane without a token of its own points at any valid token (its
+// accumulator row is discarded): the loads stay unconditional, so the MMAs
+// of different groups can overlap.  Every lane of the warp must call it.
+__device__ __forceinline__ void dn_unit_mma(const unsigned char* unit, const unsigned char* hf, int lane, float& r0,
+                                            float& r1, int j0 = 0, int j1 = kDnChunks) {
   const int c = lane & 3;
   float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll 2
@@ -226,11 +227,8 @@ __device__ __forceinline__ void dn_unit_mma(const unsigned char* unit, const uns
     const uint32_t wv[4] = {w.x, w.y, w.z, w.w}, sv[4] = {s.x, s.y, s.z, s.w};
 #pragma unroll
     for (int gg = 0; gg < 4; ++gg) {
-      uint4 a0 = make_uint4(0u, 0u, 0u, 0u), a1 = a0;
-      if (act) {
-        a0 = lds128(hf + (8 * j + 2 * gg) * 64);
-        a1 = lds128(hf + (8 * j + 2 * gg + 1) * 64);
-      }
+      const uint4 a0 = lds128(hf + (8 * j + 2 * gg) * 64);
+      const uint4 a1 = lds128(hf + (8 * j + 2 * gg + 1) * 64);
       float d0, d1, d2, d3;
       mma_16816(d0, d1, d2, d3, a0.x, a0.y, a0.z, a0.w, deq_q_even(wv[gg]), deq_q_odd(wv[gg]), 0.f, 0.f, 0.f, 0.f);
       mma_16816(d0, d1, d2, d3, a1.x, a1.y, a1.z, a1.w, deq_q_even(wv[gg] >> 8), deq_q_odd(wv[gg] >> 8), d0, d1,

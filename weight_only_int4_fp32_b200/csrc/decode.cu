@@ -365,7 +365,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     if (warp == 0) { LING_CLK(1); if (lane == 0) g_clk_sink(lg[0] + lg[E - 1]); LING_CLK(2); }
     warp_topk_fast(lg, E, K, hd.topi[warp], hd.topw[warp]);
     if (warp == 0) LING_CLK(3);
-    if (warp == 0) LING_TRACE(4);
+
   }
   __syncthreads();
   LING_TRACE(3);
@@ -455,7 +455,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       const int u = unit / kGuUnits, b = unit - u * kGuUnits;
       const int cnt = hd.uniq_cnt[u];
       const bool bval = n < cnt;
-      const unsigned char* xrow = xf + (bval ? hd.uniq_pair[u][n] / K : 0) * kXfTok + m * 32 +
+      // a column without a token reads token 0's x (its results are dropped),
+      // so that the loads below need no branch
+      const unsigned char* xrow = xf + (hd.uniq_pair[u][bval ? n : 0] / K) * kXfTok + m * 32 +
                                   half * (kGuChunks / 2) * 128;
       float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
       bool ok = issued && mbar_wait_warp(barA, pha, p.wait_limit_ns, p.err);
@@ -472,8 +474,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         for (int jj = 0; jj < kGuChunks / 8; ++jj) {
           const int jl = pc * (kGuChunks / 8) + jj;  // chunk within the half
           const uint4 wv = lds128(bufA + jl * 512 + 16 * lane);
-          const uint4 xa = bval ? lds128(xrow + jl * 128) : make_uint4(0, 0, 0, 0);
-          const uint4 xc = bval ? lds128(xrow + jl * 128 + 16) : make_uint4(0, 0, 0, 0);
+          const uint4 xa = lds128(xrow + jl * 128);
+          const uint4 xc = lds128(xrow + jl * 128 + 16);
           const uint32_t s01 = *reinterpret_cast<const uint32_t*>(bufA + kGuHalfCodes + (2 * jl) * 32 + 4 * n);
           const uint32_t s23 = *reinterpret_cast<const uint32_t*>(bufA + kGuHalfCodes + (2 * jl + 1) * 32 + 4 * n);
           const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
@@ -623,9 +625,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   auto down_item = [&](const unsigned char* base, int blk, int u) {
     const int g = lane >> 2, c = lane & 3;
     const bool act = g < hd.uniq_cnt[u];
-    const int pr = act ? hd.uniq_pair[u][g] : 0;
+    const int pr = hd.uniq_pair[u][act ? g : 0];
     float v0, v1;
-    dn_unit_mma(base, hfb + (size_t)pr * kHfStride + 16 * c, act, lane, v0, v1);
+    dn_unit_mma(base, hfb + (size_t)pr * kHfStride + 16 * c, lane, v0, v1);
     if (act) {
       const float f = (float)(1 << kHShift) * hd.topw[pr / K][pr % K];
       *reinterpret_cast<float2*>(part + ((size_t)blk * (PL::P + T) + pr) * 8 + 2 * c) = make_float2(v0 * f, v1 * f);
@@ -636,10 +638,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     if (!mbar_wait(&hd.dbar, 0, p.wait_limit_ns, p.err)) {
       hd.abort = 1;
     } else {
+      LING_TRACE(7);
+      if (warp == 0) LING_CLK(4);
       for (int it = warp; it < nitems; it += kWarps) {
         const int blk = it / U, u = it - blk * U;
         down_item(body + PL::dn + ((size_t)u * nblk + blk) * kDnUnitBytes, blk, u);
+        if (warp == 0 && it == 0) LING_CLK(5);
       }
+      if (warp == 0) { LING_CLK(15); LING_TRACE(4); }
     }
   }
   {

@@ -150,8 +150,8 @@ __global__ void __launch_bounds__(kGvThreads, 1) gv_gu_kernel(const GvParams p) 
       for (int jj = 0; jj < kGuChunks / 8; ++jj) {
         const int jl = pc * (kGuChunks / 8) + jj;
         const uint4 wv = lds128(buf + jl * 512 + 16 * lane);
-        const uint4 xa = bval ? lds128(xrow + jl * 128) : make_uint4(0, 0, 0, 0);
-        const uint4 xc = bval ? lds128(xrow + jl * 128 + 16) : make_uint4(0, 0, 0, 0);
+        const uint4 xa = lds128(xrow + jl * 128);  // a column without a token reads token 0
+        const uint4 xc = lds128(xrow + jl * 128 + 16);
         const uint32_t s01 = *reinterpret_cast<const uint32_t*>(sc + (2 * jl) * 32 + 4 * n);
         const uint32_t s23 = *reinterpret_cast<const uint32_t*>(sc + (2 * jl + 1) * 32 + 4 * n);
         const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
@@ -294,7 +294,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gv_dn_kernel(const GvParams p) 
       }
       float r0, r1;
       constexpr int kJ = kDnChunks / kGvDnThirds;
-      dn_unit_mma(units + (size_t)u * kDnUnitBytes, hfl, act, lane, r0, r1, kJ * th, kJ * th + kJ);
+      dn_unit_mma(units + (size_t)u * kDnUnitBytes, hfl, lane, r0, r1, kJ * th, kJ * th + kJ);
       if (act) *reinterpret_cast<float2*>(part + ((size_t)it * kGvMaxTok + g) * 8 + 2 * c) = make_float2(r0, r1);
     }
     dead = __syncthreads_or(dead);
