@@ -1,8 +1,9 @@
 // Token-grouped path (T > kMaxDecodeT): prefill chunks and large verify
 // batches of the W4 g32 MoE layer.
 //
-//   route        logits[t, e] = x_t . Wr_e (+ b_e) in fp32 on CUDA cores, tiles
-//                of <= 16 tokens x 64 experts
+//   route        logits[t, e] = x_t . Wr_e (+ b_e), bf16 products summed in
+//                fp32 on the tensor cores (mma.sync), tiles of 32 tokens x 64
+//                experts
 //   top-k        per token (ties to the lower index) and the renormalised
 //                softmax weights; pairs per expert counted on the fly
 //   plan         exclusive scan of the counts, tile lists for both GEMMs
@@ -28,17 +29,11 @@
 
 namespace lingmoe {
 
-constexpr int kRtThreads = 256;
-constexpr int kRtWarps = kRtThreads / 32;
-constexpr int kRtPass = 8;      // tokens per pass (register tile: 8 experts x 8 tokens per lane)
-constexpr int kRtMaxTok = 16;   // tokens per CTA
-constexpr int kRtExperts = 8 * kRtWarps;  // experts per CTA: 8 per warp
-constexpr size_t kRtSmem = (size_t)kRtPass * kXTok * sizeof(float);
 constexpr int kPlanThreads = 1024;
 constexpr int kRowThreads = kH / 8;  // 320: one thread per 8 columns of a row
 
 const char* grouped_describe() {
-  return "fp32 router GEMM + top-k + counting scatter by expert + tcgen05 grouped GEMMs "
+  return "router GEMM (bf16 mma.sync, fp32 sums) + top-k + counting scatter by expert + tcgen05 grouped GEMMs "
          "(M=256 weight rows x N<=128 positions; routed int4 dequantised to exact fp16 in shared memory, "
          "shared expert as fp16 tiles via TMA; activations via TMA; fp32 accumulators in double-buffered TMEM) "
          "+ fixed-order combine";
@@ -93,114 +88,89 @@ cudaError_t grouped_prepare(GroupedWorkspace* ws, int E, const __nv_bfloat16* sh
   return tc_encode_maps(&ws->maps, ws->xg, ws->h16, (int)ws->rows, ws->shgu16, ws->shdn16);
 }
 
-// Block-cooperative: x rows toks[0..n) (bf16) -> fp32 planes (first and
-// second halves of each 8-column chunk in separate planes, padded every 80
-// chunks) so that a warp reading consecutive chunks hits distinct banks.
-__device__ void stage_x_rows(const __nv_bfloat16* x, const int* toks, int n, float* xs) {
-  for (int v = threadIdx.x; v < n * kXChunks; v += blockDim.x) {
-    const int m = v / kXChunks, c = v - m * kXChunks;
-    const uint4 w = *reinterpret_cast<const uint4*>(x + (size_t)toks[m] * kH + 8 * c);
-    float* d = xs + (size_t)m * kXTok + xoff(c);
-    *reinterpret_cast<float4*>(d) = make_float4(bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y));
-    *reinterpret_cast<float4*>(d + kXPlane) = make_float4(bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w));
-  }
-}
-
 // ---------------------------------------------------------------- route
-// Logits of NT <= 8 staged tokens (rows t0 ..) for the CTA's experts.  A warp
-// takes 8 experts; each lane accumulates 8 experts x NT tokens over its
-// K-chunks (every 32nd chunk of 8 columns), then a reduce-scatter across the
-// warp leaves lane l with the sums for expert e0 + l/4 and tokens 2(l%4), +1.
-template <int NT>
-__device__ __forceinline__ void route_logits(const float* xs, const GroupedParams& p, int t0, int ebase,
-                                             float* logits) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  {
-    const int e0 = ebase + 8 * warp;
-    if (e0 >= p.E) return;
-    float acc[64];
-#pragma unroll
-    for (int i = 0; i < 64; ++i) acc[i] = 0.f;
-#pragma unroll 1
-    for (int c = lane; c < kXChunks; c += 32) {
-      float wf[8][8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int e = e0 + j;
-        const uint4 w = e < p.E ? ldg_stream(p.router_w + (size_t)e * kH + 8 * c) : make_uint4(0, 0, 0, 0);
-        wf[j][0] = bf16lo(w.x); wf[j][1] = bf16hi(w.x); wf[j][2] = bf16lo(w.y); wf[j][3] = bf16hi(w.y);
-        wf[j][4] = bf16lo(w.z); wf[j][5] = bf16hi(w.z); wf[j][6] = bf16lo(w.w); wf[j][7] = bf16hi(w.w);
-      }
-      const int o = xoff(c);
-#pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        const float4 a = ldsf4(xs + t * kXTok + o);
-        const float4 b = ldsf4(xs + t * kXTok + kXPlane + o);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float s = acc[8 * j + t];
-          s = fmaf(wf[j][0], a.x, s); s = fmaf(wf[j][1], a.y, s);
-          s = fmaf(wf[j][2], a.z, s); s = fmaf(wf[j][3], a.w, s);
-          s = fmaf(wf[j][4], b.x, s); s = fmaf(wf[j][5], b.y, s);
-          s = fmaf(wf[j][6], b.z, s); s = fmaf(wf[j][7], b.w, s);
-          acc[8 * j + t] = s;
-        }
-      }
-    }
-    // reduce-scatter of the 64 partial sums: after the step with offset o,
-    // lane bit o selects which half of the remaining values the lane keeps
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      const bool up = (lane & o) != 0;
-#pragma unroll
-      for (int i = 0; i < 2 * o; ++i) {
-        const float send = up ? acc[i] : acc[i + 2 * o];
-        const float keep = up ? acc[i + 2 * o] : acc[i];
-        acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-      }
-    }
-    const int e = e0 + (lane >> 2);
-    if (e < p.E) {
-      const float bias = p.router_bias ? p.router_bias[e] : 0.f;
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int t = 2 * (lane & 3) + u;
-        if (t < NT) logits[(size_t)(t0 + t) * p.E + e] = acc[u] + bias;
-      }
-    }
-  }
+// logits[t, e] = x_t . Wr_e (+ b_e): the bf16 x bf16 products are exact in
+// fp32 and are summed in fp32 by mma.sync m16n8k16 (bf16 inputs).  CTA tile:
+// 32 tokens x 64 experts, 4 warps of 16 tokens x 32 experts; K streams
+// through shared memory in stages of 128 (cp.async, double-buffered), the
+// fragments come from ldmatrix.  Rows past T or E repeat the last valid row;
+// their results are not stored.
+constexpr int kRmTok = 32, kRmExp = 64, kRmK = 128, kRmThreads = 128;
+constexpr int kRmRow = kRmK * 2 + 16;                    // 272 B: 8 rows hit 8 distinct 16-byte bank groups
+constexpr int kRmStage = (kRmTok + kRmExp) * kRmRow;     // 26112
+constexpr size_t kRmSmem = 2 * (size_t)kRmStage;
+static_assert(kH % kRmK == 0, "K stages tile the hidden size");
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// CTA (x, y): tokens [x tpc, x tpc + tpc) in passes of <= 8, experts
-// [64 y, 64 y + 64).  Splitting the experts keeps every SM streaming router
-// rows at small T too.
-__global__ void __launch_bounds__(kRtThreads, 1) grp_route_kernel(GroupedParams p, int tpc, float* logits) {
-  extern __shared__ __align__(16) float xs[];
-  __shared__ int toks[kRtPass];
-  const int t_begin = blockIdx.x * tpc, t_end = min(p.T, t_begin + tpc);
-  const int ntok = t_end - t_begin;
-  const int ebase = blockIdx.y * kRtExperts;
-  if (ntok <= 0) return;
-  const int npass = (ntok + kRtPass - 1) / kRtPass;
-  const int per = (ntok + npass - 1) / npass;
+__global__ void __launch_bounds__(kRmThreads) grp_route_kernel(GroupedParams p, float* logits) {
+  extern __shared__ __align__(128) unsigned char rsm[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t0 = blockIdx.x * kRmTok, e0 = blockIdx.y * kRmExp;
+  const int wm = warp & 1, wn = warp >> 1;  // 16-token half, 32-expert half
+  auto load_stage = [&](int kc, int buf) {
+    unsigned char* base = rsm + buf * kRmStage;
+    for (int v = tid; v < (kRmTok + kRmExp) * (kRmK / 8); v += kRmThreads) {
+      const int row = v >> 4, pc = v & 15;
+      const __nv_bfloat16* src = row < kRmTok ? p.x + (size_t)min(t0 + row, p.T - 1) * kH
+                                              : p.router_w + (size_t)min(e0 + row - kRmTok, p.E - 1) * kH;
+      cp_async16(smem_u32(base + row * kRmRow + pc * 16), src + kc * kRmK + pc * 8);
+    }
+    cp_async_commit();
+  };
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+  constexpr int NKC = kH / kRmK;
+  load_stage(0, 0);
 #pragma unroll 1
-  for (int t0 = t_begin; t0 < t_end; t0 += per) {
-    const int nt = min(per, t_end - t0);
-    if (threadIdx.x < kRtPass) toks[threadIdx.x] = t0 + min((int)threadIdx.x, nt - 1);
-    __syncthreads();
-    stage_x_rows(p.x, toks, nt, xs);
-    __syncthreads();
-    switch (nt) {
-      case 1: route_logits<1>(xs, p, t0, ebase, logits); break;
-      case 2: route_logits<2>(xs, p, t0, ebase, logits); break;
-      case 3: route_logits<3>(xs, p, t0, ebase, logits); break;
-      case 4: route_logits<4>(xs, p, t0, ebase, logits); break;
-      case 5: route_logits<5>(xs, p, t0, ebase, logits); break;
-      case 6: route_logits<6>(xs, p, t0, ebase, logits); break;
-      case 7: route_logits<7>(xs, p, t0, ebase, logits); break;
-      default: route_logits<8>(xs, p, t0, ebase, logits); break;
+  for (int kc = 0; kc < NKC; ++kc) {
+    if (kc + 1 < NKC) {
+      load_stage(kc + 1, (kc + 1) & 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
     __syncthreads();
+    const uint32_t base = smem_u32(rsm + (kc & 1) * kRmStage);
+    // A (x rows): lanes 0-15 address rows 0-15 at k 0, lanes 16-31 the same rows at k 8
+    const uint32_t arow = base + (wm * 16 + (lane & 15)) * kRmRow + (lane >> 4) * 16;
+    // B (router rows, K contiguous): matrix lane/8 = (expert octet lane/16, k half (lane/8)%2)
+    const uint32_t brow = base + (kRmTok + wn * 32 + (lane >> 4) * 8 + (lane & 7)) * kRmRow + ((lane >> 3) & 1) * 16;
+#pragma unroll
+    for (int ks = 0; ks < kRmK / 16; ++ks) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(arow + ks * 32, a0, a1, a2, a3);
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(brow + np * 16 * kRmRow + ks * 32, b0, b1, b2, b3);
+        mma_bf16_16816(acc[2 * np], a0, a1, a2, a3, b0, b1);
+        mma_bf16_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+      }
+    }
+    __syncthreads();  // the buffer is refilled two stages on
+  }
+  // accumulator (token g / g + 8, experts 2c, 2c + 1 of each 8-expert tile)
+  const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt) {
+    const int e = e0 + wn * 32 + nt * 8 + 2 * c;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int t = t0 + wm * 16 + g + 8 * hh;
+      if (t >= p.T) continue;
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+        if (e + q < p.E)
+          logits[(size_t)t * p.E + e + q] = acc[nt][2 * hh + q] + (p.router_bias ? p.router_bias[e + q] : 0.f);
+    }
   }
 }
 
@@ -392,7 +362,7 @@ __global__ void __launch_bounds__(kRowThreads) grp_combine_kernel(const float* y
 
 cudaError_t setup_grouped() {
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(grp_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRtSmem)) !=
+  if ((e = cudaFuncSetAttribute(grp_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRmSmem)) !=
       cudaSuccess)
     return e;
   if ((e = setup_grouped_gemv()) != cudaSuccess) return e;
@@ -403,10 +373,8 @@ cudaError_t launch_grouped(const GroupedParams& p, const GroupedWorkspace& ws, c
   int nl = 0;
   cudaError_t e = cudaSuccess;
   const int P = p.T * p.k;
-  const int eblocks = (p.E + kRtExperts - 1) / kRtExperts;
-  const int tpc = std::max(1, std::min(kRtMaxTok, (p.T * eblocks + 2 * p.num_sms - 1) / (2 * p.num_sms)));
-  grp_route_kernel<<<dim3((p.T + tpc - 1) / tpc, (p.E + kRtExperts - 1) / kRtExperts), kRtThreads, kRtSmem, s>>>(
-      p, tpc, ws.logits);
+  grp_route_kernel<<<dim3((p.T + kRmTok - 1) / kRmTok, (p.E + kRmExp - 1) / kRmExp), kRmThreads, kRmSmem, s>>>(
+      p, ws.logits);
   ++nl;
   grp_topk_kernel<<<(p.T + 7) / 8, 256, 0, s>>>(p, ws.logits, ws.topk_idx, ws.topk_w, ws.cnt);
   ++nl;
