@@ -326,6 +326,67 @@ def run_ours(args):
     if any(s != lm.LING_MOE_OK for s in status):
         raise RuntimeError(f"device status {status}")
 
+    # the same steps as one CUDA graph per step (stack: the 40 layer calls
+    # captured once and replayed; inputs copied into the captured buffer
+    # before each step's start event)
+    graph = None
+    if stack:
+        xs_static = torch.empty_like(inputs[0])
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            one_step(xs_static)  # warm-up outside the capture
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        cg = torch.cuda.CUDAGraph()
+        n_cap0 = sum(l.launch_count() for l in layers)
+        with torch.cuda.graph(cg):
+            one_step(xs_static)
+        per_replay = sum(l.launch_count() for l in layers) - n_cap0
+        for i in range(nwarm):
+            flush.fill_(float(i))
+            xs_static.copy_(inputs[i])
+            cg.replay()
+        torch.cuda.synchronize()
+        gs = [torch.cuda.Event(enable_timing=True) for _ in range(nsteps)]
+        ge = [torch.cuda.Event(enable_timing=True) for _ in range(nsteps)]
+        for i in range(nsteps):
+            flush.fill_(float(i))
+            xs_static.copy_(inputs[nwarm + i])
+            gs[i].record(stream)
+            cg.replay()
+            ge[i].record(stream)
+        torch.cuda.synchronize()
+        g_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(gs, ge)), dev)
+        del cg
+        graph = {"value": ws * nsteps * T / (g_ms * 1e-3), "unit": "tokens/s", "ms_per_step": g_ms / nsteps,
+                 "us_per_layer": g_ms / nsteps / len(layers) * 1e3, "gpu_launches": per_replay * nsteps,
+                 "note": "the step's layer calls captured once as one CUDA graph and replayed; "
+                         "L2 flushed and inputs copied before each step's start event"}
+
+    # warm: the same calls back to back with nothing in between (weights may
+    # partly stay in L2 between calls: router and shared expert)
+    warm = None
+    if not stack:
+        nw = min(nsteps, 100)
+        for i in range(3):
+            one_step(inputs[nwarm + i % nsteps])
+        torch.cuda.synchronize()
+        w0 = torch.cuda.Event(enable_timing=True)
+        w1 = torch.cuda.Event(enable_timing=True)
+        w0.record(stream)
+        for i in range(nw):
+            one_step(inputs[nwarm + i])
+        w1.record(stream)
+        torch.cuda.synchronize()
+        w_ms = max_over_ranks(w0.elapsed_time(w1), dev)
+        warm = {"value": ws * nw * T / (w_ms * 1e-3), "unit": "tokens/s", "us_per_layer": w_ms / nw * 1e3,
+                "calls": nw, "note": "calls back to back, no L2 flush between them"}
+
+    status = [l.status() for l in layers]
+    if any(s != lm.LING_MOE_OK for s in status):
+        raise RuntimeError(f"device status after the graph / warm runs {status}")
+
     # end to end through the host-buffer entry point (pinned buffers, copies timed)
     e2e = None
     if not stack:
@@ -377,6 +438,8 @@ def run_ours(args):
                          "bytes_per_launch": avg_bytes / calls_per_step},
             "cpu_baseline": cpu,
             "e2e": e2e,
+            "warm": warm,
+            "graph": graph,
             "gpu_launches": launches,
             "clocks": clk.summary(),
             "wall_s_timed_region": t_wall,
