@@ -39,9 +39,16 @@ L2_FLUSH_BYTES = 256 << 20
 # the command), valid only while the kernel's sources are the ones captured:
 # the sources are hashed and the figure is reported as null once they change.
 TRAFFIC = {
-    "decode_e512_t1": {"bytes": 41_036_800 + 108_544,
-                       "sources": ("decode.cu", "decode.h", "common.cuh", "layout.h"),
-                       "sha256": "de2b634dce1fb6040e1da20aabfda112fe2c9012bb29996529810a8c5352e736"},
+    "decode_e512_t1": {"bytes": 41_036_544 + 9_472,
+                       "sources": ('decode.cu', 'decode.h', 'common.cuh', 'layout.h'),
+                       "sha256": "844e57c1ead859209af68874df7195df955e778ed669d35487ec2db09dd04154"},
+    "verify_e512_t4": {"bytes": 126_062_848 + 3_859_456,
+                       "sources": ('decode.cu', 'decode.h', 'common.cuh', 'layout.h'),
+                       "sha256": "844e57c1ead859209af68874df7195df955e778ed669d35487ec2db09dd04154"},
+    # token-grouped: the dominant kernel, tc_grouped_kernel<0> (gate/up tiles)
+    "prefill_e512_t2048_zipf": {"bytes": 457_028_864 + 53_828_608,
+                                "sources": ('grouped_tc.cu', 'grouped_tc.h', 'common.cuh', 'layout.h'),
+                                "sha256": "56514f5ff591f5be46384759f168373b232e0f2534780ced74471a67e3ca4c13"},
 }
 
 
@@ -76,6 +83,19 @@ def peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+def tensor_peak():
+    """Burst bf16 dense TFLOP/s (fp16 inputs run at the same rate)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+GEMV_MAX_TOKENS = 8  # experts with at most this many tokens take the GEMV kernels, not the tensor-core tiles
 
 
 class ClockSampler:
@@ -285,11 +305,16 @@ def run_ours(args):
         else:
             layers[0].forward(x, out)
 
-    # union of routed experts per step (bytes the method must read), from the routing
+    # union of routed experts per step (bytes the method must read), from the
+    # routing; for token-grouped calls also the rows the tensor-core tiles take
+    tc_rows = []
+
     def union_of(x):
         if stack:
             return [8] * len(layers)
         _, idx, _ = layers[0].forward(x, return_routing=True)
+        cnt = torch.bincount(idx.flatten().long(), minlength=E)
+        tc_rows.append(int(cnt[cnt > GEMV_MAX_TOKENS].sum()) + T)
         return [int(torch.unique(idx).numel())]
 
     for i in range(nwarm):
@@ -383,9 +408,23 @@ def run_ours(args):
         warm = {"value": ws * nw * T / (w_ms * 1e-3), "unit": "tokens/s", "us_per_layer": w_ms / nw * 1e3,
                 "calls": nw, "note": "calls back to back, no L2 flush between them"}
 
+    # per-kernel times of the token-grouped path (a separate pass: the events
+    # around each launch are not in the timed steps above)
+    ktimes = None
+    if T > 4 and not stack:
+        layers[0].set_kernel_timing(True)
+        per = {}
+        for i in range(nsteps):
+            flush.fill_(float(i))
+            one_step(inputs[nwarm + i])
+            for name, ms in layers[0].kernel_times():
+                per.setdefault(name, []).append(ms)
+        layers[0].set_kernel_timing(False)
+        ktimes = {n: sum(v) / len(v) for n, v in per.items()}
+
     status = [l.status() for l in layers]
     if any(s != lm.LING_MOE_OK for s in status):
-        raise RuntimeError(f"device status after the graph / warm runs {status}")
+        raise RuntimeError(f"device status after the graph / warm / timing runs {status}")
 
     # end to end through the host-buffer entry point (pinned buffers, copies timed)
     e2e = None
@@ -415,6 +454,19 @@ def run_ours(args):
     avg_launch_ms = kern_ms / nsteps / calls_per_step
     achieved = (avg_bytes / calls_per_step) / (avg_launch_ms * 1e-3) / 1e9
     peak, peak_kind = peaks()
+    roofline = {"bound": "hbm", "kernel": "whole layer (one launch per call at T <= 4)", "achieved": achieved,
+                "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic_for(args.workload),
+                "peak_kind": peak_kind, "bytes_per_launch": avg_bytes / calls_per_step}
+    if ktimes is not None and "tc_gu" in ktimes:
+        # dominant kernel: the gate/up tiles; algorithmic FLOPs of the rows they take
+        tpk, tpk_kind = tensor_peak()
+        flops = sum(2.0 * r * H * 2 * I for r in tc_rows) / len(tc_rows)
+        ach_t = flops / (ktimes["tc_gu"] * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "kernel": "tc_grouped_kernel<0> (gate/up tiles)", "achieved": ach_t,
+                    "peak": tpk, "unit": "TFLOP/s", "frac": ach_t / tpk, "traffic": traffic_for(args.workload),
+                    "peak_kind": tpk_kind + " (bf16 burst; fp16 x fp16 runs at the same rate)",
+                    "flops_per_launch": flops, "kernel_ms": ktimes["tc_gu"],
+                    "kernel_ms_by_name": ktimes, "layer_hbm_gbs": achieved}
     tokens = ws * nsteps * T
     value = tokens / (kern_ms * 1e-3)
     if rank == 0:
@@ -432,10 +484,7 @@ def run_ours(args):
             "us_per_layer": avg_launch_ms * 1e3,
             "achieved_gbs": achieved,
             "frac_of_8tbs": achieved / 8000.0,
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": traffic_for(args.workload),
-                         "peak_kind": peak_kind,
-                         "bytes_per_launch": avg_bytes / calls_per_step},
+            "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "warm": warm,

@@ -132,6 +132,24 @@ int64_t ling_moe_launch_count(const ling_moe_t *h);
 /* Message of the last error on the calling host thread ("" if none). */
 const char *ling_moe_last_error(void);
 
+/* ---- per-kernel timing (measurement; off by default) ----
+ * With on != 0, every later forward call also records CUDA events on its
+ * stream around each kernel it launches (one for T <= 4, nine for larger T:
+ * route, topk, plan, scatter, gemv_gu, tc_gu, gemv_dn, tc_dn, combine).  The
+ * events add a little time of their own; do not leave timing on while
+ * capturing a stream into a graph.  on == 0 frees the events.  Returns OK,
+ * INVALID_ARG (NULL handle) or CUDA. */
+int ling_moe_set_kernel_timing(ling_moe_t *h, int on);
+/* Durations in milliseconds of the kernels of the last forward call issued
+ * while timing was on, in launch order: waits for that call's last event,
+ * writes *count (0 if no call was timed) and ms[0 .. *count).  capacity is
+ * the length of ms (at least *count, 9 is always enough).  Returns OK,
+ * INVALID_ARG (NULL handle or count, timing off, ms too short) or CUDA. */
+int ling_moe_kernel_times(ling_moe_t *h, float *ms, int capacity, int *count);
+/* Name of kernel i of the last timed call ("" if there is none).  The
+ * string is static. */
+const char *ling_moe_kernel_name(const ling_moe_t *h, int i);
+
 /* Free everything the handle owns.  NULL is a no-op.  The caller must make
  * sure no enqueued work still uses the handle. */
 void ling_moe_destroy(ling_moe_t *h);

@@ -99,6 +99,10 @@ def test_null_handle_is_rejected_everywhere():
     assert lm.lib.ling_moe_forward_host(None, 16, 1, 32, None) == lm.LING_MOE_ERR_INVALID_ARG
     assert lm.lib.ling_moe_status(None, None) == lm.LING_MOE_ERR_INVALID_ARG
     assert lm.lib.ling_moe_test_set_wait(None, 0, 0) == lm.LING_MOE_ERR_INVALID_ARG
+    assert lm.lib.ling_moe_set_kernel_timing(None, 1) == lm.LING_MOE_ERR_INVALID_ARG
+    n = ctypes.c_int(-7)
+    assert lm.lib.ling_moe_kernel_times(None, None, 0, ctypes.byref(n)) == lm.LING_MOE_ERR_INVALID_ARG
+    assert lm.lib.ling_moe_kernel_name(None, 0) == b""
     assert lm.ling_moe_describe(None) == ""
     assert lm.ling_moe_launch_count(None) == 0
     lm.ling_moe_destroy(None)  # no-op

@@ -215,6 +215,26 @@ def test_cuda_graph_replay_matches_eager(full):
         del g
 
 
+def test_kernel_timing_reports_each_launch(full):
+    _, layer, _, _ = full
+    layer.set_kernel_timing(True)
+    try:
+        for T, names in ((1, ["decode"]), (64, ["route", "topk", "plan", "scatter", "gemv_gu", "tc_gu",
+                                               "gemv_dn", "tc_dn", "combine"])):
+            x = workloads.tokens(T, seed=5, device=DEV)
+            timed = layer.forward(x)
+            times = layer.kernel_times()
+            assert [n for n, _ in times] == names
+            assert all(ms > 0 for _, ms in times)
+            layer.set_kernel_timing(False)
+            plain = layer.forward(x)
+            torch.cuda.synchronize()
+            assert torch.equal(timed, plain)  # the events change nothing
+            layer.set_kernel_timing(True)
+    finally:
+        layer.set_kernel_timing(False)
+
+
 def test_forward_host_matches_device(full):
     _, layer, _, _ = full
     for T in (1, 4, 20):

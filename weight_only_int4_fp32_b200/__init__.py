@@ -18,7 +18,8 @@ __all__ = [
     "ling_moe_config_t", "ling_moe_weights_t", "library_path", "load_library",
     "ling_moe_create", "ling_moe_forward", "ling_moe_forward_ex", "ling_moe_forward_host",
     "ling_moe_status", "ling_moe_describe", "ling_moe_launch_count", "ling_moe_last_error",
-    "ling_moe_destroy", "ling_moe_test_set_wait", "ling_moe_route_noalloc", "MoELayer", "EXPORTED",
+    "ling_moe_destroy", "ling_moe_test_set_wait", "ling_moe_route_noalloc", "ling_moe_set_kernel_timing",
+    "ling_moe_kernel_times", "MoELayer", "EXPORTED",
 ]
 
 LING_MOE_OK = 0
@@ -33,6 +34,7 @@ EXPORTED = (
     "ling_moe_create", "ling_moe_forward", "ling_moe_forward_ex", "ling_moe_forward_host",
     "ling_moe_status", "ling_moe_describe", "ling_moe_launch_count", "ling_moe_last_error",
     "ling_moe_destroy", "ling_moe_test_set_wait", "ling_moe_route_noalloc",
+    "ling_moe_set_kernel_timing", "ling_moe_kernel_times", "ling_moe_kernel_name",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -91,6 +93,9 @@ def _load():
         "ling_moe_destroy": (None, [vp]),
         "ling_moe_test_set_wait": (ci, [vp, ci, ctypes.c_uint64]),
         "ling_moe_route_noalloc": (ci, [vp, ci, vp, vp, ci, ci, vp, vp, vp]),
+        "ling_moe_set_kernel_timing": (ci, [vp, ci]),
+        "ling_moe_kernel_times": (ci, [vp, ctypes.POINTER(ctypes.c_float), ci, ctypes.POINTER(ci)]),
+        "ling_moe_kernel_name": (ctypes.c_char_p, [vp, ci]),
     }
     for name, (res, args) in sig.items():
         try:
@@ -125,6 +130,18 @@ def ling_moe_create(cfg: ling_moe_config_t, weights: ling_moe_weights_t) -> int:
     h = ctypes.c_void_p()
     _check(lib.ling_moe_create(ctypes.byref(cfg), ctypes.byref(weights), ctypes.byref(h)))
     return h.value
+
+
+def ling_moe_set_kernel_timing(h: int, on: bool) -> int:
+    return _check(lib.ling_moe_set_kernel_timing(h, 1 if on else 0))
+
+
+def ling_moe_kernel_times(h: int) -> list:
+    """[(kernel name, ms)] of the last forward call issued with timing on."""
+    ms = (ctypes.c_float * 16)()
+    n = ctypes.c_int(0)
+    _check(lib.ling_moe_kernel_times(h, ms, 16, ctypes.byref(n)))
+    return [(lib.ling_moe_kernel_name(h, i).decode(), float(ms[i])) for i in range(n.value)]
 
 
 def ling_moe_forward(h: int, x: int, T: int, out: int, stream: int = 0) -> int:
@@ -231,6 +248,13 @@ class MoELayer:
 
     def launch_count(self) -> int:
         return ling_moe_launch_count(self.handle)
+
+    def set_kernel_timing(self, on: bool = True):
+        ling_moe_set_kernel_timing(self.handle, on)
+
+    def kernel_times(self) -> list:
+        """[(kernel name, ms)] of the last forward call issued with timing on."""
+        return ling_moe_kernel_times(self.handle)
 
     def close(self):
         if getattr(self, "handle", None):

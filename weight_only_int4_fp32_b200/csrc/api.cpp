@@ -82,6 +82,11 @@ struct ling_moe {
   std::atomic<int64_t> launches{0};
   int skip_arrive_cta = -1;
   unsigned long long wait_limit_ns = kDefaultWaitNs;
+  // optional per-kernel timing: events around the launches of the last call
+  bool timing = false;
+  cudaEvent_t tev[kGroupedKernels + 1] = {};
+  int tev_kernels = 0;   // kernels timed in the last call
+  bool tev_grouped = false;
 
   cudaError_t alloc(void** p, size_t bytes) {
     *p = nullptr;
@@ -286,8 +291,14 @@ static int forward_impl(ling_moe_t* h, const void* x, int T, void* out, int32_t*
     p.skip_arrive_cta = h->skip_arrive_cta;
     p.wait_limit_ns = h->wait_limit_ns;
     h->skip_arrive_cta = -1;  // one launch only
+    if (h->timing) cudaEventRecord(h->tev[0], stream);
     e = launch_decode(p, h->decode_ctas, stream);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    if (h->timing) {
+      cudaEventRecord(h->tev[1], stream);
+      h->tev_kernels = 1;
+      h->tev_grouped = false;
+    }
     h->launches.fetch_add(1);
     return LING_MOE_OK;
   }
@@ -305,9 +316,13 @@ static int forward_impl(ling_moe_t* h, const void* x, int T, void* out, int32_t*
   gp.topk_w_out = topk_w;
   gp.num_sms = h->num_sms;
   int nl = 0;
-  e = launch_grouped(gp, h->gws, stream, &nl);
+  e = launch_grouped(gp, h->gws, stream, &nl, h->timing ? h->tev : nullptr);
   h->launches.fetch_add(nl);
   if (e != cudaSuccess) return cuda_fail(e, "grouped launch");
+  if (h->timing) {
+    h->tev_kernels = kGroupedKernels;
+    h->tev_grouped = true;
+  }
   return LING_MOE_OK;
 }
 
@@ -369,8 +384,56 @@ const char* ling_moe_describe(const ling_moe_t* h) { return h ? h->desc.c_str() 
 
 int64_t ling_moe_launch_count(const ling_moe_t* h) { return h ? h->launches.load() : 0; }
 
+static void timing_events(ling_moe_t* h, bool on) {
+  for (auto& ev : h->tev) {
+    if (ev) cudaEventDestroy(ev);
+    ev = nullptr;
+  }
+  h->timing = false;
+  h->tev_kernels = 0;
+  if (!on) return;
+  for (auto& ev : h->tev)
+    if (cudaEventCreate(&ev) != cudaSuccess) {
+      timing_events(h, false);
+      return;
+    }
+  h->timing = true;
+}
+
+int ling_moe_set_kernel_timing(ling_moe_t* h, int on) {
+  if (!h) return fail(LING_MOE_ERR_INVALID_ARG, "handle is NULL");
+  cudaError_t e = cudaSetDevice(h->device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  timing_events(h, on != 0);
+  if (on && !h->timing) return fail(LING_MOE_ERR_CUDA, "could not create the timing events");
+  return LING_MOE_OK;
+}
+
+int ling_moe_kernel_times(ling_moe_t* h, float* ms, int capacity, int* count) {
+  if (!h || !count) return fail(LING_MOE_ERR_INVALID_ARG, "handle or count is NULL");
+  if (!h->timing) return fail(LING_MOE_ERR_INVALID_ARG, "kernel timing is off");
+  const int n = h->tev_kernels;
+  *count = n;
+  if (n == 0) return LING_MOE_OK;
+  if (!ms || capacity < n) return fail(LING_MOE_ERR_INVALID_ARG, "need room for %d times", n);
+  cudaError_t e = cudaEventSynchronize(h->tev[n]);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+  for (int i = 0; i < n; ++i)
+    if ((e = cudaEventElapsedTime(&ms[i], h->tev[i], h->tev[i + 1])) != cudaSuccess)
+      return cuda_fail(e, "cudaEventElapsedTime");
+  return LING_MOE_OK;
+}
+
+const char* ling_moe_kernel_name(const ling_moe_t* h, int i) {
+  static const char* const grouped[kGroupedKernels] = {"route", "topk", "plan", "scatter", "gemv_gu",
+                                                       "tc_gu", "gemv_dn", "tc_dn", "combine"};
+  if (!h || i < 0 || i >= h->tev_kernels) return "";
+  return h->tev_grouped ? grouped[i] : "decode";
+}
+
 void ling_moe_destroy(ling_moe_t* h) {
   if (!h) return;
+  timing_events(h, false);
   h->release();
   delete h;
 }

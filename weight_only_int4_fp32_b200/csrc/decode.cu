@@ -461,6 +461,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
                                   half * (kGuChunks / 2) * 128;
       float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
       bool ok = issued && mbar_wait_warp(barA, pha, p.wait_limit_ns, p.err);
+      const uint32_t pa0 = pha;
+      int pc_next = ok ? 1 : 0;  // first piece not yet seen complete
       if (issued) pha ^= 1;
       if (warp == 0 && unit == u0) { LING_TRACE(13); LING_CLK(6); }
 #pragma unroll 1
@@ -468,6 +470,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         if (pc > 0) {
           ok = mbar_wait_warp(&hd.mbar[warp][pc], phq, p.wait_limit_ns, p.err);
           if (!ok) break;
+          pc_next = pc + 1;
           if (warp == 0 && unit == u0) LING_CLK(6 + pc);
         }
 #pragma unroll
@@ -500,7 +503,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         }
       }
       if (issued) phq ^= 1;
-      if (!ok && issued) hd.abort = 1;
+      if (!ok && issued) {
+        // a wait ran out: the unit's pieces still in flight land (bounded
+        // waits) before the buffer is reused or the CTA exits
+        hd.abort = 1;
+        if (lane == 0)
+          for (int pc = pc_next; pc < 4; ++pc)
+            mbar_wait(pc == 0 ? barA : &hd.mbar[warp][pc], pc == 0 ? pa0 : (phq ^ 1u), p.wait_limit_ns, p.err);
+        __syncwarp();
+      }
       // combine the two K halves: the second half's partials go through
       // shared memory (double-buffered by unit parity, one barrier per unit)
       float* cb = comb + par * (32 * 4) + lane * 4;

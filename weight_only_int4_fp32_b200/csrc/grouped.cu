@@ -369,18 +369,26 @@ cudaError_t setup_grouped() {
   return setup_grouped_tc();
 }
 
-cudaError_t launch_grouped(const GroupedParams& p, const GroupedWorkspace& ws, cudaStream_t s, int* nlaunch) {
+cudaError_t launch_grouped(const GroupedParams& p, const GroupedWorkspace& ws, cudaStream_t s, int* nlaunch,
+                           cudaEvent_t* marks) {
   int nl = 0;
   cudaError_t e = cudaSuccess;
+  auto mark = [&](int i) {
+    if (marks) cudaEventRecord(marks[i], s);
+  };
   const int P = p.T * p.k;
+  mark(0);
   grp_route_kernel<<<dim3((p.T + kRmTok - 1) / kRmTok, (p.E + kRmExp - 1) / kRmExp), kRmThreads, kRmSmem, s>>>(
       p, ws.logits);
   ++nl;
+  mark(1);
   grp_topk_kernel<<<(p.T + 7) / 8, 256, 0, s>>>(p, ws.logits, ws.topk_idx, ws.topk_w, ws.cnt);
   ++nl;
+  mark(2);
   grp_plan_kernel<<<1, kPlanThreads, 0, s>>>(p.T, p.E, ws.cnt, ws.fill, ws.off, ws.gu_tiles, ws.dn_tiles, ws.ntiles,
                                              ws.small, ws.nsmall);
   ++nl;
+  mark(3);
   grp_scatter_kernel<<<p.T, kRowThreads, 0, s>>>(p.x, p.k, P, ws.topk_idx, ws.off, ws.fill, ws.perm, ws.inv, ws.xg,
                                                  ws.xscale);
   ++nl;
@@ -417,16 +425,22 @@ cudaError_t launch_grouped(const GroupedParams& p, const GroupedWorkspace& ws, c
   gv.nsmall = ws.nsmall;
   gv.err = ws.err;
   gv.wait_limit_ns = 2000000000ull;
+  mark(4);
   if ((e = launch_gemv_gu(gv, p.num_sms, s)) != cudaSuccess) return e;
   ++nl;
+  mark(5);
   if ((e = launch_tc_gemm(0, ws.maps, tp, p.num_sms, s)) != cudaSuccess) return e;
   ++nl;
+  mark(6);
   if ((e = launch_gemv_dn(gv, p.num_sms, s)) != cudaSuccess) return e;
   ++nl;
+  mark(7);
   if ((e = launch_tc_gemm(1, ws.maps, tp, p.num_sms, s)) != cudaSuccess) return e;
   ++nl;
+  mark(8);
   grp_combine_kernel<<<p.T, kRowThreads, 0, s>>>(ws.y, ws.inv, p.k, P, p.out);
   ++nl;
+  mark(kGroupedKernels);
   e = cudaGetLastError();
   *nlaunch = nl;
   return e;

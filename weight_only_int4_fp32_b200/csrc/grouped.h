@@ -64,7 +64,11 @@ cudaError_t grouped_prepare(GroupedWorkspace* ws, int E, const __nv_bfloat16* sh
 cudaError_t setup_grouped();
 const char* grouped_describe();
 // Enqueues the grouped path; *nlaunch receives the number of kernels launched.
+// marks: optional, kGroupedKernels + 1 events; marks[i] is recorded just
+// before kernel i of the sequence below and marks[kGroupedKernels] after the
+// last one (per-kernel timing; nullptr records nothing).
+constexpr int kGroupedKernels = 9;  // route, topk, plan, scatter, gemv_gu, tc_gu, gemv_dn, tc_dn, combine
 cudaError_t launch_grouped(const GroupedParams& p, const GroupedWorkspace& ws, cudaStream_t stream,
-                           int* nlaunch);
+                           int* nlaunch, cudaEvent_t* marks = nullptr);
 
 }  // namespace lingmoe
