@@ -125,6 +125,19 @@ def test_prefill_t2048_zipf_sampled(full):
     compare(ref, out[sample], idx[sample], w[sample], 8, "prefill sample")
 
 
+def test_mixed_gemv_and_tile_experts_t200(full):
+    """One call whose experts split between the GEMV kernels (1..8 tokens)
+    and the tensor-core tiles (more), every output compared."""
+    _, _, host_b, layer_b = full
+    T = 200
+    xs = workloads.tokens(T, seed=31337, device=DEV)
+    out, idx, w = layer_b.forward(xs, return_routing=True)
+    torch.cuda.synchronize()
+    counts = np.bincount(idx.cpu().numpy().reshape(-1), minlength=512)
+    assert (counts > 8).any() and ((counts > 0) & (counts <= 8)).any()
+    compare(oracle.moe_layer(bits(xs), host_b, 8), out, idx, w, 8, "mixed T=200")
+
+
 # ------------------------------------------------------------------ degenerate routing
 
 def _small_layer(E, k, seed, max_tokens=16, zero_router=False):
@@ -136,7 +149,9 @@ def _small_layer(E, k, seed, max_tokens=16, zero_router=False):
 
 def test_all_logits_equal_picks_lowest_indices():
     host, layer = _small_layer(16, 8, seed=3, zero_router=True)
-    for T in (1, 4, 9):
+    # experts 0..7 get exactly T tokens each: T = 8 is the largest expert the
+    # GEMV kernels take, T = 9 the smallest tensor-core tile
+    for T in (1, 4, 8, 9):
         xs = workloads.tokens(T, seed=40 + T, device="cpu")
         out, idx, w = layer.forward(xs.to(DEV), return_routing=True)
         torch.cuda.synchronize()
