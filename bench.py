@@ -39,12 +39,12 @@ L2_FLUSH_BYTES = 256 << 20
 # the command), valid only while the kernel's sources are the ones captured:
 # the sources are hashed and the figure is reported as null once they change.
 TRAFFIC = {
-    "decode_e512_t1": {"bytes": 41_036_544 + 9_472,
+    "decode_e512_t1": {"bytes": 41_036_288 + 13_568,
                        "sources": ('decode.cu', 'decode.h', 'common.cuh', 'layout.h'),
-                       "sha256": "844e57c1ead859209af68874df7195df955e778ed669d35487ec2db09dd04154"},
-    "verify_e512_t4": {"bytes": 126_062_848 + 3_859_456,
+                       "sha256": "ed6ad3f459dbdeaf472f2b064f6568192661d8f7c5ed1856120264390f27db67"},
+    "verify_e512_t4": {"bytes": 126_536_960 + 4_990_208,
                        "sources": ('decode.cu', 'decode.h', 'common.cuh', 'layout.h'),
-                       "sha256": "844e57c1ead859209af68874df7195df955e778ed669d35487ec2db09dd04154"},
+                       "sha256": "ed6ad3f459dbdeaf472f2b064f6568192661d8f7c5ed1856120264390f27db67"},
     # token-grouped: the dominant kernel, tc_grouped_kernel<0> (gate/up tiles)
     "prefill_e512_t2048_zipf": {"bytes": 457_028_864 + 53_828_608,
                                 "sources": ('grouped_tc.cu', 'grouped_tc.h', 'common.cuh', 'layout.h'),

@@ -715,15 +715,22 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     for (int v = tid; v < nblk * T * kDnUnitRows; v += kDecodeThreads) {
       const int blk = v / (T * kDnUnitRows), rem = v - blk * T * kDnUnitRows, t = rem >> 3, r = rem & 7;
       const float* pb = part + (size_t)blk * (PL::P + T) * 8;
+      float v8[kMaxTopK];  // all loads in flight first, then the sum in slot order
+#pragma unroll
+      for (int sl = 0; sl < kMaxTopK; ++sl) v8[sl] = sl < K ? pb[(t * K + sl) * 8 + r] : 0.f;
+      const float vs = pb[(PL::P + t) * 8 + r];
       float s = 0.f;
-      for (int sl = 0; sl < K; ++sl) s += pb[(t * K + sl) * 8 + r];
-      s += pb[(PL::P + t) * 8 + r];
+#pragma unroll
+      for (int sl = 0; sl < kMaxTopK; ++sl)
+        if (sl < K) s += v8[sl];
+      s += vs;
       p.out[(size_t)t * kH + kDnUnitRows * (b0 + blk) + r] = __float2bfloat16_rn(s);
     }
   }
   // every CTA (aborted or not) counts itself out: the next launch's index
   __syncthreads();
-  if (tid == 0 && hd.dcopies) mbar_wait(&hd.dbar, 0, p.wait_limit_ns, p.err);  // no copy left in flight
+  // no copy left in flight (without an abort the phase-4 warps waited for them)
+  if (tid == 0 && hd.dcopies && aborted(hd)) mbar_wait(&hd.dbar, 0, p.wait_limit_ns, p.err);
   if (tid == 0) atomicAdd(p.sync + 3, 1ull);  // read by later launches only: no fence needed
   LING_TRACE(9);
 }
