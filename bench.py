@@ -179,21 +179,29 @@ def cpu_oracle_rate(workload: str, seconds: float = 15.0, max_tokens: int = 64):
         host["router_bias"] = workloads.zipf_router_bias(E, wl["zipf_s"]).numpy()
     T = min(wl["T"], 4)
     seeds = wl.get("token_seeds") or wl.get("call_seeds") or [1 + t for t in range(1000)]
-    n, t0 = 0, time.perf_counter()
-    calls = 0
-    while calls < max_tokens and (time.perf_counter() - t0) < seconds:
-        x = workloads.tokens(T, seed=seeds[calls % len(seeds)], device="cpu")
-        xb = x.view(torch.int16).numpy().view(np.uint16)
-        oracle.moe_layer(xb, host, 8)
-        n += T
-        calls += 1
-    dt = time.perf_counter() - t0
+
+    def timed(budget):
+        n, calls, t0 = 0, 0, time.perf_counter()
+        while calls < max_tokens and (time.perf_counter() - t0) < budget:
+            x = workloads.tokens(T, seed=seeds[calls % len(seeds)], device="cpu")
+            xb = x.view(torch.int16).numpy().view(np.uint16)
+            oracle.moe_layer(xb, host, 8)
+            n += T
+            calls += 1
+        return n, calls, time.perf_counter() - t0
+
+    from threadpoolctl import threadpool_info, threadpool_limits
+    blas = sum(i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas") or 1
+    n, calls, dt = timed(seconds * 2 / 3)  # BLAS threads as configured (all cores by default)
+    with threadpool_limits(limits=1, user_api="blas"):
+        n1, calls1, dt1 = timed(seconds / 3)
     cores = len(os.sched_getaffinity(0))
-    threads = torch.get_num_threads()
-    return {"value": n / dt, "unit": "tokens/s", "cores": cores, "threads": threads,
+    return {"value": n / dt, "unit": "tokens/s", "cores": cores, "threads": blas,
             "kind": "oracle",
             "sample": f"{calls} calls of T={T} of {workload} through the fp64 numpy oracle "
-                      f"({dt:.1f} s of host time, numpy/BLAS threads as configured: {threads})"}
+                      f"({dt:.1f} s of host time, {blas} BLAS threads)",
+            "single_thread": {"value": n1 / dt1, "unit": "tokens/s", "threads": 1,
+                              "sample": f"{calls1} calls, {dt1:.1f} s, one BLAS thread"}}
 
 
 def run_reference(args):
@@ -493,6 +501,7 @@ def run_ours(args):
             "clocks": clk.summary(),
             "wall_s_timed_region": t_wall,
             "step_us_p10_p50_p90": [sorted(step_ms)[int(q * (nsteps - 1))] * 1e3 for q in (0.1, 0.5, 0.9)],
+            "tokens_per_s_median_step": ws * T / (statistics.median(step_ms) * 1e-3),
         }
         print(json.dumps(line), flush=True)
     if ws > 1:
