@@ -419,7 +419,7 @@ def run_ours(args):
     # per-kernel times of the token-grouped path (a separate pass: the events
     # around each launch are not in the timed steps above)
     ktimes = None
-    if T > 4 and not stack:
+    if T > 8 and not stack:
         layers[0].set_kernel_timing(True)
         per = {}
         for i in range(nsteps):

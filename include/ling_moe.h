@@ -100,6 +100,8 @@ int ling_moe_create(const ling_moe_config_t *cfg, const ling_moe_weights_t *w,
  * Asynchronous: no host synchronisation and no allocation, so the call can be
  * captured into a CUDA graph.  Device-detected failures (a bounded wait that
  * gave up) are reported later by ling_moe_status.
+ * Kernels: T <= 4 one persistent decode launch; 5 <= T <= 8 two of them (the
+ * first 4 tokens, then the rest); larger T the token-grouped path (9 launches).
  * Errors: INVALID_ARG (checked on the host before anything is enqueued), CUDA. */
 int ling_moe_forward(ling_moe_t *h, const void *x, int T, void *out, void *stream);
 
@@ -134,7 +136,8 @@ const char *ling_moe_last_error(void);
 
 /* ---- per-kernel timing (measurement; off by default) ----
  * With on != 0, every later forward call also records CUDA events on its
- * stream around each kernel it launches (one for T <= 4, nine for larger T:
+ * stream around each kernel it launches (one for T <= 4, two for 5 <= T <= 8,
+ * nine for larger T:
  * route, topk, plan, scatter, gemv_gu, tc_gu, gemv_dn, tc_dn, combine).  The
  * events add a little time of their own; do not leave timing on while
  * capturing a stream into a graph.  on == 0 frees the events.  Returns OK,

@@ -90,7 +90,7 @@ def test_full_verify_t4(full):
     print("verify", rep)
 
 
-@pytest.mark.parametrize("T", [2, 3, 5, 17, 37])
+@pytest.mark.parametrize("T", [2, 3, 5, 8, 9, 17, 37])
 def test_full_ragged_token_counts(full, T):
     host, layer, _, _ = full
     xs = workloads.tokens(T, seed=500 + T, device=DEV)
@@ -280,5 +280,7 @@ def test_describe_and_launch_count(full):
     n0 = layer.launch_count()
     layer.forward(workloads.tokens(1, seed=1, device=DEV))
     assert layer.launch_count() == n0 + 1
-    layer.forward(workloads.tokens(8, seed=1, device=DEV))
-    assert layer.launch_count() > n0 + 1
+    layer.forward(workloads.tokens(8, seed=1, device=DEV))  # 5..8 tokens: two decode launches
+    assert layer.launch_count() == n0 + 3
+    layer.forward(workloads.tokens(9, seed=1, device=DEV))  # the token-grouped path: 9 kernels
+    assert layer.launch_count() == n0 + 12
