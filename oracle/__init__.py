@@ -1,4 +1,5 @@
-"""fp64 CPU oracle of the W4 g32 MoE layer.
+"""fp64 CPU oracles of the W4 g32 MoE layer (moe_ref) and of the online-FP8
+LM head (lmhead_ref, imported as oracle.lmhead_ref).
 
 TEST INFRASTRUCTURE ONLY: imported by the tests, the package smoke check and
 the benchmark's CPU-baseline arm, never by the GPU library.
