@@ -1,7 +1,8 @@
 """Benchmark of the W4 g32 MoE layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode_e512_t1|verify_e512_t4|stack40_e512_t1|prefill_e512_t2048_zipf|reduced_e32_t1]
+                    [--workload decode_e512_t1|verify_e512_t4|stack40_e512_t1|prefill_e512_t2048_zipf|reduced_e32_t1
+                               |lmhead_fp8_v157184_t1|lmhead_fp8_v157184_t8]
 
 A step is one pass of the whole layer (router, top-k, routed gate/up, down,
 shared expert, combine) over one batch of synthetic input: one token for the
@@ -512,6 +513,153 @@ def run_ours(args):
     return 0
 
 
+# ------------------------------------------------------------------ online-FP8 LM head
+
+LMHEAD_METRIC = "online-FP8 LM-head tokens/s and achieved HBM GB/s (157,184 x 2,560 e4m3, fp32 logits)"
+
+
+def lmhead_bytes(V, T):
+    """Algorithmic bytes of one call: e4m3 codes + row scales, the tokens, the fp32 logits."""
+    return V * H + 4 * V + T * H * 2 + T * V * 4
+
+
+def lmhead_oracle_rate(workload: str, seconds: float = 15.0, rows: int = 8192):
+    """The oracle (quantise the head rows and the tokens, exact dot products)
+    on a slice of the head, scaled to tokens/s of the whole vocabulary."""
+    import numpy as np
+    import torch
+    import oracle.lmhead_ref as L
+    import workloads
+    wl = workloads.LMHEAD_WORKLOADS[workload]
+    V, T = wl["vocab"], wl["T"]
+    w = workloads.lm_head_weights(rows, H, seed=wl["weight_seed"], device="cpu")
+    wb = w.view(torch.int16).numpy().view(np.uint16)
+    n, dt, t0 = 0, 0.0, time.perf_counter()
+    while dt < seconds and n < 64:
+        x = workloads.tokens(T, H, seed=wl["token_seed"] + n, device="cpu")
+        L.lm_head_fp8(x.view(torch.int16).numpy().view(np.uint16), wb)
+        n += 1
+        dt = time.perf_counter() - t0
+    per_call_full = dt / n * (V / rows)
+    return {"value": T / per_call_full, "unit": "tokens/s", "cores": len(os.sched_getaffinity(0)),
+            "kind": "oracle",
+            "sample": f"{n} calls of T={T} through the fp64 numpy oracle on {rows} of the {V} head rows "
+                      f"(each call quantises those rows and the tokens), {dt:.1f} s, scaled by {V}/{rows}"}
+
+
+def run_lmhead_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import workloads
+    wl = workloads.LMHEAD_WORKLOADS[args.workload]
+    budget = max(10.0, min(60.0, 2.0 * (args.steps + args.warmup)))
+    cpu = lmhead_oracle_rate(args.workload, seconds=budget)
+    v = cpu["value"]
+    line = {"metric": LMHEAD_METRIC, "value": v, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": wl["T"] / v * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": args.workload, "T": wl["T"], "vocab": wl["vocab"], "hidden": H},
+            "cpu_baseline": cpu,
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_lmhead(args):
+    import torch
+    import torch.distributed as dist
+    ws, rank, local = dist_env()
+    if ws > 1:
+        dist.init_process_group("nccl", init_method="env://", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import workloads
+    import weight_only_int4_fp32_b200 as lm
+    wl = workloads.LMHEAD_WORKLOADS[args.workload]
+    V, T = wl["vocab"], wl["T"]
+    w = workloads.lm_head_weights(V, H, seed=wl["weight_seed"], device=dev)
+    head = lm.LMHeadFP8(w)
+    del w
+    torch.cuda.empty_cache()
+    nsteps, nwarm = args.steps, args.warmup
+    off = rank * REPLICA_SEED_STRIDE
+    inputs = [workloads.tokens(T, H, seed=wl["token_seed"] + i + off, device=dev) for i in range(nsteps + nwarm)]
+    logits = torch.empty((T, V), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for i in range(nwarm):
+        flush.fill_(float(i))
+        head.forward(inputs[i], logits)
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(nsteps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(nsteps)]
+    n0 = head.launch_count()
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter()
+    with ClockSampler(local) as clk:
+        for i in range(nsteps):
+            flush.fill_(float(i))
+            starts[i].record(stream)
+            head.forward(inputs[nwarm + i], logits)
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall
+    launches = head.launch_count() - n0
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    kern_ms = max_over_ranks(sum(step_ms), dev)
+
+    # end to end: pinned host tokens in, fp32 logits back to pinned host memory
+    xh = [inputs[nwarm + i].cpu().pin_memory() for i in range(nsteps)]
+    lh = torch.empty((T, V), dtype=torch.float32).pin_memory()
+    for i in range(min(nwarm, 5)):
+        head.forward_host(xh[i % nsteps], lh)
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    te = time.perf_counter()
+    for i in range(nsteps):
+        flush.fill_(float(i))
+        head.forward_host(xh[i], lh)
+    te = max_over_ranks(time.perf_counter() - te, dev)
+    e2e = {"value": ws * nsteps * T / te, "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
+           "d2h_bytes_per_step": T * V * 4,
+           "note": "ling_moe_lmhead_forward_host per step: pinned H2D copy + head + D2H copy of the logits + "
+                   "stream sync; the L2 flush fill runs between steps inside this wall clock"}
+
+    bytes_per_launch = lmhead_bytes(V, T)
+    avg_ms = kern_ms / nsteps
+    achieved = bytes_per_launch / (avg_ms * 1e-3) / 1e9
+    peak, peak_kind = peaks()
+    roofline = {"bound": "hbm", "kernel": f"lmh_gemv_kernel<{T}> (one launch per call)", "achieved": achieved,
+                "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic_for(args.workload),
+                "peak_kind": peak_kind, "bytes_per_launch": bytes_per_launch}
+    if rank == 0:
+        cpu = lmhead_oracle_rate(args.workload, seconds=args.cpu_seconds) \
+            if ws == 1 and args.cpu_seconds > 0 else None
+        line = {
+            "metric": LMHEAD_METRIC, "value": ws * nsteps * T / (kern_ms * 1e-3), "unit": "tokens/s",
+            "n_gpus": ws, "steps": nsteps, "warmup": nwarm, "ms_per_step": avg_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 x e4m3, fp32 accumulate",
+            "data": "synthetic (seeded head and tokens, recipe in DESIGN.md)",
+            "config": {"workload": args.workload, "T": T, "vocab": V, "hidden": H,
+                       "l2": "flushed before every step (256 MiB write), outside the per-step events; "
+                             "the 402 MB of codes exceed L2 anyway",
+                       "parallelism": f"replicas x{ws}"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "clocks": clk.summary(), "wall_s_timed_region": t_wall,
+            "step_us_p10_p50_p90": [sorted(step_ms)[int(q * (nsteps - 1))] * 1e3 for q in (0.1, 0.5, 0.9)],
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    head.close()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -523,9 +671,10 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    lmhead = args.workload.startswith("lmhead")
     if args.impl == "reference":
-        return run_reference(args)
-    return run_ours(args)
+        return run_lmhead_reference(args) if lmhead else run_reference(args)
+    return run_lmhead(args) if lmhead else run_ours(args)
 
 
 if __name__ == "__main__":

@@ -195,6 +195,65 @@ int ling_moe_test_set_wait(ling_moe_t *h, int skip_arrive_cta, uint64_t wait_lim
 int ling_moe_route_noalloc(const void *x, int T, const void *router_w, const float *router_bias,
                            int num_experts, int top_k, int32_t *topk_idx, float *topk_w, void *stream);
 
+/* ---- online-FP8 LM head ----
+ * Source: bpdata article "Harom optimalizacio a Ling-3.0-flash MoE
+ * inferenciajanak", section "Optimalizacio 2: Online FP8 LM head kvantalas":
+ * the bf16 LM head (157,184 x 2,560 in Ling-3.0-flash) is quantised to FP8
+ * once, when the head is built, so that each decoded token reads about half
+ * as many bytes.  The pages do not fix the FP8 format or the scaling; this
+ * library takes:
+ *   FP8 = e4m3 (no infinities, largest finite 448), round to nearest even,
+ *         saturating;
+ *   weights: one fp32 scale per vocabulary row, s_w[v] = max_k |W[v,k]| / 448
+ *         (1 for an all-zero row), codes e4m3(W[v,k] / s_w[v]);
+ *   tokens: the same per token at every call, s_x[t], codes e4m3(x[t,k] / s_x[t]);
+ *   both divisions correctly rounded in fp32;
+ *   logits[t, v] = (sum_k e4m3(x)[t,k] * e4m3(W)[v,k]) * s_x[t] * s_w[v],
+ *         every product exact, the sum accumulated in fp32 (order unspecified).
+ */
+typedef struct ling_moe_lmhead ling_moe_lmhead_t; /* opaque handle */
+
+/* Quantise the head w [vocab, hidden] (bf16, DEVICE, row-major, 16-byte
+ * aligned; read only during this call) into library-owned device memory:
+ * vocab * hidden code bytes plus vocab fp32 scales, and staging buffers for
+ * ling_moe_lmhead_forward_host (8 tokens).  Synchronises the device.
+ * Limits: vocab >= 1; hidden a multiple of 512, at most 4096.
+ * Errors: INVALID_ARG (NULL, misaligned, non-positive sizes), UNSUPPORTED
+ * (hidden outside the limits, not an sm_100 GPU), OOM, CUDA.  On failure
+ * *out is NULL and nothing leaks. */
+int ling_moe_lmhead_create(const void *w, int vocab, int hidden, ling_moe_lmhead_t **out);
+
+/* logits[T, vocab] (fp32, DEVICE, 4-byte aligned, row-major) of the tokens
+ * x[T, hidden] (bf16, DEVICE, 16-byte aligned) on `stream`; 0 <= T <= 8
+ * (T == 0 enqueues nothing).  logits must not overlap x.  One kernel launch;
+ * asynchronous, no allocation, capturable into a CUDA graph.
+ * Errors: INVALID_ARG (checked before anything is enqueued), CUDA. */
+int ling_moe_lmhead_forward(ling_moe_lmhead_t *h, const void *x, int T, float *logits, void *stream);
+
+/* As ling_moe_lmhead_forward, and also writes the tokens' quantisation:
+ * x_codes [T, hidden] e4m3 bytes (16-byte aligned) and x_scales fp32 [T]
+ * (DEVICE; either may be NULL; neither may overlap x or logits). */
+int ling_moe_lmhead_forward_ex(ling_moe_lmhead_t *h, const void *x, int T, float *logits,
+                               uint8_t *x_codes, float *x_scales, void *stream);
+
+/* End-to-end call on HOST buffers: copies x_host [T, hidden] bf16 to the
+ * device, runs the head, copies logits [T, vocab] fp32 to logits_host and
+ * waits for the stream.  Pinned host buffers give asynchronous copies. */
+int ling_moe_lmhead_forward_host(ling_moe_lmhead_t *h, const void *x_host, int T, float *logits_host,
+                                 void *stream);
+
+/* The handle's quantised head: *codes = e4m3 [vocab, hidden], *scales = fp32
+ * [vocab], DEVICE pointers owned by the handle (read only; valid until
+ * ling_moe_lmhead_destroy). */
+int ling_moe_lmhead_weights(const ling_moe_lmhead_t *h, const uint8_t **codes, const float **scales);
+
+/* Number of kernel launches the handle's forward calls have enqueued. */
+int64_t ling_moe_lmhead_launch_count(const ling_moe_lmhead_t *h);
+
+/* Free everything the handle owns.  NULL is a no-op.  The caller must make
+ * sure no enqueued work still uses the handle. */
+void ling_moe_lmhead_destroy(ling_moe_lmhead_t *h);
+
 #ifdef __cplusplus
 }
 #endif

@@ -112,3 +112,34 @@ def test_python_errors_carry_the_code():
     with pytest.raises(lm.LingMoEError) as ei:
         lm.ling_moe_create(_cfg(top_k=9, num_experts=16), _weights())
     assert ei.value.code == lm.LING_MOE_ERR_UNSUPPORTED
+
+
+def _lmh_create_rc(w, vocab, hidden):
+    h = ctypes.c_void_p()
+    rc = lm.lib.ling_moe_lmhead_create(w, vocab, hidden, ctypes.byref(h))
+    return rc, h.value
+
+
+@pytest.mark.parametrize("w,vocab,hidden,code", [
+    (None, 1000, 2560, lm.LING_MOE_ERR_INVALID_ARG),
+    (0x100008, 1000, 2560, lm.LING_MOE_ERR_INVALID_ARG),      # misaligned
+    (0x100000, 0, 2560, lm.LING_MOE_ERR_INVALID_ARG),
+    (0x100000, 1000, -512, lm.LING_MOE_ERR_INVALID_ARG),
+    (0x100000, 1000, 2304, lm.LING_MOE_ERR_UNSUPPORTED),      # not a multiple of 512
+    (0x100000, 1000, 4608, lm.LING_MOE_ERR_UNSUPPORTED),      # above 4096
+])
+def test_lmhead_create_rejects_bad_arguments(w, vocab, hidden, code):
+    rc, h = _lmh_create_rc(w, vocab, hidden)
+    assert rc == code, lm.ling_moe_last_error()
+    assert h is None
+    assert lm.lib.ling_moe_lmhead_create(0x100000, 1000, 2560, None) == lm.LING_MOE_ERR_INVALID_ARG
+
+
+def test_lmhead_null_handle_is_rejected_everywhere():
+    assert lm.lib.ling_moe_lmhead_forward(None, 16, 1, 32, None) == lm.LING_MOE_ERR_INVALID_ARG
+    assert lm.lib.ling_moe_lmhead_forward_ex(None, 16, 1, 32, None, None, None) == lm.LING_MOE_ERR_INVALID_ARG
+    assert lm.lib.ling_moe_lmhead_forward_host(None, 16, 1, 32, None) == lm.LING_MOE_ERR_INVALID_ARG
+    c, s = ctypes.c_void_p(), ctypes.c_void_p()
+    assert lm.lib.ling_moe_lmhead_weights(None, ctypes.byref(c), ctypes.byref(s)) == lm.LING_MOE_ERR_INVALID_ARG
+    assert lm.lib.ling_moe_lmhead_launch_count(None) == 0
+    lm.lib.ling_moe_lmhead_destroy(None)  # no-op

@@ -19,7 +19,7 @@ __all__ = [
     "ling_moe_create", "ling_moe_forward", "ling_moe_forward_ex", "ling_moe_forward_host",
     "ling_moe_status", "ling_moe_describe", "ling_moe_launch_count", "ling_moe_last_error",
     "ling_moe_destroy", "ling_moe_test_set_wait", "ling_moe_route_noalloc", "ling_moe_set_kernel_timing",
-    "ling_moe_kernel_times", "MoELayer", "EXPORTED",
+    "ling_moe_kernel_times", "MoELayer", "LMHeadFP8", "EXPORTED",
 ]
 
 LING_MOE_OK = 0
@@ -35,6 +35,9 @@ EXPORTED = (
     "ling_moe_status", "ling_moe_describe", "ling_moe_launch_count", "ling_moe_last_error",
     "ling_moe_destroy", "ling_moe_test_set_wait", "ling_moe_route_noalloc",
     "ling_moe_set_kernel_timing", "ling_moe_kernel_times", "ling_moe_kernel_name",
+    "ling_moe_lmhead_create", "ling_moe_lmhead_forward", "ling_moe_lmhead_forward_ex",
+    "ling_moe_lmhead_forward_host", "ling_moe_lmhead_weights", "ling_moe_lmhead_launch_count",
+    "ling_moe_lmhead_destroy",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -96,6 +99,13 @@ def _load():
         "ling_moe_set_kernel_timing": (ci, [vp, ci]),
         "ling_moe_kernel_times": (ci, [vp, ctypes.POINTER(ctypes.c_float), ci, ctypes.POINTER(ci)]),
         "ling_moe_kernel_name": (ctypes.c_char_p, [vp, ci]),
+        "ling_moe_lmhead_create": (ci, [vp, ci, ci, ctypes.POINTER(vp)]),
+        "ling_moe_lmhead_forward": (ci, [vp, vp, ci, vp, vp]),
+        "ling_moe_lmhead_forward_ex": (ci, [vp, vp, ci, vp, vp, vp, vp]),
+        "ling_moe_lmhead_forward_host": (ci, [vp, vp, ci, vp, vp]),
+        "ling_moe_lmhead_weights": (ci, [vp, ctypes.POINTER(vp), ctypes.POINTER(vp)]),
+        "ling_moe_lmhead_launch_count": (i64, [vp]),
+        "ling_moe_lmhead_destroy": (None, [vp]),
     }
     for name, (res, args) in sig.items():
         try:
@@ -259,6 +269,93 @@ class MoELayer:
     def close(self):
         if getattr(self, "handle", None):
             ling_moe_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class _DeviceArray:
+    """A view of library-owned device memory for torch.as_tensor (torch
+    accepts only writable views; the callers only clone it)."""
+
+    def __init__(self, ptr: int, shape: tuple, typestr: str):
+        self.__cuda_array_interface__ = {"shape": shape, "typestr": typestr, "data": (ptr, False),
+                                         "version": 3, "strides": None}
+
+
+class LMHeadFP8:
+    """The online-FP8 LM head on the current CUDA device.
+
+    `w` is the bf16 head [vocab, hidden] (contiguous CUDA tensor); it is
+    quantised to e4m3 with one fp32 scale per row when the object is built
+    and may be freed afterwards.  Each call quantises its tokens the same
+    way and returns fp32 logits [T, vocab] (T <= 8).
+    """
+
+    MAX_TOKENS = 8
+
+    def __init__(self, w):
+        import torch  # device memory and streams only
+        if w.dtype != torch.bfloat16 or not w.is_cuda or not w.is_contiguous() or w.dim() != 2:
+            raise ValueError("w must be a contiguous 2-D bf16 CUDA tensor")
+        self.vocab, self.hidden = w.shape
+        h = ctypes.c_void_p()
+        _check(lib.ling_moe_lmhead_create(w.data_ptr(), self.vocab, self.hidden, ctypes.byref(h)))
+        self.handle = h.value
+        self._torch = torch
+
+    def _stream(self, stream):
+        if stream is None:
+            return self._torch.cuda.current_stream().cuda_stream
+        return getattr(stream, "cuda_stream", stream)
+
+    def forward(self, x, logits=None, stream=None, return_codes: bool = False):
+        torch = self._torch
+        if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous() or x.dim() != 2:
+            raise ValueError("x must be a contiguous 2-D bf16 CUDA tensor")
+        T = x.shape[0]
+        if logits is None:
+            logits = torch.empty((T, self.vocab), dtype=torch.float32, device=x.device)
+        s = self._stream(stream)
+        if return_codes:
+            xq = torch.empty((T, self.hidden), dtype=torch.uint8, device=x.device)
+            xs = torch.empty((T,), dtype=torch.float32, device=x.device)
+            _check(lib.ling_moe_lmhead_forward_ex(self.handle, x.data_ptr(), T, logits.data_ptr(),
+                                                  xq.data_ptr(), xs.data_ptr(), s))
+            return logits, xq, xs
+        _check(lib.ling_moe_lmhead_forward(self.handle, x.data_ptr(), T, logits.data_ptr(), s))
+        return logits
+
+    __call__ = forward
+
+    def forward_host(self, x_host, logits_host=None, stream=None):
+        torch = self._torch
+        T = x_host.shape[0]
+        if logits_host is None:
+            logits_host = torch.empty((T, self.vocab), dtype=torch.float32, pin_memory=True)
+        _check(lib.ling_moe_lmhead_forward_host(self.handle, x_host.data_ptr(), T, logits_host.data_ptr(),
+                                                self._stream(stream)))
+        return logits_host
+
+    def weights(self):
+        """(codes uint8 [vocab, hidden], scales fp32 [vocab]) copied from the handle's device memory."""
+        torch = self._torch
+        c, s = ctypes.c_void_p(), ctypes.c_void_p()
+        _check(lib.ling_moe_lmhead_weights(self.handle, ctypes.byref(c), ctypes.byref(s)))
+        codes = torch.as_tensor(_DeviceArray(c.value, (self.vocab, self.hidden), "|u1"), device="cuda").clone()
+        scales = torch.as_tensor(_DeviceArray(s.value, (self.vocab,), "<f4"), device="cuda").clone()
+        return codes, scales
+
+    def launch_count(self) -> int:
+        return lib.ling_moe_lmhead_launch_count(self.handle)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib.ling_moe_lmhead_destroy(self.handle)
             self.handle = None
 
     def __del__(self):

@@ -14,6 +14,7 @@
 #include "layout.h"
 #include "decode.h"
 #include "grouped.h"
+#include "lmhead.h"
 #include "repack.h"
 
 using namespace lingmoe;
@@ -473,6 +474,154 @@ int ling_moe_test_set_wait(ling_moe_t* h, int skip_arrive_cta, uint64_t wait_lim
   h->skip_arrive_cta = skip_arrive_cta < 0 ? -1 : skip_arrive_cta;
   h->wait_limit_ns = wait_limit_ns ? wait_limit_ns : kDefaultWaitNs;
   return LING_MOE_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Online-FP8 LM head
+
+struct ling_moe_lmhead {
+  int device = 0;
+  int vocab = 0;
+  int hidden = 0;
+  int nctas = 0;
+  uint8_t* codes = nullptr;      // e4m3 [vocab, hidden]
+  float* scales = nullptr;       // fp32 [vocab]
+  __nv_bfloat16* x_stage = nullptr;
+  float* logits_stage = nullptr;
+  std::atomic<int64_t> launches{0};
+  void release() {
+    for (void* p : {(void*)codes, (void*)scales, (void*)x_stage, (void*)logits_stage})
+      if (p) cudaFree(p);
+    codes = nullptr;
+    scales = nullptr;
+    x_stage = nullptr;
+    logits_stage = nullptr;
+  }
+};
+
+extern "C" {
+
+int ling_moe_lmhead_create(const void* w, int vocab, int hidden, ling_moe_lmhead_t** out) {
+  if (!out) return fail(LING_MOE_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (!w) return fail(LING_MOE_ERR_INVALID_ARG, "w is NULL");
+  if (!aligned16(w)) return fail(LING_MOE_ERR_INVALID_ARG, "w must be 16-byte aligned");
+  if (vocab <= 0 || hidden <= 0) return fail(LING_MOE_ERR_INVALID_ARG, "vocab and hidden must be positive");
+  if (hidden % 512 || hidden > kLmhMaxHidden)
+    return fail(LING_MOE_ERR_UNSUPPORTED, "hidden must be a multiple of 512 and at most %d (got %d)",
+                kLmhMaxHidden, hidden);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  cudaDeviceProp prop;
+  e = cudaGetDeviceProperties(&prop, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+  if (prop.major != 10)
+    return fail(LING_MOE_ERR_UNSUPPORTED, "needs an sm_100 GPU (got sm_%d%d)", prop.major, prop.minor);
+  e = setup_lmhead();
+  if (e != cudaSuccess) return cuda_fail(e, "LM-head kernel attributes");
+
+  ling_moe_lmhead* h = new ling_moe_lmhead();
+  h->device = dev;
+  h->vocab = vocab;
+  h->hidden = hidden;
+  h->nctas = prop.multiProcessorCount;
+  struct A { void** p; size_t n; } plan[] = {
+      {(void**)&h->codes, (size_t)vocab * hidden},
+      {(void**)&h->scales, (size_t)vocab * sizeof(float)},
+      {(void**)&h->x_stage, (size_t)kLmhMaxT * hidden * sizeof(__nv_bfloat16)},
+      {(void**)&h->logits_stage, (size_t)kLmhMaxT * vocab * sizeof(float)},
+  };
+  for (auto& a : plan) {
+    e = cudaMalloc(a.p, a.n);
+    if (e != cudaSuccess) {
+      *a.p = nullptr;
+      const int rc = cuda_fail(e, "cudaMalloc");
+      h->release();
+      delete h;
+      return rc;
+    }
+  }
+  e = launch_lmh_quantize(static_cast<const __nv_bfloat16*>(w), vocab, hidden, h->codes, h->scales, nullptr);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    const int rc = cuda_fail(e, "LM-head quantisation");
+    h->release();
+    delete h;
+    return rc;
+  }
+  *out = h;
+  return LING_MOE_OK;
+}
+
+static int lmhead_forward_impl(ling_moe_lmhead_t* h, const void* x, int T, float* logits, uint8_t* x_codes,
+                               float* x_scales, void* stream) {
+  if (!h) return fail(LING_MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (T < 0 || T > kLmhMaxT) return fail(LING_MOE_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, kLmhMaxT);
+  if (T == 0) return LING_MOE_OK;
+  if (!x || !logits) return fail(LING_MOE_ERR_INVALID_ARG, "x or logits is NULL");
+  if (!aligned16(x)) return fail(LING_MOE_ERR_INVALID_ARG, "x must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(logits) & 3u) return fail(LING_MOE_ERR_INVALID_ARG, "logits must be 4-byte aligned");
+  if (x_codes && !aligned16(x_codes)) return fail(LING_MOE_ERR_INVALID_ARG, "x_codes must be 16-byte aligned");
+  if (x_scales && (reinterpret_cast<uintptr_t>(x_scales) & 3u))
+    return fail(LING_MOE_ERR_INVALID_ARG, "x_scales must be 4-byte aligned");
+  const size_t xb = (size_t)T * h->hidden * sizeof(__nv_bfloat16), lb = (size_t)T * h->vocab * sizeof(float);
+  if (overlaps(x, xb, logits, lb)) return fail(LING_MOE_ERR_INVALID_ARG, "logits overlaps x");
+  if (x_codes && (overlaps(x_codes, (size_t)T * h->hidden, logits, lb) || overlaps(x_codes, (size_t)T * h->hidden, x, xb)))
+    return fail(LING_MOE_ERR_INVALID_ARG, "x_codes overlaps x or logits");
+  if (x_scales && (overlaps(x_scales, (size_t)T * 4, logits, lb) || overlaps(x_scales, (size_t)T * 4, x, xb)))
+    return fail(LING_MOE_ERR_INVALID_ARG, "x_scales overlaps x or logits");
+  cudaError_t e = launch_lmh_forward(h->codes, h->scales, h->vocab, h->hidden, static_cast<const __nv_bfloat16*>(x), T,
+                                     logits, x_codes, x_scales, h->nctas, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "LM-head launch");
+  h->launches.fetch_add(1);
+  return LING_MOE_OK;
+}
+
+int ling_moe_lmhead_forward(ling_moe_lmhead_t* h, const void* x, int T, float* logits, void* stream) {
+  return lmhead_forward_impl(h, x, T, logits, nullptr, nullptr, stream);
+}
+
+int ling_moe_lmhead_forward_ex(ling_moe_lmhead_t* h, const void* x, int T, float* logits, uint8_t* x_codes,
+                               float* x_scales, void* stream) {
+  return lmhead_forward_impl(h, x, T, logits, x_codes, x_scales, stream);
+}
+
+int ling_moe_lmhead_forward_host(ling_moe_lmhead_t* h, const void* x_host, int T, float* logits_host,
+                                 void* stream_v) {
+  if (!h) return fail(LING_MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (T < 0 || T > kLmhMaxT) return fail(LING_MOE_ERR_INVALID_ARG, "T=%d outside [0, %d]", T, kLmhMaxT);
+  if (T == 0) return LING_MOE_OK;
+  if (!x_host || !logits_host) return fail(LING_MOE_ERR_INVALID_ARG, "x_host or logits_host is NULL");
+  const size_t xb = (size_t)T * h->hidden * sizeof(__nv_bfloat16), lb = (size_t)T * h->vocab * sizeof(float);
+  if (overlaps(x_host, xb, logits_host, lb)) return fail(LING_MOE_ERR_INVALID_ARG, "logits_host overlaps x_host");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  cudaError_t e = cudaMemcpyAsync(h->x_stage, x_host, xb, cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "host->device copy");
+  int rc = lmhead_forward_impl(h, h->x_stage, T, h->logits_stage, nullptr, nullptr, stream_v);
+  if (rc) return rc;
+  e = cudaMemcpyAsync(logits_host, h->logits_stage, lb, cudaMemcpyDeviceToHost, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "device->host copy");
+  e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  return LING_MOE_OK;
+}
+
+int ling_moe_lmhead_weights(const ling_moe_lmhead_t* h, const uint8_t** codes, const float** scales) {
+  if (!h || !codes || !scales) return fail(LING_MOE_ERR_INVALID_ARG, "handle, codes or scales is NULL");
+  *codes = h->codes;
+  *scales = h->scales;
+  return LING_MOE_OK;
+}
+
+int64_t ling_moe_lmhead_launch_count(const ling_moe_lmhead_t* h) { return h ? h->launches.load() : 0; }
+
+void ling_moe_lmhead_destroy(ling_moe_lmhead_t* h) {
+  if (!h) return;
+  h->release();
+  delete h;
 }
 
 }  // extern "C"

@@ -1,0 +1,25 @@
+// Online-FP8 LM head: the bf16 head [vocab, hidden] quantised at build time
+// to e4m3 with one fp32 scale per vocabulary row; each call quantises the
+// tokens the same way and returns fp32 logits.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace lingmoe {
+
+constexpr int kLmhMaxT = 8;          // tokens per call
+constexpr int kLmhMaxHidden = 4096;  // hidden % 512 == 0
+
+// w [vocab, hidden] bf16 -> codes [vocab, hidden] e4m3 bytes, scales [vocab] fp32
+cudaError_t launch_lmh_quantize(const __nv_bfloat16* w, int vocab, int hidden, uint8_t* codes, float* scales,
+                                cudaStream_t s);
+// logits [T, vocab] fp32; x_codes / x_scales: optional copies of the tokens' codes and scales
+cudaError_t launch_lmh_forward(const uint8_t* codes, const float* scales, int vocab, int hidden,
+                               const __nv_bfloat16* x, int T, float* logits, uint8_t* x_codes, float* x_scales,
+                               int nctas, cudaStream_t s);
+cudaError_t setup_lmhead();
+
+}  // namespace lingmoe

@@ -16,6 +16,7 @@ it produces, in the canonical boundary layout:
   sh_up     bf16  [I, H]
   sh_down   bf16  [H, I]
   x         bf16  [T, H]        ~ N(0, 1)
+  lm head   bf16  [V, H]        ~ N(0, 0.02) * exp(U(-1, 1)) per row, V = 157,184
 
 A uniform byte carries two independent uniform 4-bit codes, so drawing
 bytes uniformly is the same as drawing each int4 code uniformly in
@@ -176,6 +177,27 @@ WORKLOADS = {
     "prefill_e512_t2048_zipf": dict(num_experts=512, T=2048, weight_seed=0, token_seed=20000,
                                     zipf_s=1.1,
                                     note="full layer, 2048-token prefill chunk, Zipf(1.1) router bias"),
+}
+
+
+VOCAB = 157_184        # LM-head vocabulary of Ling-3.0-flash
+
+
+def lm_head_weights(vocab: int = VOCAB, hidden: int = HIDDEN, seed: int = 0, device="cpu") -> torch.Tensor:
+    """LM head W [vocab, hidden] bf16: N(0, 0.02) times a per-row factor
+    exp(U(-1, 1)), so that the rows' ranges (and their FP8 scales) differ."""
+    g = _gen(seed, device)
+    w = torch.randn((vocab, hidden), generator=g, device=device, dtype=torch.float32)
+    f = torch.empty((vocab, 1), device=device, dtype=torch.float32)
+    f.uniform_(-1.0, 1.0, generator=g)
+    return (w * (0.02 * torch.exp(f))).to(torch.bfloat16)
+
+
+LMHEAD_WORKLOADS = {
+    "lmhead_fp8_v157184_t1": dict(vocab=VOCAB, T=1, weight_seed=7, token_seed=30000,
+                                  note="online-FP8 LM head, 157,184 x 2,560, one token per call"),
+    "lmhead_fp8_v157184_t8": dict(vocab=VOCAB, T=8, weight_seed=7, token_seed=40000,
+                                  note="online-FP8 LM head, 157,184 x 2,560, 8 tokens per call"),
 }
 
 
