@@ -209,14 +209,17 @@ int ling_moe_route_noalloc(const void *x, int T, const void *router_w, const flo
  *   tokens: the same per token at every call, s_x[t], codes e4m3(x[t,k] / s_x[t]);
  *   both divisions correctly rounded in fp32;
  *   logits[t, v] = (sum_k e4m3(x)[t,k] * e4m3(W)[v,k]) * s_x[t] * s_w[v],
- *         every product exact, the sum accumulated in fp32 (order unspecified).
+ *         every product exact; tensor cores sum 256 products at a time
+ *         (16 per instruction, chained), those sums are accumulated in fp32.
  */
 typedef struct ling_moe_lmhead ling_moe_lmhead_t; /* opaque handle */
 
 /* Quantise the head w [vocab, hidden] (bf16, DEVICE, row-major, 16-byte
  * aligned; read only during this call) into library-owned device memory:
- * vocab * hidden code bytes plus vocab fp32 scales, and staging buffers for
- * ling_moe_lmhead_forward_host (8 tokens).  Synchronises the device.
+ * the codes (vocab rounded up to a multiple of 32, times hidden bytes, in a
+ * tiled layout that the GEMV streams in order), vocab fp32 scales, and
+ * staging buffers for ling_moe_lmhead_forward_host (8 tokens).
+ * Synchronises the device.
  * Limits: vocab >= 1; hidden a multiple of 512, at most 4096.
  * Errors: INVALID_ARG (NULL, misaligned, non-positive sizes), UNSUPPORTED
  * (hidden outside the limits, not an sm_100 GPU), OOM, CUDA.  On failure
@@ -226,7 +229,9 @@ int ling_moe_lmhead_create(const void *w, int vocab, int hidden, ling_moe_lmhead
 /* logits[T, vocab] (fp32, DEVICE, 4-byte aligned, row-major) of the tokens
  * x[T, hidden] (bf16, DEVICE, 16-byte aligned) on `stream`; 0 <= T <= 8
  * (T == 0 enqueues nothing).  logits must not overlap x.  One kernel launch;
- * asynchronous, no allocation, capturable into a CUDA graph.
+ * asynchronous, no allocation, capturable into a CUDA graph.  Device-side
+ * failures (a bounded wait that gave up) are reported by
+ * ling_moe_lmhead_status.
  * Errors: INVALID_ARG (checked before anything is enqueued), CUDA. */
 int ling_moe_lmhead_forward(ling_moe_lmhead_t *h, const void *x, int T, float *logits, void *stream);
 
@@ -242,10 +247,17 @@ int ling_moe_lmhead_forward_ex(ling_moe_lmhead_t *h, const void *x, int T, float
 int ling_moe_lmhead_forward_host(ling_moe_lmhead_t *h, const void *x_host, int T, float *logits_host,
                                  void *stream);
 
-/* The handle's quantised head: *codes = e4m3 [vocab, hidden], *scales = fp32
- * [vocab], DEVICE pointers owned by the handle (read only; valid until
- * ling_moe_lmhead_destroy). */
-int ling_moe_lmhead_weights(const ling_moe_lmhead_t *h, const uint8_t **codes, const float **scales);
+/* The handle's quantised head in row-major order: writes codes [vocab,
+ * hidden] (e4m3 bytes, 16-byte aligned) and scales [vocab] (fp32) to the
+ * caller's DEVICE buffers on `stream` (asynchronous; one kernel launch,
+ * which ling_moe_lmhead_launch_count does not count).  The handle keeps
+ * the codes in its own tiled layout; this call is for inspection and tests. */
+int ling_moe_lmhead_weights(const ling_moe_lmhead_t *h, uint8_t *codes, float *scales, void *stream);
+
+/* Synchronise `stream` and return the handle's sticky device error: OK, or
+ * DEVICE_TIMEOUT if a bounded wait inside the kernel (2 s) gave up (the word
+ * is cleared), or CUDA if the synchronisation itself failed. */
+int ling_moe_lmhead_status(ling_moe_lmhead_t *h, void *stream);
 
 /* Number of kernel launches the handle's forward calls have enqueued. */
 int64_t ling_moe_lmhead_launch_count(const ling_moe_lmhead_t *h);

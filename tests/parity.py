@@ -8,6 +8,18 @@ The bar, per token:
   * routing weights: within 1e-5 of the oracle's, matched by expert index;
   * output: |gpu - oracle| <= 2e-2 * max(1, |oracle|) elementwise, the oracle
     taken in fp64 before any rounding.
+
+The online-FP8 LM head (compare_lmhead): codes and scales bit-exact; logits
+within the rounding bound of the GPU's arithmetic.  Every product of two
+e4m3 values is exact.  A tensor-core MMA adds 16 of them to its accumulator;
+the bound allows that step an error of 2^-21 times (|accumulator| + the sum
+of the 16 magnitudes) -- a model, not a documented guarantee: it grants the
+tensor core's internal alignment a few guard bits' worth of truncation.  16
+MMAs are chained per 256 codes, so each such chunk may be off by
+16 * 2^-21 = 2^-17 times its sum of magnitudes; the hidden / 256 chunk sums
+of a logit are added in fp32 (at most hidden / 256 roundings) and the total
+is multiplied by the two scales (two more).  So
+|gpu - exact| <= (2^-17 + (hidden / 256 + 2) * 2^-24) * sum_k |x_k w_k| * s_x * s_w.
 """
 from __future__ import annotations
 
@@ -58,3 +70,21 @@ def compare(ref: dict, out: torch.Tensor, idx: torch.Tensor | None, w: torch.Ten
     rel = err / np.maximum(1.0, np.abs(o))
     return {"near_ties": int(near.sum()), "exempt": int(exempt.sum()),
             "max_scaled_err": float(rel[~exempt].max()) if (~exempt).any() else 0.0}
+
+
+def lmhead_bound_ratio(got: np.ndarray, xq, xs, wq, ws, hidden: int, label: str = "") -> float:
+    """Check LM-head logits got [T, R] against the oracle's exact logits of the
+    same codes (x codes/scales [T], head rows' codes/scales [R]); return the
+    largest error as a fraction of the bound."""
+    import oracle.lmhead_ref as L
+    xd, wd = L.e4m3_decode(xq), L.e4m3_decode(wq)
+    scale = xs.astype(np.float64)[:, None] * ws.astype(np.float64)[None, :]
+    exact = (xd @ wd.T) * scale
+    mag = (np.abs(xd) @ np.abs(wd).T) * scale
+    u = 2.0 ** -24
+    tol = (128 * u + (hidden // 256 + 2) * u) * mag + 1e-37
+    err = np.abs(np.asarray(got, dtype=np.float64) - exact)
+    ratio = float((err / tol).max())
+    bad = int((err > tol).sum())
+    assert bad == 0, f"{label}: {bad} logits outside the bound; worst {ratio:.2f} x bound"
+    return ratio

@@ -2,12 +2,9 @@
 
 Codes and scales (of the head and of the tokens) must be bit-exact: both
 sides take every quantisation decision in the same fp32 steps.  Logits must
-lie within the rounding bound of the GPU's fp32 accumulation: every product
-of two e4m3 values is exact, a logit passes through at most
-d = 8 * (hidden / 512) + 6 fp32 additions (a lane's running sums, the sum of
-its two accumulators, five shuffle levels) and two fp32 products with the
-scales, so |gpu - exact| <= (d + 2) * 2^-24 * (sum_k |x_k w_k|) * s_x * s_w
-(first order; the test allows (d + 3)).
+lie within the rounding bound of the GPU's arithmetic derived in
+tests/parity.py; the largest measured error, as a fraction of that bound,
+is printed.
 """
 import numpy as np
 import pytest
@@ -16,11 +13,11 @@ import torch
 import oracle.lmhead_ref as L
 import workloads
 import weight_only_int4_fp32_b200 as lm
+from tests.parity import lmhead_bound_ratio
 
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
-U = 2.0 ** -24
 
 
 def _bits(t: torch.Tensor) -> np.ndarray:
@@ -32,26 +29,20 @@ def _f32(bits: np.ndarray) -> np.ndarray:
 
 
 def _check_logits(got, xq, xs, wq, ws, hidden, what):
-    """got [T, R] (GPU) against the oracle's exact logits of the same codes."""
-    xd, wd = L.e4m3_decode(xq), L.e4m3_decode(wq)
-    exact = (xd @ wd.T) * xs.astype(np.float64)[:, None] * ws.astype(np.float64)[None, :]
-    mag = (np.abs(xd) @ np.abs(wd).T) * xs.astype(np.float64)[:, None] * ws.astype(np.float64)[None, :]
-    d = 8 * (hidden // 512) + 6
-    tol = (d + 3) * U * mag + 1e-37
-    err = np.abs(got.astype(np.float64) - exact)
-    bad = err > tol
-    assert not bad.any(), (f"{what}: {int(bad.sum())} logits outside the fp32 bound; worst "
-                           f"{float((err / tol).max()):.2f} x bound")
-    return exact
+    ratio = lmhead_bound_ratio(got, xq, xs, wq, ws, hidden, what)
+    print(f"{what}: largest error {ratio:.3f} of the bound")
 
 
 def _run(head, x):
     logits, xq, xs = head.forward(x, return_codes=True)
-    torch.cuda.synchronize()
+    assert head.status() == lm.LING_MOE_OK
     return logits.cpu().numpy(), xq.cpu().numpy(), xs.cpu().numpy()
 
 
-@pytest.mark.parametrize("vocab,hidden", [(3001, 2560), (777, 512), (777, 4096), (1, 2560), (2369, 1024)])
+# vocabularies from one tile per CTA (pieces of a tile on several warps) to
+# several (tiles cut between two warps); hidden from 2 to 16 chunks per row
+@pytest.mark.parametrize("vocab,hidden", [(3001, 2560), (777, 512), (777, 4096), (1, 2560), (2369, 1024),
+                                          (20011, 2560), (9473, 1536)])
 def test_lmhead_matches_the_oracle(vocab, hidden):
     w = workloads.lm_head_weights(vocab, hidden, seed=11, device=DEV)
     head = lm.LMHeadFP8(w)

@@ -36,8 +36,8 @@ EXPORTED = (
     "ling_moe_destroy", "ling_moe_test_set_wait", "ling_moe_route_noalloc",
     "ling_moe_set_kernel_timing", "ling_moe_kernel_times", "ling_moe_kernel_name",
     "ling_moe_lmhead_create", "ling_moe_lmhead_forward", "ling_moe_lmhead_forward_ex",
-    "ling_moe_lmhead_forward_host", "ling_moe_lmhead_weights", "ling_moe_lmhead_launch_count",
-    "ling_moe_lmhead_destroy",
+    "ling_moe_lmhead_forward_host", "ling_moe_lmhead_weights", "ling_moe_lmhead_status",
+    "ling_moe_lmhead_launch_count", "ling_moe_lmhead_destroy",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -103,7 +103,8 @@ def _load():
         "ling_moe_lmhead_forward": (ci, [vp, vp, ci, vp, vp]),
         "ling_moe_lmhead_forward_ex": (ci, [vp, vp, ci, vp, vp, vp, vp]),
         "ling_moe_lmhead_forward_host": (ci, [vp, vp, ci, vp, vp]),
-        "ling_moe_lmhead_weights": (ci, [vp, ctypes.POINTER(vp), ctypes.POINTER(vp)]),
+        "ling_moe_lmhead_weights": (ci, [vp, vp, vp, vp]),
+        "ling_moe_lmhead_status": (ci, [vp, vp]),
         "ling_moe_lmhead_launch_count": (i64, [vp]),
         "ling_moe_lmhead_destroy": (None, [vp]),
     }
@@ -278,15 +279,6 @@ class MoELayer:
             pass
 
 
-class _DeviceArray:
-    """A view of library-owned device memory for torch.as_tensor (torch
-    accepts only writable views; the callers only clone it)."""
-
-    def __init__(self, ptr: int, shape: tuple, typestr: str):
-        self.__cuda_array_interface__ = {"shape": shape, "typestr": typestr, "data": (ptr, False),
-                                         "version": 3, "strides": None}
-
-
 class LMHeadFP8:
     """The online-FP8 LM head on the current CUDA device.
 
@@ -341,14 +333,17 @@ class LMHeadFP8:
                                                 self._stream(stream)))
         return logits_host
 
-    def weights(self):
-        """(codes uint8 [vocab, hidden], scales fp32 [vocab]) copied from the handle's device memory."""
+    def weights(self, stream=None):
+        """(codes uint8 [vocab, hidden], scales fp32 [vocab]): the handle's quantised head, row-major."""
         torch = self._torch
-        c, s = ctypes.c_void_p(), ctypes.c_void_p()
-        _check(lib.ling_moe_lmhead_weights(self.handle, ctypes.byref(c), ctypes.byref(s)))
-        codes = torch.as_tensor(_DeviceArray(c.value, (self.vocab, self.hidden), "|u1"), device="cuda").clone()
-        scales = torch.as_tensor(_DeviceArray(s.value, (self.vocab,), "<f4"), device="cuda").clone()
+        codes = torch.empty((self.vocab, self.hidden), dtype=torch.uint8, device="cuda")
+        scales = torch.empty((self.vocab,), dtype=torch.float32, device="cuda")
+        _check(lib.ling_moe_lmhead_weights(self.handle, codes.data_ptr(), scales.data_ptr(), self._stream(stream)))
         return codes, scales
+
+    def status(self, stream=None) -> int:
+        """Status code of the handle's device work (does not raise on DEVICE_TIMEOUT)."""
+        return lib.ling_moe_lmhead_status(self.handle, self._stream(stream))
 
     def launch_count(self) -> int:
         return lib.ling_moe_lmhead_launch_count(self.handle)

@@ -486,14 +486,16 @@ struct ling_moe_lmhead {
   int vocab = 0;
   int hidden = 0;
   int nctas = 0;
-  uint8_t* codes = nullptr;      // e4m3 [vocab, hidden]
+  uint8_t* codes = nullptr;      // e4m3, tiled (lmh_codes_bytes)
   float* scales = nullptr;       // fp32 [vocab]
   __nv_bfloat16* x_stage = nullptr;
   float* logits_stage = nullptr;
+  unsigned int* err = nullptr;   // sticky device error word
   std::atomic<int64_t> launches{0};
   void release() {
-    for (void* p : {(void*)codes, (void*)scales, (void*)x_stage, (void*)logits_stage})
+    for (void* p : {(void*)codes, (void*)scales, (void*)x_stage, (void*)logits_stage, (void*)err})
       if (p) cudaFree(p);
+    err = nullptr;
     codes = nullptr;
     scales = nullptr;
     x_stage = nullptr;
@@ -529,10 +531,11 @@ int ling_moe_lmhead_create(const void* w, int vocab, int hidden, ling_moe_lmhead
   h->hidden = hidden;
   h->nctas = prop.multiProcessorCount;
   struct A { void** p; size_t n; } plan[] = {
-      {(void**)&h->codes, (size_t)vocab * hidden},
+      {(void**)&h->codes, lmh_codes_bytes(vocab, hidden)},
       {(void**)&h->scales, (size_t)vocab * sizeof(float)},
       {(void**)&h->x_stage, (size_t)kLmhMaxT * hidden * sizeof(__nv_bfloat16)},
       {(void**)&h->logits_stage, (size_t)kLmhMaxT * vocab * sizeof(float)},
+      {(void**)&h->err, sizeof(unsigned int)},
   };
   for (auto& a : plan) {
     e = cudaMalloc(a.p, a.n);
@@ -544,7 +547,9 @@ int ling_moe_lmhead_create(const void* w, int vocab, int hidden, ling_moe_lmhead
       return rc;
     }
   }
-  e = launch_lmh_quantize(static_cast<const __nv_bfloat16*>(w), vocab, hidden, h->codes, h->scales, nullptr);
+  e = cudaMemset(h->err, 0, sizeof(unsigned int));
+  if (e == cudaSuccess)
+    e = launch_lmh_quantize(static_cast<const __nv_bfloat16*>(w), vocab, hidden, h->codes, h->scales, nullptr);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     const int rc = cuda_fail(e, "LM-head quantisation");
@@ -573,8 +578,9 @@ static int lmhead_forward_impl(ling_moe_lmhead_t* h, const void* x, int T, float
     return fail(LING_MOE_ERR_INVALID_ARG, "x_codes overlaps x or logits");
   if (x_scales && (overlaps(x_scales, (size_t)T * 4, logits, lb) || overlaps(x_scales, (size_t)T * 4, x, xb)))
     return fail(LING_MOE_ERR_INVALID_ARG, "x_scales overlaps x or logits");
-  cudaError_t e = launch_lmh_forward(h->codes, h->scales, h->vocab, h->hidden, static_cast<const __nv_bfloat16*>(x), T,
-                                     logits, x_codes, x_scales, h->nctas, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_lmh_forward(h->codes, h->scales, h->vocab, h->hidden, static_cast<const __nv_bfloat16*>(x),
+                                     T, logits, x_codes, x_scales, h->err, kDefaultWaitNs, h->nctas,
+                                     static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "LM-head launch");
   h->launches.fetch_add(1);
   return LING_MOE_OK;
@@ -609,10 +615,30 @@ int ling_moe_lmhead_forward_host(ling_moe_lmhead_t* h, const void* x_host, int T
   return LING_MOE_OK;
 }
 
-int ling_moe_lmhead_weights(const ling_moe_lmhead_t* h, const uint8_t** codes, const float** scales) {
+int ling_moe_lmhead_weights(const ling_moe_lmhead_t* h, uint8_t* codes, float* scales, void* stream_v) {
   if (!h || !codes || !scales) return fail(LING_MOE_ERR_INVALID_ARG, "handle, codes or scales is NULL");
-  *codes = h->codes;
-  *scales = h->scales;
+  if (!aligned16(codes)) return fail(LING_MOE_ERR_INVALID_ARG, "codes must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(scales) & 3u) return fail(LING_MOE_ERR_INVALID_ARG, "scales must be 4-byte aligned");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  cudaError_t e = launch_lmh_untile(h->codes, h->vocab, h->hidden, codes, stream);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(scales, h->scales, (size_t)h->vocab * sizeof(float), cudaMemcpyDeviceToDevice, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "LM-head weights copy");
+  return LING_MOE_OK;
+}
+
+int ling_moe_lmhead_status(ling_moe_lmhead_t* h, void* stream_v) {
+  if (!h) return fail(LING_MOE_ERR_INVALID_ARG, "handle is NULL");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream_v));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  unsigned int err = 0;
+  e = cudaMemcpy(&err, h->err, sizeof(err), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  if (err) {
+    cudaMemset(h->err, 0, sizeof(unsigned int));
+    cudaDeviceSynchronize();
+    return fail(LING_MOE_ERR_DEVICE_TIMEOUT, "a bounded device-side wait of the LM head gave up (error word %u)", err);
+  }
   return LING_MOE_OK;
 }
 
