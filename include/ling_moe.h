@@ -266,6 +266,13 @@ int64_t ling_moe_lmhead_launch_count(const ling_moe_lmhead_t *h);
  * sure no enqueued work still uses the handle. */
 void ling_moe_lmhead_destroy(ling_moe_lmhead_t *h);
 
+/* Test hook: skip_cta >= 0 makes that CTA of the next forward calls issue
+ * none of its weight copies, so that its waits for them run out and the
+ * launch ends with an error status (reported by ling_moe_lmhead_status)
+ * instead of hanging; -1 turns it off.  wait_limit_ns bounds every
+ * device-side wait (0 keeps the default, 2 s). */
+int ling_moe_lmhead_test_set_wait(ling_moe_lmhead_t *h, int skip_cta, uint64_t wait_limit_ns);
+
 #ifdef __cplusplus
 }
 #endif

@@ -141,5 +141,6 @@ def test_lmhead_null_handle_is_rejected_everywhere():
     assert lm.lib.ling_moe_lmhead_forward_host(None, 16, 1, 32, None) == lm.LING_MOE_ERR_INVALID_ARG
     assert lm.lib.ling_moe_lmhead_weights(None, 16, 32, None) == lm.LING_MOE_ERR_INVALID_ARG
     assert lm.lib.ling_moe_lmhead_status(None, None) == lm.LING_MOE_ERR_INVALID_ARG
+    assert lm.lib.ling_moe_lmhead_test_set_wait(None, 0, 0) == lm.LING_MOE_ERR_INVALID_ARG
     assert lm.lib.ling_moe_lmhead_launch_count(None) == 0
     lm.lib.ling_moe_lmhead_destroy(None)  # no-op

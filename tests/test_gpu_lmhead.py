@@ -139,3 +139,53 @@ def test_lmhead_one_launch_per_call_deterministic_and_host_path():
             head.forward(workloads.tokens(9, H, seed=1, device=DEV))
     finally:
         head.close()
+
+
+def test_lmhead_wait_that_runs_out_reports_an_error_and_the_next_call_is_clean():
+    """One CTA withholds its copies: its consumers' bounded waits run out
+    (50 ms), the launch ends with DEVICE_TIMEOUT instead of hanging, and the
+    next call, with the hook off, is exact again."""
+    V, H = 20011, 2560
+    w = workloads.lm_head_weights(V, H, seed=17, device=DEV)
+    head = lm.LMHeadFP8(w)
+    try:
+        x = workloads.tokens(2, H, seed=18, device=DEV)
+        good = head.forward(x)
+        assert head.status() == lm.LING_MOE_OK
+        head.test_set_wait(5, 50_000_000)
+        head.forward(x)
+        assert head.status() == lm.LING_MOE_ERR_DEVICE_TIMEOUT
+        head.test_set_wait(-1, 0)
+        again = head.forward(x)
+        assert head.status() == lm.LING_MOE_OK
+        assert torch.equal(again, good)
+    finally:
+        head.close()
+
+
+def test_lmhead_graph_capture_replays_the_call():
+    V, H = 5000, 2560
+    w = workloads.lm_head_weights(V, H, seed=19, device=DEV)
+    head = lm.LMHeadFP8(w)
+    try:
+        x = workloads.tokens(4, H, seed=20, device=DEV)
+        logits = torch.empty((4, V), dtype=torch.float32, device=DEV)
+        ref = head.forward(x).clone()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            head.forward(x, logits)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            head.forward(x, logits)
+        for _ in range(2):
+            logits.zero_()
+            g.replay()
+            torch.cuda.synchronize()
+            assert torch.equal(logits, ref)
+        assert head.status() == lm.LING_MOE_OK
+        del g
+    finally:
+        head.close()

@@ -37,7 +37,7 @@ EXPORTED = (
     "ling_moe_set_kernel_timing", "ling_moe_kernel_times", "ling_moe_kernel_name",
     "ling_moe_lmhead_create", "ling_moe_lmhead_forward", "ling_moe_lmhead_forward_ex",
     "ling_moe_lmhead_forward_host", "ling_moe_lmhead_weights", "ling_moe_lmhead_status",
-    "ling_moe_lmhead_launch_count", "ling_moe_lmhead_destroy",
+    "ling_moe_lmhead_launch_count", "ling_moe_lmhead_destroy", "ling_moe_lmhead_test_set_wait",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -107,6 +107,7 @@ def _load():
         "ling_moe_lmhead_status": (ci, [vp, vp]),
         "ling_moe_lmhead_launch_count": (i64, [vp]),
         "ling_moe_lmhead_destroy": (None, [vp]),
+        "ling_moe_lmhead_test_set_wait": (ci, [vp, ci, ctypes.c_uint64]),
     }
     for name, (res, args) in sig.items():
         try:
@@ -347,6 +348,10 @@ class LMHeadFP8:
 
     def launch_count(self) -> int:
         return lib.ling_moe_lmhead_launch_count(self.handle)
+
+    def test_set_wait(self, skip_cta: int, wait_limit_ns: int = 0):
+        """Test hook (see ling_moe_lmhead_test_set_wait)."""
+        _check(lib.ling_moe_lmhead_test_set_wait(self.handle, skip_cta, wait_limit_ns))
 
     def close(self):
         if getattr(self, "handle", None):

@@ -492,6 +492,8 @@ struct ling_moe_lmhead {
   float* logits_stage = nullptr;
   unsigned int* err = nullptr;   // sticky device error word
   std::atomic<int64_t> launches{0};
+  int skip_cta = -1;             // test hook
+  unsigned long long wait_limit_ns = kDefaultWaitNs;
   void release() {
     for (void* p : {(void*)codes, (void*)scales, (void*)x_stage, (void*)logits_stage, (void*)err})
       if (p) cudaFree(p);
@@ -579,7 +581,7 @@ static int lmhead_forward_impl(ling_moe_lmhead_t* h, const void* x, int T, float
   if (x_scales && (overlaps(x_scales, (size_t)T * 4, logits, lb) || overlaps(x_scales, (size_t)T * 4, x, xb)))
     return fail(LING_MOE_ERR_INVALID_ARG, "x_scales overlaps x or logits");
   cudaError_t e = launch_lmh_forward(h->codes, h->scales, h->vocab, h->hidden, static_cast<const __nv_bfloat16*>(x),
-                                     T, logits, x_codes, x_scales, h->err, kDefaultWaitNs, h->nctas,
+                                     T, logits, x_codes, x_scales, h->err, h->wait_limit_ns, h->skip_cta, h->nctas,
                                      static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "LM-head launch");
   h->launches.fetch_add(1);
@@ -643,6 +645,14 @@ int ling_moe_lmhead_status(ling_moe_lmhead_t* h, void* stream_v) {
 }
 
 int64_t ling_moe_lmhead_launch_count(const ling_moe_lmhead_t* h) { return h ? h->launches.load() : 0; }
+
+int ling_moe_lmhead_test_set_wait(ling_moe_lmhead_t* h, int skip_cta, uint64_t wait_limit_ns) {
+  if (!h) return fail(LING_MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (skip_cta >= h->nctas) return fail(LING_MOE_ERR_INVALID_ARG, "skip_cta out of range");
+  h->skip_cta = skip_cta < 0 ? -1 : skip_cta;
+  h->wait_limit_ns = wait_limit_ns ? wait_limit_ns : kDefaultWaitNs;
+  return LING_MOE_OK;
+}
 
 void ling_moe_lmhead_destroy(ling_moe_lmhead_t* h) {
   if (!h) return;

@@ -142,6 +142,7 @@ struct LmhParams {
   unsigned int* err;
   unsigned long long wait_limit_ns;
   int vocab, hidden, T;
+  int skip_cta;  // test hook: this CTA's producer issues no copies (-1: none)
 };
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
@@ -231,6 +232,7 @@ __global__ void __launch_bounds__(kLmhMmaThreads, 1) lmh_mma_kernel(const LmhPar
 #pragma unroll
       for (int w = 0; w < kLmhConsumers; ++w) next[w] = 0;
       unsigned long long t0 = globaltimer_ns();
+      const bool withhold = (int)blockIdx.x == p.skip_cta;
       while (left > 0 && !*stop) {
         bool moved = false;
 #pragma unroll
@@ -239,7 +241,7 @@ __global__ void __launch_bounds__(kLmhMmaThreads, 1) lmh_mma_kernel(const LmhPar
           const int r = next[w];
           if (r >= n_w) continue;
           const int s = kLmhDepth * w + r % kLmhDepth;
-          if (r >= kLmhDepth && !mbar_test(&empty[s], (r / kLmhDepth - 1) & 1)) continue;
+          if (withhold || (r >= kLmhDepth && !mbar_test(&empty[s], (r / kLmhDepth - 1) & 1))) continue;
           mbar_arrive_expect_tx(&full[s], kLmhChunkBytes);
           bulk_g2s(ring + (size_t)s * kLmhChunkBytes, base + (size_t)(cb + r) * kLmhChunkBytes, kLmhChunkBytes,
                    &full[s]);
@@ -392,9 +394,10 @@ cudaError_t launch_lmh_untile(const uint8_t* codes, int vocab, int hidden, uint8
 
 cudaError_t launch_lmh_forward(const uint8_t* codes, const float* scales, int vocab, int hidden,
                                const __nv_bfloat16* x, int T, float* logits, uint8_t* x_codes, float* x_scales,
-                               unsigned int* err, unsigned long long wait_limit_ns, int nctas, cudaStream_t s) {
+                               unsigned int* err, unsigned long long wait_limit_ns, int skip_cta, int nctas,
+                               cudaStream_t s) {
   if (hidden % 512 || hidden > kLmhMaxHidden || T < 1 || T > kLmhMaxT) return cudaErrorInvalidValue;
-  LmhParams p{codes, scales, x, logits, x_codes, x_scales, err, wait_limit_ns, vocab, hidden, T};
+  LmhParams p{codes, scales, x, logits, x_codes, x_scales, err, wait_limit_ns, vocab, hidden, T, skip_cta};
   lmh_mma_kernel<<<nctas, kLmhMmaThreads, lmh_mma_smem(hidden), s>>>(p);
   return cudaGetLastError();
 }

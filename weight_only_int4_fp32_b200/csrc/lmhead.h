@@ -24,10 +24,11 @@ cudaError_t launch_lmh_quantize(const __nv_bfloat16* w, int vocab, int hidden, u
 cudaError_t launch_lmh_untile(const uint8_t* codes, int vocab, int hidden, uint8_t* out, cudaStream_t s);
 // logits [T, vocab] fp32; x_codes / x_scales: optional copies of the tokens'
 // codes [T, hidden] and scales [T].  Bounded waits: one that runs out sets
-// bit 2 of *err.
+// bit 2 of *err.  skip_cta >= 0 (a test hook) makes that CTA issue no copies.
 cudaError_t launch_lmh_forward(const uint8_t* codes, const float* scales, int vocab, int hidden,
                                const __nv_bfloat16* x, int T, float* logits, uint8_t* x_codes, float* x_scales,
-                               unsigned int* err, unsigned long long wait_limit_ns, int nctas, cudaStream_t s);
+                               unsigned int* err, unsigned long long wait_limit_ns, int skip_cta, int nctas,
+                               cudaStream_t s);
 cudaError_t setup_lmhead();
 
 }  // namespace lingmoe
