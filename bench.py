@@ -119,7 +119,7 @@ class L2Flush:
     def __call__(self, i):
         import torch
         self.w.fill_(float(i))
-        torch.sum(self.r, out=self.s)
+        torch.sum(self.r, dim=0, out=self.s)
 
 
 GEMV_MAX_TOKENS = 8  # experts with at most this many tokens take the GEMV kernels, not the tensor-core tiles
