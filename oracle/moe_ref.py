@@ -190,13 +190,15 @@ def expert_ffn(xs, w_gate, w_up, w_down) -> np.ndarray:
 
 # ---------------------------------------------------------------- the layer
 
-def moe_layer(x_bits, weights: dict, top_k: int) -> dict:
+def moe_layer(x_bits, weights: dict, top_k: int, dequant=None) -> dict:
     """The routed-expert MoE layer for T tokens, in float64.
 
     x_bits: bf16 bit patterns [T, H].  weights: the canonical boundary layout
     (bf16 tensors as uint16 bit patterns, packed int4 as uint8, the optional
     router bias as float32) with keys router_w, router_bias, gate_q, gate_s,
-    up_q, up_s, down_q, down_s, sh_gate, sh_up, sh_down.
+    up_q, up_s, down_q, down_s, sh_gate, sh_up, sh_down.  dequant(codes,
+    scales) turns one expert matrix's packed codes and scales into float64
+    weights (default: the W4 g32 `dequantize`; the MXFP4 oracle passes its own).
 
     Returns out [T, H] (float64, before the final bf16 rounding), idx [T, k],
     w [T, k] and logits [T, E].
@@ -209,12 +211,13 @@ def moe_layer(x_bits, weights: dict, top_k: int) -> dict:
     idx, w = route(logits, top_k)
 
     out = np.zeros((T, H), dtype=np.float64)
+    deq = dequantize if dequant is None else dequant
     # routed experts: each selected expert applied to the tokens that chose it
     for e in np.unique(idx):
         toks, slots = np.nonzero(idx == e)
-        wg = dequantize(weights["gate_q"][e], weights["gate_s"][e])
-        wu = dequantize(weights["up_q"][e], weights["up_s"][e])
-        wd = dequantize(weights["down_q"][e], weights["down_s"][e])
+        wg = deq(weights["gate_q"][e], weights["gate_s"][e])
+        wu = deq(weights["up_q"][e], weights["up_s"][e])
+        wd = deq(weights["down_q"][e], weights["down_s"][e])
         y = expert_ffn(x[toks], wg, wu, wd)
         out[toks] += w[toks, slots][:, None] * y
     # the shared expert, bf16 weights, weight 1
