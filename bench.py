@@ -31,8 +31,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer decode tokens/s and achieved HBM GB/s (W4 g32, 512e top-8, T=1)"
+METRIC_MXFP4 = "MoE-layer decode tokens/s and achieved HBM GB/s (MXFP4 e2m1/e8m0, 512e top-8, T=1)"
 H, I = 2560, 768
 ROUTED_BYTES = 3_317_760        # per expert: int4 codes + bf16 scales
+ROUTED_BYTES_MXFP4 = 3_133_440  # per expert: E2M1 codes + E8M0 scale bytes
 SHARED_BYTES = 11_796_480       # bf16 shared expert
 L2_FLUSH_BYTES = 256 << 20
 
@@ -78,9 +80,19 @@ def router_bytes(E):
     return E * H * 2
 
 
-def decode_bytes(E, union):
+def decode_bytes(E, union, fmt="int4"):
     """Algorithmic bytes of one call: distinct routed experts + shared + router."""
-    return union * ROUTED_BYTES + SHARED_BYTES + router_bytes(E)
+    return union * (ROUTED_BYTES_MXFP4 if fmt == "mxfp4" else ROUTED_BYTES) + SHARED_BYTES + router_bytes(E)
+
+
+def _layer_gen(wl):
+    """The workload's weight generator and its oracle."""
+    import oracle
+    import workloads
+    if wl.get("fmt") == "mxfp4":
+        import oracle.mxfp4_ref as MX
+        return workloads.layer_weights_mxfp4, MX.moe_layer_mxfp4
+    return workloads.layer_weights, oracle.moe_layer
 
 
 def peaks():
@@ -199,8 +211,9 @@ def cpu_oracle_rate(workload: str, seconds: float = 15.0, max_tokens: int = 64):
     import workloads
     wl = workloads.WORKLOADS[workload]
     E = wl["num_experts"]
-    lw = workloads.layer_weights(E, seed=wl.get("weight_seed", 100), device="cpu" if E <= 32 else
-                                 ("cuda" if torch.cuda.is_available() else "cpu"))
+    gen, layer_fn = _layer_gen(wl)
+    lw = gen(E, seed=wl.get("weight_seed", 100), device="cpu" if E <= 32 else
+             ("cuda" if torch.cuda.is_available() else "cpu"))
     host = lw.host_arrays()
     if workload.startswith("prefill"):
         host["router_bias"] = workloads.zipf_router_bias(E, wl["zipf_s"]).numpy()
@@ -212,7 +225,7 @@ def cpu_oracle_rate(workload: str, seconds: float = 15.0, max_tokens: int = 64):
         while calls < max_tokens and (time.perf_counter() - t0) < budget:
             x = workloads.tokens(T, seed=seeds[calls % len(seeds)], device="cpu")
             xb = x.view(torch.int16).numpy().view(np.uint16)
-            oracle.moe_layer(xb, host, 8)
+            layer_fn(xb, host, 8)
             n += T
             calls += 1
         return n, calls, time.perf_counter() - t0
@@ -242,15 +255,15 @@ def run_reference(args):
     import workloads
     wl = workloads.WORKLOADS[args.workload]
     E = wl["num_experts"]
-    lw = workloads.layer_weights(E, seed=wl.get("weight_seed", 100),
-                                 device="cuda" if torch.cuda.is_available() else "cpu")
+    gen, layer_fn = _layer_gen(wl)
+    lw = gen(E, seed=wl.get("weight_seed", 100), device="cuda" if torch.cuda.is_available() else "cpu")
     host = lw.host_arrays()
     del lw
     T = wl["T"] if wl["T"] <= 4 else 4
     seeds = wl.get("token_seeds") or wl.get("call_seeds") or [1 + t for t in range(1000)]
     def step(i):
         x = workloads.tokens(T, seed=seeds[i % len(seeds)], device="cpu")
-        oracle.moe_layer(x.view(torch.int16).numpy().view(np.uint16), host, 8)
+        layer_fn(x.view(torch.int16).numpy().view(np.uint16), host, 8)
     for i in range(warm):
         step(i)
     t0 = time.perf_counter()
@@ -258,7 +271,8 @@ def run_reference(args):
         step(warm + i)
     dt = time.perf_counter() - t0
     v = steps * T / dt
-    line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": ws, "steps": steps,
+    line = {"metric": METRIC_MXFP4 if wl.get("fmt") == "mxfp4" else METRIC, "value": v, "unit": "tokens/s",
+            "n_gpus": ws, "steps": steps,
             "warmup": warm, "ms_per_step": dt * 1e3 / steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
@@ -284,16 +298,23 @@ def build_layers(workload, device):
     nlayers = wl.get("layers", 1)
     seeds = wl.get("layer_seeds") or [wl["weight_seed"]]
     layers = []
+    gen, _ = _layer_gen(wl)
+    fmt = wl.get("fmt", "int4")
     for l in range(nlayers):
-        lw = workloads.layer_weights(E, seed=seeds[l], device=device)
+        lw = gen(E, seed=seeds[l], device=device)
         w = lw.tensors()
         if workload.startswith("prefill"):
             w = dict(w)
             w["router_bias"] = workloads.zipf_router_bias(E, wl["zipf_s"]).to(device)
-        layers.append(lm.MoELayer(w, top_k=8, max_tokens=max(T, 1)))
+        layers.append(lm.MoELayer(w, top_k=8, max_tokens=max(T, 1), fmt=fmt))
         del lw, w
         torch.cuda.empty_cache()
     return layers, E, T
+
+
+def workloads_fmt(workload):
+    import workloads
+    return workloads.WORKLOADS[workload].get("fmt", "int4")
 
 
 REPLICA_SEED_STRIDE = 1_000_003  # rank r > 0 draws its token stream from seeds shifted by r times this
@@ -484,7 +505,8 @@ def run_ours(args):
                "note": "ling_moe_forward_host per step (pinned H2D copy + layer + D2H copy + stream sync), "
                        "host wall clock summed over the calls; L2 flushed before each call, outside its clock"}
 
-    per_call_bytes = [sum(decode_bytes(E, u) for u in us) for us in unions]
+    fmt = workloads_fmt(args.workload)
+    per_call_bytes = [sum(decode_bytes(E, u, fmt) for u in us) for us in unions]
     if args.workload.startswith("prefill"):
         per_call_bytes = [b + 2 * T * H * 2 for b in per_call_bytes]
     avg_bytes = sum(per_call_bytes) / len(per_call_bytes)
@@ -511,9 +533,11 @@ def run_ours(args):
         cpu = cpu_oracle_rate(args.workload if not stack else "decode_e512_t1",
                               seconds=args.cpu_seconds) if ws == 1 and args.cpu_seconds > 0 else None
         line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": nsteps,
+            "metric": METRIC_MXFP4 if fmt == "mxfp4" else METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": ws, "steps": nsteps,
             "warmup": nwarm, "ms_per_step": kern_ms / nsteps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "w4a16, fp32 accumulate",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": ("mxfp4 (e2m1, e8m0 per 32) x fp16" if fmt == "mxfp4" else "w4a16") + ", fp32 accumulate",
             "data": "synthetic (seeded weights and tokens, recipe in DESIGN.md)",
             "config": {"workload": args.workload, "T": T, "experts": E, "top_k": 8, "hidden": H,
                        "inter": I, "layers": len(layers),

@@ -93,6 +93,23 @@ typedef struct ling_moe ling_moe_t; /* opaque handle */
 int ling_moe_create(const ling_moe_config_t *cfg, const ling_moe_weights_t *w,
                     ling_moe_t **out);
 
+/* The same layer with MXFP4 routed experts (OCP Microscaling MXFP4: FP4
+ * E2M1 elements -- bit 3 sign, bits 2..1 exponent with bias 1, bit 0
+ * mantissa, values +-{0, 0.5, 1, 1.5, 2, 3, 4, 6} -- and one E8M0 scale
+ * 2^(e - 127) per 32 consecutive K elements).  The pages profile an MXFP4
+ * checkpoint of the model (bpdata article, sections "Modell es kiindulo
+ * konfiguracio" and "Optimalizacio 1: Humming MXFP4 MoE backend") without
+ * defining the format; this is the OCP definition.
+ * Weights: as ling_moe_create, except that gate_q / up_q / down_q hold E2M1
+ * codes (two per byte, low nibble = even K index) and gate_s / up_s / down_s
+ * hold E8M0 scale bytes, uint8 [E, rows, K/32].  Scale exponents above 240
+ * (scales of 2^114 and more) are not supported: they give NaN outputs.
+ * Limits: as ling_moe_create, plus max_tokens <= 8 (the decode path; the
+ * token-grouped path is not built for MXFP4): larger values return
+ * UNSUPPORTED.  Every other entry point works on the handle as documented. */
+int ling_moe_create_mxfp4(const ling_moe_config_t *cfg, const ling_moe_weights_t *w,
+                          ling_moe_t **out);
+
 /* out[T, H] (bf16) = layer(x[T, H] bf16) on `stream` (a cudaStream_t, NULL =
  * legacy default stream).  x and out are DEVICE pointers owned by the caller,
  * contiguous row-major, 16-byte aligned; out must not overlap x.

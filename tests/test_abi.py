@@ -15,7 +15,7 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "ling_moe.h")
 def declared_symbols():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(ling_moe_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(ling_moe_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_header_declares_the_binding_list():
@@ -144,3 +144,14 @@ def test_lmhead_null_handle_is_rejected_everywhere():
     assert lm.lib.ling_moe_lmhead_test_set_wait(None, 0, 0) == lm.LING_MOE_ERR_INVALID_ARG
     assert lm.lib.ling_moe_lmhead_launch_count(None) == 0
     lm.lib.ling_moe_lmhead_destroy(None)  # no-op
+
+
+def test_create_mxfp4_checks_arguments_and_its_token_limit():
+    h = ctypes.c_void_p()
+    assert lm.lib.ling_moe_create_mxfp4(None, ctypes.byref(_weights()), ctypes.byref(h)) == \
+        lm.LING_MOE_ERR_INVALID_ARG
+    rc = lm.lib.ling_moe_create_mxfp4(ctypes.byref(_cfg(max_tokens=9)), ctypes.byref(_weights()), ctypes.byref(h))
+    assert rc == lm.LING_MOE_ERR_UNSUPPORTED and h.value is None
+    assert "MXFP4" in lm.ling_moe_last_error()
+    rc = lm.lib.ling_moe_create_mxfp4(ctypes.byref(_cfg(group_size=64)), ctypes.byref(_weights()), ctypes.byref(h))
+    assert rc == lm.LING_MOE_ERR_UNSUPPORTED

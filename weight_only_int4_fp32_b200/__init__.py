@@ -16,7 +16,7 @@ __all__ = [
     "LING_MOE_OK", "LING_MOE_ERR_INVALID_ARG", "LING_MOE_ERR_CUDA", "LING_MOE_ERR_OOM",
     "LING_MOE_ERR_UNSUPPORTED", "LING_MOE_ERR_DEVICE_TIMEOUT", "LingMoEError",
     "ling_moe_config_t", "ling_moe_weights_t", "library_path", "load_library",
-    "ling_moe_create", "ling_moe_forward", "ling_moe_forward_ex", "ling_moe_forward_host",
+    "ling_moe_create", "ling_moe_create_mxfp4", "ling_moe_forward", "ling_moe_forward_ex", "ling_moe_forward_host",
     "ling_moe_status", "ling_moe_describe", "ling_moe_launch_count", "ling_moe_last_error",
     "ling_moe_destroy", "ling_moe_test_set_wait", "ling_moe_route_noalloc", "ling_moe_set_kernel_timing",
     "ling_moe_kernel_times", "MoELayer", "LMHeadFP8", "EXPORTED",
@@ -31,9 +31,9 @@ LING_MOE_ERR_DEVICE_TIMEOUT = -5
 
 # every symbol include/ling_moe.h declares
 EXPORTED = (
-    "ling_moe_create", "ling_moe_forward", "ling_moe_forward_ex", "ling_moe_forward_host",
-    "ling_moe_status", "ling_moe_describe", "ling_moe_launch_count", "ling_moe_last_error",
-    "ling_moe_destroy", "ling_moe_test_set_wait", "ling_moe_route_noalloc",
+    "ling_moe_create", "ling_moe_create_mxfp4", "ling_moe_forward", "ling_moe_forward_ex",
+    "ling_moe_forward_host", "ling_moe_status", "ling_moe_describe", "ling_moe_launch_count",
+    "ling_moe_last_error", "ling_moe_destroy", "ling_moe_test_set_wait", "ling_moe_route_noalloc",
     "ling_moe_set_kernel_timing", "ling_moe_kernel_times", "ling_moe_kernel_name",
     "ling_moe_lmhead_create", "ling_moe_lmhead_forward", "ling_moe_lmhead_forward_ex",
     "ling_moe_lmhead_forward_host", "ling_moe_lmhead_weights", "ling_moe_lmhead_status",
@@ -86,6 +86,8 @@ def _load():
     sig = {
         "ling_moe_create": (ci, [ctypes.POINTER(ling_moe_config_t), ctypes.POINTER(ling_moe_weights_t),
                                  ctypes.POINTER(vp)]),
+        "ling_moe_create_mxfp4": (ci, [ctypes.POINTER(ling_moe_config_t), ctypes.POINTER(ling_moe_weights_t),
+                                       ctypes.POINTER(vp)]),
         "ling_moe_forward": (ci, [vp, vp, ci, vp, vp]),
         "ling_moe_forward_ex": (ci, [vp, vp, ci, vp, vp, vp, vp]),
         "ling_moe_forward_host": (ci, [vp, vp, ci, vp, vp]),
@@ -141,6 +143,12 @@ def _check(rc: int) -> int:
 def ling_moe_create(cfg: ling_moe_config_t, weights: ling_moe_weights_t) -> int:
     h = ctypes.c_void_p()
     _check(lib.ling_moe_create(ctypes.byref(cfg), ctypes.byref(weights), ctypes.byref(h)))
+    return h.value
+
+
+def ling_moe_create_mxfp4(cfg: ling_moe_config_t, weights: ling_moe_weights_t) -> int:
+    h = ctypes.c_void_p()
+    _check(lib.ling_moe_create_mxfp4(ctypes.byref(cfg), ctypes.byref(weights), ctypes.byref(h)))
     return h.value
 
 
@@ -203,9 +211,11 @@ class MoELayer:
     `weights` maps the canonical names (router_w, router_bias, gate_q, gate_s,
     up_q, up_s, down_q, down_s, sh_gate, sh_up, sh_down) to contiguous CUDA
     tensors; they are copied, so they may be freed after construction.
+    fmt="int4" (W4 g32, bf16 scales) or "mxfp4" (E2M1 codes, E8M0 scale bytes).
     """
 
-    def __init__(self, weights: dict, top_k: int = 8, max_tokens: int = 1, group_size: int = 32):
+    def __init__(self, weights: dict, top_k: int = 8, max_tokens: int = 1, group_size: int = 32,
+                 fmt: str = "int4"):
         import torch  # device memory and streams only
         rw = weights["router_w"]
         E, H = rw.shape
@@ -217,7 +227,9 @@ class MoELayer:
         ptr = lambda n: (weights[n].data_ptr() if weights.get(n) is not None else None)
         w = ling_moe_weights_t(*(ptr(n) for n, _ in ling_moe_weights_t._fields_))
         self.E, self.H, self.I, self.k, self.max_tokens = E, H, I, top_k, max_tokens
-        self.handle = ling_moe_create(cfg, w)
+        if fmt not in ("int4", "mxfp4"):
+            raise ValueError("fmt must be 'int4' or 'mxfp4'")
+        self.handle = (ling_moe_create_mxfp4 if fmt == "mxfp4" else ling_moe_create)(cfg, w)
         self._torch = torch
 
     def _stream(self, stream):

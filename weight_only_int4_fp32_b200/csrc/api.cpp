@@ -55,6 +55,7 @@ void set_last_error(const char* msg) { g_last_error = msg; }
 
 struct ling_moe {
   ling_moe_config_t cfg{};
+  int codec = kCodecInt4;  // routed-weight format
   int device = 0;
   int num_sms = 0;
   int decode_ctas = 0;
@@ -142,7 +143,7 @@ extern "C" {
 
 const char* ling_moe_last_error(void) { return g_last_error.c_str(); }
 
-int ling_moe_create(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, ling_moe_t** out) {
+static int create_impl(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, int codec, ling_moe_t** out) {
   if (!out) return fail(LING_MOE_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
   if (!cfg || !w) return fail(LING_MOE_ERR_INVALID_ARG, "cfg or weights is NULL");
@@ -150,6 +151,9 @@ int ling_moe_create(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, l
   if (rc) return rc;
   rc = validate_weights(w);
   if (rc) return rc;
+  if (codec == kCodecMxfp4 && cfg->max_tokens > 2 * kMaxDecodeT)
+    return fail(LING_MOE_ERR_UNSUPPORTED, "MXFP4 weights: max_tokens must be <= %d (no token-grouped path)",
+                2 * kMaxDecodeT);
 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -172,6 +176,7 @@ int ling_moe_create(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, l
 
   ling_moe* h = new ling_moe();
   h->cfg = *cfg;
+  h->codec = codec;
   h->device = dev;
   h->num_sms = prop.multiProcessorCount;
   h->decode_ctas = prop.multiProcessorCount;
@@ -204,7 +209,8 @@ int ling_moe_create(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, l
       return rc;
     }
   }
-  if (cfg->max_tokens > kMaxDecodeT) {
+  const bool grouped = cfg->max_tokens > kMaxDecodeT && codec == kCodecInt4;
+  if (grouped) {
     h->gws.err = h->err;
     e = grouped_alloc(&h->gws, E, K, cfg->max_tokens,
                       [h](void** p, size_t n) { return h->alloc(p, n); });
@@ -227,8 +233,8 @@ int ling_moe_create(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, l
   if (e == cudaSuccess) e = cudaMemsetAsync(h->sync, 0, 4 * sizeof(unsigned long long), s);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->err, 0, 4 * sizeof(unsigned int), s);
   if (e == cudaSuccess)
-    e = launch_repack(w->gate_q, w->up_q, w->gate_s, w->up_s, w->down_q, w->down_s, h->gu, h->dn, E, s);
-  if (e == cudaSuccess && cfg->max_tokens > kMaxDecodeT)
+    e = launch_repack(w->gate_q, w->up_q, w->gate_s, w->up_s, w->down_q, w->down_s, h->gu, h->dn, E, codec, s);
+  if (e == cudaSuccess && grouped)
     e = grouped_prepare(&h->gws, E, h->sh_gate, h->sh_up, h->sh_down, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (s) cudaStreamDestroy(s);
@@ -242,14 +248,24 @@ int ling_moe_create(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, l
   char buf[1024];
   snprintf(buf, sizeof(buf),
            "ling_moe sm_%d%d %d SMs | H=%d I=%d E=%d k=%d g=%d max_tokens=%d bias=%s | "
-           "decode path (1<=T<=%d): 1 cooperative launch grid=%dx%d smem=%zuB, W4 g32 GEMV "
+           "decode path (1<=T<=%d): 1 cooperative launch grid=%dx%d smem=%zuB, %s GEMV "
            "dequant-in-register, fp32 accumulate (T<=%d: 2 such launches) | grouped path (T>%d): %s",
            prop.major, prop.minor, h->num_sms, kH, kI, E, K, kGroup, cfg->max_tokens,
            w->router_bias ? "yes" : "no", kMaxDecodeT, h->decode_ctas, kDecodeThreads,
-           decode_smem_bytes(1), 2 * kMaxDecodeT, 2 * kMaxDecodeT, grouped_describe());
+           decode_smem_bytes(1), codec == kCodecMxfp4 ? "MXFP4 (E2M1, E8M0 per 32)" : "W4 g32",
+           2 * kMaxDecodeT, 2 * kMaxDecodeT,
+           codec == kCodecMxfp4 ? "not built for MXFP4 weights" : grouped_describe());
   h->desc = buf;
   *out = h;
   return LING_MOE_OK;
+}
+
+int ling_moe_create(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, ling_moe_t** out) {
+  return create_impl(cfg, w, kCodecInt4, out);
+}
+
+int ling_moe_create_mxfp4(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, ling_moe_t** out) {
+  return create_impl(cfg, w, kCodecMxfp4, out);
 }
 
 static int forward_impl(ling_moe_t* h, const void* x, int T, void* out, int32_t* topk_idx,
@@ -300,6 +316,7 @@ static int forward_impl(ling_moe_t* h, const void* x, int T, void* out, int32_t*
       p.err = h->err;
       p.skip_arrive_cta = h->skip_arrive_cta;
       p.wait_limit_ns = h->wait_limit_ns;
+      p.codec = h->codec;
       h->skip_arrive_cta = -1;  // one launch only
       e = launch_decode(p, h->decode_ctas, stream);
       if (e != cudaSuccess) return cuda_fail(e, "decode launch");

@@ -182,6 +182,22 @@ __device__ __forceinline__ uint32_t deq_q_odd16(uint32_t w) {
   asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(0x64806480u));  // 1152
   return r;
 }
+// ---------------------------------------------------------------- routed-weight codecs (layout.h)
+// The E2M1 codes at bits P..P+3 and P+16..P+19 of a fragment word as the
+// fp16 pair (value * 2^-14, exactly): with its magnitude bits E1 E0 M at
+// fp16 bits 11..9 and its sign at bit 15, an fp16 is 2^(E - 15) (1 + M / 2)
+// for E > 0 and the subnormal M 2^-15 for E = 0, i.e. the E2M1 value times
+// 2^-14.  (The 2^14 is folded into the stored scale.)
+template <int P>
+__device__ __forceinline__ uint32_t deq_e2m1(uint32_t w) {
+  static_assert(P >= 0 && P <= 12, "nibble position");
+  uint32_t mag, sgn;
+  if constexpr (P <= 9) mag = (w << (9 - P)) & 0x0E000E00u;
+  else mag = (w >> (P - 9)) & 0x0E000E00u;
+  sgn = (w << (12 - P)) & 0x80008000u;
+  return mag | sgn;
+}
+
 // D = A B + C for one m16n8k16 tile: A 16x16 fp16 (row-major fragment),
 // B 16x8 fp16 (column-major fragment), C and D fp32.
 __device__ __forceinline__ void mma_16816(float& d0, float& d1, float& d2, float& d3, uint32_t a0, uint32_t a1,
@@ -235,6 +251,8 @@ __device__ __forceinline__ uint2 h_split2(float h0, float h1) {
 // A lane without a token of its own points at any valid token (its
 // accumulator row is discarded): the loads stay unconditional, so the MMAs
 // of different groups can overlap.  Every lane of the warp must call it.
+// C: the codec of the unit's codes (the scales already carry its factor).
+template <int C = kCodecInt4>
 __device__ __forceinline__ void dn_unit_mma(const unsigned char* unit, const unsigned char* hf, int lane, float& r0,
                                             float& r1, int j0 = 0, int j1 = kDnChunks) {
   const int c = lane & 3;
@@ -249,9 +267,16 @@ __device__ __forceinline__ void dn_unit_mma(const unsigned char* unit, const uns
       const uint4 a0 = lds128(hf + (8 * j + 2 * gg) * 64);
       const uint4 a1 = lds128(hf + (8 * j + 2 * gg + 1) * 64);
       float d0, d1, d2, d3;
-      mma_16816(d0, d1, d2, d3, a0.x, a0.y, a0.z, a0.w, deq_q_even(wv[gg]), deq_q_odd(wv[gg]), 0.f, 0.f, 0.f, 0.f);
-      mma_16816(d0, d1, d2, d3, a1.x, a1.y, a1.z, a1.w, deq_q_even(wv[gg] >> 8), deq_q_odd(wv[gg] >> 8), d0, d1,
-                d2, d3);
+      if constexpr (C == kCodecMxfp4) {
+        mma_16816(d0, d1, d2, d3, a0.x, a0.y, a0.z, a0.w, deq_e2m1<0>(wv[gg]), deq_e2m1<4>(wv[gg]), 0.f, 0.f, 0.f,
+                  0.f);
+        mma_16816(d0, d1, d2, d3, a1.x, a1.y, a1.z, a1.w, deq_e2m1<8>(wv[gg]), deq_e2m1<12>(wv[gg]), d0, d1, d2, d3);
+      } else {
+        mma_16816(d0, d1, d2, d3, a0.x, a0.y, a0.z, a0.w, deq_q_even(wv[gg]), deq_q_odd(wv[gg]), 0.f, 0.f, 0.f,
+                  0.f);
+        mma_16816(d0, d1, d2, d3, a1.x, a1.y, a1.z, a1.w, deq_q_even(wv[gg] >> 8), deq_q_odd(wv[gg] >> 8), d0, d1,
+                  d2, d3);
+      }
       acc0 = fmaf(bf16lo(sv[gg]), d0 + d2, acc0);
       acc1 = fmaf(bf16hi(sv[gg]), d1 + d3, acc1);
     }

@@ -164,7 +164,8 @@ __device__ __forceinline__ bool wait_count(const unsigned long long* ctr, unsign
   return true;
 }
 
-template <int T>
+// C: the codec of the routed weights (kCodecInt4 or kCodecMxfp4).
+template <int T, int C>
 __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const DecodeParams p) {
   using PL = Plan<T>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -252,7 +253,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       const uint32_t hi = *reinterpret_cast<const uint32_t*>(xb + t * kXbTok + 2 * (c + 8));
       const float inv = 1.0f / hd.xscale[t];
       const __half2 h0 = __floats2half2_rn(bf16lo(lo) * inv, bf16hi(lo) * inv);
-      const __half2 h1 = __floats2half2_rn(bf16lo(hi) * inv * 0.0625f, bf16hi(hi) * inv * 0.0625f);
+      // int4: the upper half meets codes dequantised as 16 q, so it carries 1/16
+      constexpr float kHiFactor = C == kCodecInt4 ? 0.0625f : 1.0f;
+      const __half2 h1 = __floats2half2_rn(bf16lo(hi) * inv * kHiFactor, bf16hi(hi) * inv * kHiFactor);
       if (__hisinf(h0.x) | __hisinf(h0.y) | __hisinf(__float2half_rn(bf16lo(hi) * inv)) |
           __hisinf(__float2half_rn(bf16hi(hi) * inv)))
         hd.xinf = 1;
@@ -486,8 +489,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
           float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
-            const uint32_t a0 = deq_q_even(wd[w]), a2 = deq_q_odd16(wd[w]);
-            const uint32_t a1 = deq_q_even(wd[w] >> 8), a3 = deq_q_odd16(wd[w] >> 8);
+            uint32_t a0, a1, a2, a3;
+            if constexpr (C == kCodecMxfp4) {
+              a0 = deq_e2m1<0>(wd[w]);
+              a2 = deq_e2m1<4>(wd[w]);
+              a1 = deq_e2m1<8>(wd[w]);
+              a3 = deq_e2m1<12>(wd[w]);
+            } else {
+              a0 = deq_q_even(wd[w]);
+              a2 = deq_q_odd16(wd[w]);
+              a1 = deq_q_even(wd[w] >> 8);
+              a3 = deq_q_odd16(wd[w] >> 8);
+            }
             if (w & 1) {
               mma_16816(d0, d1, d2, d3, a0, a1, a2, a3, bx[2 * w], bx[2 * w + 1], d0, d1, d2, d3);
               const uint32_t sw = (w == 1) ? s01 : s23;
@@ -638,7 +651,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     const bool act = g < hd.uniq_cnt[u];
     const int pr = hd.uniq_pair[u][act ? g : 0];
     float v0, v1;
-    dn_unit_mma(base, hfb + (size_t)pr * kHfStride + 16 * c, lane, v0, v1);
+    dn_unit_mma<C>(base, hfb + (size_t)pr * kHfStride + 16 * c, lane, v0, v1);
     if (act) {
       const float f = (float)(1 << kHShift) * hd.topw[pr / K][pr % K];
       *reinterpret_cast<float2*>(part + ((size_t)blk * (PL::P + T) + pr) * 8 + 2 * c) = make_float2(v0 * f, v1 * f);
@@ -742,7 +755,7 @@ extern "C" int ling_moe_trace_read(unsigned long long* host, int nctas) {
 }
 #endif
 
-template <int T>
+template <int T, int C>
 static cudaError_t launch_t(const DecodeParams& p, int nctas, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nctas);
@@ -754,22 +767,32 @@ static cudaError_t launch_t(const DecodeParams& p, int nctas, cudaStream_t strea
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, moe_decode_kernel<T>, p);
+  return cudaLaunchKernelEx(&cfg, moe_decode_kernel<T, C>, p);
 }
 
-cudaError_t launch_decode(const DecodeParams& p, int nctas, cudaStream_t stream) {
+template <int C>
+static cudaError_t launch_c(const DecodeParams& p, int nctas, cudaStream_t stream) {
   switch (p.T) {
-    case 1: return launch_t<1>(p, nctas, stream);
-    case 2: return launch_t<2>(p, nctas, stream);
-    case 3: return launch_t<3>(p, nctas, stream);
-    case 4: return launch_t<4>(p, nctas, stream);
+    case 1: return launch_t<1, C>(p, nctas, stream);
+    case 2: return launch_t<2, C>(p, nctas, stream);
+    case 3: return launch_t<3, C>(p, nctas, stream);
+    case 4: return launch_t<4, C>(p, nctas, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
+cudaError_t launch_decode(const DecodeParams& p, int nctas, cudaStream_t stream) {
+  if (p.codec == kCodecMxfp4) return launch_c<kCodecMxfp4>(p, nctas, stream);
+  if (p.codec == kCodecInt4) return launch_c<kCodecInt4>(p, nctas, stream);
+  return cudaErrorInvalidValue;
+}
+
 template <int T>
 static cudaError_t setup_t() {
-  return cudaFuncSetAttribute(moe_decode_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(moe_decode_kernel<T, kCodecInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Plan<T>::bytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(moe_decode_kernel<T, kCodecMxfp4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)Plan<T>::bytes);
 }
 
@@ -783,7 +806,7 @@ cudaError_t setup_decode() {
 
 int decode_max_ctas_per_sm() {
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, moe_decode_kernel<4>, kDecodeThreads,
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, moe_decode_kernel<4, kCodecInt4>, kDecodeThreads,
                                                     Plan<4>::bytes) != cudaSuccess)
     return 0;
   return n;

@@ -38,6 +38,7 @@ struct DecodeParams {
   unsigned int* err;             // sticky device error word
   int skip_arrive_cta;           // test hook: this CTA withholds its router rows (-1: none)
   unsigned long long wait_limit_ns;
+  int codec;                     // kCodecInt4 or kCodecMxfp4 (common.cuh): how gu / dn codes decode
 };
 
 size_t decode_smem_bytes(int T);

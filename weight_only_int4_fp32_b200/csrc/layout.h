@@ -58,6 +58,15 @@ constexpr int kDnScaleOff = kDnChunks * 512;      // 3072
 constexpr int kDnUnitBytes = kDnScaleOff + kDnChunks * 64;  // 3456
 constexpr size_t kDnExpertBytes = (size_t)kDnUnits * kDnUnitBytes;  // 1105920
 
+// Routed-weight codecs.  kCodecInt4: symmetric int4 codes, stored
+// offset-binary (q + 8), one bf16 scale per 32 K.  kCodecMxfp4: MXFP4 (OCP
+// Microscaling) -- E2M1 codes (bit 3 sign, bits 2..1 exponent with bias 1,
+// bit 0 mantissa) stored as they are, in the same nibble positions, with the
+// per-32 E8M0 scale 2^(e - 127) stored as the bf16 2^(e - 127 + 14) (the
+// kernels decode E2M1 as value * 2^-14).  Same unit layouts for both.
+constexpr int kCodecInt4 = 0;
+constexpr int kCodecMxfp4 = 1;
+
 static_assert(kGuChunks % 2 == 0, "gate/up units split into two K halves");
 static_assert(kH % 256 == 0 && kI % 256 == 0, "shape must tile by 256");
 

@@ -17,6 +17,9 @@ it produces, in the canonical boundary layout:
   sh_down   bf16  [H, I]
   x         bf16  [T, H]        ~ N(0, 1)
   lm head   bf16  [V, H]        ~ N(0, 0.02) * exp(U(-1, 1)) per row, V = 157,184
+MXFP4 layers (layer_weights_mxfp4) draw the same tensors in the same order,
+with E8M0 scale bytes uint8 [E, rows, K/32] uniform in [119, 123] in place of
+the bf16 scales (the code bytes are uniform either way).
 
 A uniform byte carries two independent uniform 4-bit codes, so drawing
 bytes uniformly is the same as drawing each int4 code uniformly in
@@ -133,6 +136,36 @@ def layer_weights(num_experts: int = NUM_EXPERTS, hidden: int = HIDDEN,
                         sh_gate, sh_up, sh_down)
 
 
+def _e8m0_bytes(shape, g, device, lo=119, hi=123):
+    """E8M0 scale bytes e uniform in [lo, hi]: scales 2^(e - 127) from 2^-8 to 2^-4."""
+    return torch.randint(lo, hi + 1, shape, generator=g, device=device, dtype=torch.uint8)
+
+
+def layer_weights_mxfp4(num_experts: int = NUM_EXPERTS, hidden: int = HIDDEN,
+                        inter: int = INTER, seed: int = 0, device="cpu",
+                        group: int = GROUP) -> LayerWeights:
+    """One MoE layer with MXFP4 routed experts, drawn in the W4 layer's order:
+    the codes are uniform bytes (two independent uniform E2M1 codes per byte,
+    all 16 codes valid), the scales E8M0 bytes uniform in [119, 123], so that
+    the weights' spread is close to the W4 layer's."""
+    E, H, I = num_experts, hidden, inter
+    if H % 2 or I % 2 or H % group or I % group:
+        raise ValueError("hidden and inter must be multiples of the group size")
+    g = _gen(seed, device)
+    router_w = _normal_bf16((E, H), 0.02, g, device)
+    gate_q = _bytes((E, I, H // 2), g, device)
+    gate_s = _e8m0_bytes((E, I, H // group), g, device)
+    up_q = _bytes((E, I, H // 2), g, device)
+    up_s = _e8m0_bytes((E, I, H // group), g, device)
+    down_q = _bytes((E, H, I // 2), g, device)
+    down_s = _e8m0_bytes((E, H, I // group), g, device)
+    sh_gate = _normal_bf16((I, H), 0.02, g, device)
+    sh_up = _normal_bf16((I, H), 0.02, g, device)
+    sh_down = _normal_bf16((H, I), 0.02, g, device)
+    return LayerWeights(router_w, gate_q, gate_s, up_q, up_s, down_q, down_s,
+                        sh_gate, sh_up, sh_down)
+
+
 def tokens(T: int, hidden: int = HIDDEN, seed: int = 0, device="cpu") -> torch.Tensor:
     """x [T, hidden] bf16 ~ N(0, 1) from one seed."""
     g = _gen(seed, device)
@@ -177,6 +210,9 @@ WORKLOADS = {
     "prefill_e512_t2048_zipf": dict(num_experts=512, T=2048, weight_seed=0, token_seed=20000,
                                     zipf_s=1.1,
                                     note="full layer, 2048-token prefill chunk, Zipf(1.1) router bias"),
+    "decode_e512_t1_mxfp4": dict(num_experts=512, T=1, weight_seed=0, fmt="mxfp4",
+                                 token_seeds=[1 + t for t in range(1000)],
+                                 note="full layer with MXFP4 routed experts, batch-1 decode, token t from seed 1+t"),
 }
 
 
