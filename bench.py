@@ -44,16 +44,21 @@ L2_FLUSH_BYTES = 256 << 20
 # the command), valid only while the kernel's sources are the ones captured:
 # the sources are hashed and the figure is reported as null once they change.
 TRAFFIC = {
-    "decode_e512_t1": {"bytes": 41_036_288 + 13_568,
+    "decode_e512_t1": {"bytes": 41_039_872 + 9_472,
                        "sources": ('decode.cu', 'decode.h', 'common.cuh', 'layout.h'),
-                       "sha256": "ed6ad3f459dbdeaf472f2b064f6568192661d8f7c5ed1856120264390f27db67"},
-    "verify_e512_t4": {"bytes": 126_536_960 + 4_990_208,
+                       "sha256": "01babd609ad0cf5bcc904feebe6f651432ef6deaf6fbd8a02fa6306d53f437d1"},
+    "verify_e512_t4": {"bytes": 129_148_160 + 3_299_584,
                        "sources": ('decode.cu', 'decode.h', 'common.cuh', 'layout.h'),
-                       "sha256": "ed6ad3f459dbdeaf472f2b064f6568192661d8f7c5ed1856120264390f27db67"},
+                       "sha256": "01babd609ad0cf5bcc904feebe6f651432ef6deaf6fbd8a02fa6306d53f437d1"},
     # online-FP8 LM head: lmh_mma_kernel, the only kernel of a call
     "lmhead_fp8_v157184_t1": {"bytes": 403_094_784 + 3_492_608,
                               "sources": ('lmhead.cu', 'lmhead.h', 'common.cuh', 'layout.h'),
                               "sha256": "d01a920b9c0a6a3a51626bf75dd07ef598df8463088f96b423c90873de2a1698"},
+    # MXFP4 routed experts (the decode kernel's E2M1 instantiation); the unit
+    # layout keeps a bf16 scale per 32, so 8 experts read 3,317,760 B each
+    "decode_e512_t1_mxfp4": {"bytes": 41_039_872 + 70_400,
+                             "sources": ('decode.cu', 'decode.h', 'common.cuh', 'layout.h'),
+                             "sha256": "01babd609ad0cf5bcc904feebe6f651432ef6deaf6fbd8a02fa6306d53f437d1"},
     # token-grouped: the dominant kernel, tc_grouped_kernel<0> (gate/up tiles)
     "prefill_e512_t2048_zipf": {"bytes": 457_028_864 + 53_828_608,
                                 "sources": ('grouped_tc.cu', 'grouped_tc.h', 'common.cuh', 'layout.h'),
