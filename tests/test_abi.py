@@ -155,3 +155,21 @@ def test_create_mxfp4_checks_arguments_and_its_token_limit():
     assert "MXFP4" in lm.ling_moe_last_error()
     rc = lm.lib.ling_moe_create_mxfp4(ctypes.byref(_cfg(group_size=64)), ctypes.byref(_weights()), ctypes.byref(h))
     assert rc == lm.LING_MOE_ERR_UNSUPPORTED
+
+
+def test_binding_rejects_wrong_tensors_before_any_call():
+    import torch
+    layer = object.__new__(lm.MoELayer)   # no handle: the checks run before the library is called
+    layer.H, layer.k, layer._torch, layer.handle = 2560, 8, torch, None
+    with pytest.raises(ValueError):
+        layer.forward(torch.zeros((1, 2560), dtype=torch.bfloat16))          # not on the GPU
+    with pytest.raises(ValueError):
+        layer.forward_host(torch.zeros((2, 2048), dtype=torch.bfloat16))     # wrong hidden
+    with pytest.raises(ValueError):
+        layer.forward_host(torch.zeros((2, 2560), dtype=torch.bfloat16), torch.zeros((2, 2560)))  # fp32 out
+    head = object.__new__(lm.LMHeadFP8)
+    head.vocab, head.hidden, head._torch, head.handle = 1000, 2560, torch, None
+    with pytest.raises(ValueError):
+        head.forward_host(torch.zeros((1, 2560), dtype=torch.bfloat16), torch.zeros((1, 999)))
+    with pytest.raises(ValueError):
+        head.forward(torch.zeros((1, 2560), dtype=torch.bfloat16))

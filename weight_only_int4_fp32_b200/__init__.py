@@ -205,6 +205,16 @@ def ling_moe_route_noalloc(x: int, T: int, router_w: int, router_bias, num_exper
                                              topk_idx, topk_w, stream))
 
 
+def _require(t, shape, dtype, cuda: bool, name: str):
+    """Raise ValueError unless t is a contiguous tensor of this shape and dtype
+    on the GPU (cuda) or the host; the C calls trust the sizes they are given."""
+    if (tuple(t.shape) != tuple(shape) or t.dtype != dtype or bool(t.is_cuda) != cuda
+            or not t.is_contiguous()):
+        where = "CUDA" if cuda else "host"
+        raise ValueError(f"{name} must be a contiguous {where} {dtype} tensor of shape {tuple(shape)}, "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+
 class MoELayer:
     """One MoE layer on the current CUDA device, built from torch tensors.
 
@@ -239,11 +249,13 @@ class MoELayer:
 
     def forward(self, x, out=None, stream=None, return_routing: bool = False):
         torch = self._torch
-        if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous() or x.dim() != 2:
-            raise ValueError("x must be a contiguous 2-D bf16 CUDA tensor")
+        if x.dim() != 2:
+            raise ValueError("x must be 2-D [T, hidden]")
         T = x.shape[0]
+        _require(x, (T, self.H), torch.bfloat16, True, "x")
         if out is None:
             out = torch.empty_like(x)
+        _require(out, (T, self.H), torch.bfloat16, True, "out")
         s = self._stream(stream)
         if return_routing:
             idx = torch.empty((T, self.k), dtype=torch.int32, device=x.device)
@@ -259,8 +271,10 @@ class MoELayer:
     def forward_host(self, x_host, out_host=None, stream=None):
         torch = self._torch
         T = x_host.shape[0]
+        _require(x_host, (T, self.H), torch.bfloat16, False, "x_host")
         if out_host is None:
             out_host = torch.empty_like(x_host)
+        _require(out_host, (T, self.H), torch.bfloat16, False, "out_host")
         ling_moe_forward_host(self.handle, x_host.data_ptr(), T, out_host.data_ptr(), self._stream(stream))
         return out_host
 
@@ -320,11 +334,13 @@ class LMHeadFP8:
 
     def forward(self, x, logits=None, stream=None, return_codes: bool = False):
         torch = self._torch
-        if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous() or x.dim() != 2:
-            raise ValueError("x must be a contiguous 2-D bf16 CUDA tensor")
+        if x.dim() != 2:
+            raise ValueError("x must be 2-D [T, hidden]")
         T = x.shape[0]
+        _require(x, (T, self.hidden), torch.bfloat16, True, "x")
         if logits is None:
             logits = torch.empty((T, self.vocab), dtype=torch.float32, device=x.device)
+        _require(logits, (T, self.vocab), torch.float32, True, "logits")
         s = self._stream(stream)
         if return_codes:
             xq = torch.empty((T, self.hidden), dtype=torch.uint8, device=x.device)
@@ -340,8 +356,10 @@ class LMHeadFP8:
     def forward_host(self, x_host, logits_host=None, stream=None):
         torch = self._torch
         T = x_host.shape[0]
+        _require(x_host, (T, self.hidden), torch.bfloat16, False, "x_host")
         if logits_host is None:
             logits_host = torch.empty((T, self.vocab), dtype=torch.float32, pin_memory=True)
+        _require(logits_host, (T, self.vocab), torch.float32, False, "logits_host")
         _check(lib.ling_moe_lmhead_forward_host(self.handle, x_host.data_ptr(), T, logits_host.data_ptr(),
                                                 self._stream(stream)))
         return logits_host
