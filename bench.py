@@ -543,7 +543,7 @@ def run_ours(args):
             "warmup": nwarm, "ms_per_step": kern_ms / nsteps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
             "dtype": ("mxfp4 (e2m1, e8m0 per 32) x fp16" if fmt == "mxfp4" else "w4a16") + ", fp32 accumulate",
-            "data": "synthetic (seeded weights and tokens, recipe in DESIGN.md)",
+            "data": "synthetic (seeded weights and tokens drawn by workloads/synth.py)",
             "config": {"workload": args.workload, "T": T, "experts": E, "top_k": 8, "hidden": H,
                        "inter": I, "layers": len(layers),
                        "l2": "flushed before every step (256 MiB write, then a 256 MiB read of another buffer "
@@ -698,7 +698,7 @@ def run_lmhead(args):
             "metric": LMHEAD_METRIC, "value": ws * nsteps * T / (kern_ms * 1e-3), "unit": "tokens/s",
             "n_gpus": ws, "steps": nsteps, "warmup": nwarm, "ms_per_step": avg_ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 x e4m3, fp32 accumulate",
-            "data": "synthetic (seeded head and tokens, recipe in DESIGN.md)",
+            "data": "synthetic (seeded head and tokens drawn by workloads/synth.py)",
             "config": {"workload": args.workload, "T": T, "vocab": V, "hidden": H,
                        "l2": "not flushed: every call streams 402 MB of codes, over 3x the 126 MB L2, "
                              "from the start of each CTA's range, so nothing of a call is left in L2 for the next",
