@@ -11,9 +11,10 @@ weights are resident in HBM when the timed region starts; L2 is flushed
 (256 MiB write, then a 256 MiB read) before every step, outside the per-step
 CUDA events.  The online-FP8 LM-head workloads stream 402 MB per call, over
 three times the L2, and are not flushed.
-Rank 0 prints one JSON line.  With N > 1 (torchrun) every rank runs its own
-independent token stream on its own GPU: replicas, no collective on the data
-path; time is the max over ranks.
+Rank 0 prints one JSON line.  With N > 1 every rank runs its own independent
+token stream on its own GPU: replicas, no collective on the data path; time is
+the max over ranks.  Started with --gpus N > 1 outside a launcher, bench.py
+starts the N ranks itself under torch.distributed.run.
 """
 from __future__ import annotations
 
@@ -32,6 +33,19 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer decode tokens/s and achieved HBM GB/s (W4 g32, 512e top-8, T=1)"
 METRIC_MXFP4 = "MoE-layer decode tokens/s and achieved HBM GB/s (MXFP4 e2m1/e8m0, 512e top-8, T=1)"
+# every other workload's line carries its own metric, so that no line claims another's
+WORKLOAD_METRIC = {
+    "decode_e512_t1": METRIC,
+    "decode_e512_t1_mxfp4": METRIC_MXFP4,
+    "reduced_e32_t1": "reduced MoE-layer decode tokens/s and achieved HBM GB/s (W4 g32, 32e top-8, T=1)",
+    "verify_e512_t4": "MoE-layer verify tokens/s and achieved HBM GB/s (W4 g32, 512e top-8, T=4 per call)",
+    "stack40_e512_t1": "40-layer MoE-stack decode tokens/s and achieved HBM GB/s (W4 g32, 512e top-8, T=1)",
+    "prefill_e512_t2048_zipf": "MoE-layer prefill tokens/s (W4 g32, 512e top-8, T=2048 per call, Zipf(1.1) routing)",
+}
+
+
+def metric_for(workload):
+    return WORKLOAD_METRIC.get(workload, f"MoE-layer tokens/s ({workload})")
 H, I = 2560, 768
 ROUTED_BYTES = 3_317_760        # per expert: int4 codes + bf16 scales
 ROUTED_BYTES_MXFP4 = 3_133_440  # per expert: E2M1 codes + E8M0 scale bytes
@@ -276,7 +290,7 @@ def run_reference(args):
         step(warm + i)
     dt = time.perf_counter() - t0
     v = steps * T / dt
-    line = {"metric": METRIC_MXFP4 if wl.get("fmt") == "mxfp4" else METRIC, "value": v, "unit": "tokens/s",
+    line = {"metric": metric_for(args.workload), "value": v, "unit": "tokens/s",
             "n_gpus": ws, "steps": steps,
             "warmup": warm, "ms_per_step": dt * 1e3 / steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -538,7 +552,7 @@ def run_ours(args):
         cpu = cpu_oracle_rate(args.workload if not stack else "decode_e512_t1",
                               seconds=args.cpu_seconds) if ws == 1 and args.cpu_seconds > 0 else None
         line = {
-            "metric": METRIC_MXFP4 if fmt == "mxfp4" else METRIC, "value": value, "unit": "tokens/s",
+            "metric": metric_for(args.workload), "value": value, "unit": "tokens/s",
             "n_gpus": ws, "steps": nsteps,
             "warmup": nwarm, "ms_per_step": kern_ms / nsteps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
@@ -715,6 +729,24 @@ def run_lmhead(args):
     return 0
 
 
+def spawn_ranks(n):
+    """Run this same command as n ranks (one per GPU) under torch.distributed.run.
+
+    Used when bench.py is started with --gpus N > 1 but not under a launcher
+    (WORLD_SIZE unset): each rank reads RANK / LOCAL_RANK / WORLD_SIZE from the
+    environment the launcher sets, rank 0 prints the one JSON line.  The
+    launcher's exit code is returned."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + sys.argv[1:]
+    env = dict(os.environ)
+    env.setdefault("OMP_NUM_THREADS", "4")
+    return subprocess.call(cmd, env=env, timeout=3600)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -726,6 +758,12 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return spawn_ranks(args.gpus)
+    ws, _, _ = dist_env()
+    if ws != args.gpus and "WORLD_SIZE" in os.environ:
+        print(f"bench.py: --gpus {args.gpus} under a launcher of WORLD_SIZE={ws}: running {ws} ranks",
+              file=sys.stderr)
     lmhead = args.workload.startswith("lmhead")
     if args.impl == "reference":
         return run_lmhead_reference(args) if lmhead else run_reference(args)

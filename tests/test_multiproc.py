@@ -78,3 +78,31 @@ def test_reference_arm_under_torchrun_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_bench_spawns_its_own_ranks_without_a_launcher():
+    """`bench.py --gpus 2` started plainly (no WORLD_SIZE) runs two ranks
+    itself under torch.distributed.run; rank 0 alone prints one line with
+    n_gpus = 2 (the reference arm needs no GPU, so this runs on CPU)."""
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+           "--workload", "reduced_e32_t1", "--steps", "2", "--warmup", "3"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+    assert d["metric"].startswith("reduced MoE-layer decode")
+
+
+def test_every_workload_line_names_its_own_metric():
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads
+    names = [w for w in workloads.WORKLOADS]
+    metrics = {bench.metric_for(w) for w in names}
+    assert len(metrics) == len(names)  # no two workloads share a metric string
+    assert bench.metric_for("decode_e512_t1") == bench.METRIC
+    assert "T=2048" in bench.metric_for("prefill_e512_t2048_zipf")
+    assert "T=4" in bench.metric_for("verify_e512_t4")
