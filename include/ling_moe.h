@@ -200,17 +200,36 @@ int ling_moe_test_set_wait(ling_moe_t *h, int skip_arrive_cta, uint64_t wait_lim
  * Limits: 0 <= T <= 4, 1 <= num_experts <= 512, 1 <= top_k <= min(8, num_experts);
  * anything else returns LING_MOE_ERR_INVALID_ARG (message in
  * ling_moe_last_error) before anything is launched.
- * Scratch: a static array of 8,448 bytes in device memory (logits of 4 x 512
- * experts plus two counters) that every GPU which loads the library holds
- * until the process exits.  Nothing is allocated, by this call or on its
- * behalf.  The first call on a device looks up that array's device address
- * (cudaGetSymbolAddress), so make the first call on each device before any
- * stream capture on it.  Every call shares the array: the counters start at
- * zero and each call leaves them at zero, but calls that overlap on the GPU
- * (two streams, or two host threads) race and must not be issued.
- * A device-side wait that runs out (2 s) writes -1 indices. */
+ * Scratch: a static array of 16,640 bytes in device memory (tagged logit
+ * slots of 4 x 512 experts, a generation word and an error word) that every
+ * GPU which loads the library holds until the process exits.  Nothing is
+ * allocated, by this call or on its behalf.  The first call on a device looks
+ * up that array's device address (cudaGetSymbolAddress) and keeps it for the
+ * life of the process, so make the first call on each device before any
+ * stream capture on it, and do not use this call across a device reset
+ * (cudaDeviceReset), after which the kept address may be stale.
+ * Every call shares the array.  Nothing in it needs to start at zero: each
+ * call tags the logits it writes with a fresh tag and reads only slots that
+ * carry it, so a call never sees an earlier call's values.  Calls that
+ * overlap on the GPU (two streams, or two host threads) race on the array and
+ * must not be issued; if they are, their own results are undefined, but the
+ * next call on its own is correct again.
+ * A device-side wait that runs out (2 s) writes -1 indices and 0 weights and
+ * sets a sticky error word, which ling_moe_route_noalloc_status reports. */
 int ling_moe_route_noalloc(const void *x, int T, const void *router_w, const float *router_bias,
                            int num_experts, int top_k, int32_t *topk_idx, float *topk_w, void *stream);
+
+/* Synchronises `stream`, then reports whether a ling_moe_route_noalloc call
+ * on the current device had a device-side wait run out since the last status
+ * call: LING_MOE_ERR_DEVICE_TIMEOUT (and clears the error word) or
+ * LING_MOE_OK.  Allocates nothing.  Errors: CUDA. */
+int ling_moe_route_noalloc_status(void *stream);
+
+/* Test hook: the next ling_moe_route_noalloc call has CTA skip_cta (-1:
+ * none) withhold its logits, so that CTA 0's wait runs out; wait_limit_ns
+ * bounds that wait for this and later calls (0 restores 2 s).  Errors:
+ * INVALID_ARG (skip_cta >= 512). */
+int ling_moe_route_noalloc_test_set_wait(int skip_cta, uint64_t wait_limit_ns);
 
 /* ---- online-FP8 LM head ----
  * Source: bpdata article "Harom optimalizacio a Ling-3.0-flash MoE

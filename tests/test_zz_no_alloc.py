@@ -59,3 +59,71 @@ def test_route_noalloc_rejects_sizes_beyond_its_scratch():
             lm.ling_moe_route_noalloc(x.data_ptr(), T, wr.data_ptr(), 0, E, k, idx.data_ptr(), w.data_ptr(), 0)
         assert e.value.code == lm.LING_MOE_ERR_INVALID_ARG
         assert "route_noalloc" in lm.ling_moe_last_error()
+
+
+def _reduced_layer(k=8):
+    lw = workloads.layer_weights(32, seed=0, device="cuda")
+    return lw, lm.MoELayer(lw.tensors(), top_k=k, max_tokens=4)
+
+
+def test_route_noalloc_wait_runs_out_then_next_call_is_correct():
+    """A call whose CTA 5 withholds its logits gives up after the shortened
+    wait: -1 indices, 0 weights, and the status call reports the time-out
+    once.  The next call routes correctly (its fresh tag ignores the slots
+    the cut-short call left behind)."""
+    lw, layer = _reduced_layer()
+    stream = torch.cuda.current_stream().cuda_stream
+    try:
+        assert lm.ling_moe_route_noalloc_status(stream) == lm.LING_MOE_OK
+        x = workloads.tokens(2, seed=901, device="cuda")
+        lm.ling_moe_route_noalloc_test_set_wait(5, 50_000_000)
+        idx, w = _route_noalloc(x, lw.router_w, None, 32, 8)
+        torch.cuda.synchronize()
+        assert (idx == -1).all() and (w == 0).all(), (idx, w)
+        assert lm.ling_moe_route_noalloc_status(stream) == lm.LING_MOE_ERR_DEVICE_TIMEOUT
+        assert lm.ling_moe_route_noalloc_status(stream) == lm.LING_MOE_OK  # read once, then cleared
+        lm.ling_moe_route_noalloc_test_set_wait(-1, 0)
+        for T, seed in ((2, 902), (4, 903)):
+            x = workloads.tokens(T, seed=seed, device="cuda")
+            idx, w = _route_noalloc(x, lw.router_w, None, 32, 8)
+            _, idx_ref, w_ref = layer.forward(x, return_routing=True)
+            torch.cuda.synchronize()
+            assert torch.equal(idx, idx_ref), (T, idx, idx_ref)
+            assert torch.allclose(w, w_ref, rtol=0, atol=1e-5), T
+        assert lm.ling_moe_route_noalloc_status(stream) == lm.LING_MOE_OK
+    finally:
+        lm.ling_moe_route_noalloc_test_set_wait(-1, 0)
+        layer.close()
+
+
+def test_route_noalloc_replayed_from_a_cuda_graph():
+    """One call outside capture (it looks up the scratch address), one call
+    captured into a CUDA graph on a side stream, then two replays with new
+    tokens copied into the captured input: each replay's routing equals
+    forward_ex on the same tokens."""
+    lw, layer = _reduced_layer()
+    T, E, k = 3, 32, 8
+    try:
+        x_static = workloads.tokens(T, seed=910, device="cuda")
+        idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+        w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+        _route_noalloc(x_static, lw.router_w, None, E, k)
+        torch.cuda.synchronize()
+        side = torch.cuda.Stream()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            lm.ling_moe_route_noalloc(x_static.data_ptr(), T, lw.router_w.data_ptr(), 0, E, k, idx.data_ptr(),
+                                      w.data_ptr(), side.cuda_stream)
+        for replay in range(2):
+            x = workloads.tokens(T, seed=911 + replay, device="cuda")
+            x_static.copy_(x)
+            graph.replay()
+            torch.cuda.synchronize()
+            _, idx_ref, w_ref = layer.forward(x, return_routing=True)
+            torch.cuda.synchronize()
+            assert torch.equal(idx, idx_ref), (replay, idx, idx_ref)
+            assert torch.allclose(w, w_ref, rtol=0, atol=1e-5), replay
+        del graph
+        assert lm.ling_moe_route_noalloc_status(torch.cuda.current_stream().cuda_stream) == lm.LING_MOE_OK
+    finally:
+        layer.close()

@@ -18,7 +18,8 @@ __all__ = [
     "ling_moe_config_t", "ling_moe_weights_t", "library_path", "load_library",
     "ling_moe_create", "ling_moe_create_mxfp4", "ling_moe_forward", "ling_moe_forward_ex", "ling_moe_forward_host",
     "ling_moe_status", "ling_moe_describe", "ling_moe_launch_count", "ling_moe_last_error",
-    "ling_moe_destroy", "ling_moe_test_set_wait", "ling_moe_route_noalloc", "ling_moe_set_kernel_timing",
+    "ling_moe_destroy", "ling_moe_test_set_wait", "ling_moe_route_noalloc", "ling_moe_route_noalloc_status",
+    "ling_moe_route_noalloc_test_set_wait", "ling_moe_set_kernel_timing",
     "ling_moe_kernel_times", "MoELayer", "LMHeadFP8", "EXPORTED",
 ]
 
@@ -34,7 +35,8 @@ EXPORTED = (
     "ling_moe_create", "ling_moe_create_mxfp4", "ling_moe_forward", "ling_moe_forward_ex",
     "ling_moe_forward_host", "ling_moe_status", "ling_moe_describe", "ling_moe_launch_count",
     "ling_moe_last_error", "ling_moe_destroy", "ling_moe_test_set_wait", "ling_moe_route_noalloc",
-    "ling_moe_set_kernel_timing", "ling_moe_kernel_times", "ling_moe_kernel_name",
+    "ling_moe_route_noalloc_status", "ling_moe_route_noalloc_test_set_wait", "ling_moe_set_kernel_timing",
+    "ling_moe_kernel_times", "ling_moe_kernel_name",
     "ling_moe_lmhead_create", "ling_moe_lmhead_forward", "ling_moe_lmhead_forward_ex",
     "ling_moe_lmhead_forward_host", "ling_moe_lmhead_weights", "ling_moe_lmhead_status",
     "ling_moe_lmhead_launch_count", "ling_moe_lmhead_destroy", "ling_moe_lmhead_test_set_wait",
@@ -98,6 +100,8 @@ def _load():
         "ling_moe_destroy": (None, [vp]),
         "ling_moe_test_set_wait": (ci, [vp, ci, ctypes.c_uint64]),
         "ling_moe_route_noalloc": (ci, [vp, ci, vp, vp, ci, ci, vp, vp, vp]),
+        "ling_moe_route_noalloc_status": (ci, [vp]),
+        "ling_moe_route_noalloc_test_set_wait": (ci, [ci, ctypes.c_uint64]),
         "ling_moe_set_kernel_timing": (ci, [vp, ci]),
         "ling_moe_kernel_times": (ci, [vp, ctypes.POINTER(ctypes.c_float), ci, ctypes.POINTER(ci)]),
         "ling_moe_kernel_name": (ctypes.c_char_p, [vp, ci]),
@@ -203,6 +207,19 @@ def ling_moe_route_noalloc(x: int, T: int, router_w: int, router_bias, num_exper
     """Routing with the library's static scratch; allocates nothing (see ling_moe.h)."""
     return _check(lib.ling_moe_route_noalloc(x, T, router_w, router_bias or None, num_experts, top_k,
                                              topk_idx, topk_w, stream))
+
+
+def ling_moe_route_noalloc_status(stream: int = 0) -> int:
+    """LING_MOE_OK, or LING_MOE_ERR_DEVICE_TIMEOUT if a routing wait gave up since the last check
+    (returned, not raised, like MoELayer.status)."""
+    rc = lib.ling_moe_route_noalloc_status(stream)
+    if rc not in (LING_MOE_OK, LING_MOE_ERR_DEVICE_TIMEOUT):
+        raise LingMoEError(rc, ling_moe_last_error())
+    return rc
+
+
+def ling_moe_route_noalloc_test_set_wait(skip_cta: int, wait_limit_ns: int) -> int:
+    return _check(lib.ling_moe_route_noalloc_test_set_wait(skip_cta, wait_limit_ns))
 
 
 def _require(t, shape, dtype, cuda: bool, name: str):

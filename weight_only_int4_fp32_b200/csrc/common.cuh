@@ -366,6 +366,81 @@ __device__ __forceinline__ void warp_topk_fast(const float* lg, int E, int k, in
   __syncwarp();
 }
 
+// The same selection with fewer dependent steps (one warp, k <= 8,
+// E <= 512): keys are 64-bit (order key of the logit, then 0xFFFF - index),
+// all distinct, so (logit desc, index asc) is plain key order.  The k-th
+// largest lane maximum (found by redux.sync rounds over the 32-bit order
+// keys, lanes that tie dropping out together) bounds the k-th largest key
+// from below, so every selected key is a candidate; the few candidates are
+// gathered in shared memory and each one's rank among them is counted.  With
+// more than 32 candidates (heavy ties) the round-by-round selection above
+// takes over.  scratch: 40 x 8 bytes of this warp's shared memory.
+// Returns the same indices and weights as warp_topk_fast.
+__device__ __forceinline__ void warp_topk_thresh(const float* lg, int E, int k, unsigned long long* scratch,
+                                                 int* out_i, float* out_w) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long key[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int e = lane + 32 * j;
+    key[j] = e < E ? ((unsigned long long)f32_order_key(lg[e]) << 32) | (unsigned long long)(0xFFFF - e) : 0ull;
+  }
+  uint32_t mx = 0u;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) mx = max(mx, (uint32_t)(key[j] >> 32));
+  uint32_t cur = mx, tau32 = 0u;
+  int counted = 0;
+#pragma unroll 1
+  for (int r = 0; r < 32 && counted < k; ++r) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, cur);
+    counted += __popc(__ballot_sync(0xffffffffu, cur == m));
+    tau32 = m;
+    cur = cur == m ? 0u : cur;
+  }
+  const unsigned long long tau = (unsigned long long)tau32 << 32;
+  unsigned int mask = 0;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) mask |= (key[j] >= tau && key[j] != 0ull ? 1u : 0u) << j;
+  const int cnt = __popc(mask);
+  int off = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, off, o);
+    if (lane >= o) off += v;
+  }
+  const int total = __shfl_sync(0xffffffffu, off, 31);
+  off -= cnt;
+  if (total > 32) {
+    warp_topk_fast(lg, E, k, out_i, out_w);
+    return;
+  }
+  unsigned long long* cand = scratch;
+  unsigned long long* sel = scratch + 32;
+#pragma unroll
+  for (int j = 0; j < 16; ++j)
+    if (mask >> j & 1u) cand[off++] = key[j];
+  __syncwarp();
+  const unsigned long long mine = lane < total ? cand[lane] : 0ull;
+  int r = 0;
+  for (int o = 0; o < total; ++o) r += cand[o] > mine;
+  __syncwarp();
+  if (lane < total && r < k) sel[r] = mine;  // the r-th selection
+  __syncwarp();
+  const unsigned long long s_l = lane < k ? sel[lane] : 0ull;
+  const float v0 = f32_from_order_key((uint32_t)(sel[0] >> 32));
+  const float vr = f32_from_order_key((uint32_t)(s_l >> 32));
+  const float ex = lane < k ? expf(vr - v0) : 0.f;
+  float s = ex;
+#pragma unroll
+  for (int o = 4; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane < k) {
+    const int e = 0xFFFF - (int)(s_l & 0xFFFFu);
+    out_i[lane] = e < E ? e : 0;
+    out_w[lane] = ex / s;
+  }
+  __syncwarp();
+}
+
 // Two-accumulator variants (even / odd elements) to halve dependent chains.
 __device__ __forceinline__ void dot8_bf16_bf16_2(uint4 w, uint4 x, float& a, float& b) {
   a = fma_bf16h<0, 0>(w.x, x.x, a);

@@ -366,7 +366,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     __syncwarp();
     if (warp == 0) LING_TRACE(12);
     if (warp == 0) { LING_CLK(1); if (lane == 0) g_clk_sink(lg[0] + lg[E - 1]); LING_CLK(2); }
-    warp_topk_fast(lg, E, K, hd.topi[warp], hd.topw[warp]);
+    warp_topk_thresh(lg, E, K, reinterpret_cast<unsigned long long*>(bufA + kMaxExperts * 4), hd.topi[warp],
+                     hd.topw[warp]);
     if (warp == 0) LING_CLK(3);
 
   }

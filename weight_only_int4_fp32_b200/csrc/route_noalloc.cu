@@ -6,9 +6,20 @@
 // and one CTA selects the top-k.  Its scratch does not come from cudaMalloc
 // or a library handle: it lives in a file-scope static __device__ array that
 // every GPU loading the library holds until the process exits.  Callers that
-// cannot allocate -- code running inside a CUDA-graph capture, a framework
-// whose memory is owned by its own pool, or a plugin that must not touch the
-// device allocator -- can still route tokens with it.
+// cannot allocate -- a framework whose device memory is owned by its own
+// pool, or a latency-critical path that must not call cudaMalloc (which can
+// synchronise the device) -- can still route tokens with it.
+//
+// Every call finds the scratch as the last call left it, so nothing in it has
+// to start at zero: each logit slot is one 64-bit word holding a call tag in
+// its upper half and the fp32 logit in its lower half, written in one store.
+// All CTAs read the generation word when they start; the call's tag is the
+// generation + 1 (never 0, the value of untouched static storage).  CTA 0
+// waits until every slot it needs carries the tag, selects, and writes the
+// tag back as the new generation.  A call therefore never reads a value from
+// an earlier call, and a call that ran out of time, or two calls that
+// overlapped on the GPU (a race the caller must avoid), leave nothing behind
+// that a later call could misread: the next call uses a fresh tag.
 #include <mutex>
 
 #include <cuda_runtime.h>
@@ -18,35 +29,51 @@
 
 namespace lingmoe {
 
-// Scratch: logits of up to kRouteMaxT tokens x kMaxExperts experts, then two
-// counters (router rows published, CTAs finished).  The counters start at
-// zero (static storage) and the last CTA of every call puts them back to
-// zero.  Calls that overlap on the GPU share the scratch and race.
+// Scratch: tagged logit slots of up to kRouteMaxT tokens x kMaxExperts
+// experts, then the generation word and the sticky error word.
 constexpr int kRouteMaxT = 4;
-constexpr size_t kRouteLogitsBytes = (size_t)kRouteMaxT * kMaxExperts * sizeof(float);  // 8192
-constexpr size_t kRouteScratchBytes = kRouteLogitsBytes + 256;
+constexpr size_t kRouteSlotBytes = (size_t)kRouteMaxT * kMaxExperts * sizeof(unsigned long long);  // 16384
+constexpr size_t kRouteGenOff = kRouteSlotBytes;
+constexpr size_t kRouteErrOff = kRouteSlotBytes + 4;
+constexpr size_t kRouteScratchBytes = kRouteSlotBytes + 256;  // 16,640
 static __device__ __align__(256) unsigned char g_route_scratch[kRouteScratchBytes];
 
 constexpr int kRouteWarps = 8;
 constexpr int kRouteThreads = kRouteWarps * 32;
 constexpr unsigned long long kRouteWaitNs = 2000000000ull;  // 2 s
 
-// scratch: logits [T][E] fp32 at offset 0; counters at kRouteLogitsBytes
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" :: "l"(p), "l"(v) : "memory");
+}
+
+// scratch: slots [T][E] at offset 0, generation and error words after them
 __global__ void __launch_bounds__(kRouteThreads)
 route_noalloc_kernel(const __nv_bfloat16* __restrict__ x, int T, const __nv_bfloat16* __restrict__ wr,
                      const float* __restrict__ bias, int E, int K, int32_t* topk_idx, float* topk_w,
-                     unsigned char* scratch) {
+                     unsigned char* scratch, int skip_cta, unsigned long long wait_ns) {
   __shared__ __align__(16) unsigned char xs[kRouteMaxT * kH * 2];
   __shared__ __align__(16) float lg[kRouteMaxT][kMaxExperts];
   __shared__ int si[kRouteMaxT][kMaxTopK];
   __shared__ float sw[kRouteMaxT][kMaxTopK];
-  __shared__ int ok_s;
-  float* logits = reinterpret_cast<float*>(scratch);
-  unsigned int* rows_done = reinterpret_cast<unsigned int*>(scratch + kRouteLogitsBytes);
-  unsigned int* ctas_done = rows_done + 1;
+  __shared__ int late;
+  __shared__ unsigned long long tk_scratch[kRouteMaxT][40];
+  unsigned long long* slots = reinterpret_cast<unsigned long long*>(scratch);
+  unsigned int* gen = reinterpret_cast<unsigned int*>(scratch + kRouteGenOff);
+  unsigned int* err = reinterpret_cast<unsigned int*>(scratch + kRouteErrOff);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int cta = blockIdx.x, ncta = gridDim.x;
 
+  // this call's tag: read before this CTA publishes anything, so CTA 0 (which
+  // moves the generation on only after every slot carries the tag) cannot
+  // have moved it yet
+  const unsigned int g0 = *reinterpret_cast<volatile unsigned int*>(gen);
+  const unsigned int tag = g0 + 1u == 0u ? 1u : g0 + 1u;
+  if (tid == 0) late = 0;
   for (int v = tid; v < T * kH / 8; v += kRouteThreads)
     reinterpret_cast<uint4*>(xs)[v] = reinterpret_cast<const uint4*>(x)[v];
   __syncthreads();
@@ -54,11 +81,11 @@ route_noalloc_kernel(const __nv_bfloat16* __restrict__ x, int T, const __nv_bflo
   // this CTA's router rows, one warp per row; the same accumulation order as
   // the decode kernel's router rows, so both entry points agree bit for bit
   const int r0 = (int)((long long)cta * E / ncta), r1 = (int)((long long)(cta + 1) * E / ncta);
-  for (int e = r0 + warp; e < r1; e += kRouteWarps) {
+  for (int e = r0 + warp; e < r1 && cta != skip_cta; e += kRouteWarps) {
     const __nv_bfloat16* row = wr + (size_t)e * kH;
-    float g0[kRouteMaxT], g1[kRouteMaxT], g2[kRouteMaxT], g3[kRouteMaxT];
+    float g0a[kRouteMaxT], g1[kRouteMaxT], g2[kRouteMaxT], g3[kRouteMaxT];
 #pragma unroll
-    for (int t = 0; t < kRouteMaxT; ++t) g0[t] = g1[t] = g2[t] = g3[t] = 0.f;
+    for (int t = 0; t < kRouteMaxT; ++t) g0a[t] = g1[t] = g2[t] = g3[t] = 0.f;
 #pragma unroll
     for (int m = 0; m < kH / 256; m += 2) {
       const int c0 = lane + 32 * m, c1 = c0 + 32;
@@ -66,7 +93,7 @@ route_noalloc_kernel(const __nv_bfloat16* __restrict__ x, int T, const __nv_bflo
 #pragma unroll
       for (int t = 0; t < kRouteMaxT; ++t) {
         if (t < T) {
-          dot8_bf16_bf16_2(w0, lds128(xs + t * kH * 2 + 16 * c0), g0[t], g1[t]);
+          dot8_bf16_bf16_2(w0, lds128(xs + t * kH * 2 + 16 * c0), g0a[t], g1[t]);
           dot8_bf16_bf16_2(w1, lds128(xs + t * kH * 2 + 16 * c1), g2[t], g3[t]);
         }
       }
@@ -74,53 +101,44 @@ route_noalloc_kernel(const __nv_bfloat16* __restrict__ x, int T, const __nv_bflo
 #pragma unroll
     for (int t = 0; t < kRouteMaxT; ++t) {
       if (t < T) {
-        const float v = warp_sum((g0[t] + g1[t]) + (g2[t] + g3[t]));
-        if (lane == 0) logits[t * E + e] = v + (bias ? bias[e] : 0.f);
+        const float v = warp_sum((g0a[t] + g1[t]) + (g2[t] + g3[t])) + (bias ? bias[e] : 0.f);
+        if (lane == 0)
+          st_relaxed_u64(slots + (size_t)t * E + e, ((unsigned long long)tag << 32) | __float_as_uint(v));
       }
-    }
-    if (lane == 0) {
-      __threadfence();
-      atomicAdd(rows_done, 1u);
     }
   }
 
-  if (cta == 0) {
-    // wait (bounded) for every row, then select
-    if (tid == 0) {
-      int ok = 1;
-      const unsigned long long t0 = globaltimer_ns();
-      while (ld_acquire_u32(rows_done) < (unsigned)E) {
-        if (globaltimer_ns() - t0 > kRouteWaitNs) { ok = 0; break; }
+  if (cta != 0) return;
+  // CTA 0: wait (bounded) until every slot carries this call's tag, then select
+  const unsigned long long t0 = globaltimer_ns();
+  for (int v = tid; v < T * E; v += kRouteThreads) {
+    unsigned long long s = ld_relaxed_u64(slots + v);
+    while ((unsigned int)(s >> 32) != tag) {
+      if (*reinterpret_cast<volatile int*>(&late) || globaltimer_ns() - t0 > wait_ns) {
+        late = 1;
+        break;
       }
-      ok_s = ok;
+      s = ld_relaxed_u64(slots + v);
     }
-    __syncthreads();
-    const bool ok = ok_s != 0;
+    lg[v / E][v % E] = __uint_as_float((unsigned int)s);
+  }
+  __syncthreads();
+  const bool ok = late == 0;
+  if (warp < T) {
     if (ok) {
-      for (int v = tid; v < T * E; v += kRouteThreads) lg[v / E][v % E] = ldcg_f32(logits + v);
-    }
-    __syncthreads();
-    if (warp < T) {
-      if (ok) {
-        warp_topk_fast(lg[warp], E, K, si[warp], sw[warp]);
-        if (lane < K) {
-          topk_idx[warp * K + lane] = si[warp][lane];
-          topk_w[warp * K + lane] = sw[warp][lane];
-        }
-      } else if (lane < K) {
-        topk_idx[warp * K + lane] = -1;  // a wait ran out: no routing
-        topk_w[warp * K + lane] = 0.f;
+      warp_topk_thresh(lg[warp], E, K, tk_scratch[warp], si[warp], sw[warp]);
+      if (lane < K) {
+        topk_idx[warp * K + lane] = si[warp][lane];
+        topk_w[warp * K + lane] = sw[warp][lane];
       }
+    } else if (lane < K) {
+      topk_idx[warp * K + lane] = -1;  // a wait ran out: no routing
+      topk_w[warp * K + lane] = 0.f;
     }
   }
-  // every CTA counts itself out; the last one zeroes the counters for the next call
-  __syncthreads();
   if (tid == 0) {
-    __threadfence();
-    if (atomicAdd(ctas_done, 1u) == (unsigned)ncta - 1u) {
-      atomicExch(rows_done, 0u);
-      atomicExch(ctas_done, 0u);
-    }
+    if (!ok) atomicOr(err, 1u);  // sticky until ling_moe_route_noalloc_status reads it
+    *reinterpret_cast<volatile unsigned int*>(gen) = tag;
   }
 }
 
@@ -129,9 +147,27 @@ void set_last_error(const char* msg);  // the library's thread-local message (ap
 namespace {
 std::mutex g_mu;
 unsigned char* g_scratch_ptr[64] = {};  // device address of the scratch, per device ordinal
+int g_skip_cta = -1;                    // test hook: next call only
+unsigned long long g_wait_ns = kRouteWaitNs;
 int reject(int code, const char* msg) {
   set_last_error(msg);
   return code;
+}
+// The scratch's device address on the current device (looked up once per device).
+int scratch_address(int* dev_out, unsigned char** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return reject(LING_MOE_ERR_CUDA, "route_noalloc: cudaGetDevice failed");
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
+    if (e != cudaSuccess || !p) return reject(LING_MOE_ERR_CUDA, "route_noalloc: cudaGetSymbolAddress failed");
+    g_scratch_ptr[dev] = static_cast<unsigned char*>(p);
+  }
+  *dev_out = dev;
+  *out = g_scratch_ptr[dev];
+  return LING_MOE_OK;
 }
 }  // namespace
 
@@ -156,24 +192,21 @@ extern "C" int ling_moe_route_noalloc(const void* x, int T, const void* router_w
       (router_bias && (reinterpret_cast<uintptr_t>(router_bias) & 3)))
     return reject(LING_MOE_ERR_INVALID_ARG, "route_noalloc: misaligned pointer");
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-    return reject(LING_MOE_ERR_CUDA, "route_noalloc: cudaGetDevice failed");
-  unsigned char* scratch;
+  unsigned char* scratch = nullptr;
+  int rc = scratch_address(&dev, &scratch);
+  if (rc) return rc;
   int nsm = 0;
-  {
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_scratch_ptr[dev]) {
-      // first call on this device: the device address of the static scratch
-      void* p = nullptr;
-      const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
-      if (e != cudaSuccess || !p) return reject(LING_MOE_ERR_CUDA, "route_noalloc: cudaGetSymbolAddress failed");
-      g_scratch_ptr[dev] = static_cast<unsigned char*>(p);
-    }
-    scratch = g_scratch_ptr[dev];
-  }
   if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0)
     return reject(LING_MOE_ERR_CUDA, "route_noalloc: SM count query failed");
   const int nctas = nsm < num_experts ? nsm : num_experts;
+  int skip;
+  unsigned long long wait_ns;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    skip = g_skip_cta;
+    g_skip_cta = -1;  // one call only
+    wait_ns = g_wait_ns;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nctas);
   cfg.blockDim = dim3(kRouteThreads);
@@ -186,7 +219,35 @@ extern "C" int ling_moe_route_noalloc(const void* x, int T, const void* router_w
   cfg.numAttrs = 1;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, route_noalloc_kernel, static_cast<const __nv_bfloat16*>(x), T,
                                            static_cast<const __nv_bfloat16*>(router_w), router_bias, num_experts,
-                                           top_k, topk_idx, topk_w, scratch);
+                                           top_k, topk_idx, topk_w, scratch, skip, wait_ns);
   if (e != cudaSuccess) return reject(LING_MOE_ERR_CUDA, cudaGetErrorString(e));
+  return LING_MOE_OK;
+}
+
+extern "C" int ling_moe_route_noalloc_status(void* stream) {
+  int dev = 0;
+  unsigned char* scratch = nullptr;
+  int rc = scratch_address(&dev, &scratch);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned int err = 0;
+  cudaError_t e = cudaMemcpyAsync(&err, scratch + kRouteErrOff, sizeof(err), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return reject(LING_MOE_ERR_CUDA, "route_noalloc: reading the error word failed");
+  if (err) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyAsync(scratch + kRouteErrOff, &zero, sizeof(zero), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return reject(LING_MOE_ERR_CUDA, "route_noalloc: clearing the error word failed");
+    return reject(LING_MOE_ERR_DEVICE_TIMEOUT, "route_noalloc: a device-side wait gave up (indices -1)");
+  }
+  return LING_MOE_OK;
+}
+
+extern "C" int ling_moe_route_noalloc_test_set_wait(int skip_cta, uint64_t wait_limit_ns) {
+  if (skip_cta >= kMaxExperts) return reject(LING_MOE_ERR_INVALID_ARG, "route_noalloc: skip_cta out of range");
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_skip_cta = skip_cta < 0 ? -1 : skip_cta;
+  g_wait_ns = wait_limit_ns ? wait_limit_ns : kRouteWaitNs;
   return LING_MOE_OK;
 }
