@@ -307,7 +307,11 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ our arm
 
-def build_layers(workload, device):
+ROTATE_LAYERS = 12       # independent copies a single-layer workload rotates over (L2 not flushed)
+ROTATE_SEED_STRIDE = 7919  # copy r > 0 of a layer draws its weights from seed + r times this
+
+
+def build_layers(workload, device, rotate=1):
     import torch
     import workloads
     import weight_only_int4_fp32_b200 as lm
@@ -316,6 +320,10 @@ def build_layers(workload, device):
     T = wl["T"]
     nlayers = wl.get("layers", 1)
     seeds = wl.get("layer_seeds") or [wl["weight_seed"]]
+    if nlayers == 1 and rotate > 1:
+        # the same workload on `rotate` independent layers: step i runs layer i % rotate
+        nlayers = rotate
+        seeds = [seeds[0] + r * ROTATE_SEED_STRIDE for r in range(rotate)]
     layers = []
     gen, _ = _layer_gen(wl)
     fmt = wl.get("fmt", "int4")
@@ -329,6 +337,18 @@ def build_layers(workload, device):
         del lw, w
         torch.cuda.empty_cache()
     return layers, E, T
+
+
+def l2_mode(workload, requested):
+    """'rotate' (single-layer decode-size workloads: steps rotate over independent
+    layers, no flush) or 'flush' (an L2 flush before every step)."""
+    if requested != "auto":
+        return requested
+    import workloads
+    wl = workloads.WORKLOADS[workload]
+    if wl.get("layers", 1) == 1 and wl["T"] <= 8 and wl["num_experts"] >= 512:
+        return "rotate"
+    return "flush"
 
 
 def workloads_fmt(workload):
@@ -365,38 +385,40 @@ def run_ours(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     import weight_only_int4_fp32_b200 as lm
-    layers, E, T = build_layers(args.workload, dev)
+    mode = l2_mode(args.workload, args.l2)
+    stack = args.workload.startswith("stack")
+    layers, E, T = build_layers(args.workload, dev, rotate=ROTATE_LAYERS if mode == "rotate" else 1)
     nsteps, nwarm = args.steps, args.warmup
     inputs = make_inputs(args.workload, nsteps + nwarm, T, dev, rank=rank)
-    stack = args.workload.startswith("stack")
-    flush = L2Flush(dev)
+    l2flush = L2Flush(dev)
+    flush = l2flush if mode == "flush" else (lambda i: None)
     out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
 
-    def one_step(x):
+    def one_step(x, i=0):
         if stack:
             for l, layer in enumerate(layers):
                 layer.forward(x[l:l + 1], out)
         else:
-            layers[0].forward(x, out)
+            layers[i % len(layers)].forward(x, out)
 
     # union of routed experts per step (bytes the method must read), from the
     # routing; for token-grouped calls also the rows the tensor-core tiles take
     tc_rows = []
 
-    def union_of(x):
+    def union_of(x, i=0):
         if stack:
             return [8] * len(layers)
-        _, idx, _ = layers[0].forward(x, return_routing=True)
+        _, idx, _ = layers[i % len(layers)].forward(x, return_routing=True)
         cnt = torch.bincount(idx.flatten().long(), minlength=E)
         tc_rows.append(int(cnt[cnt > GEMV_MAX_TOKENS].sum()) + T)
         return [int(torch.unique(idx).numel())]
 
     for i in range(nwarm):
         flush(i)
-        one_step(inputs[i])
+        one_step(inputs[i], i)
     torch.cuda.synchronize()
-    unions = [union_of(inputs[nwarm + i]) for i in range(nsteps)]
+    unions = [union_of(inputs[nwarm + i], nwarm + i) for i in range(nsteps)]
     torch.cuda.synchronize()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(nsteps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(nsteps)]
@@ -412,7 +434,7 @@ def run_ours(args):
         for i in range(nsteps):
             flush(i)
             starts[i].record(stream)
-            one_step(inputs[nwarm + i])
+            one_step(inputs[nwarm + i], nwarm + i)
             ends[i].record(stream)
         g1.record(stream)
         torch.cuda.synchronize()
@@ -507,7 +529,7 @@ def run_ours(args):
         xh = [inputs[nwarm + i].cpu().pin_memory() for i in range(nsteps)]
         oh = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
         for i in range(min(nwarm, 5)):
-            layers[0].forward_host(xh[i % nsteps], oh)
+            layers[i % len(layers)].forward_host(xh[i % nsteps], oh)
         torch.cuda.synchronize()
         if ws > 1:
             dist.barrier()
@@ -516,20 +538,38 @@ def run_ours(args):
             flush(i)
             torch.cuda.synchronize()
             t0 = time.perf_counter()
-            layers[0].forward_host(xh[i], oh)
+            layers[(nwarm + i) % len(layers)].forward_host(xh[i], oh)
             te += time.perf_counter() - t0
         te = max_over_ranks(te, dev)
         e2e = {"value": ws * nsteps * T / te, "unit": "tokens/s",
                "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2,
                "note": "ling_moe_forward_host per step (pinned H2D copy + layer + D2H copy + stream sync), "
-                       "host wall clock summed over the calls; L2 flushed before each call, outside its clock"}
+                       "host wall clock summed over the calls; " + (
+                           "steps rotate over the layers as in the timed steps" if mode == "rotate" else
+                           "L2 flushed before each call, outside its clock")}
+
+    # with rotation, the same steps on one layer with an L2 flush before each
+    # (instruction and weight bytes both come from HBM), for comparison
+    flushed = None
+    if mode == "rotate":
+        fs = [torch.cuda.Event(enable_timing=True) for _ in range(nsteps)]
+        fe = [torch.cuda.Event(enable_timing=True) for _ in range(nsteps)]
+        for i in range(nsteps):
+            l2flush(i)
+            fs[i].record(stream)
+            layers[0].forward(inputs[nwarm + i], out)
+            fe[i].record(stream)
+        torch.cuda.synchronize()
+        f_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(fs, fe)), dev)
+        flushed = {"value": ws * nsteps * T / (f_ms * 1e-3), "unit": "tokens/s", "us_per_step": f_ms / nsteps * 1e3,
+                   "note": "one layer, L2 flushed (256 MiB write + 256 MiB read) before every step, outside its events"}
 
     fmt = workloads_fmt(args.workload)
     per_call_bytes = [sum(decode_bytes(E, u, fmt) for u in us) for us in unions]
     if args.workload.startswith("prefill"):
         per_call_bytes = [b + 2 * T * H * 2 for b in per_call_bytes]
     avg_bytes = sum(per_call_bytes) / len(per_call_bytes)
-    calls_per_step = len(layers)
+    calls_per_step = len(layers) if stack else 1
     avg_launch_ms = kern_ms / nsteps / calls_per_step
     achieved = (avg_bytes / calls_per_step) / (avg_launch_ms * 1e-3) / 1e9
     peak, peak_kind = peaks()
@@ -560,8 +600,12 @@ def run_ours(args):
             "data": "synthetic (seeded weights and tokens drawn by workloads/synth.py)",
             "config": {"workload": args.workload, "T": T, "experts": E, "top_k": 8, "hidden": H,
                        "inter": I, "layers": len(layers),
-                       "l2": "flushed before every step (256 MiB write, then a 256 MiB read of another buffer "
-                             "so that no dirty lines are left), outside the per-step events",
+                       "l2": (f"not flushed: step i runs layer i mod {len(layers)} of {len(layers)} independent "
+                              f"full-shape layers, so the bytes a step reads were last read {len(layers)} steps "
+                              f"(over {len(layers) - 1} x 40 MB of other weight traffic, above the 126 MB L2) before"
+                              if mode == "rotate" else
+                              "flushed before every step (256 MiB write, then a 256 MiB read of another buffer "
+                              "so that no dirty lines are left), outside the per-step events"),
                        "parallelism": f"replicas x{ws}"},
             "us_per_layer": avg_launch_ms * 1e3,
             "achieved_gbs": achieved,
@@ -570,6 +614,7 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "e2e": e2e,
             "warm": warm,
+            "flushed": flushed,
             "graph": graph,
             "gpu_launches": launches,
             "clocks": clk.summary(),
@@ -755,6 +800,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode_e512_t1")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--l2", default="auto", choices=["auto", "rotate", "flush"],
+                    help="between steps: rotate over independent layers (decode-size workloads) or flush L2")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
