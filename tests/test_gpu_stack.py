@@ -1,9 +1,10 @@
 """The 40-layer stack (independent full-shape layers, one token per call)
 against the fp64 oracle (needs a B200 with room for all 40 layers, ~68 GB).
 
-Every layer is checked on its first 4 tokens of the stack's input recipe; all
-40 handles stay alive together, as in the benchmark, and layer 0 is run again
-at the end to show that the other 39 left it untouched.
+Every layer is checked on the first 4 tokens of the stack's input recipe and
+layers 0, 13, 26 and 39 on the first 16; all 40 handles stay alive together,
+as in the benchmark, and layer 0 is run again at the end to show that the
+other 39 left it untouched.
 """
 import numpy as np
 import pytest
@@ -18,11 +19,14 @@ pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
 TOKENS = 4
+TOKENS_FULL = 16
+FULL_LAYERS = (0, 13, 26, 39)
 
 
 def _layer_inputs(layer_index: int) -> torch.Tensor:
+    n = TOKENS_FULL if layer_index in FULL_LAYERS else TOKENS
     return torch.stack([workloads.tokens(1, seed=workloads.stack_token_seed(t, layer_index), device=DEV)[0]
-                        for t in range(TOKENS)])
+                        for t in range(n)])
 
 
 def _run_t1(layer, xs):

@@ -34,6 +34,27 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
   // SiLU(g) * u = g / (1 + e^-g) * u
   return g / (1.0f + expf(-g)) * u;
 }
+// The same for a token carried at scale 2^-sigma: g and u are the scaled
+// gate and up values (true values s g, s u with s = 2^sigma) and the result is
+// SiLU(s g) (s u) / s^2 = g u sigmoid(s g), which stays finite wherever g and
+// u are.  With s = 1 it is silu_mul bit for bit.
+__device__ __forceinline__ float silu_mul_scaled(float g, float u, float s) {
+  return g / (1.0f + expf(-(g * s))) * u;
+}
+// Largest |x| of a token as bf16 magnitude bits (0..0x7F80 for finite x) ->
+// the exponent sigma of its power-of-two scale: 0 while that |x| lies in
+// [2^-3, 16) (the range the fixed scales of h are laid out for), otherwise
+// the exponent that brings it into [2, 4), limited to [-100, 126] (a token
+// whose largest |x| is below 2^-99 has an output below bf16's smallest
+// subnormal either way).
+__device__ __forceinline__ int token_sigma(uint32_t bf16_mag_bits) {
+  if (bf16_mag_bits == 0u) return 0;
+  const int e = (int)(bf16_mag_bits >> 7) - 127;  // subnormals count as 2^-127
+  if (e >= -3 && e <= 3) return 0;
+  return max(-100, min(126, e - 1));
+}
+// 2^e for e in [-126, 127]
+__device__ __forceinline__ float pow2_int(int e) { return __uint_as_float((uint32_t)(127 + e) << 23); }
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -304,6 +325,8 @@ __device__ __forceinline__ float f32_from_order_key(uint32_t k) {
 // lanes holding it (a second redux.sync on 0xFFFF - index); the owner
 // removes the entry and rebuilds its tree.  Lane r keeps the result of
 // round r.  Lane r < k writes slot r and exp(l_r - l_0) / sum_s exp(l_s - l_0).
+// lg may hold logits divided by a power of two s (a rescaled token): the
+// weights then take wscale = s, exp(s (l_r - l_0)).
 __device__ __forceinline__ void lane_best16(const uint32_t key[16], uint32_t& bk, int& bj) {
   uint32_t k8[8];
   int j8[8];
@@ -325,7 +348,8 @@ __device__ __forceinline__ void lane_best16(const uint32_t key[16], uint32_t& bk
   bk = k8[0];
   bj = j8[0];
 }
-__device__ __forceinline__ void warp_topk_fast(const float* lg, int E, int k, int* out_i, float* out_w) {
+__device__ __forceinline__ void warp_topk_fast(const float* lg, int E, int k, int* out_i, float* out_w,
+                                               float wscale = 1.0f) {
   const int lane = threadIdx.x & 31;
   uint32_t key[16];
 #pragma unroll
@@ -355,12 +379,12 @@ __device__ __forceinline__ void warp_topk_fast(const float* lg, int E, int k, in
   }
   const float vmax = f32_from_order_key(__shfl_sync(0xffffffffu, mine_k, 0));
   const float vr = f32_from_order_key(mine_k);
-  const float ex = (lane < k) ? expf(vr - vmax) : 0.f;
+  const float ex = (lane < k) ? expf((vr - vmax) * wscale) : 0.f;
   float s = ex;
 #pragma unroll
   for (int o = 4; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if (lane < k) {
-    out_i[lane] = mine_i < E ? mine_i : 0;  // only a NaN logit could select past the end
+    out_i[lane] = (unsigned)mine_i < (unsigned)E ? mine_i : 0;  // always in [0, E)
     out_w[lane] = ex / s;
   }
   __syncwarp();
@@ -377,7 +401,7 @@ __device__ __forceinline__ void warp_topk_fast(const float* lg, int E, int k, in
 // takes over.  scratch: 40 x 8 bytes of this warp's shared memory.
 // Returns the same indices and weights as warp_topk_fast.
 __device__ __forceinline__ void warp_topk_thresh(const float* lg, int E, int k, unsigned long long* scratch,
-                                                 int* out_i, float* out_w) {
+                                                 int* out_i, float* out_w, float wscale = 1.0f) {
   const int lane = threadIdx.x & 31;
   unsigned long long key[16];
 #pragma unroll
@@ -411,7 +435,7 @@ __device__ __forceinline__ void warp_topk_thresh(const float* lg, int E, int k, 
   const int total = __shfl_sync(0xffffffffu, off, 31);
   off -= cnt;
   if (total > 32) {
-    warp_topk_fast(lg, E, k, out_i, out_w);
+    warp_topk_fast(lg, E, k, out_i, out_w, wscale);
     return;
   }
   unsigned long long* cand = scratch;
@@ -429,13 +453,13 @@ __device__ __forceinline__ void warp_topk_thresh(const float* lg, int E, int k, 
   const unsigned long long s_l = lane < k ? sel[lane] : 0ull;
   const float v0 = f32_from_order_key((uint32_t)(sel[0] >> 32));
   const float vr = f32_from_order_key((uint32_t)(s_l >> 32));
-  const float ex = lane < k ? expf(vr - v0) : 0.f;
+  const float ex = lane < k ? expf((vr - v0) * wscale) : 0.f;
   float s = ex;
 #pragma unroll
   for (int o = 4; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if (lane < k) {
     const int e = 0xFFFF - (int)(s_l & 0xFFFFu);
-    out_i[lane] = e < E ? e : 0;
+    out_i[lane] = (unsigned)e < (unsigned)E ? e : 0;  // always in [0, E)
     out_w[lane] = ex / s;
   }
   __syncwarp();

@@ -74,10 +74,9 @@ struct __align__(128) SmemHeader {  // 128-byte multiple: the body starts on a f
   uint64_t mbar[kWarps][4];
   uint64_t xbar;
   uint64_t dbar;
-  uint32_t xmax[kMaxDecodeT];
-  float xscale[kMaxDecodeT];
-  int xinf;
-  int pad0[3];
+  uint32_t xmax[kMaxDecodeT];   // largest |x| of each token, bf16 magnitude bits
+  float xscale[kMaxDecodeT];    // s_t = 2^sigma_t (1 for most tokens)
+  float xinv[kMaxDecodeT];      // 1 / s_t
   int topi[kMaxDecodeT][kMaxTopK];
   float topw[kMaxDecodeT][kMaxTopK];
   int uniq_e[kMaxDecodeT * kMaxTopK];
@@ -92,8 +91,12 @@ struct __align__(128) SmemHeader {  // 128-byte multiple: the body starts on a f
 static_assert(sizeof(SmemHeader) % 128 == 0, "header keeps the body 128-byte aligned");
 
 // x is kept twice: the bf16 input as staged (router and shared rows read it
-// with mixed-precision FMAs) and an fp16 copy scaled by 2^-sigma per token in
-// MMA B-fragment order for the routed gate/up: per chunk of 64 K, per lane
+// with mixed-precision FMAs) and an fp16 copy in MMA B-fragment order for the
+// routed gate/up.  A token whose largest |x| lies outside [2^-3, 16) is first
+// divided by its power-of-two scale s_t in place (exact); everything after
+// that runs on x / s_t: the router adds b / s_t and weighs by exp(s_t (l -
+// l_0)), h is kept as h / s_t^2 (silu_mul_scaled) and the output is
+// multiplied by s_t twice before its bf16 rounding.  Per chunk of 64 K, per lane
 // class m = lane % 4, per K block w, the pair (x[c], x[c+1]) and the pair
 // (x[c+8], x[c+9]) / 16 with c = 16 kb + 2 m (the /16 matches the 16 q form
 // in which the upper half of a block's codes is dequantised).
@@ -196,6 +199,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   if (tid < kMaxDecodeT) {
     hd.xmax[tid] = 0u;
     hd.xscale[tid] = 1.0f;
+    hd.xinv[tid] = 1.0f;
   }
   // Launch index of this call: every CTA of the earlier launches on the
   // stream has counted itself out, and no CTA of this one can before all
@@ -204,7 +208,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   const unsigned long long done_ctas = (tid == 0) ? ld_acquire_u64(p.sync + 3) : 0ull;
   if (tid == 0) {
     hd.abort = 0;
-    hd.xinf = 0;
     hd.dcopies = 0;
     mbar_init(&hd.xbar, 1);
     mbar_init(&hd.dbar, 1);
@@ -242,49 +245,66 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   if (!mbar_wait(&hd.xbar, 0, p.wait_limit_ns, p.err)) hd.abort = 1;
   LING_TRACE(1);
   // fp16 copy of x in B-fragment order, built as soon as x lands (the first
-  // weight rows are still in flight).  x is converted as is (exact for normal
-  // bf16 values below 65504); if any value overflows fp16, the token is redone
-  // scaled by 2^-sigma.
-  auto build_xh = [&]() {
+  // weight rows are still in flight), together with each token's largest |x|.
+  // A warp's 32 items never straddle two tokens (640 items per token).
+  auto build_xh = [&](bool track) {
     for (int v = tid; v < T * (kH / 4); v += kDecodeThreads) {
       const int t = v / (kH / 4), r = v - t * (kH / 4), kb = r >> 2, m = r & 3;
       const int c = 16 * kb + 2 * m;
       const uint32_t lo = *reinterpret_cast<const uint32_t*>(xb + t * kXbTok + 2 * c);
       const uint32_t hi = *reinterpret_cast<const uint32_t*>(xb + t * kXbTok + 2 * (c + 8));
-      const float inv = 1.0f / hd.xscale[t];
-      const __half2 h0 = __floats2half2_rn(bf16lo(lo) * inv, bf16hi(lo) * inv);
+      const __half2 h0 = __floats2half2_rn(bf16lo(lo), bf16hi(lo));
       // int4: the upper half meets codes dequantised as 16 q, so it carries 1/16
       constexpr float kHiFactor = C == kCodecInt4 ? 0.0625f : 1.0f;
-      const __half2 h1 = __floats2half2_rn(bf16lo(hi) * inv * kHiFactor, bf16hi(hi) * inv * kHiFactor);
-      if (__hisinf(h0.x) | __hisinf(h0.y) | __hisinf(__float2half_rn(bf16lo(hi) * inv)) |
-          __hisinf(__float2half_rn(bf16hi(hi) * inv)))
-        hd.xinf = 1;
+      const __half2 h1 = __floats2half2_rn(bf16lo(hi) * kHiFactor, bf16hi(hi) * kHiFactor);
+      if (track) {
+        const uint32_t mag = __vmaxu2(lo & 0x7FFF7FFFu, hi & 0x7FFF7FFFu);
+        const uint32_t wm = __reduce_max_sync(0xffffffffu, max(mag & 0xFFFFu, mag >> 16));
+        if (lane == 0) atomicMax(&hd.xmax[t], wm);
+      }
       *reinterpret_cast<uint2*>(xf + t * kXfTok + (kb >> 2) * 128 + m * 32 + (kb & 3) * 8) =
           make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
     }
   };
-  build_xh();
+  build_xh(true);
   __syncthreads();
-  if (hd.xinf) {
-    // rare: some |x| beyond the fp16 range; scale that token by 2^-sigma
-    for (int v = tid; v < T * kXChunks; v += kDecodeThreads) {
-      const int t = v / kXChunks, c = v - t * kXChunks;
-      const uint4 w = lds128(xb + t * kXbTok + 16 * c);
-      const float mx = fmaxf(fmaxf(fmaxf(fabsf(bf16lo(w.x)), fabsf(bf16hi(w.x))),
-                                   fmaxf(fabsf(bf16lo(w.y)), fabsf(bf16hi(w.y)))),
-                             fmaxf(fmaxf(fabsf(bf16lo(w.z)), fabsf(bf16hi(w.z))),
-                                   fmaxf(fabsf(bf16lo(w.w)), fabsf(bf16hi(w.w)))));
-      atomicMax(&hd.xmax[t], __float_as_uint(fminf(mx, 3.0e38f)));  // monotonic for non-negative floats
+  {
+    int sig[T];
+    bool any = false;
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+      sig[t] = token_sigma(hd.xmax[t]);
+      any |= sig[t] != 0;
     }
-    __syncthreads();
-    if (tid < T) {
-      const int e = (int)(hd.xmax[tid] >> 23) - 127;
-      const int sigma = e >= 14 ? e - 13 : 0;
-      hd.xscale[tid] = __uint_as_float((uint32_t)(127 + sigma) << 23);
+    if (any) {
+      // rare: a token outside the direct range; x / s_t in place, then the
+      // fp16 copy again
+      if (tid < T) {
+        const int st = token_sigma(hd.xmax[tid]);
+        hd.xscale[tid] = pow2_int(st);
+        hd.xinv[tid] = pow2_int(-st);
+      }
+      for (int v = tid; v < T * kXChunks; v += kDecodeThreads) {
+        const int t = v / kXChunks, c = v - t * kXChunks;
+        int st = 0;
+#pragma unroll
+        for (int q = 0; q < T; ++q)
+          if (q == t) st = sig[q];
+        if (st == 0) continue;
+        const float inv = pow2_int(-st);
+        uint4 w = lds128(xb + t * kXbTok + 16 * c);
+        uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+        for (int o = 0; o < 4; ++o) {
+          const __nv_bfloat162 r2 = __floats2bfloat162_rn(bf16lo(wv[o]) * inv, bf16hi(wv[o]) * inv);
+          wv[o] = *reinterpret_cast<const uint32_t*>(&r2);
+        }
+        *reinterpret_cast<uint4*>(xb + t * kXbTok + 16 * c) = w;
+      }
+      __syncthreads();
+      build_xh(false);
+      __syncthreads();
     }
-    __syncthreads();
-    build_xh();
-    __syncthreads();
   }
   LING_TRACE(15);
 
@@ -326,10 +346,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     for (int t = 0; t < T; ++t) {
       const float g = warp_sum(a0[t]);
       if (router) {
-        if (lane == 0) p.logits[(size_t)t * E + r0 + it] = g + (p.router_bias ? p.router_bias[r0 + it] : 0.f);
+        if (lane == 0)
+          p.logits[(size_t)t * E + r0 + it] = g + (p.router_bias ? p.router_bias[r0 + it] * hd.xinv[t] : 0.f);
       } else {
         const float u = warp_sum(a1[t]);
-        if (lane == 0) p.h_s[(size_t)t * kI + s0 + it - nr] = silu_mul(g, u);
+        if (lane == 0) p.h_s[(size_t)t * kI + s0 + it - nr] = silu_mul_scaled(g, u, hd.xscale[t]);
       }
     }
     if (lane == 0 && !(router && withhold)) arrive(p.sync + (router ? 0 : 1));
@@ -367,7 +388,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     if (warp == 0) LING_TRACE(12);
     if (warp == 0) { LING_CLK(1); if (lane == 0) g_clk_sink(lg[0] + lg[E - 1]); LING_CLK(2); }
     warp_topk_thresh(lg, E, K, reinterpret_cast<unsigned long long*>(bufA + kMaxExperts * 4), hd.topi[warp],
-                     hd.topw[warp]);
+                     hd.topw[warp], hd.xscale[warp]);
     if (warp == 0) LING_CLK(3);
 
   }
@@ -543,9 +564,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
           const int col = 2 * m + cc;  // the expert's token column
           if (col < cnt) {
             const int pr = hd.uniq_pair[u][col];
-            const float xs = hd.xscale[pr / K];
-            const float g = (cc ? acc1 : acc0) * xs, up = (cc ? acc3 : acc2) * xs;
-            p.h_pair[(size_t)pr * kI + i] = silu_mul(g, up);
+            p.h_pair[(size_t)pr * kI + i] = silu_mul_scaled(cc ? acc1 : acc0, cc ? acc3 : acc2, hd.xscale[pr / K]);
           }
         }
       }
@@ -738,7 +757,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       for (int sl = 0; sl < kMaxTopK; ++sl)
         if (sl < K) s += v8[sl];
       s += vs;
-      p.out[(size_t)t * kH + kDnUnitRows * (b0 + blk) + r] = __float2bfloat16_rn(s);
+      const float st = hd.xscale[t];  // back from x / s_t: the output scales as s_t^2
+      p.out[(size_t)t * kH + kDnUnitRows * (b0 + blk) + r] = __float2bfloat16_rn(s * st * st);
     }
   }
   // every CTA (aborted or not) counts itself out: the next launch's index

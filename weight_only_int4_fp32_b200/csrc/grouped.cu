@@ -175,7 +175,13 @@ __global__ void __launch_bounds__(kRmThreads) grp_route_kernel(GroupedParams p, 
 }
 
 // One warp per token: top-k of its logits, the renormalised weights, and
-// one count per selected expert.
+// one count per selected expert.  The router GEMM sums bf16 products in fp32
+// on the tensor cores, which is exact to fp32 rounding while every product
+// that matters is a normal fp32 number and no sum overflows: for a token whose
+// largest |x| lies in [2^-60, 2^101) (with |Wr| < 2^20 per row sum).  A token
+// outside that window, or with a logit that is not finite, has its logits
+// recomputed here from x / s_t (the decode path's power-of-two token scale)
+// with fp32 FMAs: keys l / s_t + b / s_t, weights exp(s_t (l - l_0)).
 __global__ void __launch_bounds__(256) grp_topk_kernel(GroupedParams p, const float* logits, int32_t* ti,
                                                        float* tw, int32_t* cnt) {
   __shared__ float lg[8][kMaxExperts];
@@ -184,9 +190,45 @@ __global__ void __launch_bounds__(256) grp_topk_kernel(GroupedParams p, const fl
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t = blockIdx.x * 8 + warp;
   if (t >= p.T) return;
-  for (int e = lane; e < p.E; e += 32) lg[warp][e] = logits[(size_t)t * p.E + e];
+  bool bad = false;
+  for (int e = lane; e < p.E; e += 32) {
+    const float v = logits[(size_t)t * p.E + e];
+    bad |= !isfinite(v);
+    lg[warp][e] = v;
+  }
+  const uint4* xr = reinterpret_cast<const uint4*>(p.x + (size_t)t * kH);
+  uint32_t mag = 0u;
+  for (int c = lane; c < kH / 8; c += 32) {
+    const uint4 w = xr[c];
+    mag = __vmaxu2(mag, __vmaxu2(__vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
+                                 __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu)));  // per half
+  }
+  mag = __reduce_max_sync(0xffffffffu, max(mag & 0xFFFFu, mag >> 16));
+  const int ex = (int)(mag >> 7) - 127;
+  bad |= mag != 0u && (ex < -60 || ex > 100);
+  float wscale = 1.0f;
+  if (__any_sync(0xffffffffu, bad)) {
+    const int st = token_sigma(mag);
+    const float inv = pow2_int(-st);
+    wscale = pow2_int(st);
+    for (int e = 0; e < p.E; ++e) {
+      const uint4* wr = reinterpret_cast<const uint4*>(p.router_w + (size_t)e * kH);
+      float a = 0.f;
+      for (int c = lane; c < kH / 8; c += 32) {
+        const uint4 xv = xr[c], wv = wr[c];
+        const uint32_t xa[4] = {xv.x, xv.y, xv.z, xv.w}, wa[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int o = 0; o < 4; ++o) {
+          a = fmaf(bf16lo(xa[o]) * inv, bf16lo(wa[o]), a);
+          a = fmaf(bf16hi(xa[o]) * inv, bf16hi(wa[o]), a);
+        }
+      }
+      a = warp_sum(a);
+      if (lane == 0) lg[warp][e] = a + (p.router_bias ? p.router_bias[e] * inv : 0.f);
+    }
+  }
   __syncwarp();
-  warp_topk_fast(lg[warp], p.E, p.k, s_idx[warp], s_w[warp]);
+  warp_topk_fast(lg[warp], p.E, p.k, s_idx[warp], s_w[warp], wscale);
   if (lane < p.k) {
     const int e = s_idx[warp][lane];
     const float w = s_w[warp][lane];
@@ -299,9 +341,11 @@ __global__ void __launch_bounds__(kPlanThreads) grp_plan_kernel(int T, int E, in
 // ---------------------------------------------------------------- scatter
 // One CTA per token: each of its k pairs takes the next position in its
 // expert's run; x_t is scaled by 2^-sigma_t (max |x_t| * 2^-sigma_t in
-// [2^14, 2^15), so fp16 holds every bf16 value of a normal-range row exactly),
-// converted to fp16 and written to its k positions and to the shared-expert
-// row P + t.
+// [2^14, 2^15), so fp16 holds every value of the row down to 2^-24 of its
+// largest exactly), converted to fp16 and written to its k positions and to
+// the shared-expert row P + t.  sigma_t runs from -100 (a token whose largest
+// |x| is below 2^-86 has an output below bf16's smallest subnormal either
+// way) to 113 (bf16's largest finite value).
 __global__ void __launch_bounds__(kRowThreads) grp_scatter_kernel(const __nv_bfloat16* x, int k, int P,
                                                                   const int32_t* ti, const int32_t* off,
                                                                   int32_t* fill, int32_t* perm, int32_t* inv,
@@ -330,7 +374,7 @@ __global__ void __launch_bounds__(kRowThreads) grp_scatter_kernel(const __nv_bfl
   if ((c & 31) == 0) atomicMax(&smax, __float_as_uint(fminf(m, 3.0e38f)));
   __syncthreads();
   const int ex = (int)(smax >> 23) - 127;
-  const int sigma = smax == 0 ? 0 : max(-100, min(100, ex - 14));
+  const int sigma = smax == 0 ? 0 : max(-100, ex - 14);  // ex <= 127: at most 113
   const float inv_s = __uint_as_float((uint32_t)(127 - sigma) << 23);
   if (c == 0) xscale[t] = __uint_as_float((uint32_t)(127 + sigma) << 23);
   __half h[8];
@@ -342,7 +386,7 @@ __global__ void __launch_bounds__(kRowThreads) grp_scatter_kernel(const __nv_bfl
 
 // ---------------------------------------------------------------- combine
 __global__ void __launch_bounds__(kRowThreads) grp_combine_kernel(const float* y, const int32_t* inv, int k, int P,
-                                                                  __nv_bfloat16* out) {
+                                                                  const float* xscale, __nv_bfloat16* out) {
   const int t = blockIdx.x, c = threadIdx.x;
   float s[8];
 #pragma unroll
@@ -354,9 +398,13 @@ __global__ void __launch_bounds__(kRowThreads) grp_combine_kernel(const float* y
     s[0] += a.x; s[1] += a.y; s[2] += a.z; s[3] += a.w;
     s[4] += b.x; s[5] += b.y; s[6] += b.z; s[7] += b.w;
   }
+  // y is kept as y / c_t^2: back to the token's scale, c_t = 2^(sigma_t + 13)
+  // in [2^-87, 2^126], then one bf16 rounding (exact products unless the
+  // result leaves fp32's range, where bf16 rounds the same way)
+  const float ct = xscale[t] * (float)(1 << kGrpUnitShift);
   __nv_bfloat162 r[4];
 #pragma unroll
-  for (int o = 0; o < 4; ++o) r[o] = __floats2bfloat162_rn(s[2 * o], s[2 * o + 1]);
+  for (int o = 0; o < 4; ++o) r[o] = __floats2bfloat162_rn(s[2 * o] * ct * ct, s[2 * o + 1] * ct * ct);
   *reinterpret_cast<uint4*>(out + (size_t)t * kH + 8 * c) = *reinterpret_cast<const uint4*>(r);
 }
 
@@ -438,7 +486,7 @@ cudaError_t launch_grouped(const GroupedParams& p, const GroupedWorkspace& ws, c
   if ((e = launch_tc_gemm(1, ws.maps, tp, p.num_sms, s)) != cudaSuccess) return e;
   ++nl;
   mark(8);
-  grp_combine_kernel<<<p.T, kRowThreads, 0, s>>>(ws.y, ws.inv, p.k, P, p.out);
+  grp_combine_kernel<<<p.T, kRowThreads, 0, s>>>(ws.y, ws.inv, p.k, P, ws.xscale, p.out);
   ++nl;
   mark(kGroupedKernels);
   e = cudaGetLastError();

@@ -206,9 +206,10 @@ __global__ void __launch_bounds__(kGvThreads, 1) gv_gu_kernel(const GvParams p) 
         const int col = 2 * mm + cc;
         if (col < m) {
           const int pos = pos0 + col;
+          // h / c_t^2 (the tensor-core tiles' convention), then the fp16 shift
           const float xs = p.xscale[p.perm[pos] / p.k];
-          const float hv = silu_mul((cc ? acc1 : acc0) * xs, (cc ? acc3 : acc2) * xs) *
-                           (1.f / (float)(1 << kTcScaleShift));
+          const float hv = silu_mul_scaled(cc ? acc1 : acc0, cc ? acc3 : acc2, xs) *
+                           (1.f / (float)(1 << kTcScaleShift)) * (1.f / (float)(1 << (2 * kGrpUnitShift)));
           const __half hh = __float2half_rn(hv);
           __half* dst = p.h16 + (size_t)pos * (2 * kI) + i;
           dst[0] = hh;

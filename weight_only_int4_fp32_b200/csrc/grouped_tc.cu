@@ -129,8 +129,11 @@ __device__ __forceinline__ void tmem_ld16x2(uint32_t ta, uint32_t tb, float va[1
     vb[i] = __uint_as_float(q[i]);
   }
 }
-// SiLU(g) * u with the fast exponential and division (relative error ~1e-6)
-__device__ __forceinline__ float tc_silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
+// SiLU(s g) (s u) / s^2 = g u sigmoid(s g) with the fast exponential and
+// division (relative error ~1e-6); g, u: the scaled gate and up values
+__device__ __forceinline__ float tc_silu_mul_scaled(float g, float u, float s) {
+  return __fdividef(g, 1.0f + __expf(-(g * s))) * u;
+}
 // 2-D tiled TMA load (no multicast) into this CTA's shared memory.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   asm volatile(
@@ -507,7 +510,9 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
             const int col = c0 + cc;
             if (col < n) {
               const float f = fb[col];
-              const float hv = tc_silu_mul(g[cc] * f * cg, u[cc] * f * cu) * (1.f / (float)(1 << kTcScaleShift));
+              // h / c_t^2 = (x-scaled gate/up product) * 2^-2*kGrpUnitShift, then the fp16 shift
+              const float hv = tc_silu_mul_scaled(g[cc] * cg, u[cc] * cu, f) *
+                               (1.f / (float)(1 << kTcScaleShift)) * (1.f / (float)(1 << (2 * kGrpUnitShift)));
               const __half hi = __float2half_rn(hv);
               hrow[(size_t)col * (2 * kI)] = hi;
               hrow[(size_t)col * (2 * kI) + kI] = __float2half_rn(hv - __half2float(hi));

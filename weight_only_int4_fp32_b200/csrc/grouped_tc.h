@@ -20,14 +20,22 @@ constexpr int kTcMTilesDn = kH / kTcTileM;      // 10
 // 2^-kTcScaleShift, which keeps both inside fp16's normal range for scales in
 // [2^-22, 32] and |h| < 2^23.
 constexpr int kTcScaleShift = 8;
+// A token's x enters as x * 2^-sigma_t with its largest |x| in [2^14, 2^15);
+// h and y are kept relative to c_t = 2^(sigma_t + kGrpUnitShift), h as
+// h / c_t^2 and y as y / c_t^2, and the combine multiplies by c_t twice.  A
+// token whose largest |x| lies in [2, 4) has c_t = 1.  So no intermediate
+// grows or shrinks with the token's magnitude: every finite bf16 token keeps
+// the same relative precision, and only the final product can overflow
+// (to the infinity bf16 rounds the exact result to) or underflow.
+constexpr int kGrpUnitShift = 13;
 
 // Tile record: (expert or E for the shared expert, m-tile, first position, positions).
 struct TcParams {
   const uint8_t* gu;        // repacked routed gate/up
   const uint8_t* dn;        // repacked routed down
   const float* xscale;      // [T] 2^sigma_t: x16 rows hold x * 2^-sigma_t
-  __half* h16;              // [rows, 2, I] h * 2^-8 as fp16 hi + lo, natural K order
-  float* y;                 // [rows, H] expert output per position, times the routing weight
+  __half* h16;              // [rows, 2, I] (h / c_t^2) * 2^-8 as fp16 hi + lo, natural K order
+  float* y;                 // [rows, H] expert output per position / c_t^2, times the routing weight
   const int32_t* perm;      // position (< P) -> pair id t*k + slot
   const float* topk_w;      // [P] routing weight per pair id
   const float* sh_scale;    // [3] 2^-c of the fp16 shared-expert copies (gate, up, down)

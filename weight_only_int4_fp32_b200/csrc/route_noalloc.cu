@@ -62,6 +62,7 @@ route_noalloc_kernel(const __nv_bfloat16* __restrict__ x, int T, const __nv_bflo
   __shared__ float sw[kRouteMaxT][kMaxTopK];
   __shared__ int late;
   __shared__ unsigned long long tk_scratch[kRouteMaxT][40];
+  __shared__ unsigned int xmag[kRouteMaxT];
   unsigned long long* slots = reinterpret_cast<unsigned long long*>(scratch);
   unsigned int* gen = reinterpret_cast<unsigned int*>(scratch + kRouteGenOff);
   unsigned int* err = reinterpret_cast<unsigned int*>(scratch + kRouteErrOff);
@@ -74,9 +75,40 @@ route_noalloc_kernel(const __nv_bfloat16* __restrict__ x, int T, const __nv_bflo
   const unsigned int g0 = *reinterpret_cast<volatile unsigned int*>(gen);
   const unsigned int tag = g0 + 1u == 0u ? 1u : g0 + 1u;
   if (tid == 0) late = 0;
-  for (int v = tid; v < T * kH / 8; v += kRouteThreads)
-    reinterpret_cast<uint4*>(xs)[v] = reinterpret_cast<const uint4*>(x)[v];
+  if (tid < kRouteMaxT) xmag[tid] = 0u;
   __syncthreads();
+  // x and each token's largest |x| (bf16 magnitude bits; a warp's 32 chunks
+  // never straddle two tokens: 320 chunks per token)
+  for (int v = tid; v < T * kH / 8; v += kRouteThreads) {
+    const uint4 w = reinterpret_cast<const uint4*>(x)[v];
+    reinterpret_cast<uint4*>(xs)[v] = w;
+    const uint32_t m2 = __vmaxu2(__vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
+                                 __vmaxu2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu));
+    const uint32_t wm = __reduce_max_sync(0xffffffffu, max(m2 & 0xFFFFu, m2 >> 16));
+    if (lane == 0) atomicMax(&xmag[v / (kH / 8)], wm);
+  }
+  __syncthreads();
+  // tokens outside the direct range are divided by their power-of-two scale
+  // s_t, exactly as the decode kernel does: the bias then enters as b / s_t
+  // and the weights as exp(s_t (l - l_0))
+  bool any = false;
+  for (int t = 0; t < T; ++t) any |= token_sigma(xmag[t]) != 0;
+  if (any) {
+    for (int v = tid; v < T * kH / 8; v += kRouteThreads) {
+      const int st = token_sigma(xmag[v / (kH / 8)]);
+      if (st == 0) continue;
+      const float inv = pow2_int(-st);
+      uint4 w = reinterpret_cast<const uint4*>(xs)[v];
+      uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+      for (int o = 0; o < 4; ++o) {
+        const __nv_bfloat162 r2 = __floats2bfloat162_rn(bf16lo(wv[o]) * inv, bf16hi(wv[o]) * inv);
+        wv[o] = *reinterpret_cast<const uint32_t*>(&r2);
+      }
+      reinterpret_cast<uint4*>(xs)[v] = w;
+    }
+    __syncthreads();
+  }
 
   // this CTA's router rows, one warp per row; the same accumulation order as
   // the decode kernel's router rows, so both entry points agree bit for bit
@@ -101,7 +133,8 @@ route_noalloc_kernel(const __nv_bfloat16* __restrict__ x, int T, const __nv_bflo
 #pragma unroll
     for (int t = 0; t < kRouteMaxT; ++t) {
       if (t < T) {
-        const float v = warp_sum((g0a[t] + g1[t]) + (g2[t] + g3[t])) + (bias ? bias[e] : 0.f);
+        const float v = warp_sum((g0a[t] + g1[t]) + (g2[t] + g3[t])) +
+                        (bias ? bias[e] * pow2_int(-token_sigma(xmag[t])) : 0.f);
         if (lane == 0)
           st_relaxed_u64(slots + (size_t)t * E + e, ((unsigned long long)tag << 32) | __float_as_uint(v));
       }
@@ -126,7 +159,7 @@ route_noalloc_kernel(const __nv_bfloat16* __restrict__ x, int T, const __nv_bflo
   const bool ok = late == 0;
   if (warp < T) {
     if (ok) {
-      warp_topk_thresh(lg[warp], E, K, tk_scratch[warp], si[warp], sw[warp]);
+      warp_topk_thresh(lg[warp], E, K, tk_scratch[warp], si[warp], sw[warp], pow2_int(token_sigma(xmag[warp])));
       if (lane < K) {
         topk_idx[warp * K + lane] = si[warp][lane];
         topk_w[warp * K + lane] = sw[warp][lane];

@@ -173,6 +173,79 @@ def tokens(T: int, hidden: int = HIDDEN, seed: int = 0, device="cpu") -> torch.T
                        dtype=torch.float32).to(torch.bfloat16)
 
 
+BF16_MAX = 3.3895313892515355e38  # largest finite bf16 (0x7F7F)
+
+# Token kinds of extreme magnitude, for the range tests: name -> what it is.
+EXTREME_KINDS = {
+    "normal": "N(0, 1)",
+    "zeros": "all zero",
+    "big": "N(0, 1) * 2^20 (|x| far beyond fp16's 65504)",
+    "fp16_edge": "N(0, 1) * 2^15 (|x| around and above fp16's 65504)",
+    "near_max": "N(0, 1) * 2^125, clipped to bf16's largest finite value",
+    "all_max": "every element +-U(0.5, 1) * bf16's largest finite value",
+    "subnormal": "every element a random nonzero bf16 subnormal",
+    "tiny": "N(0, 1) * 2^-60",
+    "mixed": "N(0, 1) with 64 positions bf16 subnormals, 16 at N(0, 1) * 2^-100 "
+             "and 4 at +-U(1, 2) * 2^30",
+    "tiny_huge": "every element a bf16 subnormal except 3 at +-U(1, 2) * 2^50",
+}
+
+
+def extreme_token(kind: str, hidden: int = HIDDEN, seed: int = 0) -> torch.Tensor:
+    """One token x [hidden] bf16 of the given kind (EXTREME_KINDS), on the CPU."""
+    g = _gen(seed, "cpu")
+    n = torch.randn(hidden, generator=g, dtype=torch.float64)
+
+    def subnormals(m):
+        mant = torch.randint(1, 128, (m,), generator=g, dtype=torch.int32)
+        sign = torch.randint(0, 2, (m,), generator=g, dtype=torch.int32) << 15
+        return (mant | sign).to(torch.int16).view(torch.bfloat16)
+
+    def positions(m):
+        return torch.randperm(hidden, generator=g)[:m]
+
+    def signs(m):
+        return torch.randint(0, 2, (m,), generator=g, dtype=torch.float64) * 2 - 1
+
+    if kind == "normal":
+        x = n.to(torch.bfloat16)
+    elif kind == "zeros":
+        x = torch.zeros(hidden, dtype=torch.bfloat16)
+    elif kind == "big":
+        x = (n * 2.0 ** 20).to(torch.bfloat16)
+    elif kind == "fp16_edge":
+        x = (n * 2.0 ** 15).to(torch.bfloat16)
+    elif kind == "near_max":
+        x = (n * 2.0 ** 125).clamp(-BF16_MAX, BF16_MAX).to(torch.bfloat16)
+    elif kind == "all_max":
+        u = torch.empty(hidden, dtype=torch.float64).uniform_(0.5, 1.0, generator=g)
+        x = (signs(hidden) * u * BF16_MAX).clamp(-BF16_MAX, BF16_MAX).to(torch.bfloat16)
+    elif kind == "subnormal":
+        x = subnormals(hidden)
+    elif kind == "tiny":
+        x = (n * 2.0 ** -60).to(torch.bfloat16)
+    elif kind == "mixed":
+        x = n.to(torch.bfloat16)
+        p = positions(84)
+        x[p[:64]] = subnormals(64)
+        x[p[64:80]] = (torch.randn(16, generator=g, dtype=torch.float64) * 2.0 ** -100).to(torch.bfloat16)
+        u = torch.empty(4, dtype=torch.float64).uniform_(1.0, 2.0, generator=g)
+        x[p[80:]] = (signs(4) * u * 2.0 ** 30).to(torch.bfloat16)
+    elif kind == "tiny_huge":
+        x = subnormals(hidden)
+        p = positions(3)
+        u = torch.empty(3, dtype=torch.float64).uniform_(1.0, 2.0, generator=g)
+        x[p] = (signs(3) * u * 2.0 ** 50).to(torch.bfloat16)
+    else:
+        raise ValueError(f"unknown token kind {kind!r}")
+    return x
+
+
+def extreme_tokens(kinds, hidden: int = HIDDEN, seed: int = 0, device="cpu") -> torch.Tensor:
+    """Tokens of the given kinds, row i of kinds[i] from seed + i."""
+    return torch.stack([extreme_token(k, hidden, seed + i) for i, k in enumerate(kinds)]).to(device)
+
+
 def token_stream(seeds, hidden: int = HIDDEN, device="cpu") -> torch.Tensor:
     """One token per seed, stacked: row i is tokens(1, seed=seeds[i])."""
     rows = [tokens(1, hidden, s, device) for s in seeds]
