@@ -114,6 +114,11 @@ int ling_moe_create_mxfp4(const ling_moe_config_t *cfg, const ling_moe_weights_t
  * legacy default stream).  x and out are DEVICE pointers owned by the caller,
  * contiguous row-major, 16-byte aligned; out must not overlap x.
  * 0 <= T <= max_tokens; T == 0 returns OK and enqueues nothing.
+ * Range: every finite bf16 x (subnormals and values up to bf16's largest
+ * included) is computed with the same relative precision, through a
+ * power-of-two scale per token; out is the exact result rounded once to bf16,
+ * so +-inf where that result overflows bf16.  Non-finite x is outside the
+ * contract (no trap, no check; the outputs are then undefined).
  * Asynchronous: no host synchronisation and no allocation, so the call can be
  * captured into a CUDA graph.  Device-detected failures (a bounded wait that
  * gave up) are reported later by ling_moe_status.
