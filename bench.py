@@ -41,6 +41,8 @@ WORKLOAD_METRIC = {
     "verify_e512_t4": "MoE-layer verify tokens/s and achieved HBM GB/s (W4 g32, 512e top-8, T=4 per call)",
     "stack40_e512_t1": "40-layer MoE-stack decode tokens/s and achieved HBM GB/s (W4 g32, 512e top-8, T=1)",
     "prefill_e512_t2048_zipf": "MoE-layer prefill tokens/s (W4 g32, 512e top-8, T=2048 per call, Zipf(1.1) routing)",
+    "prefill_e512_t2048_zipf_mxfp4": "MoE-layer prefill tokens/s (MXFP4 e2m1/e8m0, 512e top-8, T=2048 per call, "
+                                     "Zipf(1.1) routing)",
 }
 
 

@@ -103,10 +103,13 @@ int ling_moe_create(const ling_moe_config_t *cfg, const ling_moe_weights_t *w,
  * Weights: as ling_moe_create, except that gate_q / up_q / down_q hold E2M1
  * codes (two per byte, low nibble = even K index) and gate_s / up_s / down_s
  * hold E8M0 scale bytes, uint8 [E, rows, K/32].  Scale exponents above 240
- * (scales of 2^114 and more) are not supported: they give NaN outputs.
- * Limits: as ling_moe_create, plus max_tokens <= 8 (the decode path; the
- * token-grouped path is not built for MXFP4): larger values return
- * UNSUPPORTED.  Every other entry point works on the handle as documented. */
+ * (scales of 2^114 and more) are not supported: they give NaN outputs.  The
+ * token-grouped path (T > 8) feeds the tensor cores exact fp16 weights
+ * value * scale * 2^8, which holds for exponents e in [96, 132] (scales 2^-31
+ * to 2^5); outside that range its weights lose bits or overflow.
+ * Limits: as ling_moe_create.  Every other entry point works on the handle as
+ * documented; both paths (T <= 8 decode launches, T > 8 token-grouped) run
+ * for MXFP4 weights. */
 int ling_moe_create_mxfp4(const ling_moe_config_t *cfg, const ling_moe_weights_t *w,
                           ling_moe_t **out);
 

@@ -146,15 +146,15 @@ def test_lmhead_null_handle_is_rejected_everywhere():
     lm.lib.ling_moe_lmhead_destroy(None)  # no-op
 
 
-def test_create_mxfp4_checks_arguments_and_its_token_limit():
+def test_create_mxfp4_checks_arguments():
     h = ctypes.c_void_p()
     assert lm.lib.ling_moe_create_mxfp4(None, ctypes.byref(_weights()), ctypes.byref(h)) == \
         lm.LING_MOE_ERR_INVALID_ARG
-    rc = lm.lib.ling_moe_create_mxfp4(ctypes.byref(_cfg(max_tokens=9)), ctypes.byref(_weights()), ctypes.byref(h))
-    assert rc == lm.LING_MOE_ERR_UNSUPPORTED and h.value is None
-    assert "MXFP4" in lm.ling_moe_last_error()
     rc = lm.lib.ling_moe_create_mxfp4(ctypes.byref(_cfg(group_size=64)), ctypes.byref(_weights()), ctypes.byref(h))
-    assert rc == lm.LING_MOE_ERR_UNSUPPORTED
+    assert rc == lm.LING_MOE_ERR_UNSUPPORTED and h.value is None
+    rc = lm.lib.ling_moe_create_mxfp4(ctypes.byref(_cfg(top_k=9, num_experts=16)), ctypes.byref(_weights()),
+                                      ctypes.byref(h))
+    assert rc == lm.LING_MOE_ERR_UNSUPPORTED and h.value is None
 
 
 def test_binding_rejects_wrong_tensors_before_any_call():

@@ -28,15 +28,18 @@ def _calls(layer, xs, T):
     return torch.cat(outs), torch.cat(idxs), torch.cat(ws)
 
 
-@pytest.mark.parametrize("T", [1, 2, 3, 4, 5, 8])
+@pytest.mark.parametrize("T", [1, 2, 3, 4, 5, 8, 9, 17, 37, 200])
 def test_mxfp4_reduced_layer_matches_the_oracle(T):
+    """Decode path up to 8 tokens, the token-grouped path above (at T = 200
+    the 32 experts hold ~50 tokens each: tensor-core tiles; at 9..37 both the
+    GEMV kernels and the tiles run)."""
     lw = workloads.layer_weights_mxfp4(32, seed=3, device="cpu")
     host = lw.host_arrays()
     layer = lm.MoELayer({k: (None if v is None else v.to(DEV)) for k, v in lw.tensors().items()},
-                        top_k=8, max_tokens=8, fmt="mxfp4")
+                        top_k=8, max_tokens=max(T, 8), fmt="mxfp4")
     try:
         assert "MXFP4" in layer.describe()
-        xs = workloads.token_stream(range(300, 300 + 4 * T))
+        xs = workloads.token_stream(range(300, 300 + (4 if T <= 8 else 1) * T))
         out, idx, w = _calls(layer, xs.to(DEV), T)
         compare(MX.moe_layer_mxfp4(bits(xs), host, 8), out, idx, w, 8, f"mxfp4 reduced T={T}")
     finally:
@@ -92,3 +95,28 @@ def test_mxfp4_equals_int4_on_weights_both_formats_hold():
     finally:
         a.close()
         b.close()
+
+
+def test_mxfp4_prefill_t2048_zipf_every_output():
+    """The full MXFP4 layer with the Zipf(1.1) router bias at T = 2048 (the
+    prefill workload's shape) against the MXFP4 oracle, every output."""
+    lw = workloads.layer_weights_mxfp4(512, seed=0, device=DEV)
+    host = lw.host_arrays()
+    bias = workloads.zipf_router_bias(512, 1.1, seed=0)
+    wb = dict(lw.tensors())
+    wb["router_bias"] = bias.to(DEV)
+    host["router_bias"] = bias.numpy()
+    layer = lm.MoELayer(wb, top_k=8, max_tokens=2048, fmt="mxfp4")
+    del lw, wb
+    torch.cuda.empty_cache()
+    try:
+        xs = workloads.tokens(2048, seed=20000)
+        n0 = layer.launch_count()
+        out, idx, w = _calls(layer, xs.to(DEV), 2048)
+        assert layer.launch_count() - n0 == 9  # the token-grouped path
+        counts = np.bincount(idx.cpu().numpy().reshape(-1), minlength=512)
+        assert counts.max() > 1000 and ((counts > 0) & (counts <= 8)).any()  # tiles and GEMV both run
+        rep = compare(MX.moe_layer_mxfp4(bits(xs), host, 8), out, idx, w, 8, "mxfp4 prefill T=2048")
+        print("mxfp4 prefill T=2048", rep)
+    finally:
+        layer.close()

@@ -7,7 +7,7 @@ subnormals, tiny tokens whose outputs sit near bf16's smallest values, and
 tokens mixing subnormal, ordinary and huge values.  They run through the
 decode kernel (T = 1 and T = 4), the token-grouped path (T = 37 on the
 32-expert layer, which splits its experts between the GEMV kernels and the
-tensor-core tiles; T = 20 on the full layer) and the MXFP4 decode kernel,
+tensor-core tiles; T = 20 on the full layer) and both MXFP4 paths,
 with and without a router bias, and are compared with the bar of
 tests.parity.compare_range.
 """
@@ -121,14 +121,22 @@ def test_full_layer_extreme_tokens():
 
 @pytest.mark.parametrize("group", range(len(T4_GROUPS)))
 def test_mxfp4_decode_mixed_kinds(group):
+    _mxfp4_case(T4_GROUPS[group], 1400 + 10 * group, f"mxfp4 T=4 {T4_GROUPS[group]}")
+
+
+def test_mxfp4_grouped_t37_every_kind():
+    _mxfp4_case([KINDS[i % len(KINDS)] for i in range(37)], 1500, "mxfp4 grouped T=37")
+
+
+def _mxfp4_case(kinds, seed, label):
     lw = workloads.layer_weights_mxfp4(32, seed=3, device="cpu")
     host = lw.host_arrays()
-    layer = lm.MoELayer(_cuda(lw.tensors()), top_k=8, max_tokens=8, fmt="mxfp4")
+    layer = lm.MoELayer(_cuda(lw.tensors()), top_k=8, max_tokens=64, fmt="mxfp4")
     try:
-        x = workloads.extreme_tokens(T4_GROUPS[group], seed=1400 + 10 * group)
+        x = workloads.extreme_tokens(kinds, seed=seed)
         out, idx, w = _run(layer, x)
         with np.errstate(over="ignore", invalid="ignore", under="ignore"):
             ref = MX.moe_layer_mxfp4(bits(x), host, 8)
-        compare_range(ref, out, idx, w, 8, f"mxfp4 T=4 {T4_GROUPS[group]}")
+        compare_range(ref, out, idx, w, 8, label)
     finally:
         layer.close()

@@ -151,9 +151,6 @@ static int create_impl(const ling_moe_config_t* cfg, const ling_moe_weights_t* w
   if (rc) return rc;
   rc = validate_weights(w);
   if (rc) return rc;
-  if (codec == kCodecMxfp4 && cfg->max_tokens > 2 * kMaxDecodeT)
-    return fail(LING_MOE_ERR_UNSUPPORTED, "MXFP4 weights: max_tokens must be <= %d (no token-grouped path)",
-                2 * kMaxDecodeT);
 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -209,7 +206,7 @@ static int create_impl(const ling_moe_config_t* cfg, const ling_moe_weights_t* w
       return rc;
     }
   }
-  const bool grouped = cfg->max_tokens > kMaxDecodeT && codec == kCodecInt4;
+  const bool grouped = cfg->max_tokens > kMaxDecodeT;
   if (grouped) {
     h->gws.err = h->err;
     e = grouped_alloc(&h->gws, E, K, cfg->max_tokens,
@@ -254,7 +251,7 @@ static int create_impl(const ling_moe_config_t* cfg, const ling_moe_weights_t* w
            w->router_bias ? "yes" : "no", kMaxDecodeT, h->decode_ctas, kDecodeThreads,
            decode_smem_bytes(1), codec == kCodecMxfp4 ? "MXFP4 (E2M1, E8M0 per 32)" : "W4 g32",
            2 * kMaxDecodeT, 2 * kMaxDecodeT,
-           codec == kCodecMxfp4 ? "not built for MXFP4 weights" : grouped_describe());
+           grouped_describe());
   h->desc = buf;
   *out = h;
   return LING_MOE_OK;
@@ -342,6 +339,7 @@ static int forward_impl(ling_moe_t* h, const void* x, int T, void* out, int32_t*
   gp.topk_idx_out = topk_idx;
   gp.topk_w_out = topk_w;
   gp.num_sms = h->num_sms;
+  gp.codec = h->codec;
   int nl = 0;
   e = launch_grouped(gp, h->gws, stream, &nl, h->timing ? h->tev : nullptr);
   h->launches.fetch_add(nl);

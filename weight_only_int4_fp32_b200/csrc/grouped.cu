@@ -459,6 +459,7 @@ cudaError_t launch_grouped(const GroupedParams& p, const GroupedWorkspace& ws, c
   tp.xg = ws.xg;
   tp.shgu16 = ws.shgu16;
   tp.shdn16 = ws.shdn16;
+  tp.codec = p.codec;
   GvParams gv{};
   gv.gu = p.gu;
   gv.dn = p.dn;
@@ -473,6 +474,7 @@ cudaError_t launch_grouped(const GroupedParams& p, const GroupedWorkspace& ws, c
   gv.nsmall = ws.nsmall;
   gv.err = ws.err;
   gv.wait_limit_ns = 2000000000ull;
+  gv.codec = p.codec;
   mark(4);
   if ((e = launch_gemv_gu(gv, p.num_sms, s)) != cudaSuccess) return e;
   ++nl;

@@ -23,6 +23,7 @@ struct GroupedParams {
   int32_t* topk_idx_out;         // optional [T, k]
   float* topk_w_out;             // optional [T, k]
   int num_sms;
+  int codec;                     // kCodecInt4 or kCodecMxfp4 (layout.h)
 };
 
 // Positions: the T*k token-expert pairs sorted by expert occupy positions

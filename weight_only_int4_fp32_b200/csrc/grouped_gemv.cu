@@ -69,6 +69,8 @@ static_assert(kGvDnSmem <= 227 * 1024, "GEMV down shared memory over budget");
 // pieces of 2560 B; as soon as piece pc of round g is consumed, piece pc of
 // round g + 1 is requested into the same slot, and the scales of round g + 1
 // go to the second of two scale slots, so the weights stream continuously.
+// C: the codec of the routed weights (kCodecInt4 or kCodecMxfp4, layout.h).
+template <int C>
 __global__ void __launch_bounds__(kGvThreads, 1) gv_gu_kernel(const GvParams p) {
   extern __shared__ __align__(128) unsigned char sm[];
   uint64_t* mbar = reinterpret_cast<uint64_t*>(sm);
@@ -124,12 +126,15 @@ __global__ void __launch_bounds__(kGvThreads, 1) gv_gu_kernel(const GvParams p) 
       q4 = task % kGvGuTasks;
       __syncthreads();  // the previous task is done with xf
       // x rows of the expert's positions in B-fragment order: per 16-K block kb
-      // and lane class mm, (x[c], x[c+1]) and (x[c+8], x[c+9]) / 16, c = 16 kb + 2 mm
+      // and lane class mm, (x[c], x[c+1]) and (x[c+8], x[c+9]), c = 16 kb + 2 mm;
+      // int4: the second pair / 16 (it meets codes dequantised as 16 q)
       for (int v = tid; v < m * (kH / 4); v += kGvThreads) {
         const int t = v / (kH / 4), rr = v - t * (kH / 4), kb = rr >> 2, c = 16 * kb + 2 * (rr & 3);
         const __half* row = p.xg + (size_t)(pos0 + t) * kH;
         const uint32_t lo = *reinterpret_cast<const uint32_t*>(row + c);
-        const __half2 hi = __hmul2(*reinterpret_cast<const __half2*>(row + c + 8), __float2half2_rn(0.0625f));
+        const __half2 hi = C == kCodecInt4
+                               ? __hmul2(*reinterpret_cast<const __half2*>(row + c + 8), __float2half2_rn(0.0625f))
+                               : *reinterpret_cast<const __half2*>(row + c + 8);
         *reinterpret_cast<uint2*>(xf + t * kGvXfTok + (kb >> 2) * 128 + (rr & 3) * 32 + (kb & 3) * 8) =
             make_uint2(lo, *reinterpret_cast<const uint32_t*>(&hi));
       }
@@ -159,8 +164,18 @@ __global__ void __launch_bounds__(kGvThreads, 1) gv_gu_kernel(const GvParams p) 
         float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-          const uint32_t a0 = deq_q_even(wd[w]), a2 = deq_q_odd16(wd[w]);
-          const uint32_t a1 = deq_q_even(wd[w] >> 8), a3 = deq_q_odd16(wd[w] >> 8);
+          uint32_t a0, a1, a2, a3;
+          if constexpr (C == kCodecMxfp4) {
+            a0 = deq_e2m1<0>(wd[w]);
+            a2 = deq_e2m1<4>(wd[w]);
+            a1 = deq_e2m1<8>(wd[w]);
+            a3 = deq_e2m1<12>(wd[w]);
+          } else {
+            a0 = deq_q_even(wd[w]);
+            a2 = deq_q_odd16(wd[w]);
+            a1 = deq_q_even(wd[w] >> 8);
+            a3 = deq_q_odd16(wd[w] >> 8);
+          }
           if (w & 1) {
             mma_16816(d0, d1, d2, d3, a0, a1, a2, a3, bx[2 * w], bx[2 * w + 1], d0, d1, d2, d3);
             const uint32_t sw = (w == 1) ? s01 : s23;
@@ -241,6 +256,7 @@ __device__ __forceinline__ void gv_dn_issue(const GvParams& p, int gc, unsigned 
   }
 }
 
+template <int C>
 __global__ void __launch_bounds__(kGvThreads, 1) gv_dn_kernel(const GvParams p) {
   extern __shared__ __align__(128) unsigned char sm[];
   uint64_t* mbar = reinterpret_cast<uint64_t*>(sm);  // [buffer][piece]
@@ -295,7 +311,7 @@ __global__ void __launch_bounds__(kGvThreads, 1) gv_dn_kernel(const GvParams p) 
       }
       float r0, r1;
       constexpr int kJ = kDnChunks / kGvDnThirds;
-      dn_unit_mma(units + (size_t)u * kDnUnitBytes, hfl, lane, r0, r1, kJ * th, kJ * th + kJ);
+      dn_unit_mma<C>(units + (size_t)u * kDnUnitBytes, hfl, lane, r0, r1, kJ * th, kJ * th + kJ);
       if (act) *reinterpret_cast<float2*>(part + ((size_t)it * kGvMaxTok + g) * 8 + 2 * c) = make_float2(r0, r1);
     }
     dead = __syncthreads_or(dead);
@@ -322,21 +338,29 @@ __global__ void __launch_bounds__(kGvThreads, 1) gv_dn_kernel(const GvParams p) 
   }
 }
 
-cudaError_t setup_grouped_gemv() {
+template <int C>
+static cudaError_t setup_c() {
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(gv_gu_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGvGuSmem)) !=
+  if ((e = cudaFuncSetAttribute(gv_gu_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGvGuSmem)) !=
       cudaSuccess)
     return e;
-  return cudaFuncSetAttribute(gv_dn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGvDnSmem);
+  return cudaFuncSetAttribute(gv_dn_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGvDnSmem);
+}
+
+cudaError_t setup_grouped_gemv() {
+  const cudaError_t e = setup_c<kCodecInt4>();
+  return e != cudaSuccess ? e : setup_c<kCodecMxfp4>();
 }
 
 cudaError_t launch_gemv_gu(const GvParams& p, int nctas, cudaStream_t s) {
-  gv_gu_kernel<<<nctas, kGvThreads, kGvGuSmem, s>>>(p);
+  if (p.codec == kCodecMxfp4) gv_gu_kernel<kCodecMxfp4><<<nctas, kGvThreads, kGvGuSmem, s>>>(p);
+  else gv_gu_kernel<kCodecInt4><<<nctas, kGvThreads, kGvGuSmem, s>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemv_dn(const GvParams& p, int nctas, cudaStream_t s) {
-  gv_dn_kernel<<<nctas, kGvThreads, kGvDnSmem, s>>>(p);
+  if (p.codec == kCodecMxfp4) gv_dn_kernel<kCodecMxfp4><<<nctas, kGvThreads, kGvDnSmem, s>>>(p);
+  else gv_dn_kernel<kCodecInt4><<<nctas, kGvThreads, kGvDnSmem, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -21,12 +21,13 @@ struct GvParams {
   const int32_t* perm;          // position -> pair id t*k + slot
   const float* topk_w;          // [P] routing weight per pair id
   int k;
-  __half* h16;                  // [rows, 2, I] h * 2^-8 as fp16 hi + lo, natural K order (written here)
-  float* y;                     // [rows, H] routed output per position, times the routing weight
+  __half* h16;                  // [rows, 2, I] (h / c_t^2) * 2^-8 as fp16 hi + lo, natural K order (written here)
+  float* y;                     // [rows, H] routed output per position / c_t^2, times the routing weight
   const int4* small;            // [E] (expert, first position, tokens, 0)
   const int32_t* nsmall;        // number of entries in small
   unsigned int* err;            // sticky device error word
   unsigned long long wait_limit_ns;
+  int codec;                    // kCodecInt4 or kCodecMxfp4 (layout.h)
 };
 
 cudaError_t setup_grouped_gemv();

@@ -167,6 +167,22 @@ __device__ __forceinline__ uint32_t deq_pair(uint32_t v, __half2 s2, __half2 b2)
   return *reinterpret_cast<const uint32_t*>(&r);
 }
 
+// MXFP4: an E2M1 pair as fp16 (value * 2^-14, exact; deq_e2m1) times the
+// group's scale factor f = s * 2^(14 + 8) (s = 2^(e - 127), the stored bf16
+// being s * 2^14), applied as fa * fb with fa = f limited to [2^-14, 2^15] and
+// fb = f / fa, so that both factors are fp16 powers of two and each product is
+// exact: value * s * 2^8 is an fp16 multiple of 2^-24 below 65504 for
+// E8M0 exponents e in [96, 132].
+__device__ __forceinline__ void mx_factors(float f, __half2& fa, __half2& fb) {
+  const float a = fminf(fmaxf(f, 0x1p-14f), 0x1p15f);
+  fa = __float2half2_rn(a);
+  fb = __float2half2_rn(f / a);
+}
+__device__ __forceinline__ uint32_t mx_pair(uint32_t e2m1_pair, __half2 fa, __half2 fb) {
+  const __half2 r = __hmul2(__hmul2(*reinterpret_cast<const __half2*>(&e2m1_pair), fa), fb);
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
 // ---------------------------------------------------------------- shared-expert fp16 copies
 // Power-of-two exponent c with max|w| * 2^c in [2^14, 2^15) (0 for an all-zero
 // matrix), clamped so that 2^c and 2^-c stay normal fp32 numbers.
@@ -272,7 +288,7 @@ __device__ __forceinline__ void prefetch_tile(const TcParams& p, int4 tl, const 
 // Roles: warps 0-7 dequantise A, warps 8-11 drain TMEM, warp 12 issues the
 // MMAs (one thread), warp 13 issues the TMA loads (one thread).  Every role
 // walks the same sequence of tiles (blockIdx.x, + gridDim.x, ...) and stages.
-template <int MODE>
+template <int MODE, int C>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmA,
                   const TcParams p) {
@@ -399,6 +415,11 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
           const __half2 sg = __float2half2_rn(sgf), sg16 = __float2half2_rn(sgf * 0.0625f);
           const __half2 su = __float2half2_rn(suf), su16 = __float2half2_rn(suf * 0.0625f);
           const __half2 be = __float2half2_rn(1032.0f), bo = __float2half2_rn(1152.0f);
+          __half2 ga, gb, ua, ub;
+          if constexpr (C == kCodecMxfp4) {
+            mx_factors(sgf, ga, gb);
+            mx_factors(suf, ua, ub);
+          }
           uint2 cw[4];
 #pragma unroll
           for (int m = 0; m < 4; ++m) cw[m] = *reinterpret_cast<const uint2*>(slot + m * (kProd * 8) + r * 8);
@@ -410,6 +431,13 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
               const uint32_t w = ww ? cw[m].y : cw[m].x;
+              if constexpr (C == kCodecMxfp4) {
+                glo[m] = mx_pair(deq_e2m1<0>(w), ga, gb);   // gate c, c+1
+                ghi[m] = mx_pair(deq_e2m1<4>(w), ga, gb);   // gate c+8, c+9
+                ulo[m] = mx_pair(deq_e2m1<8>(w), ua, ub);   // up c, c+1
+                uhi[m] = mx_pair(deq_e2m1<12>(w), ua, ub);  // up c+8, c+9
+                continue;
+              }
               uint32_t v0, v1, v2, v3;
               asm("lop3.b32 %0, %1, 0x000F000F, 0x64006400, 0xEA;" : "=r"(v0) : "r"(w));
               asm("lop3.b32 %0, %1, 0x00F000F0, 0x64006400, 0xEA;" : "=r"(v1) : "r"(w));
@@ -442,10 +470,19 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
             const uint32_t ws = h ? sw.y : sw.x;
             const float sf = __uint_as_float((n & 1) ? (ws & 0xFFFF0000u) : (ws << 16)) * (float)(1 << kTcScaleShift);
             const __half2 s2 = __float2half2_rn(sf), s16 = __float2half2_rn(sf * 0.0625f);
+            __half2 fa, fb;
+            if constexpr (C == kCodecMxfp4) mx_factors(sf, fa, fb);
             uint32_t q0[4], q1[4], q2[4], q3[4];
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
               const uint32_t w = h ? cw[m].y : cw[m].x;
+              if constexpr (C == kCodecMxfp4) {
+                q0[m] = mx_pair(deq_e2m1<0>(w), fa, fb);   // K c, c+1
+                q1[m] = mx_pair(deq_e2m1<4>(w), fa, fb);   // c+8, c+9
+                q2[m] = mx_pair(deq_e2m1<8>(w), fa, fb);   // c+16, c+17
+                q3[m] = mx_pair(deq_e2m1<12>(w), fa, fb);  // c+24, c+25
+                continue;
+              }
               uint32_t v0, v1, v2, v3;
               asm("lop3.b32 %0, %1, 0x000F000F, 0x64006400, 0xEA;" : "=r"(v0) : "r"(w));
               asm("lop3.b32 %0, %1, 0x00F000F0, 0x64006400, 0xEA;" : "=r"(v1) : "r"(w));
@@ -635,12 +672,19 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
 }
 
 // ---------------------------------------------------------------- host
-cudaError_t setup_grouped_tc() {
+template <int C>
+static cudaError_t setup_c() {
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(tc_grouped_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if ((e = cudaFuncSetAttribute(tc_grouped_kernel<0, C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)tc_smem(0))) != cudaSuccess)
     return e;
-  return cudaFuncSetAttribute(tc_grouped_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_smem(1));
+  return cudaFuncSetAttribute(tc_grouped_kernel<1, C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)tc_smem(1));
+}
+
+cudaError_t setup_grouped_tc() {
+  const cudaError_t e = setup_c<kCodecInt4>();
+  return e != cudaSuccess ? e : setup_c<kCodecMxfp4>();
 }
 
 namespace {
@@ -686,8 +730,13 @@ cudaError_t tc_encode_maps(TcMaps* m, const __half* xg, const __half* h16, int r
 }
 
 cudaError_t launch_tc_gemm(int mode, const TcMaps& m, const TcParams& p, int nctas, cudaStream_t s) {
-  if (mode == 0) tc_grouped_kernel<0><<<nctas, kTcThreads, tc_smem(0), s>>>(m.b_x, m.a_shgu, p);
-  else tc_grouped_kernel<1><<<nctas, kTcThreads, tc_smem(1), s>>>(m.b_h, m.a_shdn, p);
+  if (p.codec == kCodecMxfp4) {
+    if (mode == 0) tc_grouped_kernel<0, kCodecMxfp4><<<nctas, kTcThreads, tc_smem(0), s>>>(m.b_x, m.a_shgu, p);
+    else tc_grouped_kernel<1, kCodecMxfp4><<<nctas, kTcThreads, tc_smem(1), s>>>(m.b_h, m.a_shdn, p);
+  } else {
+    if (mode == 0) tc_grouped_kernel<0, kCodecInt4><<<nctas, kTcThreads, tc_smem(0), s>>>(m.b_x, m.a_shgu, p);
+    else tc_grouped_kernel<1, kCodecInt4><<<nctas, kTcThreads, tc_smem(1), s>>>(m.b_h, m.a_shdn, p);
+  }
   return cudaGetLastError();
 }
 

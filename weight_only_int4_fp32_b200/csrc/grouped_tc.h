@@ -45,6 +45,7 @@ struct TcParams {
   const int32_t* ntiles;    // [0] gate/up tiles, [1] down tiles
   unsigned int* err;        // sticky device error word
   const __half* xg;         // the buffers behind the tensor maps (for L2 prefetch)
+  int codec;                // kCodecInt4 or kCodecMxfp4 (layout.h)
   const __half* shgu16;
   const __half* shdn16;
 };

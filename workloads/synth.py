@@ -286,6 +286,10 @@ WORKLOADS = {
     "decode_e512_t1_mxfp4": dict(num_experts=512, T=1, weight_seed=0, fmt="mxfp4",
                                  token_seeds=[1 + t for t in range(1000)],
                                  note="full layer with MXFP4 routed experts, batch-1 decode, token t from seed 1+t"),
+    "prefill_e512_t2048_zipf_mxfp4": dict(num_experts=512, T=2048, weight_seed=0, token_seed=20000,
+                                          zipf_s=1.1, fmt="mxfp4",
+                                          note="full layer with MXFP4 routed experts, 2048-token prefill chunk, "
+                                               "Zipf(1.1) router bias"),
 }
 
 
