@@ -145,6 +145,56 @@ int ling_moe_forward_ex(ling_moe_t *h, const void *x, int T, void *out,
 int ling_moe_forward_host(ling_moe_t *h, const void *x_host, int T, void *out_host,
                           void *stream);
 
+/* ---- Expert parallel: the layer's experts partitioned over several GPUs.
+ * The pages run the model as TP4 + EP4 on four H200s with vLLM's
+ * --enable-expert-parallel (vLLM recipe page "inclusionAI/Ling-3.0-flash",
+ * section "Launching the Server"); they give no kernel-level definition.
+ * Here each GPU (rank) holds the full router and a contiguous range of the
+ * routed experts, and one rank also holds the shared expert.  Every rank
+ * scores all experts and selects the same top-k with the same weights; it
+ * computes only the terms of the selected experts it holds (plus the shared
+ * expert where it lives) and returns their sum in fp32.  The sum of all ranks'
+ * partial outputs (an all-reduce) rounded once to bf16 (ling_moe_round_bf16)
+ * is the layer's output. */
+typedef enum { LING_MOE_FORMAT_INT4 = 0, LING_MOE_FORMAT_MXFP4 = 1 } ling_moe_format_t;
+
+typedef struct {
+  int expert_begin; /* first expert held here, 0 <= expert_begin */
+  int expert_count; /* experts held here, >= 1, expert_begin + expert_count <= num_experts */
+  int with_shared;  /* 1: this handle also computes the shared expert; 0: it does not */
+  int format;       /* ling_moe_format_t of the routed weights */
+} ling_moe_ep_t;
+
+/* An expert-parallel handle.  cfg->num_experts is the number of experts the
+ * router scores (all ranks together).  w->router_w [num_experts, H] and
+ * w->router_bias [num_experts] are the full router; gate_q / gate_s / up_q /
+ * up_s / down_q / down_s hold only the expert_count experts held here, in
+ * the layouts of ling_moe_create (int4) or ling_moe_create_mxfp4 (MXFP4)
+ * with E = expert_count; sh_gate / sh_up / sh_down are read only when
+ * with_shared = 1 (they may be NULL otherwise).  Copies what it needs, as
+ * ling_moe_create does.  Such a handle serves ling_moe_forward_partial;
+ * ling_moe_forward / _forward_ex / _forward_host return INVALID_ARG on it.
+ * Errors: as ling_moe_create; INVALID_ARG for a range outside
+ * [0, num_experts), with_shared not 0/1 or an unknown format. */
+int ling_moe_create_ep(const ling_moe_config_t *cfg, const ling_moe_weights_t *w,
+                       const ling_moe_ep_t *ep, ling_moe_t **out);
+
+/* partial[T, H] (fp32, DEVICE, 16-byte aligned, not overlapping x) = the sum,
+ * in fp32, of the routed terms w_e * Wd_e(...) of the selected experts this
+ * handle holds (slot order) plus its shared-expert term, before any bf16
+ * rounding.  On a handle from ling_moe_create it is the whole layer in fp32.
+ * topk_idx / topk_w as in ling_moe_forward_ex: every selected expert, held
+ * here or not (global indices).  Same kernels, asynchrony and errors as
+ * ling_moe_forward. */
+int ling_moe_forward_partial(ling_moe_t *h, const void *x, int T, float *partial,
+                             int32_t *topk_idx, float *topk_w, void *stream);
+
+/* out[i] (bf16) = in[i] (fp32) rounded to nearest even, i < n, on `stream`:
+ * the one rounding of the layer's output once the ranks' partial sums are
+ * added.  DEVICE pointers, 16-byte aligned, not overlapping; n a multiple of
+ * 8.  One launch; asynchronous.  Errors: INVALID_ARG, CUDA. */
+int ling_moe_round_bf16(const float *in, void *out, size_t n, void *stream);
+
 /* Synchronise `stream` and return the handle's sticky device error
  * (OK or DEVICE_TIMEOUT), or CUDA if the synchronisation itself failed. */
 int ling_moe_status(ling_moe_t *h, void *stream);

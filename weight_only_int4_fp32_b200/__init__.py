@@ -20,7 +20,9 @@ __all__ = [
     "ling_moe_status", "ling_moe_describe", "ling_moe_launch_count", "ling_moe_last_error",
     "ling_moe_destroy", "ling_moe_test_set_wait", "ling_moe_route_noalloc", "ling_moe_route_noalloc_status",
     "ling_moe_route_noalloc_test_set_wait", "ling_moe_set_kernel_timing",
-    "ling_moe_kernel_times", "MoELayer", "LMHeadFP8", "EXPORTED",
+    "ling_moe_kernel_times", "ling_moe_ep_t", "ling_moe_create_ep", "ling_moe_forward_partial",
+    "ling_moe_round_bf16", "LING_MOE_FORMAT_INT4", "LING_MOE_FORMAT_MXFP4", "round_bf16",
+    "MoELayer", "LMHeadFP8", "EXPORTED",
 ]
 
 LING_MOE_OK = 0
@@ -29,6 +31,8 @@ LING_MOE_ERR_CUDA = -2
 LING_MOE_ERR_OOM = -3
 LING_MOE_ERR_UNSUPPORTED = -4
 LING_MOE_ERR_DEVICE_TIMEOUT = -5
+LING_MOE_FORMAT_INT4 = 0
+LING_MOE_FORMAT_MXFP4 = 1
 
 # every symbol include/ling_moe.h declares
 EXPORTED = (
@@ -36,7 +40,8 @@ EXPORTED = (
     "ling_moe_forward_host", "ling_moe_status", "ling_moe_describe", "ling_moe_launch_count",
     "ling_moe_last_error", "ling_moe_destroy", "ling_moe_test_set_wait", "ling_moe_route_noalloc",
     "ling_moe_route_noalloc_status", "ling_moe_route_noalloc_test_set_wait", "ling_moe_set_kernel_timing",
-    "ling_moe_kernel_times", "ling_moe_kernel_name",
+    "ling_moe_kernel_times", "ling_moe_kernel_name", "ling_moe_create_ep", "ling_moe_forward_partial",
+    "ling_moe_round_bf16",
     "ling_moe_lmhead_create", "ling_moe_lmhead_forward", "ling_moe_lmhead_forward_ex",
     "ling_moe_lmhead_forward_host", "ling_moe_lmhead_weights", "ling_moe_lmhead_status",
     "ling_moe_lmhead_launch_count", "ling_moe_lmhead_destroy", "ling_moe_lmhead_test_set_wait",
@@ -66,6 +71,11 @@ class ling_moe_weights_t(ctypes.Structure):
         "sh_gate", "sh_up", "sh_down")]
 
 
+class ling_moe_ep_t(ctypes.Structure):
+    _fields_ = [("expert_begin", ctypes.c_int), ("expert_count", ctypes.c_int), ("with_shared", ctypes.c_int),
+                ("format", ctypes.c_int)]
+
+
 _LIB = None
 
 
@@ -90,6 +100,10 @@ def _load():
                                  ctypes.POINTER(vp)]),
         "ling_moe_create_mxfp4": (ci, [ctypes.POINTER(ling_moe_config_t), ctypes.POINTER(ling_moe_weights_t),
                                        ctypes.POINTER(vp)]),
+        "ling_moe_create_ep": (ci, [ctypes.POINTER(ling_moe_config_t), ctypes.POINTER(ling_moe_weights_t),
+                                    ctypes.POINTER(ling_moe_ep_t), ctypes.POINTER(vp)]),
+        "ling_moe_forward_partial": (ci, [vp, vp, ci, vp, vp, vp, vp]),
+        "ling_moe_round_bf16": (ci, [vp, vp, ctypes.c_size_t, vp]),
         "ling_moe_forward": (ci, [vp, vp, ci, vp, vp]),
         "ling_moe_forward_ex": (ci, [vp, vp, ci, vp, vp, vp, vp]),
         "ling_moe_forward_host": (ci, [vp, vp, ci, vp, vp]),
@@ -154,6 +168,21 @@ def ling_moe_create_mxfp4(cfg: ling_moe_config_t, weights: ling_moe_weights_t) -
     h = ctypes.c_void_p()
     _check(lib.ling_moe_create_mxfp4(ctypes.byref(cfg), ctypes.byref(weights), ctypes.byref(h)))
     return h.value
+
+
+def ling_moe_create_ep(cfg: ling_moe_config_t, weights: ling_moe_weights_t, ep: ling_moe_ep_t) -> int:
+    h = ctypes.c_void_p()
+    _check(lib.ling_moe_create_ep(ctypes.byref(cfg), ctypes.byref(weights), ctypes.byref(ep), ctypes.byref(h)))
+    return h.value
+
+
+def ling_moe_forward_partial(h: int, x: int, T: int, partial: int, topk_idx: int = None, topk_w: int = None,
+                             stream: int = 0) -> int:
+    return _check(lib.ling_moe_forward_partial(h, x, T, partial, topk_idx, topk_w, stream))
+
+
+def ling_moe_round_bf16(inp: int, out: int, n: int, stream: int = 0) -> int:
+    return _check(lib.ling_moe_round_bf16(inp, out, n, stream))
 
 
 def ling_moe_set_kernel_timing(h: int, on: bool) -> int:
@@ -232,6 +261,20 @@ def _require(t, shape, dtype, cuda: bool, name: str):
                          f"got {t.dtype} {tuple(t.shape)} on {t.device}")
 
 
+def round_bf16(partial, out=None, stream=None):
+    """bf16 round-to-nearest-even of an fp32 CUDA tensor (ling_moe_round_bf16):
+    the last step of an expert-parallel combine."""
+    import torch
+    if not partial.is_cuda or partial.dtype != torch.float32 or not partial.is_contiguous():
+        raise ValueError("partial must be a contiguous CUDA float32 tensor")
+    if out is None:
+        out = torch.empty(partial.shape, dtype=torch.bfloat16, device=partial.device)
+    _require(out, tuple(partial.shape), torch.bfloat16, True, "out")
+    s = torch.cuda.current_stream().cuda_stream if stream is None else getattr(stream, "cuda_stream", stream)
+    ling_moe_round_bf16(partial.data_ptr(), out.data_ptr(), partial.numel(), s)
+    return out
+
+
 class MoELayer:
     """One MoE layer on the current CUDA device, built from torch tensors.
 
@@ -242,11 +285,15 @@ class MoELayer:
     """
 
     def __init__(self, weights: dict, top_k: int = 8, max_tokens: int = 1, group_size: int = 32,
-                 fmt: str = "int4"):
+                 fmt: str = "int4", ep: tuple | None = None):
+        """ep = (expert_begin, expert_count, with_shared): an expert-parallel
+        handle (ling_moe_create_ep) whose routed weights hold only experts
+        [expert_begin, expert_begin + expert_count) of the router's E; it
+        serves forward_partial only."""
         import torch  # device memory and streams only
         rw = weights["router_w"]
         E, H = rw.shape
-        I = weights["sh_gate"].shape[0]
+        I = (weights["sh_gate"] if weights.get("sh_gate") is not None else weights["gate_q"][0]).shape[0]
         for k, v in weights.items():
             if v is not None and (not v.is_cuda or not v.is_contiguous()):
                 raise ValueError(f"{k} must be a contiguous CUDA tensor")
@@ -256,7 +303,14 @@ class MoELayer:
         self.E, self.H, self.I, self.k, self.max_tokens = E, H, I, top_k, max_tokens
         if fmt not in ("int4", "mxfp4"):
             raise ValueError("fmt must be 'int4' or 'mxfp4'")
-        self.handle = (ling_moe_create_mxfp4 if fmt == "mxfp4" else ling_moe_create)(cfg, w)
+        self.ep = ep
+        if ep is not None:
+            b, n, sh = ep
+            spec = ling_moe_ep_t(int(b), int(n), int(bool(sh)),
+                                 LING_MOE_FORMAT_MXFP4 if fmt == "mxfp4" else LING_MOE_FORMAT_INT4)
+            self.handle = ling_moe_create_ep(cfg, w, spec)
+        else:
+            self.handle = (ling_moe_create_mxfp4 if fmt == "mxfp4" else ling_moe_create)(cfg, w)
         self._torch = torch
 
     def _stream(self, stream):
@@ -284,6 +338,27 @@ class MoELayer:
         return out
 
     __call__ = forward
+
+    def forward_partial(self, x, out=None, stream=None, return_routing: bool = False):
+        """fp32 [T, hidden]: the sum of the terms this handle computes (all of
+        the layer on an ordinary handle), before the bf16 rounding."""
+        torch = self._torch
+        if x.dim() != 2:
+            raise ValueError("x must be 2-D [T, hidden]")
+        T = x.shape[0]
+        _require(x, (T, self.H), torch.bfloat16, True, "x")
+        if out is None:
+            out = torch.empty((T, self.H), dtype=torch.float32, device=x.device)
+        _require(out, (T, self.H), torch.float32, True, "out")
+        s = self._stream(stream)
+        idx = w = None
+        if return_routing:
+            idx = torch.empty((T, self.k), dtype=torch.int32, device=x.device)
+            w = torch.empty((T, self.k), dtype=torch.float32, device=x.device)
+        ling_moe_forward_partial(self.handle, x.data_ptr(), T, out.data_ptr(),
+                                 idx.data_ptr() if idx is not None else None,
+                                 w.data_ptr() if w is not None else None, s)
+        return (out, idx, w) if return_routing else out
 
     def forward_host(self, x_host, out_host=None, stream=None):
         torch = self._torch

@@ -16,6 +16,7 @@
 #include "grouped.h"
 #include "lmhead.h"
 #include "repack.h"
+#include "ep.h"
 
 using namespace lingmoe;
 
@@ -56,6 +57,11 @@ void set_last_error(const char* msg) { g_last_error = msg; }
 struct ling_moe {
   ling_moe_config_t cfg{};
   int codec = kCodecInt4;  // routed-weight format
+  // expert parallel: routed weights of experts [e0, e0 + e_local) of the
+  // num_experts the router scores; the shared expert is computed iff shared_on
+  int e0 = 0, e_local = 0;
+  int shared_on = 1;
+  bool partial_only = false;  // an expert-parallel handle: forward_partial only
   int device = 0;
   int num_sms = 0;
   int decode_ctas = 0;
@@ -125,9 +131,10 @@ int validate_cfg(const ling_moe_config_t* c) {
   return LING_MOE_OK;
 }
 
-int validate_weights(const ling_moe_weights_t* w) {
-  const void* req[] = {w->router_w, w->gate_q, w->gate_s, w->up_q, w->up_s,
-                       w->down_q,   w->down_s, w->sh_gate, w->sh_up, w->sh_down};
+int validate_weights(const ling_moe_weights_t* w, bool shared) {
+  const void* req[] = {w->router_w, w->gate_q, w->gate_s, w->up_q, w->up_s, w->down_q, w->down_s,
+                       shared ? w->sh_gate : w->router_w, shared ? w->sh_up : w->router_w,
+                       shared ? w->sh_down : w->router_w};
   for (const void* p : req)
     if (!p) return fail(LING_MOE_ERR_INVALID_ARG, "a required weight pointer is NULL");
   for (const void* p : req)
@@ -143,13 +150,20 @@ extern "C" {
 
 const char* ling_moe_last_error(void) { return g_last_error.c_str(); }
 
-static int create_impl(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, int codec, ling_moe_t** out) {
+static int create_impl(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, int codec,
+                       const ling_moe_ep_t* ep, ling_moe_t** out) {
   if (!out) return fail(LING_MOE_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
   if (!cfg || !w) return fail(LING_MOE_ERR_INVALID_ARG, "cfg or weights is NULL");
   int rc = validate_cfg(cfg);
   if (rc) return rc;
-  rc = validate_weights(w);
+  if (ep && (ep->expert_begin < 0 || ep->expert_count < 1 ||
+             ep->expert_begin > cfg->num_experts - ep->expert_count || (ep->with_shared & ~1)))
+    return fail(LING_MOE_ERR_INVALID_ARG, "expert range [%d, %d + %d) outside [0, %d) or with_shared not 0/1",
+                ep ? ep->expert_begin : 0, ep ? ep->expert_begin : 0, ep ? ep->expert_count : 0,
+                cfg->num_experts);
+  const bool shared = !ep || ep->with_shared;
+  rc = validate_weights(w, shared);
   if (rc) return rc;
 
   int dev = 0;
@@ -178,17 +192,22 @@ static int create_impl(const ling_moe_config_t* cfg, const ling_moe_weights_t* w
   h->num_sms = prop.multiProcessorCount;
   h->decode_ctas = prop.multiProcessorCount;
   h->decode_T = cfg->max_tokens < kMaxDecodeT ? cfg->max_tokens : kMaxDecodeT;
+  h->e0 = ep ? ep->expert_begin : 0;
+  h->e_local = ep ? ep->expert_count : cfg->num_experts;
+  h->shared_on = shared ? 1 : 0;
+  h->partial_only = ep != nullptr;
 
-  const int E = cfg->num_experts, K = cfg->top_k;
+  const int E = cfg->num_experts, K = cfg->top_k, EL = h->e_local;
+  const size_t shb = shared ? 1 : 0;
   const size_t bf = sizeof(__nv_bfloat16);
   struct A { void** p; size_t n; } plan[] = {
       {(void**)&h->router_w, (size_t)E * kH * bf},
       {(void**)&h->router_bias, w->router_bias ? (size_t)E * sizeof(float) : 0},
-      {(void**)&h->gu, (size_t)E * kGuExpertBytes},
-      {(void**)&h->dn, (size_t)E * kDnExpertBytes},
-      {(void**)&h->sh_gate, (size_t)kI * kH * bf},
-      {(void**)&h->sh_up, (size_t)kI * kH * bf},
-      {(void**)&h->sh_down, (size_t)kH * kI * bf},
+      {(void**)&h->gu, (size_t)EL * kGuExpertBytes},
+      {(void**)&h->dn, (size_t)EL * kDnExpertBytes},
+      {(void**)&h->sh_gate, shb * kI * kH * bf},
+      {(void**)&h->sh_up, shb * kI * kH * bf},
+      {(void**)&h->sh_down, shb * kH * kI * bf},
       {(void**)&h->logits, (size_t)h->decode_T * E * sizeof(float)},
       {(void**)&h->h_s, (size_t)h->decode_T * kI * sizeof(float)},
       {(void**)&h->h_pair, (size_t)h->decode_T * K * kI * sizeof(float)},
@@ -224,15 +243,18 @@ static int create_impl(const ling_moe_config_t* cfg, const ling_moe_weights_t* w
   if (e == cudaSuccess) e = cudaMemcpyAsync(h->router_w, w->router_w, (size_t)E * kH * bf, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess && w->router_bias)
     e = cudaMemcpyAsync(h->router_bias, w->router_bias, (size_t)E * sizeof(float), cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(h->sh_gate, w->sh_gate, (size_t)kI * kH * bf, cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(h->sh_up, w->sh_up, (size_t)kI * kH * bf, cudaMemcpyDeviceToDevice, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(h->sh_down, w->sh_down, (size_t)kH * kI * bf, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && shared)
+    e = cudaMemcpyAsync(h->sh_gate, w->sh_gate, (size_t)kI * kH * bf, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && shared)
+    e = cudaMemcpyAsync(h->sh_up, w->sh_up, (size_t)kI * kH * bf, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && shared)
+    e = cudaMemcpyAsync(h->sh_down, w->sh_down, (size_t)kH * kI * bf, cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->sync, 0, 4 * sizeof(unsigned long long), s);
   if (e == cudaSuccess) e = cudaMemsetAsync(h->err, 0, 4 * sizeof(unsigned int), s);
   if (e == cudaSuccess)
-    e = launch_repack(w->gate_q, w->up_q, w->gate_s, w->up_s, w->down_q, w->down_s, h->gu, h->dn, E, codec, s);
+    e = launch_repack(w->gate_q, w->up_q, w->gate_s, w->up_s, w->down_q, w->down_s, h->gu, h->dn, EL, codec, s);
   if (e == cudaSuccess && grouped)
-    e = grouped_prepare(&h->gws, E, h->sh_gate, h->sh_up, h->sh_down, s);
+    e = grouped_prepare(&h->gws, E, shared ? h->sh_gate : nullptr, h->sh_up, h->sh_down, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (s) cudaStreamDestroy(s);
   if (e != cudaSuccess) {
@@ -242,13 +264,20 @@ static int create_impl(const ling_moe_config_t* cfg, const ling_moe_weights_t* w
     return rc;
   }
 
-  char buf[1024];
+  std::string ep_desc;
+  if (ep) {
+    char eb[160];
+    snprintf(eb, sizeof(eb), " | expert parallel: experts [%d, %d) of %d, shared expert %s, fp32 partial output",
+             h->e0, h->e0 + h->e_local, E, shared ? "here" : "elsewhere");
+    ep_desc = eb;
+  }
+  char buf[1200];
   snprintf(buf, sizeof(buf),
-           "ling_moe sm_%d%d %d SMs | H=%d I=%d E=%d k=%d g=%d max_tokens=%d bias=%s | "
+           "ling_moe sm_%d%d %d SMs | H=%d I=%d E=%d k=%d g=%d max_tokens=%d bias=%s%s | "
            "decode path (1<=T<=%d): 1 cooperative launch grid=%dx%d smem=%zuB, %s GEMV "
            "dequant-in-register, fp32 accumulate (T<=%d: 2 such launches) | grouped path (T>%d): %s",
            prop.major, prop.minor, h->num_sms, kH, kI, E, K, kGroup, cfg->max_tokens,
-           w->router_bias ? "yes" : "no", kMaxDecodeT, h->decode_ctas, kDecodeThreads,
+           w->router_bias ? "yes" : "no", ep_desc.c_str(), kMaxDecodeT, h->decode_ctas, kDecodeThreads,
            decode_smem_bytes(1), codec == kCodecMxfp4 ? "MXFP4 (E2M1, E8M0 per 32)" : "W4 g32",
            2 * kMaxDecodeT, 2 * kMaxDecodeT,
            grouped_describe());
@@ -258,16 +287,27 @@ static int create_impl(const ling_moe_config_t* cfg, const ling_moe_weights_t* w
 }
 
 int ling_moe_create(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, ling_moe_t** out) {
-  return create_impl(cfg, w, kCodecInt4, out);
+  return create_impl(cfg, w, kCodecInt4, nullptr, out);
 }
 
 int ling_moe_create_mxfp4(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, ling_moe_t** out) {
-  return create_impl(cfg, w, kCodecMxfp4, out);
+  return create_impl(cfg, w, kCodecMxfp4, nullptr, out);
 }
 
+int ling_moe_create_ep(const ling_moe_config_t* cfg, const ling_moe_weights_t* w, const ling_moe_ep_t* ep,
+                       ling_moe_t** out) {
+  if (!ep) return fail(LING_MOE_ERR_INVALID_ARG, "ep is NULL");
+  if (ep->format != LING_MOE_FORMAT_INT4 && ep->format != LING_MOE_FORMAT_MXFP4)
+    return fail(LING_MOE_ERR_INVALID_ARG, "ep->format must be LING_MOE_FORMAT_INT4 or LING_MOE_FORMAT_MXFP4");
+  return create_impl(cfg, w, ep->format == LING_MOE_FORMAT_MXFP4 ? kCodecMxfp4 : kCodecInt4, ep, out);
+}
+
+// out: bf16 [T, H], or (partial) fp32 [T, H]
 static int forward_impl(ling_moe_t* h, const void* x, int T, void* out, int32_t* topk_idx,
-                        float* topk_w, void* stream_v) {
+                        float* topk_w, void* stream_v, bool partial = false) {
   if (!h) return fail(LING_MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (h->partial_only && !partial)
+    return fail(LING_MOE_ERR_INVALID_ARG, "an expert-parallel handle computes partial sums: use ling_moe_forward_partial");
   if (T < 0 || T > h->cfg.max_tokens)
     return fail(LING_MOE_ERR_INVALID_ARG, "T=%d outside [0, max_tokens=%d]", T, h->cfg.max_tokens);
   if (T == 0) return LING_MOE_OK;
@@ -275,7 +315,8 @@ static int forward_impl(ling_moe_t* h, const void* x, int T, void* out, int32_t*
   if (!aligned16(x) || !aligned16(out))
     return fail(LING_MOE_ERR_INVALID_ARG, "x and out must be 16-byte aligned");
   const size_t nbytes = (size_t)T * kH * sizeof(__nv_bfloat16);
-  if (overlaps(x, nbytes, out, nbytes)) return fail(LING_MOE_ERR_INVALID_ARG, "out overlaps x");
+  if (overlaps(x, nbytes, out, partial ? 2 * nbytes : nbytes)) return fail(LING_MOE_ERR_INVALID_ARG, "out overlaps x");
+  float* out_f32 = partial ? static_cast<float*>(out) : nullptr;
   if ((topk_idx && (reinterpret_cast<uintptr_t>(topk_idx) & 3)) ||
       (topk_w && (reinterpret_cast<uintptr_t>(topk_w) & 3)))
     return fail(LING_MOE_ERR_INVALID_ARG, "topk outputs must be 4-byte aligned");
@@ -293,7 +334,11 @@ static int forward_impl(ling_moe_t* h, const void* x, int T, void* out, int32_t*
       const int t0 = c * kMaxDecodeT, Tc = c == 0 ? (T < kMaxDecodeT ? T : kMaxDecodeT) : T - kMaxDecodeT;
       DecodeParams p{};
       p.x = static_cast<const __nv_bfloat16*>(x) + (size_t)t0 * kH;
-      p.out = static_cast<__nv_bfloat16*>(out) + (size_t)t0 * kH;
+      p.out = partial ? nullptr : static_cast<__nv_bfloat16*>(out) + (size_t)t0 * kH;
+      p.out_f32 = partial ? out_f32 + (size_t)t0 * kH : nullptr;
+      p.e0 = h->e0;
+      p.e_local = h->e_local;
+      p.shared_on = h->shared_on;
       p.T = Tc;
       p.E = h->cfg.num_experts;
       p.k = h->cfg.top_k;
@@ -328,7 +373,11 @@ static int forward_impl(ling_moe_t* h, const void* x, int T, void* out, int32_t*
   }
   GroupedParams gp{};
   gp.x = static_cast<const __nv_bfloat16*>(x);
-  gp.out = static_cast<__nv_bfloat16*>(out);
+  gp.out = partial ? nullptr : static_cast<__nv_bfloat16*>(out);
+  gp.out_f32 = out_f32;
+  gp.e0 = h->e0;
+  gp.e_local = h->e_local;
+  gp.shared_on = h->shared_on;
   gp.T = T;
   gp.E = h->cfg.num_experts;
   gp.k = h->cfg.top_k;
@@ -360,8 +409,26 @@ int ling_moe_forward_ex(ling_moe_t* h, const void* x, int T, void* out, int32_t*
   return forward_impl(h, x, T, out, topk_idx, topk_w, stream);
 }
 
+int ling_moe_forward_partial(ling_moe_t* h, const void* x, int T, float* partial, int32_t* topk_idx,
+                             float* topk_w, void* stream) {
+  return forward_impl(h, x, T, partial, topk_idx, topk_w, stream, true);
+}
+
+int ling_moe_round_bf16(const float* in, void* out, size_t n, void* stream) {
+  if (n == 0) return LING_MOE_OK;
+  if (!in || !out) return fail(LING_MOE_ERR_INVALID_ARG, "in or out is NULL");
+  if (!aligned16(in) || !aligned16(out) || (n & 7))
+    return fail(LING_MOE_ERR_INVALID_ARG, "in and out must be 16-byte aligned and n a multiple of 8");
+  if (overlaps(in, n * sizeof(float), out, n * sizeof(__nv_bfloat16)))
+    return fail(LING_MOE_ERR_INVALID_ARG, "out overlaps in");
+  const cudaError_t e = launch_round_bf16(in, static_cast<__nv_bfloat16*>(out), n, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LING_MOE_OK : cuda_fail(e, "round launch");
+}
+
 int ling_moe_forward_host(ling_moe_t* h, const void* x_host, int T, void* out_host, void* stream_v) {
   if (!h) return fail(LING_MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (h->partial_only)
+    return fail(LING_MOE_ERR_INVALID_ARG, "an expert-parallel handle computes partial sums: use ling_moe_forward_partial");
   if (T < 0 || T > h->cfg.max_tokens)
     return fail(LING_MOE_ERR_INVALID_ARG, "T=%d outside [0, max_tokens=%d]", T, h->cfg.max_tokens);
   if (T == 0) return LING_MOE_OK;

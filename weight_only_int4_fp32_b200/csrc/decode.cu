@@ -187,7 +187,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   const int s0 = cta * kI / ncta, s1 = (cta + 1) * kI / ncta;
   const int b0 = cta * kDnUnits / ncta, b1 = (cta + 1) * kDnUnits / ncta;
   const int nblk = b1 - b0;
-  const int nr = r1 - r0, n12 = nr + (s1 - s0);
+  const int nr = r1 - r0, n12 = nr + (p.shared_on ? s1 - s0 : 0);
+  const bool ep = p.e_local != E;  // only experts [e0, e0 + e_local) are computed here
 
   uint64_t* barA = &hd.mbar[warp][0];  // phases 1-2 items, piece 0 of a gate/up unit, phase-4 copies
   uint32_t pha = 0, phq = 0;           // phq: parity of pieces 1-3 (always used together)
@@ -238,7 +239,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   if (warp < n12) issue12(warp);
 
   // L2 prefetch of the shared down rows this CTA will need
-  if (warp == kWarps - 1 && lane == 0 && nblk > 0)
+  if (p.shared_on && warp == kWarps - 1 && lane == 0 && nblk > 0)
     prefetch_l2_bulk(p.sh_down + (size_t)b0 * kDnUnitRows * kI, (uint32_t)nblk * 2 * kShDnBytes);
 
   // x (bf16) lands in shared memory; every warp waits for it once
@@ -394,7 +395,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   }
   __syncthreads();
   LING_TRACE(3);
-  if (T == 1) {
+  if (T == 1 && !ep) {
     // one token: the selected experts are already distinct
     if (tid < K) {
       hd.uniq_e[tid] = hd.topi[0][tid];
@@ -407,17 +408,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     }
     if (tid == 0) hd.nuniq = K;
   } else if (warp == 0 && !aborted(hd)) {
-    // union of the selected experts, in first-occurrence order (t-major)
+    // union of the selected experts held here, in first-occurrence order
+    // (t-major), as indices into the local weights
     const int npairs = T * K;
     const int pe = (lane < npairs) ? hd.topi[lane / K][lane % K] : -1 - lane;
-    bool first = lane < npairs;
+    bool first = lane < npairs && (unsigned)(pe - p.e0) < (unsigned)p.e_local;
     for (int j = 0; j < npairs; ++j) {
       const int ej = __shfl_sync(0xffffffffu, pe, j);
       if (j < lane && ej == pe) first = false;
     }
     const unsigned fm = __ballot_sync(0xffffffffu, first);
     const int myu = first ? __popc(fm & ((1u << lane) - 1u)) : -1;
-    if (first) hd.uniq_e[myu] = pe;
+    if (first) hd.uniq_e[myu] = pe - p.e0;
     int cnt = 0;
     for (int j = 0; j < npairs; ++j) {
       const int ej = __shfl_sync(0xffffffffu, pe, j);
@@ -597,7 +599,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   const int nmine_r = warp < nbatch ? (nbatch - warp + kWarps - 1) / kWarps : 0;
   const int sh_first = kWarps - 1 - warp;  // shared down: half-blocks of 4 rows
   const int nsub = 2 * nblk;
-  const int nmine_s = (!aborted(hd) && sh_first < nsub) ? (nsub - sh_first + kWarps - 1) / kWarps : 0;
+  const int nmine_s = (p.shared_on && !aborted(hd) && sh_first < nsub) ? (nsub - sh_first + kWarps - 1) / kWarps : 0;
   auto issue4 = [&](int s) {
     if (lane == 0) {
       if (s < nmine_r) {
@@ -625,7 +627,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   float* part = reinterpret_cast<float*>(body + PL::part);
   if (tid == 0 && !aborted(hd)) {
     const unsigned long long ep1 = hd.epoch + 1;
-    if (wait_count(p.sync + 1, ep1 * (unsigned long long)kI, p.wait_limit_ns, p.err, &hd.abort))
+    if (!p.shared_on || wait_count(p.sync + 1, ep1 * (unsigned long long)kI, p.wait_limit_ns, p.err, &hd.abort))
       wait_count(p.sync + 2, ep1 * (unsigned long long)ncta, p.wait_limit_ns, p.err, &hd.abort);
   }
   __syncthreads();
@@ -633,7 +635,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     // routed h (per pair) then shared h (per token), in batches whose loads
     // are all in flight before the first shared store
     constexpr int kB = 5;
-    const int nh = npairs * (kI / 4), nall = nh + T * (kI / 4);
+    const int nh = npairs * (kI / 4), nall = nh + (p.shared_on ? T * (kI / 4) : 0);
     for (int v0 = tid; v0 < nall; v0 += kB * kDecodeThreads) {
       float4 hv[kB];
 #pragma unroll
@@ -744,21 +746,25 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   __syncthreads();
   LING_TRACE(8);
   if (!aborted(hd)) {
-    // fixed-order sum: routed slots 0..k-1, then the shared expert
+    // fixed-order sum: routed slots 0..k-1 (those computed here), then the
+    // shared expert (if computed here)
     for (int v = tid; v < nblk * T * kDnUnitRows; v += kDecodeThreads) {
       const int blk = v / (T * kDnUnitRows), rem = v - blk * T * kDnUnitRows, t = rem >> 3, r = rem & 7;
       const float* pb = part + (size_t)blk * (PL::P + T) * 8;
       float v8[kMaxTopK];  // all loads in flight first, then the sum in slot order
 #pragma unroll
-      for (int sl = 0; sl < kMaxTopK; ++sl) v8[sl] = sl < K ? pb[(t * K + sl) * 8 + r] : 0.f;
-      const float vs = pb[(PL::P + t) * 8 + r];
+      for (int sl = 0; sl < kMaxTopK; ++sl)
+        v8[sl] = sl < K && (unsigned)(hd.topi[t][sl] - p.e0) < (unsigned)p.e_local ? pb[(t * K + sl) * 8 + r] : 0.f;
+      const float vs = p.shared_on ? pb[(PL::P + t) * 8 + r] : 0.f;
       float s = 0.f;
 #pragma unroll
       for (int sl = 0; sl < kMaxTopK; ++sl)
         if (sl < K) s += v8[sl];
       s += vs;
       const float st = hd.xscale[t];  // back from x / s_t: the output scales as s_t^2
-      p.out[(size_t)t * kH + kDnUnitRows * (b0 + blk) + r] = __float2bfloat16_rn(s * st * st);
+      const size_t o = (size_t)t * kH + kDnUnitRows * (b0 + blk) + r;
+      if (p.out_f32) p.out_f32[o] = s * st * st;
+      else p.out[o] = __float2bfloat16_rn(s * st * st);
     }
   }
   // every CTA (aborted or not) counts itself out: the next launch's index

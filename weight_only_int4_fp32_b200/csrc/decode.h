@@ -39,6 +39,14 @@ struct DecodeParams {
   int skip_arrive_cta;           // test hook: this CTA withholds its router rows (-1: none)
   unsigned long long wait_limit_ns;
   int codec;                     // kCodecInt4 or kCodecMxfp4 (common.cuh): how gu / dn codes decode
+  // Expert parallel: gu / dn hold experts [e0, e0 + e_local) of the E the
+  // router scores; the selection and its weights still run over all E, only
+  // the local experts' terms are computed.  shared_on = 0 leaves the shared
+  // expert out (its weights are not read).  out_f32 != nullptr: the sum of the
+  // computed terms goes there in fp32 (times s_t^2) instead of a bf16 out.
+  int e0, e_local;
+  int shared_on;
+  float* out_f32;                // [T, H] or nullptr
 };
 
 size_t decode_smem_bytes(int T);

@@ -82,8 +82,9 @@ cudaError_t grouped_prepare(GroupedWorkspace* ws, int E, const __nv_bfloat16* sh
   // columns (whose results are discarded); keep them finite
   if ((e = cudaMemsetAsync(ws->xg, 0, ws->rows * kH * sizeof(__half), stream)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(ws->h16, 0, ws->rows * 2 * kI * sizeof(__half), stream)) != cudaSuccess) return e;
-  if ((e = launch_tc_prep_shared(sh_gate, sh_up, sh_down, ws->shgu16, ws->shdn16, ws->sh_scale, ws->amax,
-                                 stream)) != cudaSuccess)
+  // (no shared expert on this handle: its fp16 copies are never read)
+  if (sh_gate && (e = launch_tc_prep_shared(sh_gate, sh_up, sh_down, ws->shgu16, ws->shdn16, ws->sh_scale, ws->amax,
+                                            stream)) != cudaSuccess)
     return e;
   return tc_encode_maps(&ws->maps, ws->xg, ws->h16, (int)ws->rows, ws->shgu16, ws->shdn16);
 }
@@ -232,11 +233,13 @@ __global__ void __launch_bounds__(256) grp_topk_kernel(GroupedParams p, const fl
   if (lane < p.k) {
     const int e = s_idx[warp][lane];
     const float w = s_w[warp][lane];
-    ti[t * p.k + lane] = e;
+    // the pair's expert as an index into the local weights, -1 if not held here
+    const int el = (unsigned)(e - p.e0) < (unsigned)p.e_local ? e - p.e0 : -1;
+    ti[t * p.k + lane] = el;
     tw[t * p.k + lane] = w;
     if (p.topk_idx_out) p.topk_idx_out[t * p.k + lane] = e;
     if (p.topk_w_out) p.topk_w_out[t * p.k + lane] = w;
-    atomicAdd(&cnt[e], 1);
+    if (el >= 0) atomicAdd(&cnt[el], 1);
   }
 }
 
@@ -255,7 +258,10 @@ __device__ __forceinline__ void write_ntile(int idx, int e, int pos0, int n, int
   for (int mt = 0; mt < kTcMTilesDn; ++mt) dn_tiles[idx * kTcMTilesDn + mt] = make_int4(e, mt, pos0, n);
 }
 
-__global__ void __launch_bounds__(kPlanThreads) grp_plan_kernel(int T, int E, int32_t* cnt, int32_t* fill,
+// The shared expert's rows are positions Pall + t (Pall = T * k, where the
+// scatter writes them), whether or not every routed pair is held here.
+__global__ void __launch_bounds__(kPlanThreads) grp_plan_kernel(int T, int E, int shared_on, int Pall, int32_t* cnt,
+                                                                int32_t* fill,
                                                                 int32_t* off, int4* gu_tiles, int4* dn_tiles,
                                                                 int32_t* ntiles, int4* small, int32_t* nsmall) {
   constexpr int NV = 10;  // [0] pairs, [1 + b] N-tiles of width bucket b, [9] GEMV experts
@@ -263,7 +269,7 @@ __global__ void __launch_bounds__(kPlanThreads) grp_plan_kernel(int T, int E, in
   __shared__ int wbase[kPlanThreads / 32][NV];
   __shared__ int total[NV];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int c = t < E ? cnt[t] : (t == E ? T : 0);
+  const int c = t < E ? cnt[t] : (t == E && shared_on ? T : 0);
   const bool gemv = t < E && c > 0 && c <= kGvMaxTok;
   const int full = gemv ? 0 : c / kTcTileN, rem = gemv ? 0 : c % kTcTileN;
   const int pb = rem > 0 ? (rem + 15) / 16 - 1 : -1;
@@ -318,7 +324,7 @@ __global__ void __launch_bounds__(kPlanThreads) grp_plan_kernel(int T, int E, in
   if (t == E) off[E] = P;
   if (gemv) small[excl[9]] = make_int4(t, excl[0], c, 0);
   if (t <= E && !gemv) {
-    const int pos_base = t < E ? excl[0] : P;
+    const int pos_base = t < E ? excl[0] : Pall;
     const int i7 = bstart[7] + excl[8];
     for (int q = 0; q < full; ++q) write_ntile(i7 + q, t, pos_base + kTcTileN * q, kTcTileN, gu_tiles, dn_tiles);
     if (pb >= 0) {
@@ -346,7 +352,7 @@ __global__ void __launch_bounds__(kPlanThreads) grp_plan_kernel(int T, int E, in
 // the shared-expert row P + t.  sigma_t runs from -100 (a token whose largest
 // |x| is below 2^-86 has an output below bf16's smallest subnormal either
 // way) to 113 (bf16's largest finite value).
-__global__ void __launch_bounds__(kRowThreads) grp_scatter_kernel(const __nv_bfloat16* x, int k, int P,
+__global__ void __launch_bounds__(kRowThreads) grp_scatter_kernel(const __nv_bfloat16* x, int k, int P, int shared_on,
                                                                   const int32_t* ti, const int32_t* off,
                                                                   int32_t* fill, int32_t* perm, int32_t* inv,
                                                                   __half* xg, float* xscale) {
@@ -356,13 +362,13 @@ __global__ void __launch_bounds__(kRowThreads) grp_scatter_kernel(const __nv_bfl
   if (c == 0) smax = 0;
   if (c < k) {
     const int pp = t * k + c;
-    const int e = ti[pp];
-    const int pos = off[e] + atomicAdd(&fill[e], 1);
-    perm[pos] = pp;
+    const int e = ti[pp];  // -1: an expert not held here (no position)
+    const int pos = e >= 0 ? off[e] + atomicAdd(&fill[e], 1) : -1;
+    if (pos >= 0) perm[pos] = pp;
     inv[pp] = pos;
     spos[c] = pos;
   }
-  if (c == k) spos[k] = P + t;
+  if (c == k) spos[k] = shared_on ? P + t : -1;
   __syncthreads();
   const uint4 w = *reinterpret_cast<const uint4*>(x + (size_t)t * kH + 8 * c);
   const float f[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
@@ -381,18 +387,21 @@ __global__ void __launch_bounds__(kRowThreads) grp_scatter_kernel(const __nv_bfl
 #pragma unroll
   for (int o = 0; o < 8; ++o) h[o] = __float2half_rn(f[o] * inv_s);
   const uint4 hv = *reinterpret_cast<const uint4*>(h);
-  for (int i = 0; i <= k; ++i) *reinterpret_cast<uint4*>(xg + (size_t)spos[i] * kH + 8 * c) = hv;
+  for (int i = 0; i <= k; ++i)
+    if (spos[i] >= 0) *reinterpret_cast<uint4*>(xg + (size_t)spos[i] * kH + 8 * c) = hv;
 }
 
 // ---------------------------------------------------------------- combine
 __global__ void __launch_bounds__(kRowThreads) grp_combine_kernel(const float* y, const int32_t* inv, int k, int P,
-                                                                  const float* xscale, __nv_bfloat16* out) {
+                                                                  int shared_on, const float* xscale,
+                                                                  __nv_bfloat16* out, float* out_f32) {
   const int t = blockIdx.x, c = threadIdx.x;
   float s[8];
 #pragma unroll
   for (int o = 0; o < 8; ++o) s[o] = 0.f;
   for (int i = 0; i <= k; ++i) {
-    const int pos = i < k ? inv[t * k + i] : P + t;
+    const int pos = i < k ? inv[t * k + i] : (shared_on ? P + t : -1);
+    if (pos < 0) continue;  // an expert (or the shared expert) not computed here
     const float4 a = ldcg_f4(reinterpret_cast<const float4*>(y + (size_t)pos * kH + 8 * c));
     const float4 b = ldcg_f4(reinterpret_cast<const float4*>(y + (size_t)pos * kH + 8 * c + 4));
     s[0] += a.x; s[1] += a.y; s[2] += a.z; s[3] += a.w;
@@ -402,6 +411,13 @@ __global__ void __launch_bounds__(kRowThreads) grp_combine_kernel(const float* y
   // in [2^-87, 2^126], then one bf16 rounding (exact products unless the
   // result leaves fp32's range, where bf16 rounds the same way)
   const float ct = xscale[t] * (float)(1 << kGrpUnitShift);
+  if (out_f32) {
+    const float4 a = make_float4(s[0] * ct * ct, s[1] * ct * ct, s[2] * ct * ct, s[3] * ct * ct);
+    const float4 b = make_float4(s[4] * ct * ct, s[5] * ct * ct, s[6] * ct * ct, s[7] * ct * ct);
+    *reinterpret_cast<float4*>(out_f32 + (size_t)t * kH + 8 * c) = a;
+    *reinterpret_cast<float4*>(out_f32 + (size_t)t * kH + 8 * c + 4) = b;
+    return;
+  }
   __nv_bfloat162 r[4];
 #pragma unroll
   for (int o = 0; o < 4; ++o) r[o] = __floats2bfloat162_rn(s[2 * o] * ct * ct, s[2 * o + 1] * ct * ct);
@@ -433,12 +449,12 @@ cudaError_t launch_grouped(const GroupedParams& p, const GroupedWorkspace& ws, c
   grp_topk_kernel<<<(p.T + 7) / 8, 256, 0, s>>>(p, ws.logits, ws.topk_idx, ws.topk_w, ws.cnt);
   ++nl;
   mark(2);
-  grp_plan_kernel<<<1, kPlanThreads, 0, s>>>(p.T, p.E, ws.cnt, ws.fill, ws.off, ws.gu_tiles, ws.dn_tiles, ws.ntiles,
-                                             ws.small, ws.nsmall);
+  grp_plan_kernel<<<1, kPlanThreads, 0, s>>>(p.T, p.e_local, p.shared_on, P, ws.cnt, ws.fill, ws.off, ws.gu_tiles,
+                                             ws.dn_tiles, ws.ntiles, ws.small, ws.nsmall);
   ++nl;
   mark(3);
-  grp_scatter_kernel<<<p.T, kRowThreads, 0, s>>>(p.x, p.k, P, ws.topk_idx, ws.off, ws.fill, ws.perm, ws.inv, ws.xg,
-                                                 ws.xscale);
+  grp_scatter_kernel<<<p.T, kRowThreads, 0, s>>>(p.x, p.k, P, p.shared_on, ws.topk_idx, ws.off, ws.fill, ws.perm,
+                                                 ws.inv, ws.xg, ws.xscale);
   ++nl;
   TcParams tp{};
   tp.gu = p.gu;
@@ -450,7 +466,7 @@ cudaError_t launch_grouped(const GroupedParams& p, const GroupedWorkspace& ws, c
   tp.topk_w = ws.topk_w;
   tp.sh_scale = ws.sh_scale;
   tp.k = p.k;
-  tp.E = p.E;
+  tp.E = p.e_local;  // tiles of expert e_local are the shared expert's
   tp.P = P;
   tp.gu_tiles = ws.gu_tiles;
   tp.dn_tiles = ws.dn_tiles;
@@ -488,7 +504,7 @@ cudaError_t launch_grouped(const GroupedParams& p, const GroupedWorkspace& ws, c
   if ((e = launch_tc_gemm(1, ws.maps, tp, p.num_sms, s)) != cudaSuccess) return e;
   ++nl;
   mark(8);
-  grp_combine_kernel<<<p.T, kRowThreads, 0, s>>>(ws.y, ws.inv, p.k, P, ws.xscale, p.out);
+  grp_combine_kernel<<<p.T, kRowThreads, 0, s>>>(ws.y, ws.inv, p.k, P, p.shared_on, ws.xscale, p.out, p.out_f32);
   ++nl;
   mark(kGroupedKernels);
   e = cudaGetLastError();

@@ -24,6 +24,12 @@ struct GroupedParams {
   float* topk_w_out;             // optional [T, k]
   int num_sms;
   int codec;                     // kCodecInt4 or kCodecMxfp4 (layout.h)
+  // Expert parallel (as DecodeParams): gu / dn hold experts [e0, e0 + e_local)
+  // of the E the router scores; shared_on = 0 leaves the shared expert out;
+  // out_f32 != nullptr takes the fp32 sum instead of the bf16 out.
+  int e0, e_local;
+  int shared_on;
+  float* out_f32;
 };
 
 // Positions: the T*k token-expert pairs sorted by expert occupy positions
