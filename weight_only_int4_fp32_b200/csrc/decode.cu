@@ -167,8 +167,11 @@ __device__ __forceinline__ bool wait_count(const unsigned long long* ctr, unsign
   return true;
 }
 
-// C: the codec of the routed weights (kCodecInt4 or kCodecMxfp4).
-template <int T, int C>
+// C: the codec of the routed weights (kCodecInt4 or kCodecMxfp4).  EP: the
+// variant that honours an expert range, shared_on and out_f32 (expert-parallel
+// handles and fp32 partial outputs); the ordinary variant computes every
+// expert and the shared expert into a bf16 out, with none of that code.
+template <int T, int C, bool EP>
 __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const DecodeParams p) {
   using PL = Plan<T>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -187,8 +190,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   const int s0 = cta * kI / ncta, s1 = (cta + 1) * kI / ncta;
   const int b0 = cta * kDnUnits / ncta, b1 = (cta + 1) * kDnUnits / ncta;
   const int nblk = b1 - b0;
-  const int nr = r1 - r0, n12 = nr + (p.shared_on ? s1 - s0 : 0);
-  const bool ep = p.e_local != E;  // only experts [e0, e0 + e_local) are computed here
+  const bool sh_on = !EP || p.shared_on;                   // the shared expert is computed here
+  const int e0 = EP ? p.e0 : 0, e_local = EP ? p.e_local : E;  // the experts held here
+  const bool ep = EP && e_local != E;
+  const int nr = r1 - r0, n12 = nr + (sh_on ? s1 - s0 : 0);
 
   uint64_t* barA = &hd.mbar[warp][0];  // phases 1-2 items, piece 0 of a gate/up unit, phase-4 copies
   uint32_t pha = 0, phq = 0;           // phq: parity of pieces 1-3 (always used together)
@@ -239,7 +244,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   if (warp < n12) issue12(warp);
 
   // L2 prefetch of the shared down rows this CTA will need
-  if (p.shared_on && warp == kWarps - 1 && lane == 0 && nblk > 0)
+  if (sh_on && warp == kWarps - 1 && lane == 0 && nblk > 0)
     prefetch_l2_bulk(p.sh_down + (size_t)b0 * kDnUnitRows * kI, (uint32_t)nblk * 2 * kShDnBytes);
 
   // x (bf16) lands in shared memory; every warp waits for it once
@@ -412,14 +417,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     // (t-major), as indices into the local weights
     const int npairs = T * K;
     const int pe = (lane < npairs) ? hd.topi[lane / K][lane % K] : -1 - lane;
-    bool first = lane < npairs && (unsigned)(pe - p.e0) < (unsigned)p.e_local;
+    bool first = lane < npairs && (unsigned)(pe - e0) < (unsigned)e_local;
     for (int j = 0; j < npairs; ++j) {
       const int ej = __shfl_sync(0xffffffffu, pe, j);
       if (j < lane && ej == pe) first = false;
     }
     const unsigned fm = __ballot_sync(0xffffffffu, first);
     const int myu = first ? __popc(fm & ((1u << lane) - 1u)) : -1;
-    if (first) hd.uniq_e[myu] = pe - p.e0;
+    if (first) hd.uniq_e[myu] = pe - e0;
     int cnt = 0;
     for (int j = 0; j < npairs; ++j) {
       const int ej = __shfl_sync(0xffffffffu, pe, j);
@@ -599,7 +604,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   const int nmine_r = warp < nbatch ? (nbatch - warp + kWarps - 1) / kWarps : 0;
   const int sh_first = kWarps - 1 - warp;  // shared down: half-blocks of 4 rows
   const int nsub = 2 * nblk;
-  const int nmine_s = (p.shared_on && !aborted(hd) && sh_first < nsub) ? (nsub - sh_first + kWarps - 1) / kWarps : 0;
+  const int nmine_s = (sh_on && !aborted(hd) && sh_first < nsub) ? (nsub - sh_first + kWarps - 1) / kWarps : 0;
   auto issue4 = [&](int s) {
     if (lane == 0) {
       if (s < nmine_r) {
@@ -627,7 +632,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   float* part = reinterpret_cast<float*>(body + PL::part);
   if (tid == 0 && !aborted(hd)) {
     const unsigned long long ep1 = hd.epoch + 1;
-    if (!p.shared_on || wait_count(p.sync + 1, ep1 * (unsigned long long)kI, p.wait_limit_ns, p.err, &hd.abort))
+    if (!sh_on || wait_count(p.sync + 1, ep1 * (unsigned long long)kI, p.wait_limit_ns, p.err, &hd.abort))
       wait_count(p.sync + 2, ep1 * (unsigned long long)ncta, p.wait_limit_ns, p.err, &hd.abort);
   }
   __syncthreads();
@@ -635,7 +640,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     // routed h (per pair) then shared h (per token), in batches whose loads
     // are all in flight before the first shared store
     constexpr int kB = 5;
-    const int nh = npairs * (kI / 4), nall = nh + (p.shared_on ? T * (kI / 4) : 0);
+    const int nh = npairs * (kI / 4), nall = nh + (sh_on ? T * (kI / 4) : 0);
     for (int v0 = tid; v0 < nall; v0 += kB * kDecodeThreads) {
       float4 hv[kB];
 #pragma unroll
@@ -754,8 +759,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       float v8[kMaxTopK];  // all loads in flight first, then the sum in slot order
 #pragma unroll
       for (int sl = 0; sl < kMaxTopK; ++sl)
-        v8[sl] = sl < K && (unsigned)(hd.topi[t][sl] - p.e0) < (unsigned)p.e_local ? pb[(t * K + sl) * 8 + r] : 0.f;
-      const float vs = p.shared_on ? pb[(PL::P + t) * 8 + r] : 0.f;
+        v8[sl] = sl < K && (!ep || (unsigned)(hd.topi[t][sl] - e0) < (unsigned)e_local) ? pb[(t * K + sl) * 8 + r]
+                                                                                        : 0.f;
+      const float vs = sh_on ? pb[(PL::P + t) * 8 + r] : 0.f;
       float s = 0.f;
 #pragma unroll
       for (int sl = 0; sl < kMaxTopK; ++sl)
@@ -763,7 +769,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       s += vs;
       const float st = hd.xscale[t];  // back from x / s_t: the output scales as s_t^2
       const size_t o = (size_t)t * kH + kDnUnitRows * (b0 + blk) + r;
-      if (p.out_f32) p.out_f32[o] = s * st * st;
+      if (EP && p.out_f32) p.out_f32[o] = s * st * st;
       else p.out[o] = __float2bfloat16_rn(s * st * st);
     }
   }
@@ -782,7 +788,7 @@ extern "C" int ling_moe_trace_read(unsigned long long* host, int nctas) {
 }
 #endif
 
-template <int T, int C>
+template <int T, int C, bool EP>
 static cudaError_t launch_t(const DecodeParams& p, int nctas, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nctas);
@@ -794,33 +800,42 @@ static cudaError_t launch_t(const DecodeParams& p, int nctas, cudaStream_t strea
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, moe_decode_kernel<T, C>, p);
+  return cudaLaunchKernelEx(&cfg, moe_decode_kernel<T, C, EP>, p);
 }
 
-template <int C>
+template <int C, bool EP>
 static cudaError_t launch_c(const DecodeParams& p, int nctas, cudaStream_t stream) {
   switch (p.T) {
-    case 1: return launch_t<1, C>(p, nctas, stream);
-    case 2: return launch_t<2, C>(p, nctas, stream);
-    case 3: return launch_t<3, C>(p, nctas, stream);
-    case 4: return launch_t<4, C>(p, nctas, stream);
+    case 1: return launch_t<1, C, EP>(p, nctas, stream);
+    case 2: return launch_t<2, C, EP>(p, nctas, stream);
+    case 3: return launch_t<3, C, EP>(p, nctas, stream);
+    case 4: return launch_t<4, C, EP>(p, nctas, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
 cudaError_t launch_decode(const DecodeParams& p, int nctas, cudaStream_t stream) {
-  if (p.codec == kCodecMxfp4) return launch_c<kCodecMxfp4>(p, nctas, stream);
-  if (p.codec == kCodecInt4) return launch_c<kCodecInt4>(p, nctas, stream);
+  const bool ep = p.e0 != 0 || p.e_local != p.E || !p.shared_on || p.out_f32 != nullptr;
+  if (p.codec == kCodecMxfp4)
+    return ep ? launch_c<kCodecMxfp4, true>(p, nctas, stream) : launch_c<kCodecMxfp4, false>(p, nctas, stream);
+  if (p.codec == kCodecInt4)
+    return ep ? launch_c<kCodecInt4, true>(p, nctas, stream) : launch_c<kCodecInt4, false>(p, nctas, stream);
   return cudaErrorInvalidValue;
+}
+
+template <int T, int C, bool EP>
+static cudaError_t set_smem() {
+  return cudaFuncSetAttribute(moe_decode_kernel<T, C, EP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)Plan<T>::bytes);
 }
 
 template <int T>
 static cudaError_t setup_t() {
-  cudaError_t e = cudaFuncSetAttribute(moe_decode_kernel<T, kCodecInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)Plan<T>::bytes);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(moe_decode_kernel<T, kCodecMxfp4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)Plan<T>::bytes);
+  cudaError_t e;
+  if ((e = set_smem<T, kCodecInt4, false>()) != cudaSuccess) return e;
+  if ((e = set_smem<T, kCodecInt4, true>()) != cudaSuccess) return e;
+  if ((e = set_smem<T, kCodecMxfp4, false>()) != cudaSuccess) return e;
+  return set_smem<T, kCodecMxfp4, true>();
 }
 
 cudaError_t setup_decode() {
@@ -833,7 +848,7 @@ cudaError_t setup_decode() {
 
 int decode_max_ctas_per_sm() {
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, moe_decode_kernel<4, kCodecInt4>, kDecodeThreads,
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, moe_decode_kernel<4, kCodecInt4, true>, kDecodeThreads,
                                                     Plan<4>::bytes) != cudaSuccess)
     return 0;
   return n;
