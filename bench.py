@@ -1,7 +1,7 @@
 """Benchmark of the W4 g32 MoE layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode_e512_t1|verify_e512_t4|stack40_e512_t1|prefill_e512_t2048_zipf|reduced_e32_t1
+                    [--workload decode_e512_t1|verify_e512_t4|verify_e512_t8|stack40_e512_t1|prefill_e512_t2048_zipf|reduced_e32_t1
                                |lmhead_fp8_v157184_t1|lmhead_fp8_v157184_t8]
 
 A step is one pass of the whole layer (router, top-k, routed gate/up, down,
@@ -39,6 +39,7 @@ WORKLOAD_METRIC = {
     "decode_e512_t1_mxfp4": METRIC_MXFP4,
     "reduced_e32_t1": "reduced MoE-layer decode tokens/s and achieved HBM GB/s (W4 g32, 32e top-8, T=1)",
     "verify_e512_t4": "MoE-layer verify tokens/s and achieved HBM GB/s (W4 g32, 512e top-8, T=4 per call)",
+    "verify_e512_t8": "MoE-layer verify tokens/s and achieved HBM GB/s (W4 g32, 512e top-8, T=8 per call)",
     "stack40_e512_t1": "40-layer MoE-stack decode tokens/s and achieved HBM GB/s (W4 g32, 512e top-8, T=1)",
     "prefill_e512_t2048_zipf": "MoE-layer prefill tokens/s (W4 g32, 512e top-8, T=2048 per call, Zipf(1.1) routing)",
     "prefill_e512_t2048_zipf_mxfp4": "MoE-layer prefill tokens/s (MXFP4 e2m1/e8m0, 512e top-8, T=2048 per call, "
@@ -238,7 +239,7 @@ def cpu_oracle_rate(workload: str, seconds: float = 15.0, max_tokens: int = 64):
     host = lw.host_arrays()
     if workload.startswith("prefill"):
         host["router_bias"] = workloads.zipf_router_bias(E, wl["zipf_s"]).numpy()
-    T = min(wl["T"], 4)
+    T = min(wl["T"], 8)
     seeds = wl.get("token_seeds") or wl.get("call_seeds") or [1 + t for t in range(1000)]
 
     def timed(budget):
@@ -280,7 +281,7 @@ def run_reference(args):
     lw = gen(E, seed=wl.get("weight_seed", 100), device="cuda" if torch.cuda.is_available() else "cpu")
     host = lw.host_arrays()
     del lw
-    T = wl["T"] if wl["T"] <= 4 else 4
+    T = wl["T"] if wl["T"] <= 8 else 8
     seeds = wl.get("token_seeds") or wl.get("call_seeds") or [1 + t for t in range(1000)]
     def step(i):
         x = workloads.tokens(T, seed=seeds[i % len(seeds)], device="cpu")
@@ -371,7 +372,8 @@ def make_inputs(workload, n, T, device, rank=0):
         seeds = [1 + t for t in range(n)] if workload.startswith("decode") else list(range(n))
         return [workloads.tokens(1, seed=s + off, device=device) for s in seeds]
     if workload.startswith("verify"):
-        return [workloads.tokens(4, seed=10000 + i + off, device=device) for i in range(n)]
+        seeds = wl["call_seeds"]
+        return [workloads.tokens(T, seed=seeds[0] + i + off, device=device) for i in range(n)]
     if workload.startswith("stack"):
         return [torch.stack([workloads.tokens(1, seed=workloads.stack_token_seed(t, l) + off, device=device)[0]
                              for l in range(wl["layers"])]) for t in range(n)]
@@ -575,7 +577,7 @@ def run_ours(args):
     avg_launch_ms = kern_ms / nsteps / calls_per_step
     achieved = (avg_bytes / calls_per_step) / (avg_launch_ms * 1e-3) / 1e9
     peak, peak_kind = peaks()
-    roofline = {"bound": "hbm", "kernel": "whole layer (one launch per call at T <= 4)", "achieved": achieved,
+    roofline = {"bound": "hbm", "kernel": "whole layer (one launch per call at T <= 8)", "achieved": achieved,
                 "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic_for(args.workload),
                 "peak_kind": peak_kind, "bytes_per_launch": avg_bytes / calls_per_step}
     if ktimes is not None and "tc_gu" in ktimes:

@@ -57,7 +57,7 @@ def test_mxfp4_full_layer_matches_the_oracle_and_the_launch_count():
             xs = workloads.token_stream(seeds)
             n0 = layer.launch_count()
             out, idx, w = _calls(layer, xs.to(DEV), T)
-            assert layer.launch_count() - n0 == (len(seeds) // T) * (1 if T <= 4 else 2)
+            assert layer.launch_count() - n0 == len(seeds) // T  # one decode launch per call up to 8 tokens
             compare(MX.moe_layer_mxfp4(bits(xs), host, 8), out, idx, w, 8, f"mxfp4 full T={T}")
     finally:
         layer.close()

@@ -5,7 +5,7 @@ The token kinds (workloads.EXTREME_KINDS) cover the input format's range:
 and, for "all_max", router logits beyond fp32's range), tokens made of bf16
 subnormals, tiny tokens whose outputs sit near bf16's smallest values, and
 tokens mixing subnormal, ordinary and huge values.  They run through the
-decode kernel (T = 1 and T = 4), the token-grouped path (T = 37 on the
+decode kernel (T = 1, 4 and 8), the token-grouped path (T = 37 on the
 32-expert layer, which splits its experts between the GEMV kernels and the
 tensor-core tiles; T = 20 on the full layer) and both MXFP4 paths,
 with and without a router bias, and are compared with the bar of
@@ -83,6 +83,14 @@ def test_decode_t4_mixed_kinds(reduced_layers, group, bias):
     x = workloads.extreme_tokens(T4_GROUPS[group], seed=800 + 10 * group)
     out, idx, w = _run(layer, x)
     compare_range(_oracle(x, host), out, idx, w, 8, f"decode T=4 {T4_GROUPS[group]} bias={bias}")
+
+
+@pytest.mark.parametrize("bias", [False, True])
+def test_decode_t8_mixed_kinds(reduced_layers, bias):
+    host, layer = reduced_layers[bias]
+    x = workloads.extreme_tokens(T4_GROUPS[0] + T4_GROUPS[1], seed=850)
+    out, idx, w = _run(layer, x)
+    compare_range(_oracle(x, host), out, idx, w, 8, f"decode T=8 bias={bias}")
 
 
 @pytest.mark.parametrize("bias", [False, True])

@@ -275,11 +275,11 @@ static int create_impl(const ling_moe_config_t* cfg, const ling_moe_weights_t* w
   snprintf(buf, sizeof(buf),
            "ling_moe sm_%d%d %d SMs | H=%d I=%d E=%d k=%d g=%d max_tokens=%d bias=%s%s | "
            "decode path (1<=T<=%d): 1 cooperative launch grid=%dx%d smem=%zuB, %s GEMV "
-           "dequant-in-register, fp32 accumulate (T<=%d: 2 such launches) | grouped path (T>%d): %s",
+           "dequant-in-register, fp32 accumulate, expert union deduplicated over the call's tokens | "
+           "grouped path (T>%d): %s",
            prop.major, prop.minor, h->num_sms, kH, kI, E, K, kGroup, cfg->max_tokens,
            w->router_bias ? "yes" : "no", ep_desc.c_str(), kMaxDecodeT, h->decode_ctas, kDecodeThreads,
-           decode_smem_bytes(1), codec == kCodecMxfp4 ? "MXFP4 (E2M1, E8M0 per 32)" : "W4 g32",
-           2 * kMaxDecodeT, 2 * kMaxDecodeT,
+           decode_smem_bytes(1), codec == kCodecMxfp4 ? "MXFP4 (E2M1, E8M0 per 32)" : "W4 g32", kMaxDecodeT,
            grouped_describe());
   h->desc = buf;
   *out = h;
@@ -322,13 +322,10 @@ static int forward_impl(ling_moe_t* h, const void* x, int T, void* out, int32_t*
     return fail(LING_MOE_ERR_INVALID_ARG, "topk outputs must be 4-byte aligned");
   cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
   cudaError_t e;
-  // Up to kMaxDecodeT tokens: one decode launch.  Up to twice that: the
-  // first kMaxDecodeT tokens and the rest as two decode launches in stream
-  // order (the handle's decode workspace is reused; experts common to both
-  // chunks are read twice) -- measured faster than the token-grouped path
-  // for 5..8 tokens.  Beyond: the token-grouped path.
-  if (T <= kMaxDecodeT || (T <= 2 * kMaxDecodeT && h->decode_T == kMaxDecodeT)) {
-    const int nchunk = T > kMaxDecodeT ? 2 : 1;
+  // Up to kMaxDecodeT (8) tokens: one decode launch, each distinct expert of
+  // the tokens' union read once.  Beyond: the token-grouped path.
+  if (T <= kMaxDecodeT) {
+    const int nchunk = 1;
     if (h->timing) cudaEventRecord(h->tev[0], stream);
     for (int c = 0; c < nchunk; ++c) {
       const int t0 = c * kMaxDecodeT, Tc = c == 0 ? (T < kMaxDecodeT ? T : kMaxDecodeT) : T - kMaxDecodeT;

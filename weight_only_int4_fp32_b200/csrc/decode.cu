@@ -31,6 +31,8 @@
 // "Single-GPU int4": symmetric W4, group 32, routed experts only) and the
 // bpdata article "Harom optimalizacio a Ling-3.0-flash MoE inferenciajanak"
 // ("Modell es kiindulo konfiguracio": 8 of 512 routed experts + 1 shared).
+#include <type_traits>
+
 #include "common.cuh"
 #include "decode.h"
 
@@ -58,16 +60,25 @@ __device__ __forceinline__ void g_clk_sink(float) {}
 
 constexpr int kWarps = kDecodeWarps;
 constexpr int kBufA = kGuHalfBytes;                 // per-warp buffer, phases 1-3 (one K half of a unit)
-constexpr int kDnBatch = 2;                         // routed down units per copy batch
-constexpr int kBufB = kDnBatch * kDnUnitBytes;      // per-warp buffer, phase 4
 constexpr int kShDnBytes = 4 * kI * 2;              // 4 shared-down rows (half a row-block)
+// routed down units per copy batch (one above 4 tokens: shared memory goes to
+// h), and the per-warp phase-4 buffer (a batch or a shared-down block)
+template <int T> __host__ __device__ constexpr int dn_batch() { return T > 4 ? 1 : 2; }
+template <int T> __host__ __device__ constexpr int dn_buf() { return T > 4 ? kShDnBytes : 2 * kDnUnitBytes; }
+// Routed h staged in shared memory as fp16 hi + lo A fragments: every pair up
+// to 4 tokens (indexed by pair); above, at most kHfCapBig pairs at a time,
+// experts taken in union order, so that phase 4 runs in at most two passes
+// (the first takes more than kHfCapBig - 8 pairs, leaving at most 33 of 64).
+constexpr int kHfCapBig = 38;
+template <int T> __host__ __device__ constexpr int hf_cap() { return T > 4 ? kHfCapBig : T * kMaxTopK; }
 constexpr int kMaxBlkPerCta = 4;                    // 8-row down blocks per CTA (>= 320 / nctas, nctas >= 80)
 constexpr int kDnPrefBlk = 3;                       // T = 1: routed down units kept in shared memory
                                                     // when the CTA has <= 3 row-blocks (>= 107 CTAs)
 constexpr int kGuPiece = kGuHalfCodes / 4;          // 2560 B: 5 chunks of a gate/up half-unit
 constexpr int kPairs = kDecodeWarps / 2;            // phase-3 warp pairs (one K half each)
 constexpr int kRowBytes = kH * 2;                   // one bf16 row of H
-static_assert(kBufB >= kShDnBytes, "phase-4 buffer holds a shared-down block");
+static_assert(dn_buf<8>() >= kShDnBytes && dn_buf<1>() >= kShDnBytes && dn_buf<8>() >= kDnUnitBytes,
+              "phase-4 buffer holds a batch or a shared-down block");
 static_assert(kBufA >= 2 * kRowBytes, "phase-1/2 buffer holds a gate and an up row");
 
 struct __align__(128) SmemHeader {  // 128-byte multiple: the body starts on a full line
@@ -82,6 +93,10 @@ struct __align__(128) SmemHeader {  // 128-byte multiple: the body starts on a f
   int uniq_e[kMaxDecodeT * kMaxTopK];
   int uniq_cnt[kMaxDecodeT * kMaxTopK];
   int uniq_pair[kMaxDecodeT * kMaxTopK][kMaxDecodeT];
+  int uniq_slot[kMaxDecodeT * kMaxTopK];  // T > 4: the expert's first h row in its pass
+  int slot_pair[2][kHfCapBig];            // T > 4: pair id of each h row, per pass
+  int nslot[2];                           // T > 4: h rows per pass
+  int u_split;                            // T > 4: experts [0, u_split) form the first pass
   int nuniq;
   int dcopies;  // T = 1: routed down copies into the dedicated region were issued
   unsigned long long epoch;  // launch index (see the arrival counters)
@@ -114,11 +129,11 @@ struct Plan {
   static constexpr size_t comb = xf + (size_t)T * kXfTok;                   // float [pairs][2][32][4]
   static constexpr size_t bufA = comb + (size_t)kPairs * 2 * 32 * 16;       // [warps][kBufA]
   static constexpr size_t endA = bufA + (size_t)kWarps * kBufA;
-  static constexpr size_t hf = 0;                                           // [P][kHfStride] h as MMA A fragments
-  static constexpr size_t hs = hf + (size_t)P * kHfStride;                  // float [T][kHsTok]
+  static constexpr size_t hf = 0;                                           // [hf_cap][kHfStride] h as MMA A fragments
+  static constexpr size_t hs = hf + (size_t)hf_cap<T>() * kHfStride;        // float [T][kHsTok]
   static constexpr size_t part = hs + (size_t)T * kHsTok * 4;               // float [blk][P + T][8]
   static constexpr size_t bufB = part + (size_t)kMaxBlkPerCta * (P + T) * 32;
-  static constexpr size_t endB = bufB + (size_t)kWarps * kBufB;
+  static constexpr size_t endB = bufB + (size_t)kWarps * dn_buf<T>();
   // T = 1: the CTA's routed down units, [expert slot][row-block] x kDnUnitBytes
   static constexpr size_t dn = endB;
   static constexpr size_t endD = dn + (T == 1 ? (size_t)kMaxTopK * kDnPrefBlk * kDnUnitBytes : 0);
@@ -134,7 +149,11 @@ size_t decode_smem_bytes(int T) {
     case 1: return Plan<1>::bytes;
     case 2: return Plan<2>::bytes;
     case 3: return Plan<3>::bytes;
-    default: return Plan<4>::bytes;
+    case 4: return Plan<4>::bytes;
+    case 5: return Plan<5>::bytes;
+    case 6: return Plan<6>::bytes;
+    case 7: return Plan<7>::bytes;
+    default: return Plan<8>::bytes;
   }
 }
 
@@ -199,7 +218,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   uint32_t pha = 0, phq = 0;           // phq: parity of pieces 1-3 (always used together)
   const bool use_d = (T == 1) && nblk <= kDnPrefBlk;
   unsigned char* bufA = body + PL::bufA + (size_t)warp * kBufA;
-  unsigned char* bufB = body + PL::bufB + (size_t)warp * kBufB;
+  unsigned char* bufB = body + PL::bufB + (size_t)warp * dn_buf<T>();
   unsigned char* xb = body + PL::xb;
   unsigned char* xf = body + PL::xf;
   if (tid < kMaxDecodeT) {
@@ -215,6 +234,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   if (tid == 0) {
     hd.abort = 0;
     hd.dcopies = 0;
+    hd.nslot[1] = 0;  // one phase-4 pass unless the union sets a second
     mbar_init(&hd.xbar, 1);
     mbar_init(&hd.dbar, 1);
     fence_mbar_init();
@@ -321,10 +341,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     pha ^= 1;
     const bool router = it < nr;
     float a0[T], a1[T];
-    {
-      float g0[T], g1[T], g2[T], g3[T], u0_[T], u1_[T], u2_[T], u3_[T];
+    // tokens [T0, T0 + TG): one pass over the staged row(s); more than 4
+    // tokens take two passes, so the accumulators stay those of 4 tokens
+    auto dots = [&](auto t0c, auto tgc) {
+      constexpr int T0 = decltype(t0c)::value, TG = decltype(tgc)::value;
+      float g0[TG], g1[TG], g2[TG], g3[TG], u0_[TG], u1_[TG], u2_[TG], u3_[TG];
 #pragma unroll
-      for (int t = 0; t < T; ++t) g0[t] = g1[t] = g2[t] = g3[t] = u0_[t] = u1_[t] = u2_[t] = u3_[t] = 0.f;
+      for (int t = 0; t < TG; ++t) g0[t] = g1[t] = g2[t] = g3[t] = u0_[t] = u1_[t] = u2_[t] = u3_[t] = 0.f;
 #pragma unroll
       for (int m = 0; m < kXChunks / 32; m += 2) {
         const int c0 = lane + 32 * m, c1 = c0 + 32;
@@ -332,8 +355,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         const uint4 w10 = router ? w00 : lds128(bufA + kRowBytes + 16 * c0);
         const uint4 w11 = router ? w01 : lds128(bufA + kRowBytes + 16 * c1);
 #pragma unroll
-        for (int t = 0; t < T; ++t) {
-          const uint4 xv0 = lds128(xb + t * kXbTok + 16 * c0), xv1 = lds128(xb + t * kXbTok + 16 * c1);
+        for (int t = 0; t < TG; ++t) {
+          const uint4 xv0 = lds128(xb + (T0 + t) * kXbTok + 16 * c0), xv1 = lds128(xb + (T0 + t) * kXbTok + 16 * c1);
           dot8_bf16_bf16_2(w00, xv0, g0[t], g1[t]);
           dot8_bf16_bf16_2(w01, xv1, g2[t], g3[t]);
           if (!router) {
@@ -343,10 +366,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         }
       }
 #pragma unroll
-      for (int t = 0; t < T; ++t) {
-        a0[t] = (g0[t] + g1[t]) + (g2[t] + g3[t]);
-        a1[t] = (u0_[t] + u1_[t]) + (u2_[t] + u3_[t]);
+      for (int t = 0; t < TG; ++t) {
+        a0[T0 + t] = (g0[t] + g1[t]) + (g2[t] + g3[t]);
+        a1[T0 + t] = (u0_[t] + u1_[t]) + (u2_[t] + u3_[t]);
       }
+    };
+    if constexpr (T <= 4) {
+      dots(std::integral_constant<int, 0>{}, std::integral_constant<int, T>{});
+    } else {
+      dots(std::integral_constant<int, 0>{}, std::integral_constant<int, 4>{});
+      dots(std::integral_constant<int, 4>{}, std::integral_constant<int, T - 4>{});
     }
 #pragma unroll
     for (int t = 0; t < T; ++t) {
@@ -412,7 +441,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       }
     }
     if (tid == 0) hd.nuniq = K;
-  } else if (warp == 0 && !aborted(hd)) {
+  } else if (T <= 4 && warp == 0 && !aborted(hd)) {
     // union of the selected experts held here, in first-occurrence order
     // (t-major), as indices into the local weights
     const int npairs = T * K;
@@ -437,6 +466,70 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       if (p.topk_idx_out) p.topk_idx_out[lane] = hd.topi[t][s];
       if (p.topk_w_out) p.topk_w_out[lane] = hd.topw[t][s];
     }
+  } else if (T > 4 && warp == 0 && !aborted(hd)) {
+    // the same union over up to 64 pairs (lane l holds pairs l and l + 32),
+    // then the h rows of phase 4: experts in union order fill passes of at
+    // most kHfCapBig pairs
+    const int npairs = T * K;
+    int pe[2];
+    bool first[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int j = lane + 32 * hh;
+      pe[hh] = j < npairs ? hd.topi[j / K][j % K] : -1 - j;
+      first[hh] = j < npairs && (unsigned)(pe[hh] - e0) < (unsigned)e_local;
+    }
+    for (int j = 0; j < npairs; ++j) {
+      const int ej = __shfl_sync(0xffffffffu, j < 32 ? pe[0] : pe[1], j & 31);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+        if (j < lane + 32 * hh && ej == pe[hh]) first[hh] = false;
+    }
+    const unsigned fm0 = __ballot_sync(0xffffffffu, first[0]), fm1 = __ballot_sync(0xffffffffu, first[1]);
+    const unsigned below = (1u << lane) - 1u;
+    const int myu[2] = {first[0] ? __popc(fm0 & below) : -1, first[1] ? __popc(fm0) + __popc(fm1 & below) : -1};
+    int cnt[2] = {0, 0};
+    for (int j = 0; j < npairs; ++j) {
+      const int ej = __shfl_sync(0xffffffffu, j < 32 ? pe[0] : pe[1], j & 31);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+        if (first[hh] && ej == pe[hh]) hd.uniq_pair[myu[hh]][cnt[hh]++] = j;
+    }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh)
+      if (first[hh]) {
+        hd.uniq_e[myu[hh]] = pe[hh] - e0;
+        hd.uniq_cnt[myu[hh]] = cnt[hh];
+      }
+    const int nu = __popc(fm0) + __popc(fm1);
+    if (lane == 0) hd.nuniq = nu;
+    __syncwarp();
+    if (lane == 0) {
+      int pass = 0, rows = 0;
+      hd.u_split = nu;
+      for (int u = 0; u < nu; ++u) {
+        const int c = hd.uniq_cnt[u];
+        if (pass == 0 && rows + c > kHfCapBig) {
+          hd.nslot[0] = rows;
+          hd.u_split = u;
+          pass = 1;
+          rows = 0;
+        }
+        hd.uniq_slot[u] = rows;
+        for (int g = 0; g < c; ++g) hd.slot_pair[pass][rows + g] = hd.uniq_pair[u][g];
+        rows += c;
+      }
+      hd.nslot[pass] = rows;
+      if (pass == 0) hd.nslot[1] = 0;
+    }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int j = lane + 32 * hh;
+      if (cta == 0 && j < npairs) {
+        if (p.topk_idx_out) p.topk_idx_out[j] = hd.topi[j / K][j % K];
+        if (p.topk_w_out) p.topk_w_out[j] = hd.topw[j / K][j % K];
+      }
+    }
   }
   __syncthreads();
   const int U = aborted(hd) ? 0 : hd.nuniq;
@@ -456,21 +549,39 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       const int u = unit / kGuUnits, b = unit - u * kGuUnits;
       const uint8_t* src = p.gu + ((size_t)hd.uniq_e[u] * kGuUnits + b) * kGuUnitBytes;
       mbar_arrive_expect_tx(barA, kGuPiece + kGuHalfScales);
-      bulk_g2s(bufA + kGuHalfCodes, src + kGuScaleOff + half * kGuHalfScales, kGuHalfScales, barA);
-      bulk_g2s(bufA, src + half * kGuHalfCodes, kGuPiece, barA);
-      for (int pc = 1; pc < 4; ++pc) {
-        mbar_arrive_expect_tx(&hd.mbar[warp][pc], kGuPiece);
-        bulk_g2s(bufA + pc * kGuPiece, src + half * kGuHalfCodes + pc * kGuPiece, kGuPiece, &hd.mbar[warp][pc]);
+      if (T > 4) {  // read once: evict first (see the down-unit prefetch)
+        const uint64_t once = l2_evict_first_policy();
+        bulk_g2s_hint(bufA + kGuHalfCodes, src + kGuScaleOff + half * kGuHalfScales, kGuHalfScales, barA, once);
+        bulk_g2s_hint(bufA, src + half * kGuHalfCodes, kGuPiece, barA, once);
+        for (int pc = 1; pc < 4; ++pc) {
+          mbar_arrive_expect_tx(&hd.mbar[warp][pc], kGuPiece);
+          bulk_g2s_hint(bufA + pc * kGuPiece, src + half * kGuHalfCodes + pc * kGuPiece, kGuPiece,
+                        &hd.mbar[warp][pc], once);
+        }
+      } else {
+        bulk_g2s(bufA + kGuHalfCodes, src + kGuScaleOff + half * kGuHalfScales, kGuHalfScales, barA);
+        bulk_g2s(bufA, src + half * kGuHalfCodes, kGuPiece, barA);
+        for (int pc = 1; pc < 4; ++pc) {
+          mbar_arrive_expect_tx(&hd.mbar[warp][pc], kGuPiece);
+          bulk_g2s(bufA + pc * kGuPiece, src + half * kGuHalfCodes + pc * kGuPiece, kGuPiece, &hd.mbar[warp][pc]);
+        }
       }
     }
   };
   const bool first_issued = u0 + pair < u1 && __shfl_sync(0xffffffffu, !aborted(hd), 0);  // one view per warp
   if (first_issued) issue3(u0 + pair);
+  // routed down units of this CTA (contiguous per expert) into L2 as soon as
+  // the routing is known.  Above 4 tokens the union's weights (~200 MB at 8
+  // tokens) outgrow L2: the gate/up units, read once, stream with an
+  // evict-first hint and these with evict-last, so that they are still there
+  // at phase 4 (without the hints: 1.24x the algorithmic DRAM reads at 8
+  // tokens).
   if (!use_d && warp == kWarps - 1 && nblk > 0) {
-    // routed down units of this CTA (contiguous per expert) into L2
+    const uint64_t keep = T > 4 ? l2_evict_last_policy() : 0;
     for (int u = lane; u < U; u += 32) {
       const uint8_t* src = p.dn + ((size_t)hd.uniq_e[u] * kDnUnits + b0) * kDnUnitBytes;
-      prefetch_l2_bulk(src, (uint32_t)nblk * kDnUnitBytes);
+      if (T > 4) prefetch_l2_bulk_hint(src, (uint32_t)nblk * kDnUnitBytes, keep);
+      else prefetch_l2_bulk(src, (uint32_t)nblk * kDnUnitBytes);
     }
   }
 
@@ -598,8 +709,23 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
 
   // ---- phase 4: down projections and the output
   // Region A is free now; start this warp's first phase-4 copy before waiting.
+  constexpr int kDnBatch = dn_batch<T>();
   const int npairs = T * K;
   const int nitems = nblk * U;
+  // above 4 tokens the items of the first pass's experts come first (pass-major,
+  // then row-block, then expert); a copy batch is one item there
+  const int npass = (T > 4 && hd.nslot[1] > 0) ? 2 : 1;  // the same value in every thread
+  const int U1 = npass == 2 ? hd.u_split : U, n1 = nblk * U1;
+  auto item_bu = [&](int it, int& blk, int& u) {
+    if (it < n1) {
+      blk = it / U1;
+      u = it - blk * U1;
+    } else {
+      const int i2 = it - n1, U2 = U - U1;
+      blk = i2 / U2;
+      u = U1 + (i2 - blk * U2);
+    }
+  };
   const int nbatch = use_d ? 0 : (nitems + kDnBatch - 1) / kDnBatch;
   const int nmine_r = warp < nbatch ? (nbatch - warp + kWarps - 1) / kWarps : 0;
   const int sh_first = kWarps - 1 - warp;  // shared down: half-blocks of 4 rows
@@ -612,7 +738,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         const int it0 = bi * kDnBatch, n = min(kDnBatch, nitems - it0);
         mbar_arrive_expect_tx(barA, (uint32_t)n * kDnUnitBytes);
         for (int bI = 0; bI < n; ++bI) {
-          const int it = it0 + bI, blk = it / U, u = it - blk * U;
+          int blk, u;
+          item_bu(it0 + bI, blk, u);
           bulk_g2s(bufB + bI * kDnUnitBytes,
                    p.dn + ((size_t)hd.uniq_e[u] * kDnUnits + b0 + blk) * kDnUnitBytes, kDnUnitBytes, barA);
         }
@@ -636,18 +763,23 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
       wait_count(p.sync + 2, ep1 * (unsigned long long)ncta, p.wait_limit_ns, p.err, &hd.abort);
   }
   __syncthreads();
-  if (!aborted(hd)) {
-    // routed h (per pair) then shared h (per token), in batches whose loads
-    // are all in flight before the first shared store
+  // routed h as fp16 hi + lo A fragments (h row r: pair r up to 4 tokens;
+  // above, row r of the pass, pair slot_pair[pass][r]) and, with the first
+  // pass, the shared h per token; in batches whose loads are all in flight
+  // before the first shared store
+  auto stage = [&](int pass) {
     constexpr int kB = 5;
-    const int nh = npairs * (kI / 4), nall = nh + (sh_on ? T * (kI / 4) : 0);
+    const int nrow = T <= 4 ? npairs : hd.nslot[pass];
+    const int nh = nrow * (kI / 4), nall = nh + (pass == 0 && sh_on ? T * (kI / 4) : 0);
     for (int v0 = tid; v0 < nall; v0 += kB * kDecodeThreads) {
       float4 hv[kB];
 #pragma unroll
       for (int b = 0; b < kB; ++b) {
         const int v = v0 + b * kDecodeThreads;
         if (v < nh) {
-          hv[b] = ldcg_f4(reinterpret_cast<const float4*>(p.h_pair) + v);
+          const int row = v / (kI / 4);
+          const int pr = T <= 4 ? row : hd.slot_pair[pass][row];
+          hv[b] = ldcg_f4(reinterpret_cast<const float4*>(p.h_pair) + (size_t)pr * (kI / 4) + (v - row * (kI / 4)));
         } else if (v < nall) {
           hv[b] = ldcg_f4(reinterpret_cast<const float4*>(p.h_s) + (v - nh));
         }
@@ -657,8 +789,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         const int v = v0 + b * kDecodeThreads;
         if (v < nh) {
           // h * 2^-8 as fp16 hi + lo in MMA A-fragment order
-          const int pr = v / (kI / 4), k = 4 * (v - pr * (kI / 4));
-          unsigned char* dst = hfb + (size_t)pr * kHfStride + hf_off(k);
+          const int row = v / (kI / 4), k = 4 * (v - row * (kI / 4));
+          unsigned char* dst = hfb + (size_t)row * kHfStride + hf_off(k);
           *reinterpret_cast<uint2*>(dst) = h_split2(hv[b].x, hv[b].y);
           *reinterpret_cast<uint2*>(dst + 16) = h_split2(hv[b].z, hv[b].w);
         } else if (v < nall) {
@@ -667,7 +799,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         }
       }
     }
-  }
+  };
+  if (!aborted(hd)) stage(0);
   __syncthreads();
   LING_TRACE(6);
   // one routed down unit (8 output rows of expert slot u, row-block blk) on
@@ -677,8 +810,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     const int g = lane >> 2, c = lane & 3;
     const bool act = g < hd.uniq_cnt[u];
     const int pr = hd.uniq_pair[u][act ? g : 0];
+    const int hrow = T <= 4 ? pr : hd.uniq_slot[u] + (act ? g : 0);
     float v0, v1;
-    dn_unit_mma<C>(base, hfb + (size_t)pr * kHfStride + 16 * c, lane, v0, v1);
+    dn_unit_mma<C>(base, hfb + (size_t)hrow * kHfStride + 16 * c, lane, v0, v1);
     if (act) {
       const float f = (float)(1 << kHShift) * hd.topw[pr / K][pr % K];
       *reinterpret_cast<float2*>(part + ((size_t)blk * (PL::P + T) + pr) * 8 + 2 * c) = make_float2(v0 * f, v1 * f);
@@ -702,16 +836,25 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
   {
     const int r = lane & 3, q = lane >> 2;
     const bool run = !aborted(hd);
-    for (int s = 0; s < nseq; ++s) {
-      if (s > 0) issue4(s);
-      if (!mbar_wait(barA, pha, p.wait_limit_ns, p.err)) { hd.abort = 1; break; }
+    int issued = nseq > 0 ? 1 : 0;  // copies requested: item sequence 0 went out above
+    // one step of this warp's sequence; false when its wait ran out
+    auto step = [&](int s) -> bool {
+      if (s >= issued) {
+        issue4(s);
+        issued = s + 1;
+      }
+      if (!mbar_wait(barA, pha, p.wait_limit_ns, p.err)) {
+        hd.abort = 1;
+        return false;
+      }
       pha ^= 1;
-      if (!run) continue;
+      if (!run) return true;
       if (s < nmine_r) {
         const int it0 = (warp + s * kWarps) * kDnBatch, n = min(kDnBatch, nitems - it0);
 #pragma unroll 1
         for (int bI = 0; bI < n; ++bI) {
-          const int it = it0 + bI, blk = it / U, u = it - blk * U;
+          int blk, u;
+          item_bu(it0 + bI, blk, u);
           down_item(bufB + bI * kDnUnitBytes, blk, u);
         }
       } else {
@@ -746,7 +889,29 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
         }
       }
       __syncwarp();
+      return true;
+    };
+    // this warp's items of the first pass (with one pass: its whole sequence)
+    const int s_p0 = npass == 2 ? min(nmine_r, n1 > warp ? (n1 - warp + kWarps - 1) / kWarps : 0) : nseq;
+    int s = 0;
+    for (; s < s_p0; ++s)
+      if (!step(s)) {
+        s = nseq;
+        break;
+      }
+    if (npass == 2) {
+      // the second pass's h rows replace the first's once every warp is done
+      // with them; this warp's next copy is requested before the barrier
+      if (s < nseq && s >= issued) {
+        issue4(s);
+        issued = s + 1;
+      }
+      __syncthreads();
+      if (!aborted(hd)) stage(1);
+      __syncthreads();
     }
+    for (; s < nseq; ++s)
+      if (!step(s)) break;
   }
   __syncthreads();
   LING_TRACE(8);
@@ -810,6 +975,10 @@ static cudaError_t launch_c(const DecodeParams& p, int nctas, cudaStream_t strea
     case 2: return launch_t<2, C, EP>(p, nctas, stream);
     case 3: return launch_t<3, C, EP>(p, nctas, stream);
     case 4: return launch_t<4, C, EP>(p, nctas, stream);
+    case 5: return launch_t<5, C, EP>(p, nctas, stream);
+    case 6: return launch_t<6, C, EP>(p, nctas, stream);
+    case 7: return launch_t<7, C, EP>(p, nctas, stream);
+    case 8: return launch_t<8, C, EP>(p, nctas, stream);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -843,13 +1012,17 @@ cudaError_t setup_decode() {
   if ((e = setup_t<1>()) != cudaSuccess) return e;
   if ((e = setup_t<2>()) != cudaSuccess) return e;
   if ((e = setup_t<3>()) != cudaSuccess) return e;
-  return setup_t<4>();
+  if ((e = setup_t<4>()) != cudaSuccess) return e;
+  if ((e = setup_t<5>()) != cudaSuccess) return e;
+  if ((e = setup_t<6>()) != cudaSuccess) return e;
+  if ((e = setup_t<7>()) != cudaSuccess) return e;
+  return setup_t<8>();
 }
 
 int decode_max_ctas_per_sm() {
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, moe_decode_kernel<4, kCodecInt4, true>, kDecodeThreads,
-                                                    Plan<4>::bytes) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, moe_decode_kernel<8, kCodecInt4, true>, kDecodeThreads,
+                                                    Plan<8>::bytes) != cudaSuccess)
     return 0;
   return n;
 }

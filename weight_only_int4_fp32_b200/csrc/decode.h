@@ -1,4 +1,5 @@
-// Host-visible interface of the decode / verify kernel (1 <= T <= kMaxDecodeT).
+// Host-visible interface of the decode / verify kernel (1 <= T <= kMaxDecodeT),
+// one launch per call for up to 8 tokens (a verify window of 8).
 #pragma once
 
 #include <cstddef>
@@ -8,7 +9,7 @@
 
 namespace lingmoe {
 
-constexpr int kMaxDecodeT = 4;     // tokens per call handled by the decode kernel
+constexpr int kMaxDecodeT = 8;     // tokens per call handled by the decode kernel
 constexpr int kDecodeWarps = 12;
 constexpr int kDecodeThreads = kDecodeWarps * 32;
 

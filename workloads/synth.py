@@ -277,6 +277,9 @@ WORKLOADS = {
     "verify_e512_t4": dict(num_experts=512, T=4, weight_seed=0,
                            call_seeds=[10000 + i for i in range(250)],
                            note="full layer, 4-token verify batch, 250 calls (seed 10000+i)"),
+    "verify_e512_t8": dict(num_experts=512, T=8, weight_seed=0,
+                           call_seeds=[30000 + i for i in range(250)],
+                           note="full layer, 8-token verify window, 250 calls (seed 30000+i), one launch each"),
     "stack40_e512_t1": dict(num_experts=512, T=1, layers=40,
                             layer_seeds=[100 + l for l in range(40)], tokens=200,
                             note="40 independent full layers back to back, 200 tokens"),
