@@ -61,25 +61,29 @@ L2_FLUSH_BYTES = 256 << 20
 # the command), valid only while the kernel's sources are the ones captured:
 # the sources are hashed and the figure is reported as null once they change.
 TRAFFIC = {
-    "decode_e512_t1": {"bytes": 41_039_872 + 9_472,
+    "decode_e512_t1": {"bytes": 41_048_576 + 0,
                        "sources": ('decode.cu', 'decode.h', 'common.cuh', 'layout.h'),
-                       "sha256": "01babd609ad0cf5bcc904feebe6f651432ef6deaf6fbd8a02fa6306d53f437d1"},
-    "verify_e512_t4": {"bytes": 129_148_160 + 3_299_584,
+                       "sha256": "552ed47622eede2e2df282a8a05ebdbc331566fa577d31df841c3c22beb4b4f8"},
+    "verify_e512_t4": {"bytes": 132_519_424 + 2_881_536,
                        "sources": ('decode.cu', 'decode.h', 'common.cuh', 'layout.h'),
-                       "sha256": "01babd609ad0cf5bcc904feebe6f651432ef6deaf6fbd8a02fa6306d53f437d1"},
+                       "sha256": "552ed47622eede2e2df282a8a05ebdbc331566fa577d31df841c3c22beb4b4f8"},
+    # one launch for the 8-token window (the union, ~62 experts, read once)
+    "verify_e512_t8": {"bytes": 220_087_552 + 3_197_696,
+                       "sources": ('decode.cu', 'decode.h', 'common.cuh', 'layout.h'),
+                       "sha256": "552ed47622eede2e2df282a8a05ebdbc331566fa577d31df841c3c22beb4b4f8"},
     # online-FP8 LM head: lmh_mma_kernel, the only kernel of a call
-    "lmhead_fp8_v157184_t1": {"bytes": 403_094_784 + 3_492_608,
+    "lmhead_fp8_v157184_t1": {"bytes": 403_095_296 + 3_477_504,
                               "sources": ('lmhead.cu', 'lmhead.h', 'common.cuh', 'layout.h'),
-                              "sha256": "d01a920b9c0a6a3a51626bf75dd07ef598df8463088f96b423c90873de2a1698"},
+                              "sha256": "97b9d0faf1db3059f55fc99a28f7971773752ba535a85e10db5243403a1fbea5"},
     # MXFP4 routed experts (the decode kernel's E2M1 instantiation); the unit
     # layout keeps a bf16 scale per 32, so 8 experts read 3,317,760 B each
-    "decode_e512_t1_mxfp4": {"bytes": 41_039_872 + 70_400,
+    "decode_e512_t1_mxfp4": {"bytes": 41_050_368 + 16_896,
                              "sources": ('decode.cu', 'decode.h', 'common.cuh', 'layout.h'),
-                             "sha256": "01babd609ad0cf5bcc904feebe6f651432ef6deaf6fbd8a02fa6306d53f437d1"},
+                             "sha256": "552ed47622eede2e2df282a8a05ebdbc331566fa577d31df841c3c22beb4b4f8"},
     # token-grouped: the dominant kernel, tc_grouped_kernel<0> (gate/up tiles)
-    "prefill_e512_t2048_zipf": {"bytes": 457_028_864 + 53_828_608,
+    "prefill_e512_t2048_zipf": {"bytes": 456_468_224 + 53_267_456,
                                 "sources": ('grouped_tc.cu', 'grouped_tc.h', 'common.cuh', 'layout.h'),
-                                "sha256": "56514f5ff591f5be46384759f168373b232e0f2534780ced74471a67e3ca4c13"},
+                                "sha256": "e2b129a4ebb03a66cf5653d3cce844530c5625db49547d188882ce7315df1735"},
 }
 
 
@@ -392,6 +396,11 @@ def run_ours(args):
     mode = l2_mode(args.workload, args.l2)
     stack = args.workload.startswith("stack")
     layers, E, T = build_layers(args.workload, dev, rotate=ROTATE_LAYERS if mode == "rotate" else 1)
+    if args.tokens:
+        # a verify window of fewer tokens on the same layers (verify-cost sweeps)
+        if not args.workload.startswith("verify") or not 1 <= args.tokens <= T:
+            raise SystemExit(f"--tokens applies to the verify workloads, 1..{T} tokens")
+        T = args.tokens
     nsteps, nwarm = args.steps, args.warmup
     inputs = make_inputs(args.workload, nsteps + nwarm, T, dev, rank=rank)
     l2flush = L2Flush(dev)
@@ -596,7 +605,9 @@ def run_ours(args):
         cpu = cpu_oracle_rate(args.workload if not stack else "decode_e512_t1",
                               seconds=args.cpu_seconds) if ws == 1 and args.cpu_seconds > 0 else None
         line = {
-            "metric": metric_for(args.workload), "value": value, "unit": "tokens/s",
+            "metric": metric_for(args.workload) if not args.tokens else
+                      f"MoE-layer verify tokens/s and achieved HBM GB/s (W4 g32, 512e top-8, T={T} per call)",
+            "value": value, "unit": "tokens/s",
             "n_gpus": ws, "steps": nsteps,
             "warmup": nwarm, "ms_per_step": kern_ms / nsteps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
@@ -804,6 +815,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode_e512_t1")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="verify workloads: calls of this many tokens (1..the workload's T) instead")
     ap.add_argument("--l2", default="auto", choices=["auto", "rotate", "flush"],
                     help="between steps: rotate over independent layers (decode-size workloads) or flush L2")
     args = ap.parse_args()
