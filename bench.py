@@ -47,6 +47,32 @@ WORKLOAD_METRIC = {
 }
 
 
+# The default run (no --workload) also times these, briefly, and attaches a
+# compact record of each to the one JSON line under "secondary".
+SECONDARY = ("verify_e512_t4", "verify_e512_t8", "decode_e512_t1_mxfp4", "stack40_e512_t1",
+             "prefill_e512_t2048_zipf", "prefill_e512_t2048_zipf_mxfp4", "lmhead_fp8_v157184_t1")
+_CAPTURE = None  # a list while secondary workloads run: lines are collected, not printed
+
+
+def emit(line):
+    if _CAPTURE is not None:
+        _CAPTURE.append(line)
+    else:
+        print(json.dumps(line), flush=True)
+
+
+def compact(line):
+    """The figures of a workload line that the secondary record keeps."""
+    r = line.get("roofline") or {}
+    e = line.get("e2e") or {}
+    return {"metric": line["metric"], "value": line["value"], "unit": line["unit"],
+            "ms_per_step": line["ms_per_step"], "steps": line["steps"], "warmup": line["warmup"],
+            "step_us_p10_p50_p90": line.get("step_us_p10_p50_p90"),
+            "roofline": {k: r.get(k) for k in ("bound", "kernel", "achieved", "peak", "unit", "frac", "traffic")},
+            "e2e": {k: e.get(k) for k in ("value", "unit")} if e else None,
+            "config": line.get("config"), "clocks": line.get("clocks")}
+
+
 def metric_for(workload):
     return WORKLOAD_METRIC.get(workload, f"MoE-layer tokens/s ({workload})")
 H, I = 2560, 768
@@ -637,7 +663,7 @@ def run_ours(args):
             "step_us_p10_p50_p90": [sorted(step_ms)[int(q * (nsteps - 1))] * 1e3 for q in (0.1, 0.5, 0.9)],
             "tokens_per_s_median_step": ws * T / (statistics.median(step_ms) * 1e-3),
         }
-        print(json.dumps(line), flush=True)
+        emit(line)
     if ws > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -781,7 +807,7 @@ def run_lmhead(args):
             "clocks": clk.summary(), "wall_s_timed_region": t_wall,
             "step_us_p10_p50_p90": [sorted(step_ms)[int(q * (nsteps - 1))] * 1e3 for q in (0.1, 0.5, 0.9)],
         }
-        print(json.dumps(line), flush=True)
+        emit(line)
     if ws > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -815,6 +841,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode_e512_t1")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-secondary", dest="secondary", action="store_false",
+                    help="default run: skip the short runs of the other workloads")
     ap.add_argument("--tokens", type=int, default=0,
                     help="verify workloads: calls of this many tokens (1..the workload's T) instead")
     ap.add_argument("--l2", default="auto", choices=["auto", "rotate", "flush"],
@@ -831,7 +859,37 @@ def main():
     lmhead = args.workload.startswith("lmhead")
     if args.impl == "reference":
         return run_lmhead_reference(args) if lmhead else run_reference(args)
+    if args.secondary and ws == 1 and "--workload" not in sys.argv:
+        return run_with_secondary(args)
     return run_lmhead(args) if lmhead else run_ours(args)
+
+
+def run_with_secondary(args):
+    """The headline workload as usual, then each SECONDARY workload for a
+    short run (at most 50 steps, 3 warm-up, no CPU baseline); one JSON line,
+    the headline's, with the others' compact records under "secondary"."""
+    global _CAPTURE
+    import copy
+    import torch
+    _CAPTURE = []
+    try:
+        rc = run_ours(args)
+        line = _CAPTURE.pop()
+        sec = {}
+        for wl in SECONDARY:
+            a = copy.copy(args)
+            a.workload, a.steps, a.warmup, a.cpu_seconds, a.tokens = wl, min(args.steps, 50), 3, 0.0, 0
+            try:
+                (run_lmhead if wl.startswith("lmhead") else run_ours)(a)
+                sec[wl] = compact(_CAPTURE.pop())
+            except Exception as exc:  # a failing secondary workload does not lose the headline line
+                sec[wl] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+            torch.cuda.empty_cache()
+        line["secondary"] = sec
+    finally:
+        _CAPTURE = None
+    print(json.dumps(line), flush=True)
+    return rc
 
 
 if __name__ == "__main__":

@@ -2,7 +2,8 @@
 
 ling_moe_route_noalloc keeps its scratch in a static device array instead of
 allocating it, for callers that cannot allocate device memory where they
-route tokens.  Its routing must equal what ling_moe_forward_ex reports for the
+route tokens.  Its routing is checked against the fp64 oracle's routing and
+must equal what ling_moe_forward_ex reports for the
 same router weights and tokens: the same fp32 accumulation order gives the
 same logits, so indices and weights match exactly (well inside the 1e-5
 weight tolerance of the other tests).  Two calls in a row on each token count
@@ -47,6 +48,37 @@ def test_route_noalloc_matches_forward_ex(E, with_bias):
                 assert torch.allclose(w, w_ref, rtol=0, atol=1e-5), (E, T, call)
     finally:
         layer.close()
+
+
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_route_noalloc_against_the_oracle(with_bias):
+    """The selection and weights straight against the fp64 oracle's routing,
+    including tokens of extreme magnitude (the power-of-two token scale)."""
+    import numpy as np
+    import oracle
+    from tests.parity import W_TOL, bits
+    E, k = 512, 8
+    lw = workloads.layer_weights(E, seed=0, device="cuda")
+    bias = workloads.zipf_router_bias(E, 1.1) if with_bias else None
+    wr64 = oracle.bf16_bits_to_f64(bits(lw.router_w))
+    kinds = [["normal"], ["normal", "big", "tiny", "mixed"], ["near_max", "all_max", "subnormal"]]
+    for seed, ks in enumerate(kinds):
+        x = workloads.extreme_tokens(ks, seed=4000 + 10 * seed).cuda()
+        idx, w = _route_noalloc(x, lw.router_w, bias.cuda() if bias is not None else None, E, k)
+        torch.cuda.synchronize()
+        logits = oracle.router_logits(oracle.bf16_bits_to_f64(bits(x)), wr64,
+                                      bias.numpy() if bias is not None else None)
+        ref_idx, ref_w = oracle.route(logits, k)
+        srt = -np.sort(-logits, axis=1)
+        near = np.abs(srt[:, k - 1] - srt[:, k]) <= 1e-5 * np.abs(logits).max(axis=1)
+        gi, gw = idx.cpu().numpy(), w.cpu().numpy()
+        for t in range(len(ks)):
+            if near[t]:
+                continue
+            assert set(gi[t].tolist()) == set(ref_idx[t].tolist()), (ks[t], gi[t], ref_idx[t])
+            ref = dict(zip(ref_idx[t].tolist(), ref_w[t].tolist()))
+            for e, wv in zip(gi[t].tolist(), gw[t].tolist()):
+                assert abs(wv - ref[e]) <= W_TOL, (ks[t], e, wv, ref[e])
 
 
 def test_route_noalloc_rejects_sizes_beyond_its_scratch():
