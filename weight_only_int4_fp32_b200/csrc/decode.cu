@@ -424,6 +424,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) moe_decode_kernel(const Dec
     if (warp == 0) { LING_CLK(1); if (lane == 0) g_clk_sink(lg[0] + lg[E - 1]); LING_CLK(2); }
     warp_topk_thresh(lg, E, K, reinterpret_cast<unsigned long long*>(bufA + kMaxExperts * 4), hd.topi[warp],
                      hd.topw[warp], hd.xscale[warp]);
+    // the phase-3 bulk copies overwrite this scratch: order these generic
+    // writes before them
+    fence_async_smem();
     if (warp == 0) LING_CLK(3);
 
   }
