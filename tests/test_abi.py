@@ -173,3 +173,45 @@ def test_binding_rejects_wrong_tensors_before_any_call():
         head.forward_host(torch.zeros((1, 2560), dtype=torch.bfloat16), torch.zeros((1, 999)))
     with pytest.raises(ValueError):
         head.forward(torch.zeros((1, 2560), dtype=torch.bfloat16))
+
+
+def _ep_rc(cfg, w, ep):
+    h = ctypes.c_void_p()
+    rc = lm.lib.ling_moe_create_ep(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(ep) if ep is not None else None,
+                                   ctypes.byref(h))
+    return rc, h.value
+
+
+@pytest.mark.parametrize("begin,count,shared,fmt", [
+    (-1, 4, 1, 0),      # range starts before 0
+    (0, 0, 1, 0),       # no expert
+    (510, 4, 1, 0),     # past the router's experts
+    (0, 4, 2, 0),       # with_shared not 0/1
+    (0, 4, 1, 7),       # unknown format
+])
+def test_create_ep_rejects_bad_ranges_before_the_gpu(begin, count, shared, fmt):
+    rc, h = _ep_rc(_cfg(), _weights(), lm.ling_moe_ep_t(begin, count, shared, fmt))
+    assert rc == lm.LING_MOE_ERR_INVALID_ARG and h is None
+    rc, h = _ep_rc(_cfg(), _weights(), None)
+    assert rc == lm.LING_MOE_ERR_INVALID_ARG and h is None
+
+
+def test_create_ep_needs_shared_weights_only_where_it_computes_them():
+    w = _weights()
+    w.sh_gate = w.sh_up = w.sh_down = None
+    rc, _ = _ep_rc(_cfg(), w, lm.ling_moe_ep_t(0, 4, 1, 0))
+    assert rc == lm.LING_MOE_ERR_INVALID_ARG  # the shared expert is computed here: its weights are required
+    assert "NULL" in lm.ling_moe_last_error()
+    import torch
+    if not torch.cuda.is_available():  # with a GPU the fake pointers would reach the copies
+        rc, _ = _ep_rc(_cfg(), w, lm.ling_moe_ep_t(0, 4, 0, 0))
+        assert rc == lm.LING_MOE_ERR_CUDA  # accepted on the host, then no device to copy to
+
+
+def test_partial_and_round_reject_bad_arguments():
+    assert lm.lib.ling_moe_forward_partial(None, None, 1, None, None, None, None) == lm.LING_MOE_ERR_INVALID_ARG
+    assert lm.lib.ling_moe_round_bf16(None, None, 8, None) == lm.LING_MOE_ERR_INVALID_ARG
+    assert lm.lib.ling_moe_round_bf16(0x100000, 0x200000, 7, None) == lm.LING_MOE_ERR_INVALID_ARG  # n % 8
+    assert lm.lib.ling_moe_round_bf16(0x100004, 0x200000, 8, None) == lm.LING_MOE_ERR_INVALID_ARG  # alignment
+    assert lm.lib.ling_moe_round_bf16(0x100000, 0x100010, 64, None) == lm.LING_MOE_ERR_INVALID_ARG  # overlap
+    assert lm.lib.ling_moe_round_bf16(0x100000, 0x200000, 0, None) == lm.LING_MOE_OK  # nothing to do
