@@ -33,17 +33,23 @@
 namespace lingmoe {
 
 // ---------------------------------------------------------------- roles and sizes
-constexpr int kProdWarps = 8;                  // one A row per thread
+// A producer group is 8 warps, one A row per thread.  Gate/up runs two
+// groups that take alternate pipeline stages (its dequantisation per stage is
+// a dependent chain per warp, so a second group doubles the stages in work);
+// down, whose shared memory holds two B parts per stage, runs one.
+constexpr int kProdWarps = 8;                  // warps per producer group
 constexpr int kEpiWarps = 4;                   // TMEM lane quadrants 0..3
-constexpr int kMmaWarp = kProdWarps + kEpiWarps;  // 12
-constexpr int kTmaWarp = kMmaWarp + 1;            // 13
-constexpr int kTcThreads = (kTmaWarp + 1) * 32;   // 448
-constexpr int kProd = kProdWarps * 32;            // 256
+constexpr int kProd = kProdWarps * 32;            // 256 rows per group
 static_assert(kProd == kTcTileM, "one producer thread per A row");
+__host__ __device__ constexpr int tc_groups(int mode) { return mode == 0 ? 2 : 1; }
+__host__ __device__ constexpr int tc_mma_warp(int mode) { return tc_groups(mode) * kProdWarps + kEpiWarps; }
+__host__ __device__ constexpr int tc_threads(int mode) { return (tc_mma_warp(mode) + 2) * 32; }  // + MMA, TMA warps
 static_assert(kProdWarps % 4 == 0, "epilogue warps must start at a multiple of 4");
 
 constexpr int kTcK = 64;                        // K per stage: one 128-byte swizzle row of fp16
-constexpr int kTcStages = 3;
+// pipeline stages: gate/up 4 (its B stage is half the size), down 3
+// an even count for gate/up, so that every stage slot belongs to one group
+__host__ __device__ constexpr int tc_stages(int mode) { return mode == 0 ? 4 : 3; }
 constexpr int kStageA = kTcTileM * kTcK * 2;    // 32 KB
 constexpr int kStageBPart = kTcTileN * kTcK * 2;  // 16 KB per B part
 constexpr int kBoxRows = 32;                    // B rows per TMA box
@@ -58,10 +64,12 @@ constexpr int kRawStage = kRawCodes + kProd * 8;  // 10 KB
 constexpr unsigned long long kTcWaitNs = 2000000000ull;
 
 __host__ __device__ constexpr int tc_bparts(int mode) { return mode == 0 ? 1 : 2; }
-__host__ __device__ constexpr int tc_raw_stages(int mode) { return mode == 0 ? 4 : 2; }
+// down's code ring depth; gate/up loads its codes straight into registers
+__host__ __device__ constexpr int tc_raw_stages(int mode) { return mode == 0 ? 0 : 2; }
 __host__ __device__ constexpr int tc_nk(int mode) { return (mode == 0 ? kH : kI) / kTcK; }
 __host__ __device__ constexpr size_t tc_bar_off(int mode) {
-  return (size_t)kTcStages * (kStageA + tc_bparts(mode) * kStageBPart) + (size_t)tc_raw_stages(mode) * kRawStage;
+  return (size_t)tc_stages(mode) * (kStageA + tc_bparts(mode) * kStageBPart) +
+         (size_t)tc_groups(mode) * tc_raw_stages(mode) * kRawStage;
 }
 // after the barriers: per epilogue warp, per TMEM buffer, 128 column factors
 constexpr int kFacOff = 256;
@@ -285,17 +293,22 @@ __device__ __forceinline__ void prefetch_tile(const TcParams& p, int4 tl, const 
 // MODE 1, down: A row r is output row 256 mt + r; B = the hi and lo halves of
 // h, both accumulated into one TMEM tile; the epilogue writes y = w (Wd h).
 //
-// Roles: warps 0-7 dequantise A, warps 8-11 drain TMEM, warp 12 issues the
-// MMAs (one thread), warp 13 issues the TMA loads (one thread).  Every role
-// walks the same sequence of tiles (blockIdx.x, + gridDim.x, ...) and stages.
+// Roles: the producer warps dequantise A (gate/up: warps 0-15 in two groups
+// of 8 taking alternate stages; down: warps 0-7), the next 4 warps drain
+// TMEM, then one warp issues the MMAs (one thread) and one the TMA loads (one
+// thread).  Every role walks the same sequence of tiles (blockIdx.x,
+// + gridDim.x, ...) and stages.
 template <int MODE, int C>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(tc_threads(MODE), 1)
 tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmA,
                   const TcParams p) {
   constexpr int NB = tc_bparts(MODE);
   constexpr int R = tc_raw_stages(MODE);
   constexpr int NK = tc_nk(MODE);
-  constexpr int S = kTcStages;
+  constexpr int S = tc_stages(MODE);
+  constexpr int NG = tc_groups(MODE);
+  constexpr int kMmaWarp = tc_mma_warp(MODE);
+  constexpr int kPW = NG * kProdWarps;  // producer warps
   extern __shared__ __align__(1024) unsigned char smem_raw_tc[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw_tc) + 1023) & ~uintptr_t(1023));
@@ -341,25 +354,32 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < kProdWarps) {
+  if (warp < kPW) {
     // ------------------------------------------------ producers: A row r
-    const int r = tid;
+    // group pg takes the stages g = NG q + pg, q = 0, 1, ...
+    const int r = tid & (kProd - 1), pg = tid / kProd;
     const int total = ntl * NK;
-    const uint32_t raw0 = smem_u32(sRaw);
-    // cp.async the codes and the scale word of groups 2kk, 2kk+1 of row r for
-    // stage q into raw slot q % R (one commit group per stage, empty or not)
+    constexpr int RR = R > 0 ? R : 1;
+    const uint32_t raw0 = smem_u32(sRaw) + pg * R * kRawStage;
+    // the codes and the scale word of groups 2kk, 2kk+1 of row r for the
+    // group's q-th stage: gate/up loads them into registers (nc, nsw) one own
+    // stage ahead; down cp.asyncs them into its raw slot q % R (one commit
+    // group per stage, empty or not)
     int jn = -1;
     int4 tln = make_int4(0, 0, 0, 0);
+    uint2 nc[4] = {};
+    uint32_t nsw = 0;
     auto issue = [&](int q) {
-      if (q < total) {
-        const int j = q / NK, kk = q - j * NK;
+      const int gq = NG * q + pg;
+      if (gq < total) {
+        const int j = gq / NK, kk = gq - j * NK;
         if (j != jn) {
           tln = tiles[blockIdx.x + j * gridDim.x];
           jn = j;
         }
         const int4 tl = tln;
         if (tl.x < p.E) {
-          const uint32_t slot = raw0 + (q % R) * kRawStage;
+          const uint32_t slot = raw0 + (q % RR) * kRawStage;
           if (MODE == 0) {
             // row i (gate and up), K blocks 2 kh, 2 kh + 1 of chunk kk: 8 bytes
             // from each of the four fragment lanes 4 (i % 8) + m, and the
@@ -369,8 +389,8 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
             const uint8_t* ub = p.gu + ((size_t)tl.x * kGuUnits + (i >> 3)) * kGuUnitBytes;
 #pragma unroll
             for (int m = 0; m < 4; ++m)
-              cp_async8(slot + m * (kProd * 8) + r * 8, ub + kk * 512 + 16 * (4 * (i & 7) + m) + 8 * kh);
-            cp_async4(slot + kRawCodes + r * 4, ub + kGuScaleOff + (2 * kk + kh) * 32 + 4 * (i & 7));
+              nc[m] = __ldg(reinterpret_cast<const uint2*>(ub + kk * 512 + 16 * (4 * (i & 7) + m) + 8 * kh));
+            nsw = __ldg(reinterpret_cast<const unsigned int*>(ub + kGuScaleOff + (2 * kk + kh) * 32 + 4 * (i & 7)));
           } else {
             // output row n, groups G = 2 kk and G + 1: 8 bytes from each of the
             // four fragment lanes 4 (n % 8) + m, and the two scale words of
@@ -384,16 +404,30 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
           }
         }
       }
-      cp_async_commit();
+      if (MODE == 1) cp_async_commit();
     };
+    if constexpr (MODE == 0) {
+      issue(0);
+    } else {
 #pragma unroll 1
-    for (int q = 0; q < R - 1; ++q) issue(q);
+      for (int q = 0; q < R - 1; ++q) issue(q);
+    }
     int jc = -1;
     int4 tl = make_int4(0, 0, 0, 0);
 #pragma unroll 1
-    for (int g = 0; g < total; ++g) {
-      issue(g + R - 1);
-      cp_async_wait<R - 1>();
+    for (int q = 0; NG * q + pg < total; ++q) {
+      const int g = NG * q + pg;
+      uint2 cw[4];
+      uint32_t sw0 = 0;
+      if constexpr (MODE == 0) {
+#pragma unroll
+        for (int m = 0; m < 4; ++m) cw[m] = nc[m];
+        sw0 = nsw;
+        issue(q + 1);
+      } else {
+        issue(q + R - 1);
+        cp_async_wait<R - 1>();
+      }
       const int j = g / NK, kk = g - j * NK;
       if (j != jc) {
         tl = tiles[blockIdx.x + j * gridDim.x];
@@ -404,12 +438,12 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
       if (lane == 0) ok = tc_wait(&empty[s], ((g / S) & 1) ^ 1, p.err, abort_flag);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       if (tl.x < p.E) {
-        const unsigned char* slot = sRaw + (g % R) * kRawStage;
+        const unsigned char* slot = sRaw + (pg * R + q % RR) * kRawStage;
         if (MODE == 0) {
           // exact fp16 q * s * 2^8 for gate row il and up row 128 + il, K blocks
           // 2 kh and 2 kh + 1 of this stage (natural K order)
           const int il = r & 127, kh = r >> 7;
-          const uint32_t sw = *reinterpret_cast<const uint32_t*>(slot + kRawCodes + r * 4);
+          const uint32_t sw = sw0;
           const float sgf = __uint_as_float(sw << 16) * (float)(1 << kTcScaleShift);
           const float suf = __uint_as_float(sw & 0xFFFF0000u) * (float)(1 << kTcScaleShift);
           const __half2 sg = __float2half2_rn(sgf), sg16 = __float2half2_rn(sgf * 0.0625f);
@@ -420,9 +454,6 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
             mx_factors(sgf, ga, gb);
             mx_factors(suf, ua, ub);
           }
-          uint2 cw[4];
-#pragma unroll
-          for (int m = 0; m < 4; ++m) cw[m] = *reinterpret_cast<const uint2*>(slot + m * (kProd * 8) + r * 8);
           unsigned char* ag = sA + s * kStageA + il * 128;
           unsigned char* au = sA + s * kStageA + (128 + il) * 128;
 #pragma unroll
@@ -461,7 +492,6 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
           const int n = kTcTileM * tl.y + r;
           const uint2 sw = *reinterpret_cast<const uint2*>(slot + kRawCodes + r * 8);
           const __half2 be = __float2half2_rn(1032.0f), bo = __float2half2_rn(1152.0f);
-          uint2 cw[4];
 #pragma unroll
           for (int m = 0; m < 4; ++m) cw[m] = *reinterpret_cast<const uint2*>(slot + m * (kProd * 8) + r * 8);
           unsigned char* a = sA + s * kStageA + r * 128;
@@ -510,7 +540,7 @@ tc_grouped_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
     // ------------------------------------------------ epilogue: TMEM lanes 32 qd .. 32 qd + 31
     const int qd = warp & 3;
     const int l = 32 * qd + lane;  // accumulator row within an M-half
-    float* facw = fac_s + (warp - kProdWarps) * (2 * kTcTileN);
+    float* facw = fac_s + (warp - kPW) * (2 * kTcTileN);
 #pragma unroll 1
     for (int j = 0; j < ntl; ++j) {
       const int b = j & 1;
@@ -731,11 +761,11 @@ cudaError_t tc_encode_maps(TcMaps* m, const __half* xg, const __half* h16, int r
 
 cudaError_t launch_tc_gemm(int mode, const TcMaps& m, const TcParams& p, int nctas, cudaStream_t s) {
   if (p.codec == kCodecMxfp4) {
-    if (mode == 0) tc_grouped_kernel<0, kCodecMxfp4><<<nctas, kTcThreads, tc_smem(0), s>>>(m.b_x, m.a_shgu, p);
-    else tc_grouped_kernel<1, kCodecMxfp4><<<nctas, kTcThreads, tc_smem(1), s>>>(m.b_h, m.a_shdn, p);
+    if (mode == 0) tc_grouped_kernel<0, kCodecMxfp4><<<nctas, tc_threads(0), tc_smem(0), s>>>(m.b_x, m.a_shgu, p);
+    else tc_grouped_kernel<1, kCodecMxfp4><<<nctas, tc_threads(1), tc_smem(1), s>>>(m.b_h, m.a_shdn, p);
   } else {
-    if (mode == 0) tc_grouped_kernel<0, kCodecInt4><<<nctas, kTcThreads, tc_smem(0), s>>>(m.b_x, m.a_shgu, p);
-    else tc_grouped_kernel<1, kCodecInt4><<<nctas, kTcThreads, tc_smem(1), s>>>(m.b_h, m.a_shdn, p);
+    if (mode == 0) tc_grouped_kernel<0, kCodecInt4><<<nctas, tc_threads(0), tc_smem(0), s>>>(m.b_x, m.a_shgu, p);
+    else tc_grouped_kernel<1, kCodecInt4><<<nctas, tc_threads(1), tc_smem(1), s>>>(m.b_h, m.a_shdn, p);
   }
   return cudaGetLastError();
 }
