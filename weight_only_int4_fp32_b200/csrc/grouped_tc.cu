@@ -6,11 +6,13 @@
 //   down:     Y_e[m_e, 2560] = w * (H_e Wd_e^T)                    K = 768
 // as tiles of M = 256 weight rows (two M=128 MMAs) x N <= 128 positions.
 //
-// The weights are the A operand.  Routed weights are dequantised by 8
+// The weights are the A operand.  Routed weights are dequantised by
 // producer warps into exact fp16 values q * s * 2^8 (q has at most 4
 // significant bits and s is a bf16, so the product fits fp16's 11 bits) and
-// written into 128-byte-swizzled K-major shared-memory tiles; their int4
-// codes and scales arrive ahead of use through a per-thread cp.async ring.
+// written into 128-byte-swizzled K-major shared-memory tiles.  Their int4
+// codes and scales arrive ahead of use: gate/up loads them into registers one
+// stage ahead (two producer groups, 4 stages), down through a per-thread
+// cp.async ring (one group, 3 stages).
 // The shared expert's weights are pre-converted fp16 copies that TMA loads
 // directly.  The activations are the B operand, fetched by TMA from buffers
 // in position order: x (fp16, exact after a per-token power-of-two scale) for
@@ -36,7 +38,8 @@ namespace lingmoe {
 // A producer group is 8 warps, one A row per thread.  Gate/up runs two
 // groups that take alternate pipeline stages (its dequantisation per stage is
 // a dependent chain per warp, so a second group doubles the stages in work);
-// down, whose shared memory holds two B parts per stage, runs one.
+// down, whose shared memory holds two B parts per stage, runs one (two
+// groups there need an even stage count, and its two stages measured slower).
 constexpr int kProdWarps = 8;                  // warps per producer group
 constexpr int kEpiWarps = 4;                   // TMEM lane quadrants 0..3
 constexpr int kProd = kProdWarps * 32;            // 256 rows per group
@@ -256,7 +259,7 @@ cudaError_t launch_tc_prep_shared(const __nv_bfloat16* g, const __nv_bfloat16* u
 // ---------------------------------------------------------------- L2 prefetch of a tile
 // Everything one tile reads is contiguous: its 256 weight rows (routed units
 // or fp16 shared rows) and its B rows (positions pos0 .. pos0 + n - 1).
-// Issued for the next tile while the current one runs, so that the cp.async
+// Issued for the next tile while the current one runs, so that the code
 // and TMA loads of the main loop find their data in L2.
 template <int MODE>
 __device__ __forceinline__ void prefetch_tile(const TcParams& p, int4 tl, const __half* xg, const __half* h16,
