@@ -87,29 +87,29 @@ L2_FLUSH_BYTES = 256 << 20
 # the command), valid only while the kernel's sources are the ones captured:
 # the sources are hashed and the figure is reported as null once they change.
 TRAFFIC = {
-    "decode_e512_t1": {"bytes": 41_048_576 + 0,
+    "decode_e512_t1": {"bytes": 41_048_320 + 1_280,
                        "sources": ('decode.cu', 'decode.h', 'common.cuh', 'layout.h'),
-                       "sha256": "552ed47622eede2e2df282a8a05ebdbc331566fa577d31df841c3c22beb4b4f8"},
-    "verify_e512_t4": {"bytes": 132_519_424 + 2_881_536,
+                       "sha256": "722bfd0b89f3542e928f71abd6a629ed2429a8e24c609c3c311ed185a0bb212a"},
+    "verify_e512_t4": {"bytes": 132_140_288 + 2_912_768,
                        "sources": ('decode.cu', 'decode.h', 'common.cuh', 'layout.h'),
-                       "sha256": "552ed47622eede2e2df282a8a05ebdbc331566fa577d31df841c3c22beb4b4f8"},
+                       "sha256": "722bfd0b89f3542e928f71abd6a629ed2429a8e24c609c3c311ed185a0bb212a"},
     # one launch for the 8-token window (the union, ~62 experts, read once)
-    "verify_e512_t8": {"bytes": 220_087_552 + 3_197_696,
+    "verify_e512_t8": {"bytes": 219_967_232 + 3_237_632,
                        "sources": ('decode.cu', 'decode.h', 'common.cuh', 'layout.h'),
-                       "sha256": "552ed47622eede2e2df282a8a05ebdbc331566fa577d31df841c3c22beb4b4f8"},
+                       "sha256": "722bfd0b89f3542e928f71abd6a629ed2429a8e24c609c3c311ed185a0bb212a"},
     # online-FP8 LM head: lmh_mma_kernel, the only kernel of a call
     "lmhead_fp8_v157184_t1": {"bytes": 403_095_296 + 3_477_504,
                               "sources": ('lmhead.cu', 'lmhead.h', 'common.cuh', 'layout.h'),
                               "sha256": "97b9d0faf1db3059f55fc99a28f7971773752ba535a85e10db5243403a1fbea5"},
     # MXFP4 routed experts (the decode kernel's E2M1 instantiation); the unit
     # layout keeps a bf16 scale per 32, so 8 experts read 3,317,760 B each
-    "decode_e512_t1_mxfp4": {"bytes": 41_050_368 + 16_896,
+    "decode_e512_t1_mxfp4": {"bytes": 41_051_136 + 37_888,
                              "sources": ('decode.cu', 'decode.h', 'common.cuh', 'layout.h'),
-                             "sha256": "552ed47622eede2e2df282a8a05ebdbc331566fa577d31df841c3c22beb4b4f8"},
+                             "sha256": "722bfd0b89f3542e928f71abd6a629ed2429a8e24c609c3c311ed185a0bb212a"},
     # token-grouped: the dominant kernel, tc_grouped_kernel<0> (gate/up tiles)
-    "prefill_e512_t2048_zipf": {"bytes": 456_468_224 + 53_267_456,
+    "prefill_e512_t2048_zipf": {"bytes": 459_126_272 + 52_561_920,
                                 "sources": ('grouped_tc.cu', 'grouped_tc.h', 'common.cuh', 'layout.h'),
-                                "sha256": "e2b129a4ebb03a66cf5653d3cce844530c5625db49547d188882ce7315df1735"},
+                                "sha256": "458c7407873c6c414b9498241e25dd17313a763852a163987dc634a7406c5806"},
 }
 
 
